@@ -1,0 +1,280 @@
+/*
+ * la2_oracle.c -- CPU fp64 oracle for Lightning Attention-2 (causal linear
+ * attention with per-head decay), forward and backward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: only the tests, the smoke check and the benchmark's CPU
+ * baseline do.  It shares no code, header or constant with the CUDA library.
+ *
+ * What it computes (per independent sequence of length T, identity feature
+ * map, no normaliser, no 1/sqrt(d) scale):
+ *
+ *     o_t = sum_{s<=t} lambda^(t-s) (q_t . k_s) v_s
+ *
+ * This is causal linear attention as the "Lightning Attention" explainer page
+ * (lizeman.github.io llm-arch-kb, section 1 "Premise") writes it, with the
+ * feature map phi set to the identity (section 2, "Let phi ... Qin et al. use
+ * the identity"), the denominator dropped (the default configuration pairs the
+ * identity map with a normalisation gate instead of a divisor), and a per-head
+ * decay lambda in (0,1] on the term of lag t-s, lambda = 1 giving the plain
+ * prefix sum of section 1.
+ *
+ * Functions:
+ *   la2o_forward            serial prefix-sum recurrence of section 1,
+ *                           S_t = lambda S_{t-1} + k_t v_t^T,  o_t = S_t^T q_t.
+ *   la2o_backward           gradients of L = sum_t do_t . o_t by the two
+ *                           recurrences that differentiate the one above:
+ *                           dq_t = S_t do_t (forward sweep);
+ *                           R_t = lambda R_{t+1} + q_t do_t^T,
+ *                           dk_t = R_t v_t, dv_t = R_t^T k_t (reverse sweep).
+ *   la2o_forward_blocked    the tiled algorithm of section 2 (steps 1-4:
+ *                           intra-tile masked product, inter-tile product with
+ *                           the running state, state update), with the decay
+ *                           folded into each step.  The decay exponents are not
+ *                           printed on the pages; they are derived from the
+ *                           definition above:
+ *                             intra weight   lambda^(r-c), r >= c
+ *                             inter weight   lambda^(r+1) on row r
+ *                             state update   KV <- lambda^TB KV
+ *                                                  + sum_r lambda^(TB-1-r) k_r v_r^T
+ *   la2o_backward_blocked   the mirrored tiling for the backward (the pages say
+ *                           only that tiling covers the backward too): dq by a
+ *                           forward-direction blocked scan, dk and dv by a
+ *                           reverse-direction blocked scan with
+ *                             intra weight   lambda^(c-r), c >= r
+ *                             inter weight   lambda^(TB-r) on row r
+ *                             state update   R <- lambda^TB R
+ *                                                 + sum_r lambda^r q_r do_r^T
+ *
+ * Layout: sequence-major, row-major: x[n][t][j] for sequence n, position t,
+ * feature j.  lam[n] is the decay of sequence n.  All arithmetic is double.
+ * Sequences are independent; they are split across OpenMP threads.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static void set_threads(int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+}
+
+int la2o_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* lambda^n for an integer n >= 0, by the C library's pow in double. */
+static double lpow(double lam, int n) { return pow(lam, (double)n); }
+
+/* ---------------------------------------------------------------- forward */
+
+void la2o_forward(int NS, int T, int d, int e, const double *lam,
+                  const double *q, const double *k, const double *v,
+                  double *o, int nthreads)
+{
+    set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < NS; ++n) {
+        const double *qn = q + (size_t)n * T * d;
+        const double *kn = k + (size_t)n * T * d;
+        const double *vn = v + (size_t)n * T * e;
+        double *on = o + (size_t)n * T * e;
+        double *S = (double *)calloc((size_t)d * e, sizeof(double)); /* S[i][j] */
+        const double l = lam[n];
+        for (int t = 0; t < T; ++t) {
+            const double *qt = qn + (size_t)t * d, *kt = kn + (size_t)t * d;
+            const double *vt = vn + (size_t)t * e;
+            /* S_t = lambda S_{t-1} + k_t v_t^T */
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < e; ++j)
+                    S[(size_t)i * e + j] = l * S[(size_t)i * e + j] + kt[i] * vt[j];
+            /* o_t = S_t^T q_t */
+            double *ot = on + (size_t)t * e;
+            for (int j = 0; j < e; ++j) ot[j] = 0.0;
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < e; ++j) ot[j] += qt[i] * S[(size_t)i * e + j];
+        }
+        free(S);
+    }
+}
+
+/* --------------------------------------------------------------- backward */
+
+void la2o_backward(int NS, int T, int d, int e, const double *lam,
+                   const double *q, const double *k, const double *v,
+                   const double *dout, double *dq, double *dk, double *dv,
+                   int nthreads)
+{
+    set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < NS; ++n) {
+        const double *qn = q + (size_t)n * T * d;
+        const double *kn = k + (size_t)n * T * d;
+        const double *vn = v + (size_t)n * T * e;
+        const double *gn = dout + (size_t)n * T * e;
+        double *dqn = dq + (size_t)n * T * d;
+        double *dkn = dk + (size_t)n * T * d;
+        double *dvn = dv + (size_t)n * T * e;
+        double *S = (double *)calloc((size_t)d * e, sizeof(double));
+        const double l = lam[n];
+
+        /* forward sweep: dq_t = S_t do_t, S_t as in the forward pass */
+        for (int t = 0; t < T; ++t) {
+            const double *kt = kn + (size_t)t * d, *vt = vn + (size_t)t * e;
+            const double *gt = gn + (size_t)t * e;
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < e; ++j)
+                    S[(size_t)i * e + j] = l * S[(size_t)i * e + j] + kt[i] * vt[j];
+            double *dqt = dqn + (size_t)t * d;
+            for (int i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < e; ++j) acc += S[(size_t)i * e + j] * gt[j];
+                dqt[i] = acc;
+            }
+        }
+
+        /* reverse sweep: R_t = lambda R_{t+1} + q_t do_t^T,
+           dk_t = R_t v_t, dv_t = R_t^T k_t                     */
+        double *R = S;
+        memset(R, 0, sizeof(double) * (size_t)d * e);
+        for (int t = T - 1; t >= 0; --t) {
+            const double *qt = qn + (size_t)t * d, *kt = kn + (size_t)t * d;
+            const double *vt = vn + (size_t)t * e, *gt = gn + (size_t)t * e;
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < e; ++j)
+                    R[(size_t)i * e + j] = l * R[(size_t)i * e + j] + qt[i] * gt[j];
+            double *dkt = dkn + (size_t)t * d, *dvt = dvn + (size_t)t * e;
+            for (int i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < e; ++j) acc += R[(size_t)i * e + j] * vt[j];
+                dkt[i] = acc;
+            }
+            for (int j = 0; j < e; ++j) dvt[j] = 0.0;
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < e; ++j) dvt[j] += R[(size_t)i * e + j] * kt[i];
+        }
+        free(S);
+    }
+}
+
+/* ------------------------------------------------------- blocked variants */
+
+/*
+ * One blocked scan, used for the forward pass and for every backward output:
+ *
+ *   dir = +1:  x_t = sum_{s<=t} lambda^(t-s) (a_t . b_s) c_s
+ *   dir = -1:  x_t = sum_{s>=t} lambda^(s-t) (a_t . b_s) c_s
+ *
+ * a, b are [T][da]; c, x are [T][dc].  Tiles are the contiguous ranges
+ * [i*TB, min((i+1)*TB, T)); the last one may be short.  For dir = +1 the tiles
+ * are visited first to last, for dir = -1 last to first.  Within tile i, with
+ * local row r and local column c:
+ *
+ *   dir = +1:  x_r = sum_{c<=r} lambda^(r-c) (a_r . b_c) c_c  +  lambda^(r+1) a_r^T W
+ *              W  <- lambda^TB W + sum_c lambda^(TB-1-c) b_c c_c^T
+ *   dir = -1:  x_r = sum_{c>=r} lambda^(c-r) (a_r . b_c) c_c  +  lambda^(TB-r) a_r^T W
+ *              W  <- lambda^TB W + sum_c lambda^c b_c c_c^T
+ *
+ * W (da x dc) starts at zero.  Every exponent is measured from a tile's first
+ * row, so a short last tile needs no special case: in the forward direction
+ * the state after it is never used, and in the reverse direction it is the
+ * first tile visited, where W is still zero, and the state it leaves behind is
+ * sum_c lambda^c b_c c_c^T, exactly the lag from the start of the tile.
+ */
+static void blocked_scan(int T, int da, int dc, int TB, int dir, double lam,
+                         const double *a, const double *b, const double *c,
+                         double *x)
+{
+    const int nb = (T + TB - 1) / TB;
+    double *W = (double *)calloc((size_t)da * dc, sizeof(double));
+    double *Wn = (double *)calloc((size_t)da * dc, sizeof(double));
+    const double lTB = lpow(lam, TB);
+    for (int step = 0; step < nb; ++step) {
+        const int i = dir > 0 ? step : nb - 1 - step;
+        const int t0 = i * TB;
+        const int len = (t0 + TB <= T) ? TB : T - t0;
+        for (int r = 0; r < len; ++r) {
+            const double *ar = a + (size_t)(t0 + r) * da;
+            double *xr = x + (size_t)(t0 + r) * dc;
+            for (int j = 0; j < dc; ++j) xr[j] = 0.0;
+            /* intra-tile: masked, decayed left product */
+            for (int cc = 0; cc < len; ++cc) {
+                int lag = dir > 0 ? r - cc : cc - r;
+                if (lag < 0) continue;
+                const double *bc = b + (size_t)(t0 + cc) * da;
+                double s = 0.0;
+                for (int u = 0; u < da; ++u) s += ar[u] * bc[u];
+                s *= lpow(lam, lag);
+                const double *ccv = c + (size_t)(t0 + cc) * dc;
+                for (int j = 0; j < dc; ++j) xr[j] += s * ccv[j];
+            }
+            /* inter-tile: right product with the running state */
+            const double w = dir > 0 ? lpow(lam, r + 1) : lpow(lam, TB - r);
+            for (int u = 0; u < da; ++u) {
+                const double au = w * ar[u];
+                for (int j = 0; j < dc; ++j) xr[j] += au * W[(size_t)u * dc + j];
+            }
+        }
+        /* state update, using the unmasked tile */
+        for (size_t z = 0; z < (size_t)da * dc; ++z) Wn[z] = lTB * W[z];
+        for (int cc = 0; cc < len; ++cc) {
+            const double w = dir > 0 ? lpow(lam, TB - 1 - cc) : lpow(lam, cc);
+            const double *bc = b + (size_t)(t0 + cc) * da;
+            const double *ccv = c + (size_t)(t0 + cc) * dc;
+            for (int u = 0; u < da; ++u) {
+                const double bu = w * bc[u];
+                for (int j = 0; j < dc; ++j) Wn[(size_t)u * dc + j] += bu * ccv[j];
+            }
+        }
+        double *tmp = W; W = Wn; Wn = tmp;
+    }
+    free(W);
+    free(Wn);
+}
+
+void la2o_forward_blocked(int NS, int T, int d, int e, int TB, const double *lam,
+                          const double *q, const double *k, const double *v,
+                          double *o, int nthreads)
+{
+    set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < NS; ++n)
+        blocked_scan(T, d, e, TB, +1, lam[n], q + (size_t)n * T * d,
+                     k + (size_t)n * T * d, v + (size_t)n * T * e,
+                     o + (size_t)n * T * e);
+}
+
+/*
+ * Blocked backward.  Differentiating o_t = sum_{s<=t} lambda^(t-s)(q_t.k_s) v_s
+ * against L = sum_t do_t . o_t gives
+ *   dq_t = sum_{s<=t} lambda^(t-s) (do_t . v_s) k_s   forward scan (a=do, b=v, c=k)
+ *   dk_s = sum_{t>=s} lambda^(t-s) (v_s . do_t) q_t   reverse scan (a=v, b=do, c=q)
+ *   dv_s = sum_{t>=s} lambda^(t-s) (k_s . q_t) do_t   reverse scan (a=k, b=q, c=do)
+ */
+void la2o_backward_blocked(int NS, int T, int d, int e, int TB, const double *lam,
+                           const double *q, const double *k, const double *v,
+                           const double *dout, double *dq, double *dk, double *dv,
+                           int nthreads)
+{
+    set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < NS; ++n) {
+        const double *qn = q + (size_t)n * T * d, *kn = k + (size_t)n * T * d;
+        const double *vn = v + (size_t)n * T * e, *gn = dout + (size_t)n * T * e;
+        blocked_scan(T, e, d, TB, +1, lam[n], gn, vn, kn, dq + (size_t)n * T * d);
+        blocked_scan(T, e, d, TB, -1, lam[n], vn, gn, qn, dk + (size_t)n * T * d);
+        blocked_scan(T, d, e, TB, -1, lam[n], kn, qn, gn, dv + (size_t)n * T * e);
+    }
+}

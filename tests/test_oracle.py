@@ -1,0 +1,200 @@
+"""Pins for the fp64 CPU oracle, against things other than the oracle itself.
+
+Each check is chosen so that a plausible slip in the oracle (a dropped term, a
+wrong exponent or sign, a transposed operand, an off-by-one in a sweep) fails:
+
+* brute force: the O(T^2) masked sum of the definition, and the matrix forms
+  of its three gradients, on tiny inputs with d != e;
+* finite differences of L = sum dO * O (O is linear in each single input
+  coordinate, so central differences are exact up to rounding);
+* a hand-worked example (tests/golden/hand_T3.json);
+* closed forms: T = 1, lambda = 1 (textbook masked product), lambda -> 0;
+* invariants: causality, linearity in V, homogeneity in Q;
+* the tiled algorithm of the pages with the derived decay exponents equals the
+  serial recurrence for every tile size, including short last tiles.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.filterwarnings("ignore::DeprecationWarning")
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+def _decay_matrix(T, lam):
+    t = np.arange(T)
+    lag = t[:, None] - t[None, :]
+    D = np.where(lag >= 0, np.power(lam, np.maximum(lag, 0).astype(np.float64)), 0.0)
+    return D
+
+
+def _brute(q, k, v, do, lam):
+    """Per-sequence masked products: the definition written as matrices."""
+    D = _decay_matrix(q.shape[0], lam)
+    A = (q @ k.T) * D            # A_ts = lam^(t-s) (q_t . k_s), s <= t
+    G = (do @ v.T) * D           # G_ts = lam^(t-s) (do_t . v_s)
+    o = A @ v
+    dq = G @ k
+    dk = G.T @ q
+    dv = A.T @ do
+    return o, dq, dk, dv
+
+
+def _rel(a, b):
+    return np.max(np.abs(a - b)) / max(np.max(np.abs(b)), 1e-300)
+
+
+LAMS = [1.0, 0.9, 0.5, 2.0 ** -20]
+
+
+@pytest.mark.parametrize("T,d,e", [(1, 3, 2), (5, 1, 1), (17, 3, 8), (64, 8, 3)])
+def test_brute_force_forward_and_gradients(oracle_mod, T, d, e):
+    rng = np.random.default_rng(1234 + T)
+    ns = len(LAMS)
+    q, k = _rand(rng, ns, T, d), _rand(rng, ns, T, d)
+    v, do = _rand(rng, ns, T, e), _rand(rng, ns, T, e)
+    lam = np.array(LAMS)
+    o = oracle_mod.forward(q, k, v, lam)
+    dq, dk, dv = oracle_mod.backward(q, k, v, lam, do)
+    for n in range(ns):
+        ref = _brute(q[n], k[n], v[n], do[n], lam[n])
+        for got, want in zip((o[n], dq[n], dk[n], dv[n]), ref):
+            assert _rel(got, want) <= 1e-12
+
+
+@pytest.mark.parametrize("lam", [1.0, 0.9])
+def test_finite_differences(oracle_mod, lam):
+    rng = np.random.default_rng(7)
+    T, d, e = 6, 3, 2
+    q, k, v, do = _rand(rng, T, d), _rand(rng, T, d), _rand(rng, T, e), _rand(rng, T, e)
+
+    def loss(qq, kk, vv):
+        return float(np.sum(do * oracle_mod.forward(qq[None], kk[None], vv[None], [lam])[0]))
+
+    dq, dk, dv = (g[0] for g in oracle_mod.backward(q[None], k[None], v[None], [lam], do[None]))
+    h = 0.5
+    for x, g, idx in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        fd = np.zeros_like(x)
+        for i in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[i] += h
+            xm[i] -= h
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[idx], args_m[idx] = xp, xm
+            fd[i] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        assert np.max(np.abs(fd - g)) <= 1e-10 * max(1.0, np.max(np.abs(g)))
+
+
+def test_hand_worked_example(oracle_mod):
+    with open(os.path.join(GOLDEN, "hand_T3.json")) as f:
+        g = json.load(f)
+    col = lambda key: np.array(g[key], dtype=np.float64)[None, :, None]
+    q, k, v, do = col("q"), col("k"), col("v"), col("do")
+    o = oracle_mod.forward(q, k, v, [g["lambda"]])
+    dq, dk, dv = oracle_mod.backward(q, k, v, [g["lambda"]], do)
+    for key, got in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv)):
+        np.testing.assert_array_equal(got[0, :, 0], np.array(g[key]))
+    for blk in (1, 2, 3):
+        np.testing.assert_array_equal(oracle_mod.forward_blocked(q, k, v, [g["lambda"]], blk)[0, :, 0],
+                                      np.array(g["o"]))
+        got = oracle_mod.backward_blocked(q, k, v, [g["lambda"]], do, blk)
+        for key, x in zip(("dq", "dk", "dv"), got):
+            np.testing.assert_array_equal(x[0, :, 0], np.array(g[key]))
+
+
+def test_T1_closed_form(oracle_mod):
+    rng = np.random.default_rng(3)
+    d, e = 5, 4
+    q, k, v, do = _rand(rng, 3, 1, d), _rand(rng, 3, 1, d), _rand(rng, 3, 1, e), _rand(rng, 3, 1, e)
+    lam = np.array([1.0, 0.3, 1e-9])
+    o = oracle_mod.forward(q, k, v, lam)
+    dq, dk, dv = oracle_mod.backward(q, k, v, lam, do)
+    for n in range(3):
+        qk = q[n, 0] @ k[n, 0]
+        dov = do[n, 0] @ v[n, 0]
+        np.testing.assert_allclose(o[n, 0], qk * v[n, 0], rtol=1e-14, atol=0)
+        np.testing.assert_allclose(dq[n, 0], dov * k[n, 0], rtol=1e-14, atol=0)
+        np.testing.assert_allclose(dk[n, 0], dov * q[n, 0], rtol=1e-14, atol=0)
+        np.testing.assert_allclose(dv[n, 0], qk * do[n, 0], rtol=1e-14, atol=0)
+
+
+def test_lambda_one_is_textbook_causal_linear_attention(oracle_mod):
+    rng = np.random.default_rng(11)
+    T, d, e = 40, 6, 7
+    q, k, v = _rand(rng, T, d), _rand(rng, T, d), _rand(rng, T, e)
+    want = np.tril(q @ k.T) @ v
+    got = oracle_mod.forward(q[None], k[None], v[None], [1.0])[0]
+    assert _rel(got, want) <= 1e-12
+    # and, as a prefix sum, o_t = q_t^T sum_{s<=t} k_s v_s^T
+    S = np.cumsum(k[:, :, None] * v[:, None, :], axis=0)
+    assert _rel(got, np.einsum("td,tde->te", q, S)) <= 1e-12
+
+
+def test_tiny_lambda_keeps_only_the_diagonal(oracle_mod):
+    rng = np.random.default_rng(5)
+    T, d, e = 12, 4, 3
+    q, k, v = _rand(rng, T, d), _rand(rng, T, d), _rand(rng, T, e)
+    lam = 2.0 ** -30
+    got = oracle_mod.forward(q[None], k[None], v[None], [lam])[0]
+    want = np.sum(q * k, axis=1)[:, None] * v
+    assert np.max(np.abs(got - want)) <= 1e-7 * np.max(np.abs(want))
+
+
+def test_causality(oracle_mod):
+    rng = np.random.default_rng(9)
+    T, d, e, tp = 30, 4, 5, 17
+    q, k, v = _rand(rng, T, d), _rand(rng, T, d), _rand(rng, T, e)
+    base = oracle_mod.forward(q[None], k[None], v[None], [0.95])[0]
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    q2[tp:] += 1.0
+    k2[tp:] -= 2.0
+    v2[tp:] *= 3.0
+    pert = oracle_mod.forward(q2[None], k2[None], v2[None], [0.95])[0]
+    np.testing.assert_array_equal(pert[:tp], base[:tp])
+    assert np.all(np.abs(pert[tp:] - base[tp:]).max(axis=1) > 0)
+
+
+def test_linearity_and_homogeneity(oracle_mod):
+    rng = np.random.default_rng(13)
+    T, d, e = 25, 3, 4
+    q, k, v1, v2 = _rand(rng, T, d), _rand(rng, T, d), _rand(rng, T, e), _rand(rng, T, e)
+    f = lambda qq, vv: oracle_mod.forward(qq[None], k[None], vv[None], [0.8])[0]
+    assert _rel(f(q, 2.0 * v1 - 3.0 * v2), 2.0 * f(q, v1) - 3.0 * f(q, v2)) <= 1e-12
+    assert _rel(f(-1.5 * q, v1), -1.5 * f(q, v1)) <= 1e-12
+
+
+@pytest.mark.parametrize("T", [1, 7, 64, 65, 129, 300])
+@pytest.mark.parametrize("block", [1, 2, 3, 5, 64, 128, 256, "T"])
+def test_blocked_equals_serial(oracle_mod, T, block):
+    blk = T if block == "T" else block
+    rng = np.random.default_rng(T * 1000 + blk)
+    d, e = 4, 3
+    lam = np.array([1.0, 0.97, 0.5])
+    q, k = _rand(rng, 3, T, d), _rand(rng, 3, T, d)
+    v, do = _rand(rng, 3, T, e), _rand(rng, 3, T, e)
+    o = oracle_mod.forward(q, k, v, lam)
+    grads = oracle_mod.backward(q, k, v, lam, do)
+    ob = oracle_mod.forward_blocked(q, k, v, lam, blk)
+    gb = oracle_mod.backward_blocked(q, k, v, lam, do, blk)
+    assert _rel(ob, o) <= 1e-12
+    for a, b in zip(gb, grads):
+        assert _rel(a, b) <= 1e-12
+
+
+def test_sequences_are_independent_and_use_their_own_decay(oracle_mod):
+    rng = np.random.default_rng(21)
+    T, d, e = 20, 3, 2
+    q, k, v = _rand(rng, 4, T, d), _rand(rng, 4, T, d), _rand(rng, 4, T, e)
+    lam = np.array([0.5, 1.0, 0.9, 0.99])
+    together = oracle_mod.forward(q, k, v, lam)
+    for n in range(4):
+        alone = oracle_mod.forward(q[n:n + 1], k[n:n + 1], v[n:n + 1], lam[n:n + 1])
+        np.testing.assert_array_equal(together[n], alone[0])
