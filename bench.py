@@ -1,0 +1,402 @@
+#!/usr/bin/env python3
+"""Throughput of the Lightning Attention-2 hot path (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = la2_fwd + la2_bwd over one batch of the named workload (default:
+the TNL-400M-shaped layer), inputs resident in HBM.  Prints one JSON line.
+Under torchrun (N > 1) every rank runs its own replica (the path has no
+exchange step), the timed region is bracketed by a barrier and device
+synchronisation on every rank, and the slowest rank's time is reported.
+
+`--impl reference` times the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the same workload (the pages ship no runnable reference).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from causal_linear_attention_la2_b200 import inputs as I  # noqa: E402
+
+METRIC = "fwd+bwd tokens/sec and TFLOP/s (fraction of bf16 TC peak) vs T, 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+# ------------------------------------------------------------------ helpers
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "causal_linear_attention_la2_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def flops_per_token_head(w: I.Workload) -> float:
+    """Credited fwd+bwd FLOPs per (token, head): 3 x (2 T_B (d + e) + 4 d e)."""
+    return 3.0 * (2.0 * w.block * (w.d + w.e) + 4.0 * w.d * w.e)
+
+
+def elem_bytes(w: I.Workload) -> int:
+    return 2 if w.dtype == "bf16" else 4
+
+
+def bwd_algorithmic_bytes(w: I.Workload) -> float:
+    """la2_bwd reads q, k, v, dO and writes dq, dk, dv, each once."""
+    return float(elem_bytes(w)) * w.sequences * w.T * (3 * w.d + 4 * w.e)
+
+
+def fwd_algorithmic_bytes(w: I.Workload) -> float:
+    return float(elem_bytes(w)) * w.sequences * w.T * (2 * w.d + 2 * w.e)
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"la2_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], 0.0, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = max(smax, float(parts[2]))
+                except ValueError:
+                    continue
+                for n, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- CPU oracle
+
+class OracleSample:
+    """Fwd+bwd of the fp64 oracle on a sample of whole sequences of a workload.
+
+    A sequence is one (b, h); H of them carry the per-head work of w.T tokens,
+    so a sample of n sequences stands for n * T / H tokens of the metric.
+    """
+
+    def __init__(self, w: I.Workload, x, target_s: float):
+        import oracle
+        oracle.build()
+        self.oracle = oracle
+        self.w = w
+        self.cores = len(os.sched_getaffinity(0))
+        B, H = w.B, w.H
+        self.lam = np.broadcast_to(x["lam"].numpy().astype(np.float64)[None, :],
+                                   (B, H)).reshape(-1)
+        self.q, self.k, self.v, self.do = (x[n].reshape(B * H, w.T, -1)
+                                           for n in ("q", "k", "v", "do"))
+        n = self.cores
+        dt = self.run(n)
+        if dt < target_s / 2:
+            n = min(64 * self.cores, max(n, int(n * target_s / max(dt, 1e-3))))
+        self.n = n
+
+    def run(self, n=None):
+        n = self.n if n is None else n
+        idx = np.arange(n) % (self.w.B * self.w.H)
+        t = torch.from_numpy(idx)
+        qs, ks, vs, ds = self.q[t], self.k[t], self.v[t], self.do[t]
+        t0 = time.perf_counter()
+        self.oracle.forward(qs, ks, vs, self.lam[idx], nthreads=self.cores)
+        self.oracle.backward(qs, ks, vs, self.lam[idx], ds, nthreads=self.cores)
+        return time.perf_counter() - t0
+
+    def rate(self):
+        dt = self.run()
+        tokens = self.n * self.w.T / self.w.H
+        return {"value": tokens / dt, "unit": "tokens/s", "cores": self.cores, "kind": "oracle",
+                "sample": f"{self.n} whole sequences (b,h) of T={self.w.T}, d={self.w.d}, "
+                          f"e={self.w.e}: {tokens:.0f} token-equivalents in {dt:.2f} s"}
+
+
+def oracle_rate(w: I.Workload, x, target_s: float = 12.0):
+    return OracleSample(w, x, target_s).rate()
+
+
+# -------------------------------------------------------------- main paths
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = torch.device("cuda") if torch.cuda.is_available() else torch.device("cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return 0
+    x = I.make_workload_inputs(w, seed=args.seed)
+    # each step is one bounded sample; the whole run stays within a few minutes
+    per_step = min(args.ref_seconds, 150.0 / max(1, args.steps))
+    sample = OracleSample(w, x, per_step)  # its calibration run doubles as warm-up
+    rates = []
+    base = None
+    for _ in range(max(1, args.steps)):
+        r = sample.rate()
+        rates.append(r["value"])
+        base = r
+    value = statistics.median(rates)
+    base = dict(base, value=value)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * w.tokens / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args),
+        "cpu_baseline": base,
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, args):
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "e": w.e,
+            "block": w.block, "global_batch": w.B * args.gpus, "seq_len": w.T,
+            "parallelism": f"replicas{args.gpus}",
+            "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"}
+
+
+def run_ours(args, w, world, rank, local):
+    from causal_linear_attention_la2_b200 import la2
+    la2.load()
+    dev = torch.device("cuda", local)
+    x = I.make_workload_inputs(w, seed=args.seed)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    lam = x["lam"].to(dev)
+    out = torch.empty_like(v)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    launches = 0
+
+    def step():
+        nonlocal launches
+        la2.la2_fwd(q, k, v, lam, out=out, block=w.block)
+        launches += la2.la2_last_launch_count()
+        la2.la2_bwd(q, k, v, lam, do, dq=dq, dk=dk, dv=dv, block=w.block)
+        launches += la2.la2_last_launch_count()
+
+    for _ in range(args.warmup):
+        flush.fill_(0.0)
+        step()
+    torch.cuda.synchronize(dev)
+    assert la2.la2_device_status(reset=True) == 0, "kernel reported a device fault in warm-up"
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    launches = 0
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        s, m, e = ev[i]
+        s.record(stream)
+        la2.la2_fwd(q, k, v, lam, out=out, block=w.block)
+        launches += la2.la2_last_launch_count()
+        m.record(stream)
+        la2.la2_bwd(q, k, v, lam, do, dq=dq, dk=dk, dv=dv, block=w.block)
+        launches += la2.la2_last_launch_count()
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    fwd_ms = [s.elapsed_time(m) for s, m, _ in ev]
+    bwd_ms = [m.elapsed_time(e) for _, m, e in ev]
+    step_ms = sum(fwd_ms) / len(fwd_ms) + sum(bwd_ms) / len(bwd_ms)
+    step_ms = max_over_ranks(step_ms, world)
+    assert la2.la2_device_status(reset=True) == 0, "kernel reported a device fault"
+
+    # end to end through the public API: pinned host in -> device -> host out
+    hosts = {n: x[n].pin_memory() for n in ("q", "k", "v", "do")}
+    houts = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (out, dq, dk, dv)]
+    h2d = sum(t.numel() * t.element_size() for t in hosts.values())
+    d2h = sum(t.numel() * t.element_size() for t in houts)
+    e2e_steps = max(2, min(args.steps, 5))
+
+    def e2e_step():
+        qd, kd, vd, dd = (hosts[n].to(dev, non_blocking=True) for n in ("q", "k", "v", "do"))
+        la2.la2_fwd(qd, kd, vd, lam, out=out, block=w.block)
+        la2.la2_bwd(qd, kd, vd, lam, dd, dq=dq, dk=dk, dv=dv, block=w.block)
+        for h, dsrc in zip(houts, (out, dq, dk, dv)):
+            h.copy_(dsrc, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1) / e2e_steps, world)
+    barrier(world)
+
+    if rank != 0:
+        return 0
+
+    pk, pk_kind = peaks()
+    hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    tc = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    tokens_per_step = w.tokens * world
+    value = tokens_per_step / (step_ms * 1e-3)
+    bwd_avg_ms = sum(bwd_ms) / len(bwd_ms)
+    achieved = bwd_algorithmic_bytes(w) / (bwd_avg_ms * 1e-3) / 1e9
+    traffic = None
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            t = json.load(f)
+        ent = t.get(w.name, {})
+        if ent.get("source_hash") == kernel_source_hash():
+            traffic = ent.get("bwd_dram_bytes_per_launch")
+    except (OSError, ValueError):
+        pass
+    tflops = flops_per_token_head(w) * w.T * w.sequences * world / (step_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic", "config": workload_config(w, args),
+        "tflops": tflops, "tc_frac": tflops / (tc * world), "tc_peak_tflops": tc,
+        "fwd_ms": sum(fwd_ms) / len(fwd_ms), "bwd_ms": bwd_avg_ms,
+        "roofline": {"bound": "hbm", "kernel": "la2_scan_bf16_sm100 (la2_bwd launch)",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": traffic,
+                     "peak_kind": f"{pk_kind} hbm_gbs"},
+        "e2e": {"value": tokens_per_step / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_rate(w, x, target_s=args.ref_seconds)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="tnl400m", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--ref-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be at least 3")
+    w = I.WORKLOADS[args.workload]
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            return run_reference(args, w, world, rank)
+        return run_ours(args, w, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,286 @@
+// la2_api.cu -- the C ABI of libla2.so (declared in include/la2.h): argument
+// validation, TMA descriptor set-up and kernel launch.  Everything numerical
+// happens in the kernels of scan_bf16_sm100.cuh and scan_f32.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "la2.h"
+#include "scan_bf16_sm100.cuh"
+#include "scan_f32.cuh"
+
+namespace {
+
+__device__ int g_la2_status = 0;  // device status word (see la2_device_status)
+
+thread_local int t_last_launches = 0;
+
+constexpr int kMaxDevices = 64;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+struct DeviceState {
+    std::once_flag once;
+    int* status = nullptr;
+    bool ok = false;
+};
+DeviceState g_dev[kMaxDevices];
+
+// Per-device set-up: address of the status word, dynamic shared-memory limits.
+bool device_setup(int* dev_out, int** status_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+    DeviceState& s = g_dev[dev];
+    std::call_once(s.once, [&s] {
+        void* p = nullptr;
+        bool ok = cudaGetSymbolAddress(&p, g_la2_status) == cudaSuccess;
+        s.status = static_cast<int*>(p);
+        ok = ok && cudaFuncSetAttribute(la2::la2_scan_bf16_sm100<64>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        la2::ScanSmem<64>::kBytes) == cudaSuccess;
+        ok = ok && cudaFuncSetAttribute(la2::la2_scan_bf16_sm100<128>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        la2::ScanSmem<128>::kBytes) == cudaSuccess;
+        ok = ok && cudaFuncSetAttribute(la2::la2_scan_f32,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(la2::f32_scan_smem_bytes(128, 128, 256))) ==
+                       cudaSuccess;
+        s.ok = ok;
+    });
+    if (!s.ok) return false;
+    *dev_out = dev;
+    *status_out = s.status;
+    return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Tensor map over a contiguous [BH, T, D] bf16 tensor, box 64 x 128 x 1, 128B swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, int BH, int T, int D) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(T),
+                                static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                                   static_cast<cuuint64_t>(T) * static_cast<cuuint64_t>(D) * 2};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(la2::kTB), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+struct RoleDesc {
+    const void* a;
+    const void* b;
+    const void* c;
+    void* x;
+    int da, dc, dir;
+};
+
+la2_status common_checks(int B, int H, int T, int d, int e, int block, la2_dtype dtype,
+                         bool* empty) {
+    if (dtype != LA2_DTYPE_F32 && dtype != LA2_DTYPE_BF16) return LA2_ERR_INVALID_ARG;
+    if (block != 64 && block != 128 && block != 256) return LA2_ERR_INVALID_ARG;
+    if (B < 0 || H < 0 || T < 0 || d <= 0 || e <= 0) return LA2_ERR_INVALID_ARG;
+    *empty = (B == 0 || H == 0 || T == 0);
+    if (*empty) return LA2_OK;
+    if (static_cast<long long>(B) * H > (1LL << 24)) return LA2_ERR_UNSUPPORTED;
+    if (dtype == LA2_DTYPE_BF16) {
+        if ((d != 64 && d != 128) || (e != 64 && e != 128)) return LA2_ERR_UNSUPPORTED;
+        if (block != la2::kTB) return LA2_ERR_UNSUPPORTED;
+    } else {
+        if (d > 128 || e > 128) return LA2_ERR_UNSUPPORTED;
+    }
+    return LA2_OK;
+}
+
+// Launches one bf16 grid over `n` roles that share (DA, DC).
+la2_status launch_bf16(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
+                       int* status, cudaStream_t stream) {
+    la2::ScanParams p;
+    std::memset(&p, 0, sizeof(p));
+    const int BH = B * H;
+    const int da = roles[0].da, dc = roles[0].dc;
+    for (int r = 0; r < n; ++r) {
+        if (!make_map(&p.role[r].ta, roles[r].a, BH, T, da) ||
+            !make_map(&p.role[r].tb, roles[r].b, BH, T, da) ||
+            !make_map(&p.role[r].tc, roles[r].c, BH, T, dc) ||
+            !make_map(&p.role[r].tx, roles[r].x, BH, T, dc))
+            return LA2_ERR_CUDA;
+        p.role[r].dir = roles[r].dir;
+    }
+    p.decay = decay;
+    p.status = status;
+    p.H = H;
+    p.T = T;
+    p.nroles = n;
+    p.nslices = dc / la2::kSlice;
+    const dim3 grid(static_cast<unsigned>(BH * n * p.nslices));
+    if (da == 128)
+        la2::la2_scan_bf16_sm100<128><<<grid, la2::kThreads, la2::ScanSmem<128>::kBytes, stream>>>(p);
+    else
+        la2::la2_scan_bf16_sm100<64><<<grid, la2::kThreads, la2::ScanSmem<64>::kBytes, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return LA2_ERR_CUDA;
+    ++t_last_launches;
+    return LA2_OK;
+}
+
+la2_status launch_f32(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
+                      int block, cudaStream_t stream) {
+    la2::F32Params p;
+    std::memset(&p, 0, sizeof(p));
+    int da_max = 0, dc_max = 0;
+    for (int r = 0; r < n; ++r) {
+        p.role[r].a = static_cast<const float*>(roles[r].a);
+        p.role[r].b = static_cast<const float*>(roles[r].b);
+        p.role[r].c = static_cast<const float*>(roles[r].c);
+        p.role[r].x = static_cast<float*>(roles[r].x);
+        p.role[r].da = roles[r].da;
+        p.role[r].dc = roles[r].dc;
+        p.role[r].dir = roles[r].dir;
+        da_max = roles[r].da > da_max ? roles[r].da : da_max;
+        dc_max = roles[r].dc > dc_max ? roles[r].dc : dc_max;
+    }
+    p.decay = decay;
+    p.H = H;
+    p.T = T;
+    p.TB = block;
+    p.nroles = n;
+    const size_t smem = la2::f32_scan_smem_bytes(da_max, dc_max, block);
+    const dim3 grid(static_cast<unsigned>(B * H * n));
+    la2::la2_scan_f32<<<grid, la2::kF32Threads, smem, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return LA2_ERR_CUDA;
+    ++t_last_launches;
+    return LA2_OK;
+}
+
+la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
+                     int block, la2_dtype dtype, cudaStream_t stream) {
+    int dev = 0;
+    int* status = nullptr;
+    if (!device_setup(&dev, &status)) return LA2_ERR_CUDA;
+    if (dtype == LA2_DTYPE_F32) return launch_f32(roles, n, decay, B, H, T, block, stream);
+    // group roles with identical (DA, DC) into one grid
+    RoleDesc group[3];
+    bool done[3] = {false, false, false};
+    for (int r = 0; r < n; ++r) {
+        if (done[r]) continue;
+        int m = 0;
+        for (int s = r; s < n; ++s)
+            if (!done[s] && roles[s].da == roles[r].da && roles[s].dc == roles[r].dc) {
+                group[m++] = roles[s];
+                done[s] = true;
+            }
+        const la2_status st = launch_bf16(group, m, decay, B, H, T, status, stream);
+        if (st != LA2_OK) return st;
+    }
+    return LA2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block, la2_dtype dtype,
+                           int is_bwd) {
+    (void)is_bwd;
+    bool empty = false;
+    const la2_status st = common_checks(B, H, T, d, e, block, dtype, &empty);
+    if (st != LA2_OK) return static_cast<size_t>(-1);
+    return 0;
+}
+
+la2_status la2_fwd(const void* q, const void* k, const void* v, const float* decay, void* out,
+                   int B, int H, int T, int d, int e, int block, la2_dtype dtype,
+                   void* workspace, size_t workspace_bytes, la2_stream_t stream) {
+    (void)workspace;
+    (void)workspace_bytes;
+    t_last_launches = 0;
+    bool empty = false;
+    la2_status st = common_checks(B, H, T, d, e, block, dtype, &empty);
+    if (st != LA2_OK || empty) return st;
+    if (!q || !k || !v || !decay || !out) return LA2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(decay) & 3u))
+        return LA2_ERR_INVALID_ARG;
+    const RoleDesc r = {q, k, v, out, d, e, +1};
+    return run_roles(&r, 1, decay, B, H, T, block, dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+la2_status la2_bwd(const void* q, const void* k, const void* v, const float* decay,
+                   const void* dout, void* dq, void* dk, void* dv, int B, int H, int T, int d,
+                   int e, int block, la2_dtype dtype, void* workspace, size_t workspace_bytes,
+                   la2_stream_t stream) {
+    (void)workspace;
+    (void)workspace_bytes;
+    t_last_launches = 0;
+    bool empty = false;
+    la2_status st = common_checks(B, H, T, d, e, block, dtype, &empty);
+    if (st != LA2_OK || empty) return st;
+    if (!q || !k || !v || !decay || !dout || !dq || !dk || !dv) return LA2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(decay) & 3u))
+        return LA2_ERR_INVALID_ARG;
+    // dq = scan(+1; dO, v, k), dk = scan(-1; v, dO, q), dv = scan(-1; k, q, dO)
+    const RoleDesc roles[3] = {
+        {dout, v, k, dq, e, d, +1},
+        {v, dout, q, dk, e, d, -1},
+        {k, q, dout, dv, d, e, -1},
+    };
+    return run_roles(roles, 3, decay, B, H, T, block, dtype,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+const char* la2_status_str(la2_status s) {
+    switch (s) {
+        case LA2_OK: return "LA2_OK";
+        case LA2_ERR_INVALID_ARG: return "LA2_ERR_INVALID_ARG";
+        case LA2_ERR_UNSUPPORTED: return "LA2_ERR_UNSUPPORTED";
+        case LA2_ERR_WORKSPACE: return "LA2_ERR_WORKSPACE";
+        case LA2_ERR_CUDA: return "LA2_ERR_CUDA";
+        case LA2_ERR_TIMEOUT: return "LA2_ERR_TIMEOUT";
+    }
+    return "LA2_UNKNOWN_STATUS";
+}
+
+la2_status la2_device_status(int* code, int reset) {
+    if (!code) return LA2_ERR_INVALID_ARG;
+    int dev = 0;
+    int* status = nullptr;
+    if (!device_setup(&dev, &status)) return LA2_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return LA2_ERR_CUDA;
+    if (cudaMemcpy(code, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return LA2_ERR_CUDA;
+    if (reset) {
+        const int zero = 0;
+        if (cudaMemcpy(status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+            return LA2_ERR_CUDA;
+    }
+    return LA2_OK;
+}
+
+int la2_last_launch_count(void) { return t_last_launches; }
+
+}  // extern "C"

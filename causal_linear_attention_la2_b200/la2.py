@@ -1,0 +1,168 @@
+"""ctypes binding of libla2.so -- argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels; this module
+only turns torch tensors into device pointers and sizes, passes the caller's
+current CUDA stream, and raises on a non-OK status.  There is no fallback: if
+the library is missing or a shape is unsupported, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libla2.so")
+
+LA2_OK = 0
+LA2_ERR_INVALID_ARG = 1
+LA2_ERR_UNSUPPORTED = 2
+LA2_ERR_WORKSPACE = 3
+LA2_ERR_CUDA = 4
+LA2_ERR_TIMEOUT = 5
+
+LA2_DTYPE_F32 = 0
+LA2_DTYPE_BF16 = 1
+
+# Every entry point include/la2.h declares.
+EXPORTS = ("la2_workspace_bytes", "la2_fwd", "la2_bwd", "la2_status_str", "la2_device_status",
+           "la2_last_launch_count")
+
+
+class LA2Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {la2_status_str(status)} ({status})")
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libla2.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libla2.so not found at {path}; build it with "
+                           "`python -m causal_linear_attention_la2_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.la2_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+    lib.la2_workspace_bytes.restype = sz
+    lib.la2_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
+    lib.la2_fwd.restype = i
+    lib.la2_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
+    lib.la2_bwd.restype = i
+    lib.la2_status_str.argtypes = [i]
+    lib.la2_status_str.restype = ctypes.c_char_p
+    lib.la2_device_status.argtypes = [ctypes.POINTER(ctypes.c_int), i]
+    lib.la2_device_status.restype = i
+    lib.la2_last_launch_count.argtypes = []
+    lib.la2_last_launch_count.restype = i
+    _lib = lib
+    return lib
+
+
+def la2_status_str(status: int) -> str:
+    return load().la2_status_str(int(status)).decode()
+
+
+def la2_workspace_bytes(B, H, T, d, e, block, dtype, is_bwd) -> int:
+    return int(load().la2_workspace_bytes(B, H, T, d, e, block, dtype, int(is_bwd)))
+
+
+def la2_device_status(reset: bool = True) -> int:
+    code = ctypes.c_int(0)
+    st = load().la2_device_status(ctypes.byref(code), int(reset))
+    if st != LA2_OK:
+        raise LA2Error(st, "la2_device_status")
+    return code.value
+
+
+def la2_last_launch_count() -> int:
+    return int(load().la2_last_launch_count())
+
+
+# ---------------------------------------------------------------- raw C calls
+
+def la2_fwd_raw(q, k, v, decay, out, B, H, T, d, e, block, dtype, workspace=0, ws_bytes=0,
+                stream=0) -> int:
+    """The C call with integer pointers; returns the status code."""
+    return int(load().la2_fwd(q, k, v, decay, out, B, H, T, d, e, block, dtype, workspace,
+                              ws_bytes, stream))
+
+
+def la2_bwd_raw(q, k, v, decay, dout, dq, dk, dv, B, H, T, d, e, block, dtype, workspace=0,
+                ws_bytes=0, stream=0) -> int:
+    return int(load().la2_bwd(q, k, v, decay, dout, dq, dk, dv, B, H, T, d, e, block, dtype,
+                              workspace, ws_bytes, stream))
+
+
+# ------------------------------------------------------------- torch wrappers
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return LA2_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return LA2_DTYPE_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; expected bfloat16 or float32")
+
+
+def _check(t: torch.Tensor, name: str, shape, dtype) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream_ptr(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def la2_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, decay: torch.Tensor,
+            out: torch.Tensor | None = None, block: int = 128, stream=None) -> torch.Tensor:
+    """o[b,h,t] = sum_{s<=t} decay[h]^(t-s) (q[b,h,t] . k[b,h,s]) v[b,h,s], on q's device."""
+    B, H, T, d = q.shape
+    e = v.shape[-1]
+    dt = _dtype_code(q)
+    _check(q, "q", (B, H, T, d), q.dtype)
+    _check(k, "k", (B, H, T, d), q.dtype)
+    _check(v, "v", (B, H, T, e), q.dtype)
+    _check(decay, "decay", (H,), torch.float32)
+    if out is None:
+        out = torch.empty((B, H, T, e), dtype=q.dtype, device=q.device)
+    _check(out, "out", (B, H, T, e), q.dtype)
+    st = la2_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(), out.data_ptr(),
+                     B, H, T, d, e, block, dt, 0, 0, _stream_ptr(stream))
+    if st != LA2_OK:
+        raise LA2Error(st, "la2_fwd")
+    return out
+
+
+def la2_bwd(q, k, v, decay, dout, dq=None, dk=None, dv=None, block: int = 128, stream=None):
+    """(dq, dk, dv) of sum(dout * la2_fwd(q, k, v, decay)); decay is not differentiated."""
+    B, H, T, d = q.shape
+    e = v.shape[-1]
+    dt = _dtype_code(q)
+    for t, n, shp in ((q, "q", (B, H, T, d)), (k, "k", (B, H, T, d)), (v, "v", (B, H, T, e)),
+                      (dout, "dout", (B, H, T, e))):
+        _check(t, n, shp, q.dtype)
+    _check(decay, "decay", (H,), torch.float32)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n, shp in ((dq, "dq", (B, H, T, d)), (dk, "dk", (B, H, T, d)), (dv, "dv", (B, H, T, e))):
+        _check(t, n, shp, q.dtype)
+    st = la2_bwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(), dout.data_ptr(),
+                     dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, T, d, e, block, dt, 0, 0,
+                     _stream_ptr(stream))
+    if st != LA2_OK:
+        raise LA2Error(st, "la2_bwd")
+    return dq, dk, dv

@@ -1,0 +1,122 @@
+/*
+ * la2.h -- C ABI of the Lightning Attention-2 library (libla2.so), sm_100a.
+ *
+ * The operation (per batch b and head h, identity feature map, no normaliser,
+ * no 1/sqrt(d) scale inside the call):
+ *
+ *     o_t = sum_{s<=t} lambda_h^(t-s) (q_t . k_s) v_s
+ *
+ * Causal linear attention is defined on the "Lightning Attention" explainer
+ * page (lizeman.github.io llm-arch-kb), section 1 "Premise" (numerator of the
+ * out_t formula and the prefix-sum recurrence S_t = S_{t-1} + phi(k_t) v_t^T),
+ * with phi the identity as in its section 2.  lambda_h in (0,1] is a per-head
+ * decay on the lag t-s; lambda_h = 1 is the plain prefix sum.  The tiled
+ * computation (intra-tile masked left product, inter-tile right product with
+ * the running d x e state, state update) is the derivation of section 2,
+ * steps 1-4, with the decay folded into each step; the backward uses the same
+ * tiling, as the Lightning Attention-2 abstract (mlsanity.com/paper/2401.04658)
+ * says, run in the reverse direction for dk and dv.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or retains them past the call.
+ *   - q, k, dq, dk are [B, H, T, d] contiguous (d fastest); v, out, dout, dv
+ *     are [B, H, T, e] contiguous.  All share the element type `dtype`.
+ *     Every tensor pointer must be 16-byte aligned.
+ *   - decay is a device array of H floats (fp32) holding lambda_h in (0, 1];
+ *     values outside that range are the caller's error and are not checked.
+ *   - block is the tile length T_B (64, 128 or 256).  It changes the order of
+ *     floating-point operations only, never the mathematical result.  T need
+ *     not be a multiple of block: the last tile is short.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream).  Argument
+ *     errors are reported synchronously and launch nothing.  A failed launch
+ *     returns LA2_ERR_CUDA.  Faults detected inside a kernel (a bounded wait
+ *     that ran out) are recorded in a device status word that
+ *     la2_device_status() reads.
+ *   - B, H or T equal to 0 is an empty problem: LA2_OK, nothing is launched
+ *     and no pointer is dereferenced.
+ */
+#ifndef LA2_H_
+#define LA2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque CUDA stream handle (a cudaStream_t / CUstream). */
+typedef struct CUstream_st *la2_stream_t;
+
+typedef enum {
+    LA2_OK = 0,
+    LA2_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad block/dtype, misaligned pointer */
+    LA2_ERR_UNSUPPORTED = 2,  /* well-formed but not implemented for this dtype/shape; never a fallback */
+    LA2_ERR_WORKSPACE = 3,    /* workspace missing or smaller than la2_workspace_bytes() */
+    LA2_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed (launch, tensor-map encode, ...) */
+    LA2_ERR_TIMEOUT = 5       /* a kernel's bounded wait ran out (see la2_device_status) */
+} la2_status;
+
+typedef enum {
+    LA2_DTYPE_F32 = 0,   /* fp32 in, fp32 out, fp32 arithmetic (SIMT kernels) */
+    LA2_DTYPE_BF16 = 1   /* bf16 in, bf16 out, fp32 accumulation and fp32 state (tcgen05) */
+} la2_dtype;
+
+/*
+ * Bytes of device workspace la2_fwd (is_bwd = 0) or la2_bwd (is_bwd = 1) needs
+ * for these sizes.  The value does not grow with T (the only state carried
+ * along a sequence is the d x e matrix, held on chip).  0 means the call
+ * accepts workspace = NULL.  Returns (size_t)-1 for arguments the call would
+ * reject.
+ */
+size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block,
+                           la2_dtype dtype, int is_bwd);
+
+/*
+ * Forward: out[b,h,t,:] = sum_{s<=t} decay[h]^(t-s) (q[b,h,t,:] . k[b,h,s,:]) v[b,h,s,:].
+ *
+ * Supported: dtype F32 with 1 <= d, e <= 128 and any block; dtype BF16 with
+ * d, e in {64, 128} and block = 128.  Anything else well-formed returns
+ * LA2_ERR_UNSUPPORTED.  out must not alias an input.
+ */
+la2_status la2_fwd(const void *q, const void *k, const void *v, const float *decay,
+                   void *out, int B, int H, int T, int d, int e, int block,
+                   la2_dtype dtype, void *workspace, size_t workspace_bytes,
+                   la2_stream_t stream);
+
+/*
+ * Backward of L = sum dout * out with respect to q, k and v (decay is not
+ * differentiated):
+ *   dq[t] = sum_{s<=t} lambda^(t-s) (dout_t . v_s) k_s
+ *   dk[s] = sum_{t>=s} lambda^(t-s) (v_s . dout_t) q_t
+ *   dv[s] = sum_{t>=s} lambda^(t-s) (k_s . q_t) dout_t
+ * Nothing is saved by la2_fwd; the backward recomputes what it needs.  Same
+ * support matrix as la2_fwd.  dq, dk, dv must not alias each other or an
+ * input.
+ */
+la2_status la2_bwd(const void *q, const void *k, const void *v, const float *decay,
+                   const void *dout, void *dq, void *dk, void *dv,
+                   int B, int H, int T, int d, int e, int block, la2_dtype dtype,
+                   void *workspace, size_t workspace_bytes, la2_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char *la2_status_str(la2_status status);
+
+/*
+ * Reads (and, if reset != 0, clears) the device status word of the current
+ * device: 0 when no kernel has reported a fault, otherwise a code whose low
+ * byte is the la2_status value and whose upper bits say where the kernel gave
+ * up.  Synchronises with the device.  Returns LA2_ERR_CUDA if the read fails.
+ */
+la2_status la2_device_status(int *code, int reset);
+
+/* Number of kernel launches the last successful la2_fwd / la2_bwd call made
+ * on this host thread. */
+int la2_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA2_H_ */

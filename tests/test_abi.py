@@ -1,0 +1,112 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+include/la2.h declares, and rejects bad arguments synchronously (before any
+CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from causal_linear_attention_la2_b200 import la2
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "la2.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from causal_linear_attention_la2_b200 import build
+    build.build()
+    return la2.load()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(la2_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_python_export_list():
+    assert _declared_functions() == sorted(la2.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings(lib):
+    names = {0: "LA2_OK", 1: "LA2_ERR_INVALID_ARG", 2: "LA2_ERR_UNSUPPORTED",
+             3: "LA2_ERR_WORKSPACE", 4: "LA2_ERR_CUDA", 5: "LA2_ERR_TIMEOUT"}
+    for code, name in names.items():
+        assert la2.la2_status_str(code) == name
+    assert la2.la2_status_str(99) == "LA2_UNKNOWN_STATUS"
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null value; validation fails before it is used
+
+
+def _fwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, decay=FAKE, out=FAKE, B=1, H=2, T=256, d=128, e=128,
+             block=128, dtype=la2.LA2_DTYPE_BF16)
+    a.update(kw)
+    return la2.la2_fwd_raw(a["q"], a["k"], a["v"], a["decay"], a["out"], a["B"], a["H"], a["T"],
+                           a["d"], a["e"], a["block"], a["dtype"])
+
+
+def _bwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, decay=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, B=1, H=2,
+             T=256, d=128, e=128, block=128, dtype=la2.LA2_DTYPE_BF16)
+    a.update(kw)
+    return la2.la2_bwd_raw(a["q"], a["k"], a["v"], a["decay"], a["dout"], a["dq"], a["dk"],
+                           a["dv"], a["B"], a["H"], a["T"], a["d"], a["e"], a["block"], a["dtype"])
+
+
+@pytest.mark.parametrize("kw", [dict(block=100), dict(block=0), dict(dtype=7), dict(B=-1),
+                                dict(H=-2), dict(T=-5), dict(d=0), dict(e=-1)])
+def test_invalid_arguments(lib, kw):
+    assert _fwd(**kw) == la2.LA2_ERR_INVALID_ARG
+    assert _bwd(**kw) == la2.LA2_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name", ["q", "k", "v", "decay", "out"])
+def test_null_pointers_forward(lib, name):
+    assert _fwd(**{name: 0}) == la2.LA2_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name", ["q", "k", "v", "decay", "dout", "dq", "dk", "dv"])
+def test_null_pointers_backward(lib, name):
+    assert _bwd(**{name: 0}) == la2.LA2_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name", ["q", "k", "v", "out"])
+def test_misaligned_pointers(lib, name):
+    assert _fwd(**{name: FAKE + 8}) == la2.LA2_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw", [dict(d=96), dict(e=32), dict(d=256), dict(block=64),
+                                dict(block=256)])
+def test_bf16_unsupported_shapes(lib, kw):
+    assert _fwd(**kw) == la2.LA2_ERR_UNSUPPORTED
+    assert _bwd(**kw) == la2.LA2_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("kw", [dict(d=129), dict(e=200)])
+def test_f32_unsupported_shapes(lib, kw):
+    assert _fwd(dtype=la2.LA2_DTYPE_F32, **kw) == la2.LA2_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(H=0), dict(T=0)])
+def test_empty_problem_is_ok_and_touches_nothing(lib, kw):
+    # null pointers are fine for an empty problem: nothing is dereferenced or launched
+    assert _fwd(q=0, k=0, v=0, decay=0, out=0, **kw) == la2.LA2_OK
+    assert _bwd(q=0, k=0, v=0, decay=0, dout=0, dq=0, dk=0, dv=0, **kw) == la2.LA2_OK
+    assert la2.la2_last_launch_count() == 0
+
+
+def test_workspace_is_flat_in_T(lib):
+    sizes = {la2.la2_workspace_bytes(1, 16, T, 128, 128, 128, la2.LA2_DTYPE_BF16, 1)
+             for T in (1, 1024, 65536, 1 << 20)}
+    assert len(sizes) == 1
+    assert la2.la2_workspace_bytes(1, 16, 1024, 128, 128, 100, la2.LA2_DTYPE_BF16, 0) == 2 ** 64 - 1

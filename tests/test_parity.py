@@ -1,0 +1,159 @@
+"""GPU parity: libla2.so (through its C ABI) against the fp64 CPU oracle.
+
+Criterion, per output tensor (o, dq, dk, dv):  max|gpu - oracle| / rms(oracle)
+<= 1e-5 for fp32 inputs and <= 2e-2 for bf16 inputs (fp32 accumulation), with
+the oracle evaluated on the very same (already rounded) inputs.  Small cases
+are compared in full; the full-size workloads on whole sampled sequences
+(every output row of the sampled (b, h)), in the same launch configuration the
+benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+from causal_linear_attention_la2_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-5, "bf16": 2e-2}
+
+
+@pytest.fixture(scope="module")
+def la2mod():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from causal_linear_attention_la2_b200 import build, la2
+    build.build()
+    la2.load()
+    return la2
+
+
+def _err(gpu, ref):
+    gpu = gpu.detach().float().cpu().numpy().astype(np.float64)
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    return float(np.max(np.abs(gpu - ref))) / max(rms, 1e-300)
+
+
+def _run_gpu(la2mod, x, block, fill_nan=True):
+    dev = torch.device("cuda")
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    lam = x["lam"].to(dev)
+    out = torch.empty_like(v)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if fill_nan:
+        for t in (out, dq, dk, dv):
+            t.fill_(float("nan"))
+    la2mod.la2_fwd(q, k, v, lam, out=out, block=block)
+    la2mod.la2_bwd(q, k, v, lam, do, dq=dq, dk=dk, dv=dv, block=block)
+    torch.cuda.synchronize()
+    assert la2mod.la2_device_status(reset=True) == 0
+    return out, dq, dk, dv
+
+
+def _check(la2mod, oracle_mod, x, block, tol, heads=None):
+    o, dq, dk, dv = _run_gpu(la2mod, x, block)
+    B, H = x["q"].shape[:2]
+    lam = np.broadcast_to(x["lam"].numpy().astype(np.float64)[None, :], (B, H))
+    if heads is None:
+        qs, ks, vs, ds, ls = x["q"], x["k"], x["v"], x["do"], lam
+        gpu = (o, dq, dk, dv)
+    else:
+        bi, hi = (np.asarray(z, dtype=np.int64) for z in heads)
+        tb, th = torch.from_numpy(bi), torch.from_numpy(hi)
+        qs, ks, vs, ds = (x[n][tb, th] for n in ("q", "k", "v", "do"))
+        ls = lam[bi, hi]
+        gpu = tuple(t[tb.cuda(), th.cuda()] for t in (o, dq, dk, dv))
+    ro = oracle_mod.forward(qs, ks, vs, ls)
+    rdq, rdk, rdv = oracle_mod.backward(qs, ks, vs, ls, ds)
+    errs = {n: _err(g, r) for n, g, r in zip(("o", "dq", "dk", "dv"), gpu, (ro, rdq, rdk, rdv))}
+    for n, g in zip(("o", "dq", "dk", "dv"), gpu):
+        assert torch.isfinite(g.float()).all(), f"{n} has non-finite entries"
+    bad = {n: e for n, e in errs.items() if not e <= tol}
+    assert not bad, f"errors {errs} exceed {tol}"
+    return errs
+
+
+# ------------------------------------------------------------------ fp32 path
+
+def test_tiny_f32_workload(la2mod, oracle_mod):
+    w = I.WORKLOADS["tiny_f32"]
+    _check(la2mod, oracle_mod, I.make_workload_inputs(w, seed=0), w.block, TOL["f32"])
+
+
+@pytest.mark.parametrize("block", [64, 128, 256])
+@pytest.mark.parametrize("T,d,e", [(1, 64, 64), (300, 64, 64), (517, 3, 5), (200, 100, 37),
+                                   (129, 128, 128)])
+def test_f32_shapes_and_blocks(la2mod, oracle_mod, block, T, d, e):
+    x = I.make_inputs(2, 3, T, d, e, "f32", seed=T + d, decay="tnl")
+    _check(la2mod, oracle_mod, x, block, TOL["f32"])
+
+
+# ------------------------------------------------------------------ bf16 path
+
+@pytest.mark.parametrize("T", [1, 64, 127, 128, 129, 300, 1000])
+@pytest.mark.parametrize("d,e", [(128, 128), (64, 64), (64, 128), (128, 64)])
+def test_bf16_shapes_with_ragged_tails(la2mod, oracle_mod, T, d, e):
+    x = I.make_inputs(2, 3, T, d, e, "bf16", seed=T * 7 + d + e, decay="tnl")
+    _check(la2mod, oracle_mod, x, 128, TOL["bf16"])
+
+
+@pytest.mark.parametrize("decay", ["ones", "tiny", "tnl"])
+def test_bf16_decays(la2mod, oracle_mod, decay):
+    x = I.make_inputs(1, 4, 777, 128, 128, "bf16", seed=3, decay=decay)
+    _check(la2mod, oracle_mod, x, 128, TOL["bf16"])
+
+
+def test_bf16_tiny_decay_keeps_only_diagonal(la2mod, oracle_mod):
+    x = I.make_inputs(1, 2, 256, 64, 64, "bf16", seed=4)
+    x["lam"] = torch.tensor([2.0 ** -20, 0.5], dtype=torch.float32)
+    _check(la2mod, oracle_mod, x, 128, TOL["bf16"])
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_bf16_seeds_multi_head(la2mod, oracle_mod, seed):
+    x = I.make_inputs(3, 8, 640, 128, 128, "bf16", seed=seed)
+    _check(la2mod, oracle_mod, x, 128, TOL["bf16"])
+
+
+def test_repeat_calls_are_bitwise_identical(la2mod):
+    x = I.make_inputs(2, 4, 700, 128, 128, "bf16", seed=5)
+    a = _run_gpu(la2mod, x, 128)
+    b = _run_gpu(la2mod, x, 128)
+    for t, u in zip(a, b):
+        assert torch.equal(t, u)
+
+
+def test_outputs_do_not_write_past_their_end(la2mod):
+    dev = torch.device("cuda")
+    x = I.make_inputs(1, 2, 333, 128, 64, "bf16", seed=6)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    lam = x["lam"].to(dev)
+    n_o, n_q = v.numel(), q.numel()
+    guard = 4096
+    buf_o = torch.full((n_o + guard,), 7.0, dtype=torch.bfloat16, device=dev)
+    buf_q = torch.full((n_q + guard,), 7.0, dtype=torch.bfloat16, device=dev)
+    buf_k = torch.full((n_q + guard,), 7.0, dtype=torch.bfloat16, device=dev)
+    buf_v = torch.full((n_o + guard,), 7.0, dtype=torch.bfloat16, device=dev)
+    la2mod.la2_fwd(q, k, v, lam, out=buf_o[:n_o].view_as(v))
+    la2mod.la2_bwd(q, k, v, lam, do, dq=buf_q[:n_q].view_as(q), dk=buf_k[:n_q].view_as(k),
+                   dv=buf_v[:n_o].view_as(v))
+    torch.cuda.synchronize()
+    for b in (buf_o, buf_q, buf_k, buf_v):
+        assert torch.all(b[-guard:] == 7.0)
+
+
+# -------------------------------------------------- full-size named workloads
+
+FULL = ["tnl400m", "tnl15b", "tnl15b_nodecay", "long", "sweep_T1024_blk128",
+        "sweep_T131072_blk128", "sweep_T92160_blk128"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_workload_sampled_sequences(la2mod, oracle_mod, name):
+    w = I.WORKLOADS[name]
+    x = I.make_workload_inputs(w, seed=0)
+    B, H = w.B, w.H
+    # first and last sequence (smallest and largest decay) and one in the middle
+    bi = np.array([0, B // 2, B - 1])
+    hi = np.array([0, H // 2, H - 1])
+    _check(la2mod, oracle_mod, x, w.block, TOL[w.dtype], heads=(bi, hi))
