@@ -66,16 +66,18 @@ def flops_per_token_head(w: I.Workload) -> float:
 
 
 def elem_bytes(w: I.Workload) -> int:
+    """Bytes per input element (outputs are always fp32)."""
     return 2 if w.dtype == "bf16" else 4
 
 
 def bwd_algorithmic_bytes(w: I.Workload) -> float:
-    """la2_bwd reads q, k, v, dO and writes dq, dk, dv, each once."""
-    return float(elem_bytes(w)) * w.sequences * w.T * (3 * w.d + 4 * w.e)
+    """la2_bwd reads q, k, v, dO and writes fp32 dq, dk, dv, each once."""
+    return float(w.sequences) * w.T * (elem_bytes(w) * (2 * w.d + 2 * w.e) + 4 * (2 * w.d + w.e))
 
 
 def fwd_algorithmic_bytes(w: I.Workload) -> float:
-    return float(elem_bytes(w)) * w.sequences * w.T * (2 * w.d + 2 * w.e)
+    """la2_fwd reads q, k, v and writes fp32 o, each once."""
+    return float(w.sequences) * w.T * (elem_bytes(w) * (2 * w.d + w.e) + 4 * w.e)
 
 
 class ClockSampler:
@@ -257,8 +259,9 @@ def run_ours(args, w, world, rank, local):
     x = I.make_workload_inputs(w, seed=args.seed)
     q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
     lam = x["lam"].to(dev)
-    out = torch.empty_like(v)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = torch.empty(v.shape, **f32)
+    dq, dk, dv = torch.empty(q.shape, **f32), torch.empty(k.shape, **f32), torch.empty(v.shape, **f32)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 

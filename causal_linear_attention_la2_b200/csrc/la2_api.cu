@@ -56,6 +56,12 @@ bool device_setup(int* dev_out, int** status_out) {
         bool ok = cudaGetSymbolAddress(&p, g_la2_status) == cudaSuccess;
         s.status = static_cast<int*>(p);
         ok = ok && cudaFuncSetAttribute(la2::la2_scan_bf16_sm100<64>,
+                                        cudaFuncAttributePreferredSharedMemoryCarveout,
+                                        100) == cudaSuccess;
+        ok = ok && cudaFuncSetAttribute(la2::la2_scan_bf16_sm100<128>,
+                                        cudaFuncAttributePreferredSharedMemoryCarveout,
+                                        100) == cudaSuccess;
+        ok = ok && cudaFuncSetAttribute(la2::la2_scan_bf16_sm100<64>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         la2::ScanSmem<64>::kBytes) == cudaSuccess;
         ok = ok && cudaFuncSetAttribute(la2::la2_scan_bf16_sm100<128>,
@@ -126,9 +132,9 @@ la2_status launch_bf16(const RoleDesc* roles, int n, const float* decay, int B, 
     for (int r = 0; r < n; ++r) {
         if (!make_map(&p.role[r].ta, roles[r].a, BH, T, da) ||
             !make_map(&p.role[r].tb, roles[r].b, BH, T, da) ||
-            !make_map(&p.role[r].tc, roles[r].c, BH, T, dc) ||
-            !make_map(&p.role[r].tx, roles[r].x, BH, T, dc))
+            !make_map(&p.role[r].tc, roles[r].c, BH, T, dc))
             return LA2_ERR_CUDA;
+        p.role[r].x = static_cast<float*>(roles[r].x);
         p.role[r].dir = roles[r].dir;
     }
     p.decay = decay;
@@ -137,6 +143,7 @@ la2_status launch_bf16(const RoleDesc* roles, int n, const float* decay, int B, 
     p.T = T;
     p.nroles = n;
     p.nslices = dc / la2::kSlice;
+    p.dc = dc;
     const dim3 grid(static_cast<unsigned>(BH * n * p.nslices));
     if (da == 128)
         la2::la2_scan_bf16_sm100<128><<<grid, la2::kThreads, la2::ScanSmem<128>::kBytes, stream>>>(p);

@@ -1,5 +1,5 @@
-// scan_bf16_sm100.cuh -- the bf16 tcgen05 kernel of the Lightning Attention-2
-// hot path.
+// scan_bf16_sm100.cuh -- the bf16-input tcgen05 kernel of the Lightning
+// Attention-2 hot path.
 //
 // One kernel computes every output of the forward and the backward pass as a
 // "decayed scan" over tiles of T_B = 128 rows:
@@ -16,25 +16,32 @@
 // derivation of the "Lightning Attention" page (lizeman.github.io llm-arch-kb,
 // section 2, steps 1-4) with the decay folded in:
 //
-//   S   = A_i B_i^T                                  (tcgen05, fp32 in TMEM)
-//   P   = S * lambda^|r-c| on the causal side, else 0 (registers -> bf16 smem)
-//   X   = diag(w_x) A_i W + P C_i                    (tcgen05, fp32 in TMEM)
-//   W  <- lambda^T_B W + (diag(w_s) B_i)^T C_i       (tcgen05 + fp32 registers)
+//   S   = A_i B_i^T                                   tcgen05, fp32 in TMEM
+//   P   = S * lambda^|r-c| on the causal side, else 0 registers -> TMEM
+//   X   = diag(w_x) A_i W + P C_i                     tcgen05, fp32 in TMEM
+//   W  <- lambda^T_B W + (diag(w_s) B_i)^T C_i        tcgen05 + fp32 registers
 //
 // with w_x = lambda^(r+1), w_s = lambda^(T_B-1-r) for dir = +1 and
 // w_x = lambda^(T_B-r), w_s = lambda^r for dir = -1.  W is the d x e state,
-// kept on chip in fp32 for the whole sequence (a bf16 copy in shared memory
-// feeds the MMA); nothing per tile goes back to HBM except X.
+// carried on chip in fp32 for the whole sequence; nothing per tile goes back
+// to HBM except X, which is written in fp32.
+//
+// Precision: inputs are bf16 and every product of two inputs is exact in the
+// fp32 accumulators.  The three operands the kernel forms itself (P, W and
+// diag(w_s) B) are fp32 values; each is fed to the tensor core as the sum of
+// two bf16 terms (hi + lo, relative residue ~2^-16), i.e. as two MMAs.
 //
 // Work split: one CTA per (sequence, role, 64-column slice of c/x).  Each CTA
 // runs its tiles serially (the state makes the scan sequential); two CTAs fit
-// on an SM (256 TMEM columns and ~100 KB of shared memory each), so one CTA's
+// on an SM (256 TMEM columns and ~113 KB of shared memory each), so one CTA's
 // TMA traffic overlaps the other's math.
 //
 // Shared-memory tiles are 128-byte swizzled, as TMA writes them; the A and B
 // tiles serve both K-major (for S) and MN-major (for the state update)
-// descriptors.  The A buffer is reused for P once S and A.W are done; the C
-// buffer is reused as the staging tile of the X store.
+// descriptors.  Once S and A W are computed the A buffer takes the lo part of
+// diag(w_s) B, and the B buffer its hi part in place.  P (hi and lo) lives in
+// TMEM over the columns of S it was computed from and feeds the MMA as its A
+// operand straight from TMEM.
 #pragma once
 #include "ptx_sm100.cuh"
 
@@ -46,21 +53,23 @@ constexpr int kThreads = 128;   // one thread per TMEM lane / tile row
 constexpr uint32_t kTmemCols = 256;
 
 struct ScanRole {
-    CUtensorMap ta, tb, tc, tx;  // a, b: [B*H, T, DA]; c, x: [B*H, T, DC]; bf16
-    int dir;                     // +1 or -1
-    int pad_[15];
+    CUtensorMap ta, tb, tc;  // a, b: [B*H, T, DA]; c: [B*H, T, DC]; bf16
+    float* x;                // [B*H, T, DC] fp32
+    int dir;                 // +1 or -1
 };
 
 struct ScanParams {
     ScanRole role[3];
     const float* decay;  // [H]
     int* status;         // device status word
-    int H, T, nroles, nslices;
+    int H, T, nroles, nslices, dc;
 };
 
-// Device status codes: low byte = la2_status (5 = timeout), next byte = where.
-__device__ __forceinline__ void report_timeout(int* status, int where) {
-    atomicCAS(status, 0, 5 | (where << 8));
+// Device status codes: low byte = la2_status, next byte = where.
+constexpr int kDevTimeout = 5;
+constexpr int kDevMisaligned = 4;
+__device__ __forceinline__ void report_status(int* status, int code, int where) {
+    atomicCAS(status, 0, code | (where << 8));
 }
 
 // Byte offset of the 16-byte chunk q (0..7) of row r inside a 128-byte
@@ -71,19 +80,20 @@ __device__ __forceinline__ uint32_t sw128(int r, int q) {
 
 template <int DA>
 struct ScanSmem {
-    static constexpr uint32_t kA = 0;                                 // A tile, then P (T_B x T_B)
-    static constexpr uint32_t kB = kA + kTB * kTB * 2;                // B tile (T_B x DA)
-    static constexpr uint32_t kC = kB + kTB * DA * 2;                 // C slice, then X staging
-    static constexpr uint32_t kW = kC + kTB * kSlice * 2;             // bf16 state slice (DA x 64)
-    static constexpr uint32_t kPow = kW + DA * kSlice * 2;            // lambda^n, n = 0..256
-    static constexpr uint32_t kBarLoad = kPow + 1040;
+    static constexpr uint32_t kA = 0;                         // A tile, then lo(w_s B)
+    static constexpr uint32_t kB = kA + kTB * DA * 2;         // B tile, then hi(w_s B)
+    static constexpr uint32_t kC = kB + kTB * DA * 2;         // C slice (T_B x 64)
+    static constexpr uint32_t kWhi = kC + kTB * kSlice * 2;   // hi(W) (DA x 64)
+    static constexpr uint32_t kWlo = kWhi + DA * kSlice * 2;  // lo(W)
+    static constexpr uint32_t kPow = kWlo + DA * kSlice * 2;  // lambda^n, n = 0..T_B
+    static constexpr uint32_t kBarLoad = kPow + 528;
     static constexpr uint32_t kBarMma = kBarLoad + 8;
     static constexpr uint32_t kTmemSlot = kBarMma + 8;
     static constexpr uint32_t kEnd = kTmemSlot + 16;
-    // Requested dynamic smem: payload + 1 KB for aligning the base, padded so
-    // that at most two CTAs share an SM (their TMEM adds up to 512 columns).
-    static constexpr uint32_t kBytesRaw = kEnd + 1024;
-    static constexpr uint32_t kBytes = kBytesRaw > 78 * 1024 ? kBytesRaw : 78 * 1024;
+    // The dynamic shared memory base is 1024-byte aligned (checked at run
+    // time).  Small tiles are padded so that at most two CTAs share an SM:
+    // their TMEM then adds up to the SM's 512 columns.
+    static constexpr uint32_t kBytes = kEnd > 78 * 1024 ? kEnd : 78 * 1024;
 };
 
 template <int DA>
@@ -92,16 +102,18 @@ la2_scan_bf16_sm100(const __grid_constant__ ScanParams p)
 {
     static_assert(DA == 64 || DA == 128, "DA must be 64 or 128");
     using L = ScanSmem<DA>;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
-    const uint32_t base = raw + pad;
-    uint8_t* gbase = smem_raw + pad;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t base = smem_u32(smem_raw);
+    if (base & 1023u) {  // 128-byte swizzled tiles need a 1024-byte aligned base
+        if (threadIdx.x == 0) report_status(p.status, kDevMisaligned, 0);
+        return;
+    }
 
-    const uint32_t sA = base + L::kA, sB = base + L::kB, sC = base + L::kC, sW = base + L::kW;
-    float* pw = reinterpret_cast<float*>(gbase + L::kPow);
+    const uint32_t sA = base + L::kA, sB = base + L::kB, sC = base + L::kC;
+    const uint32_t sWhi = base + L::kWhi, sWlo = base + L::kWlo;
+    float* pw = reinterpret_cast<float*>(smem_raw + L::kPow);
     const uint32_t bar_load = base + L::kBarLoad, bar_mma = base + L::kBarMma;
-    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gbase + L::kTmemSlot);
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem_raw + L::kTmemSlot);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int idx = blockIdx.x;
@@ -115,13 +127,15 @@ la2_scan_bf16_sm100(const __grid_constant__ ScanParams p)
     const int nb = (T + kTB - 1) / kTB;
     const int x0 = slice * kSlice;
     const float lam = p.decay[bh % p.H];
+    float* xg = R.x + static_cast<size_t>(bh) * T * p.dc + x0;
 
     // ---- set-up: powers of lambda, zero state copy, barriers, TMEM
     {
-        const float l2 = log2f(lam);
-        for (int n = tid; n <= 256; n += kThreads) pw[n] = exp2f(static_cast<float>(n) * l2);
-        for (uint32_t off = tid * 16; off < static_cast<uint32_t>(DA * kSlice * 2); off += kThreads * 16)
-            st_shared_v4(sW + off, 0u, 0u, 0u, 0u);
+        const double l2 = log2(static_cast<double>(lam));
+        for (int n = tid; n <= kTB; n += kThreads) pw[n] = static_cast<float>(exp2(n * l2));
+        for (uint32_t off = tid * 16; off < static_cast<uint32_t>(2 * DA * kSlice * 2);
+             off += kThreads * 16)
+            st_shared_v4(sWhi + off, 0u, 0u, 0u, 0u);  // hi(W) and lo(W) are adjacent
     }
     if (warp == 0) {
         tmem_alloc(base + L::kTmemSlot, kTmemCols);
@@ -134,7 +148,6 @@ la2_scan_bf16_sm100(const __grid_constant__ ScanParams p)
         prefetch_tmap(&R.ta);
         prefetch_tmap(&R.tb);
         prefetch_tmap(&R.tc);
-        prefetch_tmap(&R.tx);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -146,27 +159,22 @@ la2_scan_bf16_sm100(const __grid_constant__ ScanParams p)
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const float lamTB = pw[kTB];
 
-    constexpr uint32_t kBytesAB = 2u * kTB * DA * 2;
-    constexpr uint32_t kBytesC = kTB * kSlice * 2;
-    constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);   // S  = A B^T
-    constexpr uint32_t kIdX = idesc_bf16_f32(128, kSlice, 0, 1); // X  = A W, X += P C
-    constexpr uint32_t kIdW = idesc_bf16_f32(DA, kSlice, 1, 1);  // dW = B^T C
+    constexpr uint32_t kTxBytes = 2u * kTB * DA * 2 + kTB * kSlice * 2;
+    constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);    // S  = A B^T
+    constexpr uint32_t kIdX = idesc_bf16_f32(128, kSlice, 0, 1);  // X  = A W, X += P C
+    constexpr uint32_t kIdW = idesc_bf16_f32(DA, kSlice, 1, 1);   // dW = B^T C
 
-    auto issue_ab = [&](int i) {
+    auto issue_loads = [&](int i) {
+        mbar_arrive_expect_tx(bar_load, kTxBytes);
 #pragma unroll
         for (int g = 0; g < DA / 64; ++g) {
             tma_load_3d(sA + g * 16384, &R.ta, bar_load, g * 64, i * kTB, bh);
             tma_load_3d(sB + g * 16384, &R.tb, bar_load, g * 64, i * kTB, bh);
         }
+        tma_load_3d(sC, &R.tc, bar_load, x0, i * kTB, bh);
     };
-    auto issue_c = [&](int i) { tma_load_3d(sC, &R.tc, bar_load, x0, i * kTB, bh); };
 
-    if (tid == 0 && nb > 0) {
-        const int i0 = dir > 0 ? 0 : nb - 1;
-        mbar_arrive_expect_tx(bar_load, kBytesAB + kBytesC);
-        issue_ab(i0);
-        issue_c(i0);
-    }
+    if (tid == 0 && nb > 0) issue_loads(dir > 0 ? 0 : nb - 1);
 
     float w[kSlice];  // fp32 state row (row j of W, this CTA's 64 columns)
 #pragma unroll
@@ -179,14 +187,18 @@ la2_scan_bf16_sm100(const __grid_constant__ ScanParams p)
 
     for (int step = 0; step < nb; ++step) {
         const int i = dir > 0 ? step : nb - 1 - step;
+        const int rows = min(kTB, T - i * kTB);
 
         // (1) tiles A_i, B_i, C_i have landed
         bool ok = true;
         if (tid == 0) ok = mbar_wait(bar_load, ph_load);
         ph_load ^= 1;
-        if (!__syncthreads_and(ok)) { if (tid == 0) report_timeout(p.status, 1); break; }
+        if (!__syncthreads_and(ok)) {
+            if (tid == 0) report_status(p.status, kDevTimeout, 1);
+            break;
+        }
 
-        // (2) S = A B^T and X = A W
+        // (2) S = A B^T;  X = A hi(W) + A lo(W)
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
@@ -199,23 +211,33 @@ la2_scan_bf16_sm100(const __grid_constant__ ScanParams p)
             for (int s = 0; s < DA / 16; ++s) {
                 const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
                 mma_bf16_ss(tX, sdesc_sw128(sA + off, 16, 1024),
-                            sdesc_sw128(sW + s * 2048, DA * kSlice * 2, 1024), kIdX, s > 0);
+                            sdesc_sw128(sWhi + s * 2048, 16384, 1024), kIdX, s > 0);
+            }
+#pragma unroll
+            for (int s = 0; s < DA / 16; ++s) {
+                const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+                mma_bf16_ss(tX, sdesc_sw128(sA + off, 16, 1024),
+                            sdesc_sw128(sWlo + s * 2048, 16384, 1024), kIdX, 1);
             }
             mma_commit(bar_mma);
             ok = mbar_wait(bar_mma, ph_mma);
         }
         ph_mma ^= 1;
-        if (!__syncthreads_and(ok)) { if (tid == 0) report_timeout(p.status, 2); break; }
+        if (!__syncthreads_and(ok)) {
+            if (tid == 0) report_status(p.status, kDevTimeout, 2);
+            break;
+        }
         tc_fence_after();
 
-        // (3a) P = decay-masked S, bf16, into the A buffer (K-major, swizzled)
+        // (3a) P = decay-masked S as hi + lo bf16, written into TMEM over the
+        //      32 columns of S each chunk came from: [hi (16 cols) | lo (16 cols)]
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
             const bool zero = dir > 0 ? (cc > warp) : (cc < warp);  // warp-uniform
-            uint32_t pk[16];
+            uint32_t hi[16], lo[16];
             if (zero) {
 #pragma unroll
-                for (int u = 0; u < 16; ++u) pk[u] = 0u;
+                for (int u = 0; u < 16; ++u) hi[u] = lo[u] = 0u;
             } else {
                 float s[32];
                 tmem_ld32(tS + lane_off + cc * 32, s);
@@ -226,14 +248,11 @@ la2_scan_bf16_sm100(const __grid_constant__ ScanParams p)
                     const int lag1 = dir > 0 ? r - c0 - 1 : c0 + 1 - r;
                     const float p0 = lag0 >= 0 ? s[2 * u] * pw[lag0 < 0 ? 0 : lag0] : 0.f;
                     const float p1 = lag1 >= 0 ? s[2 * u + 1] * pw[lag1 < 0 ? 0 : lag1] : 0.f;
-                    pk[u] = pack_bf16x2(p0, p1);
+                    split_pack2(p0, p1, hi[u], lo[u]);
                 }
             }
-            const uint32_t region = sA + (cc >> 1) * 16384;
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                st_shared_v4(region + sw128(r, (cc & 1) * 4 + u), pk[4 * u], pk[4 * u + 1],
-                             pk[4 * u + 2], pk[4 * u + 3]);
+            tmem_st16(tS + lane_off + cc * 32, hi);
+            tmem_st16(tS + lane_off + cc * 32 + 16, lo);
         }
 
         // (3b) X row r *= w_x(r)   (the inter-tile term, still alone in X)
@@ -249,21 +268,22 @@ la2_scan_bf16_sm100(const __grid_constant__ ScanParams p)
             }
         }
 
-        // (3c) B row r *= w_s(r), in place (B is not needed unscaled any more)
+        // (3c) row r of w_s(r) B: hi part in place in the B buffer, lo part
+        //      into the (now free) A buffer at the same offset
         {
             const float ws = dir > 0 ? pw[kTB - 1 - r] : pw[r];
 #pragma unroll
             for (int g = 0; g < DA / 64; ++g) {
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    const uint32_t addr = sB + g * 16384 + sw128(r, q);
-                    uint32_t v0, v1, v2, v3;
-                    ld_shared_v4(addr, v0, v1, v2, v3);
-                    v0 = pack_bf16x2(bf16lo_to_f32(v0) * ws, bf16hi_to_f32(v0) * ws);
-                    v1 = pack_bf16x2(bf16lo_to_f32(v1) * ws, bf16hi_to_f32(v1) * ws);
-                    v2 = pack_bf16x2(bf16lo_to_f32(v2) * ws, bf16hi_to_f32(v2) * ws);
-                    v3 = pack_bf16x2(bf16lo_to_f32(v3) * ws, bf16hi_to_f32(v3) * ws);
-                    st_shared_v4(addr, v0, v1, v2, v3);
+                    const uint32_t off = g * 16384 + sw128(r, q);
+                    uint32_t v[4], h[4], l[4];
+                    ld_shared_v4(sB + off, v[0], v[1], v[2], v[3]);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        split_pack2(bf16lo_to_f32(v[u]) * ws, bf16hi_to_f32(v[u]) * ws, h[u], l[u]);
+                    st_shared_v4(sB + off, h[0], h[1], h[2], h[3]);
+                    st_shared_v4(sA + off, l[0], l[1], l[2], l[3]);
                 }
             }
         }
@@ -272,50 +292,49 @@ la2_scan_bf16_sm100(const __grid_constant__ ScanParams p)
         tc_fence_before();
         __syncthreads();
 
-        // (4) X += P C ;  dW = (diag(w_s) B)^T C
+        // (4) X += hi(P) C + lo(P) C;  dW = hi(w_s B)^T C + lo(w_s B)^T C
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int s = 0; s < kTB / 16; ++s) {
-                const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-                mma_bf16_ss(tX, sdesc_sw128(sA + off, 16, 1024),
-                            sdesc_sw128(sC + s * 2048, kTB * kSlice * 2, 1024), kIdX, 1);
+                const uint32_t pcol = (s >> 1) * 32 + (s & 1) * 8;
+                const uint64_t cdesc = sdesc_sw128(sC + s * 2048, 16384, 1024);
+                mma_bf16_ts(tX, tS + pcol, cdesc, kIdX, 1);
+                mma_bf16_ts(tX, tS + pcol + 16, cdesc, kIdX, 1);
             }
 #pragma unroll
             for (int s = 0; s < kTB / 16; ++s) {
-                mma_bf16_ss(tD, sdesc_sw128(sB + s * 2048, 16384, 1024),
-                            sdesc_sw128(sC + s * 2048, kTB * kSlice * 2, 1024), kIdW, s > 0);
+                const uint64_t cdesc = sdesc_sw128(sC + s * 2048, 16384, 1024);
+                mma_bf16_ss(tD, sdesc_sw128(sB + s * 2048, 16384, 1024), cdesc, kIdW, s > 0);
+                mma_bf16_ss(tD, sdesc_sw128(sA + s * 2048, 16384, 1024), cdesc, kIdW, 1);
             }
             mma_commit(bar_mma);
             ok = mbar_wait(bar_mma, ph_mma);
         }
         ph_mma ^= 1;
-        if (!__syncthreads_and(ok)) { if (tid == 0) report_timeout(p.status, 3); break; }
+        if (!__syncthreads_and(ok)) {
+            if (tid == 0) report_status(p.status, kDevTimeout, 3);
+            break;
+        }
         tc_fence_after();
 
-        // (5) A and B buffers are free: start the next tile's A, B loads
-        const bool has_next = step + 1 < nb;
-        const int inext = dir > 0 ? i + 1 : i - 1;
-        if (tid == 0 && has_next) {
-            mbar_arrive_expect_tx(bar_load, kBytesAB + kBytesC);
-            issue_ab(inext);
-        }
+        // (5) all smem tiles are free: start the next tile's loads
+        if (tid == 0 && step + 1 < nb) issue_loads(dir > 0 ? i + 1 : i - 1);
 
-        // (6a) X row r -> bf16 -> C buffer (store staging)
+        // (6a) X row r -> fp32 -> global (rows past T are not stored)
 #pragma unroll
         for (int cc = 0; cc < kSlice / 32; ++cc) {
             float x[32];
             tmem_ld32(tX + lane_off + cc * 32, x);
-            uint32_t pk[16];
+            if (r < rows) {
+                float* dst = xg + static_cast<size_t>(i * kTB + r) * p.dc + cc * 32;
 #pragma unroll
-            for (int u = 0; u < 16; ++u) pk[u] = pack_bf16x2(x[2 * u], x[2 * u + 1]);
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                st_shared_v4(sC + sw128(r, cc * 4 + u), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2],
-                             pk[4 * u + 3]);
+                for (int u = 0; u < 8; ++u)
+                    st_global_v4(dst + 4 * u, x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
+            }
         }
 
-        // (6b) W <- lambda^T_B W + dW (fp32, registers); bf16 copy for the next tile
+        // (6b) W <- lambda^T_B W + dW (fp32, registers); hi/lo bf16 copies for the next tile
 #pragma unroll
         for (int cc = 0; cc < kSlice / 32; ++cc) {
             float dw[32];
@@ -326,28 +345,21 @@ la2_scan_bf16_sm100(const __grid_constant__ ScanParams p)
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int c = cc * 32 + u * 8;
-                    st_shared_v4(sW + sw128(wrow, cc * 4 + u),
-                                 pack_bf16x2(w[c + 0], w[c + 1]), pack_bf16x2(w[c + 2], w[c + 3]),
-                                 pack_bf16x2(w[c + 4], w[c + 5]), pack_bf16x2(w[c + 6], w[c + 7]));
+                    uint32_t h[4], l[4];
+#pragma unroll
+                    for (int z = 0; z < 4; ++z)
+                        split_pack2(w[c + 2 * z], w[c + 2 * z + 1], h[z], l[z]);
+                    const uint32_t off = sw128(wrow, cc * 4 + u);
+                    st_shared_v4(sWhi + off, h[0], h[1], h[2], h[3]);
+                    st_shared_v4(sWlo + off, l[0], l[1], l[2], l[3]);
                 }
             }
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-
-        // (7) store X_i; once its staging is read, load the next C slice there
-        if (tid == 0) {
-            tma_store_3d(&R.tx, sC, x0, i * kTB, bh);
-            bulk_commit();
-            if (has_next) {
-                bulk_wait_read0();
-                issue_c(inext);
-            }
-        }
     }
 
-    if (tid == 0) bulk_wait0();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {

@@ -128,7 +128,9 @@ def _stream_ptr(stream) -> int:
 
 def la2_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, decay: torch.Tensor,
             out: torch.Tensor | None = None, block: int = 128, stream=None) -> torch.Tensor:
-    """o[b,h,t] = sum_{s<=t} decay[h]^(t-s) (q[b,h,t] . k[b,h,s]) v[b,h,s], on q's device."""
+    """o[b,h,t] = sum_{s<=t} decay[h]^(t-s) (q[b,h,t] . k[b,h,s]) v[b,h,s], on q's device.
+
+    q, k, v: bf16 or fp32; the output is always fp32."""
     B, H, T, d = q.shape
     e = v.shape[-1]
     dt = _dtype_code(q)
@@ -137,8 +139,8 @@ def la2_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, decay: torch.Tens
     _check(v, "v", (B, H, T, e), q.dtype)
     _check(decay, "decay", (H,), torch.float32)
     if out is None:
-        out = torch.empty((B, H, T, e), dtype=q.dtype, device=q.device)
-    _check(out, "out", (B, H, T, e), q.dtype)
+        out = torch.empty((B, H, T, e), dtype=torch.float32, device=q.device)
+    _check(out, "out", (B, H, T, e), torch.float32)
     st = la2_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(), out.data_ptr(),
                      B, H, T, d, e, block, dt, 0, 0, _stream_ptr(stream))
     if st != LA2_OK:
@@ -155,11 +157,12 @@ def la2_bwd(q, k, v, decay, dout, dq=None, dk=None, dv=None, block: int = 128, s
                       (dout, "dout", (B, H, T, e))):
         _check(t, n, shp, q.dtype)
     _check(decay, "decay", (H,), torch.float32)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty((B, H, T, d), **f32) if dq is None else dq
+    dk = torch.empty((B, H, T, d), **f32) if dk is None else dk
+    dv = torch.empty((B, H, T, e), **f32) if dv is None else dv
     for t, n, shp in ((dq, "dq", (B, H, T, d)), (dk, "dk", (B, H, T, d)), (dv, "dv", (B, H, T, e))):
-        _check(t, n, shp, q.dtype)
+        _check(t, n, shp, torch.float32)
     st = la2_bwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(), dout.data_ptr(),
                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, T, d, e, block, dt, 0, 0,
                      _stream_ptr(stream))

@@ -21,8 +21,9 @@
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library
  *     never allocates, frees or retains them past the call.
  *   - q, k, dq, dk are [B, H, T, d] contiguous (d fastest); v, out, dout, dv
- *     are [B, H, T, e] contiguous.  All share the element type `dtype`.
- *     Every tensor pointer must be 16-byte aligned.
+ *     are [B, H, T, e] contiguous.  The inputs q, k, v, dout have the element
+ *     type `dtype`; the outputs out, dq, dk, dv are always fp32 (see
+ *     la2_dtype).  Every tensor pointer must be 16-byte aligned.
  *   - decay is a device array of H floats (fp32) holding lambda_h in (0, 1];
  *     values outside that range are the caller's error and are not checked.
  *   - block is the tile length T_B (64, 128 or 256).  It changes the order of
@@ -58,9 +59,16 @@ typedef enum {
     LA2_ERR_TIMEOUT = 5       /* a kernel's bounded wait ran out (see la2_device_status) */
 } la2_status;
 
+/*
+ * Input element type.  Outputs are fp32 in both cases: the accuracy contract
+ * of this library is max|out - exact| <= 2e-2 * rms(exact) for bf16 inputs
+ * (1e-5 for fp32 inputs), and the outputs of this operation have
+ * max/rms ~ 10, where a bf16 result's own rounding (half an ulp, up to 2^-5
+ * of rms) would already exceed that bound.
+ */
 typedef enum {
-    LA2_DTYPE_F32 = 0,   /* fp32 in, fp32 out, fp32 arithmetic (SIMT kernels) */
-    LA2_DTYPE_BF16 = 1   /* bf16 in, bf16 out, fp32 accumulation and fp32 state (tcgen05) */
+    LA2_DTYPE_F32 = 0,   /* fp32 inputs; fp32 arithmetic on SIMT cores */
+    LA2_DTYPE_BF16 = 1   /* bf16 inputs; tcgen05 tensor cores, fp32 accumulation and state */
 } la2_dtype;
 
 /*

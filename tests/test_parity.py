@@ -38,8 +38,9 @@ def _run_gpu(la2mod, x, block, fill_nan=True):
     dev = torch.device("cuda")
     q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
     lam = x["lam"].to(dev)
-    out = torch.empty_like(v)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = torch.empty(v.shape, **f32)
+    dq, dk, dv = torch.empty(q.shape, **f32), torch.empty(k.shape, **f32), torch.empty(v.shape, **f32)
     if fill_nan:
         for t in (out, dq, dk, dv):
             t.fill_(float("nan"))
@@ -130,10 +131,10 @@ def test_outputs_do_not_write_past_their_end(la2mod):
     lam = x["lam"].to(dev)
     n_o, n_q = v.numel(), q.numel()
     guard = 4096
-    buf_o = torch.full((n_o + guard,), 7.0, dtype=torch.bfloat16, device=dev)
-    buf_q = torch.full((n_q + guard,), 7.0, dtype=torch.bfloat16, device=dev)
-    buf_k = torch.full((n_q + guard,), 7.0, dtype=torch.bfloat16, device=dev)
-    buf_v = torch.full((n_o + guard,), 7.0, dtype=torch.bfloat16, device=dev)
+    buf_o = torch.full((n_o + guard,), 7.0, dtype=torch.float32, device=dev)
+    buf_q = torch.full((n_q + guard,), 7.0, dtype=torch.float32, device=dev)
+    buf_k = torch.full((n_q + guard,), 7.0, dtype=torch.float32, device=dev)
+    buf_v = torch.full((n_o + guard,), 7.0, dtype=torch.float32, device=dev)
     la2mod.la2_fwd(q, k, v, lam, out=buf_o[:n_o].view_as(v))
     la2mod.la2_bwd(q, k, v, lam, do, dq=buf_q[:n_q].view_as(q), dk=buf_k[:n_q].view_as(k),
                    dv=buf_v[:n_o].view_as(v))
