@@ -231,25 +231,22 @@ la2_scan_bf16_sm100(const __grid_constant__ ScanParams p)
 
         // (3a) P = decay-masked S as hi + lo bf16, written into TMEM over the
         //      32 columns of S each chunk came from: [hi (16 cols) | lo (16 cols)]
+        //      Every chunk is loaded before it is overwritten, also chunks the
+        //      mask zeroes entirely: storing over S columns that were not read
+        //      first made the following TMEM-operand MMAs about 10x slower.
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
-            const bool zero = dir > 0 ? (cc > warp) : (cc < warp);  // warp-uniform
             uint32_t hi[16], lo[16];
-            if (zero) {
+            float s[32];
+            tmem_ld32(tS + lane_off + cc * 32, s);
 #pragma unroll
-                for (int u = 0; u < 16; ++u) hi[u] = lo[u] = 0u;
-            } else {
-                float s[32];
-                tmem_ld32(tS + lane_off + cc * 32, s);
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int c0 = cc * 32 + 2 * u;
-                    const int lag0 = dir > 0 ? r - c0 : c0 - r;
-                    const int lag1 = dir > 0 ? r - c0 - 1 : c0 + 1 - r;
-                    const float p0 = lag0 >= 0 ? s[2 * u] * pw[lag0 < 0 ? 0 : lag0] : 0.f;
-                    const float p1 = lag1 >= 0 ? s[2 * u + 1] * pw[lag1 < 0 ? 0 : lag1] : 0.f;
-                    split_pack2(p0, p1, hi[u], lo[u]);
-                }
+            for (int u = 0; u < 16; ++u) {
+                const int c0 = cc * 32 + 2 * u;
+                const int lag0 = dir > 0 ? r - c0 : c0 - r;
+                const int lag1 = dir > 0 ? r - c0 - 1 : c0 + 1 - r;
+                const float p0 = lag0 >= 0 ? s[2 * u] * pw[lag0 < 0 ? 0 : lag0] : 0.f;
+                const float p1 = lag1 >= 0 ? s[2 * u + 1] * pw[lag1 < 0 ? 0 : lag1] : 0.f;
+                split_pack2(p0, p1, hi[u], lo[u]);
             }
             tmem_st16(tS + lane_off + cc * 32, hi);
             tmem_st16(tS + lane_off + cc * 32 + 16, lo);
