@@ -81,20 +81,23 @@ bool device_setup(int* dev_out, int** status_out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Tensor map over a contiguous [BH, T, D] bf16 tensor, box 64 x 128 x 1, 128B swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, int BH, int T, int D) {
+// Tensor map over a contiguous [BH, T, D] tensor with 128-byte rows per box
+// (64 bf16 or 32 fp32 elements) x 128 rows x 1, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, int BH, int T, int D, bool fp32) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
+    const cuuint64_t esz = fp32 ? 4 : 2;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(T),
                                 static_cast<cuuint64_t>(BH)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
-                                   static_cast<cuuint64_t>(T) * static_cast<cuuint64_t>(D) * 2};
-    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(la2::kTB), 1};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * esz,
+                                   static_cast<cuuint64_t>(T) * static_cast<cuuint64_t>(D) * esz};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esz),
+                               static_cast<cuuint32_t>(la2::kTB), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-           CUDA_SUCCESS;
+    return enc(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+               const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 struct RoleDesc {
@@ -130,11 +133,11 @@ la2_status launch_bf16(const RoleDesc* roles, int n, const float* decay, int B, 
     const int BH = B * H;
     const int da = roles[0].da, dc = roles[0].dc;
     for (int r = 0; r < n; ++r) {
-        if (!make_map(&p.role[r].ta, roles[r].a, BH, T, da) ||
-            !make_map(&p.role[r].tb, roles[r].b, BH, T, da) ||
-            !make_map(&p.role[r].tc, roles[r].c, BH, T, dc))
+        if (!make_map(&p.role[r].ta, roles[r].a, BH, T, da, false) ||
+            !make_map(&p.role[r].tb, roles[r].b, BH, T, da, false) ||
+            !make_map(&p.role[r].tc, roles[r].c, BH, T, dc, false) ||
+            !make_map(&p.role[r].tx, roles[r].x, BH, T, dc, true))
             return LA2_ERR_CUDA;
-        p.role[r].x = static_cast<float*>(roles[r].x);
         p.role[r].dir = roles[r].dir;
     }
     p.decay = decay;

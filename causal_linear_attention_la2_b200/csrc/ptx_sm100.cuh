@@ -222,6 +222,22 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
         : "memory");
 }
 
+// 16 consecutive 32-bit TMEM columns of this thread's lane (warp-collective),
+// waited for inside the same asm statement.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr) : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // 16 consecutive 32-bit TMEM columns of this thread's lane (warp-collective).
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
     asm volatile(
@@ -231,6 +247,13 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
            "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]),
            "r"(v[13]), "r"(v[14]), "r"(v[15])
         : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16f(uint32_t taddr, const float (&v)[16]) {
+    uint32_t u[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(v[i]);
+    tmem_st16(taddr, u);
 }
 
 __device__ __forceinline__ void tmem_wait_ld() {
@@ -270,13 +293,13 @@ __device__ __forceinline__ void split_bf16(float x, uint32_t& hi, uint32_t& lo) 
     lo = static_cast<uint32_t>(__bfloat16_as_ushort(l));
 }
 
-// Packs the hi and lo parts of (x0, x1) into two bf16x2 words.
+// Packs the hi and lo parts of (x0, x1) into two bf16x2 words (x0 in the low
+// half): hi = bf16(x), lo = bf16(x - hi), both round-to-nearest-even.
 __device__ __forceinline__ void split_pack2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-    uint32_t h0, l0, h1, l1;
-    split_bf16(x0, h0, l0);
-    split_bf16(x1, h1, l1);
-    hi = h0 | (h1 << 16);
-    lo = l0 | (l1 << 16);
+    hi = pack_bf16x2(x0, x1);
+    const float h0 = __uint_as_float(hi << 16);
+    const float h1 = __uint_as_float(hi & 0xFFFF0000u);
+    lo = pack_bf16x2(x0 - h0, x1 - h1);
 }
 
 __device__ __forceinline__ void st_global_v4(void* p, float a, float b, float c, float d) {
