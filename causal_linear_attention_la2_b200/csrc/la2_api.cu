@@ -1,16 +1,18 @@
 // la2_api.cu -- the C ABI of libla2.so (declared in include/la2.h): argument
 // validation, TMA descriptor set-up and kernel launch.  Everything numerical
-// happens in the kernels of scan_bf16_sm100.cuh and scan_f32.cuh.
+// happens in the kernels of scan_ws_sm100.cuh (bf16 inputs) and scan_f32.cuh
+// (fp32 inputs).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
 #include "la2.h"
-#include "scan_bf16_sm100.cuh"
 #include "scan_f32.cuh"
+#include "scan_ws_sm100.cuh"
 
 namespace {
 
@@ -39,6 +41,13 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+template <int DA, int DC>
+bool set_ws_attrs() {
+    return cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                la2::ws::Smem<DA, DC>::kBytes) == cudaSuccess;
+}
+
 struct DeviceState {
     std::once_flag once;
     int* status = nullptr;
@@ -55,18 +64,8 @@ bool device_setup(int* dev_out, int** status_out) {
         void* p = nullptr;
         bool ok = cudaGetSymbolAddress(&p, g_la2_status) == cudaSuccess;
         s.status = static_cast<int*>(p);
-        ok = ok && cudaFuncSetAttribute(la2::la2_scan_bf16_sm100<64>,
-                                        cudaFuncAttributePreferredSharedMemoryCarveout,
-                                        100) == cudaSuccess;
-        ok = ok && cudaFuncSetAttribute(la2::la2_scan_bf16_sm100<128>,
-                                        cudaFuncAttributePreferredSharedMemoryCarveout,
-                                        100) == cudaSuccess;
-        ok = ok && cudaFuncSetAttribute(la2::la2_scan_bf16_sm100<64>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        la2::ScanSmem<64>::kBytes) == cudaSuccess;
-        ok = ok && cudaFuncSetAttribute(la2::la2_scan_bf16_sm100<128>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        la2::ScanSmem<128>::kBytes) == cudaSuccess;
+        ok = ok && set_ws_attrs<64, 64>() && set_ws_attrs<64, 128>() && set_ws_attrs<128, 64>() &&
+             set_ws_attrs<128, 128>();
         ok = ok && cudaFuncSetAttribute(la2::la2_scan_f32,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         static_cast<int>(la2::f32_scan_smem_bytes(128, 128, 256))) ==
@@ -92,7 +91,7 @@ bool make_map(CUtensorMap* m, const void* ptr, int BH, int T, int D, bool fp32) 
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * esz,
                                    static_cast<cuuint64_t>(T) * static_cast<cuuint64_t>(D) * esz};
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esz),
-                               static_cast<cuuint32_t>(la2::kTB), 1};
+                               static_cast<cuuint32_t>(la2::ws::kTB), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -118,26 +117,32 @@ la2_status common_checks(int B, int H, int T, int d, int e, int block, la2_dtype
     if (static_cast<long long>(B) * H > (1LL << 24)) return LA2_ERR_UNSUPPORTED;
     if (dtype == LA2_DTYPE_BF16) {
         if ((d != 64 && d != 128) || (e != 64 && e != 128)) return LA2_ERR_UNSUPPORTED;
-        if (block != la2::kTB) return LA2_ERR_UNSUPPORTED;
+        if (block != la2::ws::kTB) return LA2_ERR_UNSUPPORTED;
     } else {
         if (d > 128 || e > 128) return LA2_ERR_UNSUPPORTED;
     }
     return LA2_OK;
 }
 
-// Launches one bf16 grid over `n` roles that share (DA, DC).
-la2_status launch_bf16(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
-                       int* status, cudaStream_t stream) {
-    la2::ScanParams p;
+template <int DA, int DC>
+void launch_ws(const la2::ws::Params& p, unsigned grid, cudaStream_t stream) {
+    la2::ws::la2_scan_ws<DA, DC><<<grid, la2::ws::kThreads, la2::ws::Smem<DA, DC>::kBytes, stream>>>(p);
+}
+
+// Launches the warp-specialised kernel over `n` roles that share (DA, DC):
+// one CTA per (sequence, role).
+la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
+                          int* status, cudaStream_t stream) {
+    la2::ws::Params p;
     std::memset(&p, 0, sizeof(p));
     const int BH = B * H;
     const int da = roles[0].da, dc = roles[0].dc;
     for (int r = 0; r < n; ++r) {
         if (!make_map(&p.role[r].ta, roles[r].a, BH, T, da, false) ||
             !make_map(&p.role[r].tb, roles[r].b, BH, T, da, false) ||
-            !make_map(&p.role[r].tc, roles[r].c, BH, T, dc, false) ||
-            !make_map(&p.role[r].tx, roles[r].x, BH, T, dc, true))
+            !make_map(&p.role[r].tc, roles[r].c, BH, T, dc, false))
             return LA2_ERR_CUDA;
+        p.role[r].x = static_cast<float*>(roles[r].x);
         p.role[r].dir = roles[r].dir;
     }
     p.decay = decay;
@@ -145,13 +150,11 @@ la2_status launch_bf16(const RoleDesc* roles, int n, const float* decay, int B, 
     p.H = H;
     p.T = T;
     p.nroles = n;
-    p.nslices = dc / la2::kSlice;
-    p.dc = dc;
-    const dim3 grid(static_cast<unsigned>(BH * n * p.nslices));
-    if (da == 128)
-        la2::la2_scan_bf16_sm100<128><<<grid, la2::kThreads, la2::ScanSmem<128>::kBytes, stream>>>(p);
-    else
-        la2::la2_scan_bf16_sm100<64><<<grid, la2::kThreads, la2::ScanSmem<64>::kBytes, stream>>>(p);
+    const unsigned grid = static_cast<unsigned>(BH * n);
+    if (da == 128 && dc == 128) launch_ws<128, 128>(p, grid, stream);
+    else if (da == 128) launch_ws<128, 64>(p, grid, stream);
+    else if (dc == 128) launch_ws<64, 128>(p, grid, stream);
+    else launch_ws<64, 64>(p, grid, stream);
     if (cudaGetLastError() != cudaSuccess) return LA2_ERR_CUDA;
     ++t_last_launches;
     return LA2_OK;
@@ -203,7 +206,7 @@ la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, in
                 group[m++] = roles[s];
                 done[s] = true;
             }
-        const la2_status st = launch_bf16(group, m, decay, B, H, T, status, stream);
+        const la2_status st = launch_bf16_ws(group, m, decay, B, H, T, status, stream);
         if (st != LA2_OK) return st;
     }
     return LA2_OK;

@@ -1,6 +1,6 @@
 // scan_f32.cuh -- fp32 SIMT kernel of the Lightning Attention-2 path.
 //
-// Same decayed scan as the tcgen05 kernel (see scan_bf16_sm100.cuh), in plain
+// Same decayed scan as the tcgen05 kernel (see scan_ws_sm100.cuh), in plain
 // fp32 FFMA so that fp32 inputs keep fp32 accuracy (tensor cores would round
 // operands to bf16/tf32).  The tile length T_B (64, 128 or 256) is honoured:
 // the state W is carried from tile to tile and updated once per tile; inside a
