@@ -43,9 +43,49 @@ EncodeTiledFn encode_fn() {
 
 template <int DA, int DC>
 bool set_ws_attrs() {
-    return cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC>,
+    return cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC, false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                la2::ws::Smem<DA, DC>::kBytes) == cudaSuccess &&
+           cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC, true>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 la2::ws::Smem<DA, DC>::kBytes) == cudaSuccess;
+}
+
+// Sequence segments for the bf16 kernel.  Each CTA takes one (sequence,
+// role, segment) and fills one SM; when there are fewer (sequence, role)
+// units than the B200's 148 SMs, each sequence is cut into segments so that
+// the grid fills the GPU (a state pre-pass hands each segment its incoming
+// state).  The count depends on the number of units only, never on T, so the
+// workspace it needs is flat in T; per call it is further capped so that a
+// segment holds at least two tiles.
+constexpr int kTargetCTAs = 148;
+constexpr int kMaxSegments = 32;
+
+int max_segments(long long units) {
+    if (units <= 0 || units >= kTargetCTAs) return 1;
+    const long long g = kTargetCTAs / units;
+    return static_cast<int>(g < kMaxSegments ? g : kMaxSegments);
+}
+
+struct SegPlan {
+    int nseg, seg_tiles;
+};
+
+SegPlan plan_segments(long long units, int T) {
+    const int nb = (T + la2::ws::kTB - 1) / la2::ws::kTB;
+    int g = max_segments(units);
+    const int cap = nb / 2 > 1 ? nb / 2 : 1;
+    if (g > cap) g = cap;
+    SegPlan sp;
+    sp.seg_tiles = (nb + g - 1) / g;
+    sp.nseg = (nb + sp.seg_tiles - 1) / sp.seg_tiles;
+    return sp;
+}
+
+// Workspace bytes of one bf16 launch over `units` (sequence, role) units.
+size_t seg_workspace_bytes(long long units, int da, int dc) {
+    return static_cast<size_t>(max_segments(units) - 1) * static_cast<size_t>(units) *
+           static_cast<size_t>(da) * static_cast<size_t>(dc) * sizeof(float);
 }
 
 struct DeviceState {
@@ -125,14 +165,20 @@ la2_status common_checks(int B, int H, int T, int d, int e, int block, la2_dtype
 }
 
 template <int DA, int DC>
-void launch_ws(const la2::ws::Params& p, unsigned grid, cudaStream_t stream) {
-    la2::ws::la2_scan_ws<DA, DC><<<grid, la2::ws::kThreads, la2::ws::Smem<DA, DC>::kBytes, stream>>>(p);
+void launch_ws(const la2::ws::Params& p, unsigned units, cudaStream_t stream) {
+    constexpr size_t smem = la2::ws::Smem<DA, DC>::kBytes;
+    if (p.nseg > 1)
+        la2::ws::la2_scan_ws<DA, DC, true>
+            <<<units * static_cast<unsigned>(p.nseg - 1), la2::ws::kThreads, smem, stream>>>(p);
+    la2::ws::la2_scan_ws<DA, DC, false>
+        <<<units * static_cast<unsigned>(p.nseg), la2::ws::kThreads, smem, stream>>>(p);
 }
 
 // Launches the warp-specialised kernel over `n` roles that share (DA, DC):
-// one CTA per (sequence, role).
+// one CTA per (sequence, role, segment), preceded by the state pre-pass when
+// sequences are split into segments.
 la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
-                          int* status, cudaStream_t stream) {
+                          int* status, float* seg_state, cudaStream_t stream) {
     la2::ws::Params p;
     std::memset(&p, 0, sizeof(p));
     const int BH = B * H;
@@ -150,13 +196,18 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
     p.H = H;
     p.T = T;
     p.nroles = n;
-    const unsigned grid = static_cast<unsigned>(BH * n);
-    if (da == 128 && dc == 128) launch_ws<128, 128>(p, grid, stream);
-    else if (da == 128) launch_ws<128, 64>(p, grid, stream);
-    else if (dc == 128) launch_ws<64, 128>(p, grid, stream);
-    else launch_ws<64, 64>(p, grid, stream);
+    const SegPlan sp = plan_segments(static_cast<long long>(BH) * n, T);
+    p.nseg = sp.nseg;
+    p.seg_tiles = sp.seg_tiles;
+    p.seg_state = seg_state;
+    if (sp.nseg > 1 && !seg_state) return LA2_ERR_WORKSPACE;
+    const unsigned units = static_cast<unsigned>(BH * n);
+    if (da == 128 && dc == 128) launch_ws<128, 128>(p, units, stream);
+    else if (da == 128) launch_ws<128, 64>(p, units, stream);
+    else if (dc == 128) launch_ws<64, 128>(p, units, stream);
+    else launch_ws<64, 64>(p, units, stream);
     if (cudaGetLastError() != cudaSuccess) return LA2_ERR_CUDA;
-    ++t_last_launches;
+    t_last_launches += sp.nseg > 1 ? 2 : 1;
     return LA2_OK;
 }
 
@@ -189,13 +240,10 @@ la2_status launch_f32(const RoleDesc* roles, int n, const float* decay, int B, i
     return LA2_OK;
 }
 
-la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
-                     int block, la2_dtype dtype, cudaStream_t stream) {
-    int dev = 0;
-    int* status = nullptr;
-    if (!device_setup(&dev, &status)) return LA2_ERR_CUDA;
-    if (dtype == LA2_DTYPE_F32) return launch_f32(roles, n, decay, B, H, T, block, stream);
-    // group roles with identical (DA, DC) into one grid
+// Groups roles with identical (DA, DC); each group is one launch (two with the
+// state pre-pass).  Calls `f(group, m)` per group, in a fixed order.
+template <class F>
+la2_status for_role_groups(const RoleDesc* roles, int n, F&& f) {
     RoleDesc group[3];
     bool done[3] = {false, false, false};
     for (int r = 0; r < n; ++r) {
@@ -206,10 +254,39 @@ la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, in
                 group[m++] = roles[s];
                 done[s] = true;
             }
-        const la2_status st = launch_bf16_ws(group, m, decay, B, H, T, status, stream);
+        const la2_status st = f(group, m);
         if (st != LA2_OK) return st;
     }
     return LA2_OK;
+}
+
+size_t bf16_workspace_bytes(const RoleDesc* roles, int n, int B, int H) {
+    size_t total = 0;
+    for_role_groups(roles, n, [&](const RoleDesc* g, int m) {
+        total += seg_workspace_bytes(static_cast<long long>(B) * H * m, g[0].da, g[0].dc);
+        total = (total + 255) & ~static_cast<size_t>(255);
+        return LA2_OK;
+    });
+    return total;
+}
+
+la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
+                     int block, la2_dtype dtype, void* workspace, size_t ws_bytes,
+                     cudaStream_t stream) {
+    int dev = 0;
+    int* status = nullptr;
+    if (dtype == LA2_DTYPE_BF16 && bf16_workspace_bytes(roles, n, B, H) > 0 &&
+        (workspace == nullptr || ws_bytes < bf16_workspace_bytes(roles, n, B, H)))
+        return LA2_ERR_WORKSPACE;
+    if (!device_setup(&dev, &status)) return LA2_ERR_CUDA;
+    if (dtype == LA2_DTYPE_F32) return launch_f32(roles, n, decay, B, H, T, block, stream);
+    size_t off = 0;
+    return for_role_groups(roles, n, [&](const RoleDesc* g, int m) {
+        float* seg = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) + off) : nullptr;
+        off += seg_workspace_bytes(static_cast<long long>(B) * H * m, g[0].da, g[0].dc);
+        off = (off + 255) & ~static_cast<size_t>(255);
+        return launch_bf16_ws(g, m, decay, B, H, T, status, seg, stream);
+    });
 }
 
 }  // namespace
@@ -218,18 +295,20 @@ extern "C" {
 
 size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block, la2_dtype dtype,
                            int is_bwd) {
-    (void)is_bwd;
     bool empty = false;
     const la2_status st = common_checks(B, H, T, d, e, block, dtype, &empty);
     if (st != LA2_OK) return static_cast<size_t>(-1);
-    return 0;
+    if (empty || dtype != LA2_DTYPE_BF16) return 0;
+    const RoleDesc fwd[1] = {{nullptr, nullptr, nullptr, nullptr, d, e, +1}};
+    const RoleDesc bwd[3] = {{nullptr, nullptr, nullptr, nullptr, e, d, +1},
+                             {nullptr, nullptr, nullptr, nullptr, e, d, -1},
+                             {nullptr, nullptr, nullptr, nullptr, d, e, -1}};
+    return is_bwd ? bf16_workspace_bytes(bwd, 3, B, H) : bf16_workspace_bytes(fwd, 1, B, H);
 }
 
 la2_status la2_fwd(const void* q, const void* k, const void* v, const float* decay, void* out,
                    int B, int H, int T, int d, int e, int block, la2_dtype dtype,
                    void* workspace, size_t workspace_bytes, la2_stream_t stream) {
-    (void)workspace;
-    (void)workspace_bytes;
     t_last_launches = 0;
     bool empty = false;
     la2_status st = common_checks(B, H, T, d, e, block, dtype, &empty);
@@ -238,16 +317,16 @@ la2_status la2_fwd(const void* q, const void* k, const void* v, const float* dec
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
         (reinterpret_cast<uintptr_t>(decay) & 3u))
         return LA2_ERR_INVALID_ARG;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return LA2_ERR_INVALID_ARG;
     const RoleDesc r = {q, k, v, out, d, e, +1};
-    return run_roles(&r, 1, decay, B, H, T, block, dtype, reinterpret_cast<cudaStream_t>(stream));
+    return run_roles(&r, 1, decay, B, H, T, block, dtype, workspace, workspace_bytes,
+                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 la2_status la2_bwd(const void* q, const void* k, const void* v, const float* decay,
                    const void* dout, void* dq, void* dk, void* dv, int B, int H, int T, int d,
                    int e, int block, la2_dtype dtype, void* workspace, size_t workspace_bytes,
                    la2_stream_t stream) {
-    (void)workspace;
-    (void)workspace_bytes;
     t_last_launches = 0;
     bool empty = false;
     la2_status st = common_checks(B, H, T, d, e, block, dtype, &empty);
@@ -262,7 +341,8 @@ la2_status la2_bwd(const void* q, const void* k, const void* v, const float* dec
         {v, dout, q, dk, e, d, -1},
         {k, q, dout, dv, d, e, -1},
     };
-    return run_roles(roles, 3, decay, B, H, T, block, dtype,
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return LA2_ERR_INVALID_ARG;
+    return run_roles(roles, 3, decay, B, H, T, block, dtype, workspace, workspace_bytes,
                      reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -60,7 +60,11 @@ struct Params {
     Role role[3];
     const float* decay;  // [H]
     int* status;         // device status word
+    float* seg_state;    // [B*H][nroles][nseg - 1][DA][DC] fp32: local end state of each
+                         // segment but the last (written by the state pass)
     int H, T, nroles;
+    int nseg;            // segments per (sequence, role); 1 = no split
+    int seg_tiles;       // tiles per segment (the last may be shorter)
 };
 
 enum Bar {
@@ -116,7 +120,15 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
 }
 
-template <int DA, int DC>
+// kState = false: the scan itself.  One CTA per (sequence, role, segment); a
+//   segment starts from the state the segments before it leave behind,
+//   W_in(g) = sum_{g' < g} lambda^(T_B n (g-1-g')) S_g' (n tiles per segment),
+//   read from seg_state.
+// kState = true: the state pre-pass.  One CTA per (sequence, role, segment
+//   but the last); it runs only the state recurrence of its segment from zero,
+//   W <- lambda^T_B W + (diag(w_s) B_i)^T C_i, and writes W (fp32) to
+//   seg_state.  Loads B and C only.
+template <int DA, int DC, bool kState>
 __global__ void __launch_bounds__(kThreads, 1)
 la2_scan_ws(const __grid_constant__ Params p)
 {
@@ -135,12 +147,18 @@ la2_scan_ws(const __grid_constant__ Params p)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + L::kAbort);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int role_id = blockIdx.x % p.nroles;
-    const int bh = blockIdx.x / p.nroles;
+    const int segs_in_grid = kState ? p.nseg - 1 : p.nseg;
+    const int g = blockIdx.x % segs_in_grid;
+    const int unit = blockIdx.x / segs_in_grid;  // (sequence, role)
+    const int role_id = unit % p.nroles;
+    const int bh = unit / p.nroles;
     const Role& R = p.role[role_id];
     const int dir = R.dir;
     const int T = p.T;
     const int nb = (T + kTB - 1) / kTB;
+    // this CTA's steps (in scan order): [s0, s0 + ns)
+    const int s0 = g * p.seg_tiles;
+    const int ns = max(0, min(p.seg_tiles, nb - s0));
     const float lam = p.decay[bh % p.H];
 
     // ---- set-up
@@ -155,7 +173,8 @@ la2_scan_ws(const __grid_constant__ Params p)
         tmem_relinquish();
     }
     if (tid == 0) {
-        const uint32_t counts[NBAR] = {1, 1, 1, 1, 1, 1, 1, 1, 256, 256, 256, 256, 256, 256, 2};
+        const uint32_t counts[NBAR] = {1, 1, 1, 1, 1, 1, 1, 1, 256, 256, 256, 256, 256, 256,
+                                       kState ? 1u : 2u};
         for (int b = 0; b < NBAR; ++b) mbar_init(bar(b), counts[b]);
         *abort_flag = 0;
         fence_mbar_init();
@@ -169,11 +188,15 @@ la2_scan_ws(const __grid_constant__ Params p)
     // TMEM: S / P (128 columns), X in two buffers (DC each), dW (DC)
     const uint32_t tS = tmem, tD = tmem + 128 + 2 * DC;
     auto tX = [&](int b) { return tmem + 128 + static_cast<uint32_t>(b * DC); };
-    auto tile_of = [&](int step) { return dir > 0 ? step : nb - 1 - step; };
+    auto tile_of = [&](int step) { return dir > 0 ? s0 + step : nb - 1 - (s0 + step); };
+    // fp32 state slot of segment gg of this (sequence, role)
+    auto seg_slot = [&](int gg) {
+        return p.seg_state + (static_cast<size_t>(unit) * (p.nseg - 1) + gg) * (DA * DC);
+    };
 
     if (warp == 0) {
         // ================================================= TMA producer
-        if (lane == 0 && nb > 0) {
+        if (lane == 0 && ns > 0) {
             prefetch_tmap(&R.ta);
             prefetch_tmap(&R.tb);
             prefetch_tmap(&R.tc);
@@ -193,25 +216,27 @@ la2_scan_ws(const __grid_constant__ Params p)
                 for (int g = 0; g < DC / 64; ++g)
                     tma_load_3d(sC + g * 16384, &R.tc, bar(FULL_C), g * 64, i * kTB, bh);
             };
-            load_a(tile_of(0));
+            if (!kState) load_a(tile_of(0));
             load_b(tile_of(0), 0);
-            if (nb > 1) load_b(tile_of(1), 1);
+            if (ns > 1) load_b(tile_of(1), 1);
             load_c(tile_of(0));
-            for (int s = 0; s < nb; ++s) {
+            for (int s = 0; s < ns; ++s) {
                 const uint32_t ph = s & 1;
                 // A is free once S and X = A W of tile s are done; B buffer s % 2 once
                 // dW of tile s is done; C once X += P C is done too.  Waiting in
                 // this order keeps every waiter within one phase of its barrier.
-                if (!wait_bar(bar(B_S), ph, abort_flag, p.status, 13)) break;
-                if (!wait_bar(bar(B_X), ph, abort_flag, p.status, 10)) break;
-                if (s + 1 < nb) load_a(tile_of(s + 1));
+                if (!kState) {
+                    if (!wait_bar(bar(B_S), ph, abort_flag, p.status, 13)) break;
+                    if (!wait_bar(bar(B_X), ph, abort_flag, p.status, 10)) break;
+                    if (s + 1 < ns) load_a(tile_of(s + 1));
+                }
                 if (!wait_bar(bar(B_D), ph, abort_flag, p.status, 11)) break;
-                if (s + 2 < nb) load_b(tile_of(s + 2), s & 1);
-                if (!wait_bar(bar(B_PC), ph, abort_flag, p.status, 12)) break;
-                if (s + 1 < nb) load_c(tile_of(s + 1));
+                if (s + 2 < ns) load_b(tile_of(s + 2), s & 1);
+                if (!kState && !wait_bar(bar(B_PC), ph, abort_flag, p.status, 12)) break;
+                if (s + 1 < ns) load_c(tile_of(s + 1));
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 && !kState) {
         // ================================================= MMA issuer 1
         // S, then X += P C, tile after tile: S of the next tile overwrites the
         // P this thread's previous MMAs read, and MMAs issued by one thread
@@ -219,7 +244,7 @@ la2_scan_ws(const __grid_constant__ Params p)
         if (lane == 0) {
             constexpr uint32_t kIdS = idesc_bf16_f32(128, kTB, 0, 0);
             constexpr uint32_t kIdX = idesc_bf16_f32(128, DC, 0, 1);
-            for (int s = 0; s < nb; ++s) {
+            for (int s = 0; s < ns; ++s) {
                 const uint32_t ph = s & 1;
                 const uint32_t sBs = sB + (s & 1) * L::kBsz;
                 if (!wait_bar(bar(FULL_A), ph, abort_flag, p.status, 20)) break;
@@ -249,29 +274,36 @@ la2_scan_ws(const __grid_constant__ Params p)
         }
     } else if (warp == 2) {
         // ================================================= MMA issuer 2
-        // X = A hi(W) + A lo(W) into X buffer s % 2, then dW
+        // X = A hi(W) + A lo(W) into X buffer s % 2 (not in the state pass), then dW
         if (lane == 0) {
             constexpr uint32_t kIdX = idesc_bf16_f32(128, DC, 0, 1);
             constexpr uint32_t kIdW = idesc_bf16_f32(DA, DC, 1, 1);
-            for (int s = 0; s < nb; ++s) {
+            for (int s = 0; s < ns; ++s) {
                 const uint32_t ph = s & 1;
                 const uint32_t sBs = sB + (s & 1) * L::kBsz;
-                // W of tile s is written (and dW of tile s-1 read) by the epilogue;
-                // X buffer s % 2 was read out after tile s-2
-                if (s > 0 && !wait_bar(bar(B_WR), ph ^ 1, abort_flag, p.status, 30)) break;
-                if (s > 1 && !wait_bar(bar(B_XF0 + (s & 1)), ((s - 2) >> 1) & 1, abort_flag, p.status, 33))
-                    break;
-                if (!wait_bar(bar(FULL_A), ph, abort_flag, p.status, 34)) break;
-                tc_fence_after();
-                const uint32_t xt = tX(s & 1);
+                // B_WR completes once when the epilogue has set the initial state
+                // (main pass) and once per tile when it has updated W and read dW
+                if (kState) {
+                    if (s > 0 && !wait_bar(bar(B_WR), ph ^ 1, abort_flag, p.status, 30)) break;
+                } else {
+                    if (!wait_bar(bar(B_WR), ph, abort_flag, p.status, 30)) break;
+                    // X buffer s % 2 was read out after tile s-2
+                    if (s > 1 &&
+                        !wait_bar(bar(B_XF0 + (s & 1)), ((s - 2) >> 1) & 1, abort_flag, p.status, 33))
+                        break;
+                    if (!wait_bar(bar(FULL_A), ph, abort_flag, p.status, 34)) break;
+                    tc_fence_after();
+                    const uint32_t xt = tX(s & 1);
 #pragma unroll 1
-                for (int k = 0; k < DA / 16; ++k) {
-                    const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                    const uint64_t adesc = sdesc_sw128(sA + off, 16, 1024);
-                    mma_bf16_ss(xt, adesc, sdesc_sw128(sW + k * 2048, DA * 128, 1024), kIdX, k > 0);
-                    mma_bf16_ss(xt, adesc, sdesc_sw128(sW + L::kWsz + k * 2048, DA * 128, 1024), kIdX, 1);
+                    for (int k = 0; k < DA / 16; ++k) {
+                        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+                        const uint64_t adesc = sdesc_sw128(sA + off, 16, 1024);
+                        mma_bf16_ss(xt, adesc, sdesc_sw128(sW + k * 2048, DA * 128, 1024), kIdX, k > 0);
+                        mma_bf16_ss(xt, adesc, sdesc_sw128(sW + L::kWsz + k * 2048, DA * 128, 1024),
+                                    kIdX, 1);
+                    }
+                    mma_commit(bar(B_X));
                 }
-                mma_commit(bar(B_X));
                 if (!wait_bar(bar(B_BS), ph, abort_flag, p.status, 31)) break;
                 if (!wait_bar(bar(FULL_C), ph, abort_flag, p.status, 32)) break;
                 tc_fence_after();
@@ -293,10 +325,15 @@ la2_scan_ws(const __grid_constant__ Params p)
         const int r = quad * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const float ws = dir > 0 ? pw[kTB - 1 - r] : pw[r];
-        for (int s = 0; s < nb; ++s) {
+        for (int s = 0; s < ns; ++s) {
             const uint32_t ph = s & 1;
-            if (!wait_bar(bar(B_S), ph, abort_flag, p.status, 40)) break;
+            if (kState) {  // no S in the state pass: B only has to have landed
+                if (!wait_bar(bar(FULL_B0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 42)) break;
+            } else {
+                if (!wait_bar(bar(B_S), ph, abort_flag, p.status, 40)) break;
+            }
             tc_fence_after();
+            if (!kState) {
             // P = decay-masked S, hi + lo bf16, over the 16 columns of S each
             // group of 16 came from: [hi (8 cols) | lo (8 cols)], the A-operand
             // layout of one K = 16 step.  Every group is loaded before it is
@@ -304,16 +341,16 @@ la2_scan_ws(const __grid_constant__ Params p)
             // columns that were not read first made the following TMEM-operand
             // MMAs about 10x slower.
 #pragma unroll 1
-            for (int g = part; g < kTB / 16; g += 2) {
+            for (int grp = part; grp < kTB / 16; grp += 2) {
                 const int lo_g = 2 * quad, hi_g = 2 * quad + 1;
-                const int kind = (g == lo_g || g == hi_g) ? 1 : ((dir > 0) == (g < lo_g) ? 2 : 0);
+                const int kind = (grp == lo_g || grp == hi_g) ? 1 : ((dir > 0) == (grp < lo_g) ? 2 : 0);
                 uint32_t pk[16];
                 float sv[16];
-                tmem_ld16(tS + lane_off + g * 16, sv);
+                tmem_ld16(tS + lane_off + grp * 16, sv);
                 if (kind == 2) {
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
-                        const int c0 = g * 16 + 2 * u;
+                        const int c0 = grp * 16 + 2 * u;
                         const float p0 = sv[2 * u] * pw[dir > 0 ? r - c0 : c0 - r];
                         const float p1 = sv[2 * u + 1] * pw[dir > 0 ? r - c0 - 1 : c0 + 1 - r];
                         split_pack2(p0, p1, pk[u], pk[8 + u]);
@@ -321,7 +358,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                 } else if (kind == 1) {
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
-                        const int c0 = g * 16 + 2 * u;
+                        const int c0 = grp * 16 + 2 * u;
                         const int lag0 = dir > 0 ? r - c0 : c0 - r;
                         const int lag1 = dir > 0 ? r - c0 - 1 : c0 + 1 - r;
                         const float p0 = lag0 >= 0 ? sv[2 * u] * pw[lag0 < 0 ? 0 : lag0] : 0.f;
@@ -332,11 +369,12 @@ la2_scan_ws(const __grid_constant__ Params p)
 #pragma unroll
                     for (int u = 0; u < 16; ++u) pk[u] = 0u;
                 }
-                tmem_st16(tS + lane_off + g * 16, pk);
+                tmem_st16(tS + lane_off + grp * 16, pk);
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(B_P));
+            }
             // row r of w_s B (S, which reads B unscaled, is done): hi in place,
             // lo into its own buffer once the previous tile's dW, its only
             // reader, is done.  Part p does the chunks of half p of the row.
@@ -368,100 +406,166 @@ la2_scan_ws(const __grid_constant__ Params p)
         const float lamTB = pw[kTB];
         const bool owns_w_row = (DA == 128) || (lane < 16);
         const int wrow = (DA == 128) ? r : quad * 16 + (lane & 15);
-        float* xg = R.x + static_cast<size_t>(bh) * T * DC;
-        const int grp = lane >> 3, j = lane & 7;
-        for (int s = 0; s < nb; ++s) {
-            const uint32_t ph = s & 1;
-            const int i = tile_of(s);
-            const uint32_t xt = tX(s & 1);
-            // X row r *= w_x(r)   (the inter-tile term, still alone in X)
-            if (!wait_bar(bar(B_X), ph, abort_flag, p.status, 50)) break;
-            tc_fence_after();
+        if (kState) {
+            // state pass: W (fp32) lives in the first X buffer's TMEM columns
+            const uint32_t tW = tX(0);
+            for (int s = 0; s < ns; ++s) {
+                const uint32_t ph = s & 1;
+                if (!wait_bar(bar(B_D), ph, abort_flag, p.status, 56)) break;
+                tc_fence_after();
 #pragma unroll 1
-            for (int k = 0; k < kCols / 16; ++k) {
-                float x[16];
-                const uint32_t col = c0 + k * 16;
-                tmem_ld16(xt + lane_off + col, x);
+                for (int k = 0; k < kCols / 16; ++k) {
+                    float d[16], w[16];
+                    const uint32_t col = c0 + k * 16;
+                    tmem_ld16(tD + lane_off + col, d);
+                    if (s == 0) {  // TMEM starts undefined: the first update is W = dW
 #pragma unroll
-                for (int u = 0; u < 16; ++u) x[u] *= wx;
-                tmem_st16f(xt + lane_off + col, x);
+                        for (int u = 0; u < 16; ++u) w[u] = d[u];
+                    } else {
+                        tmem_ld16(tW + lane_off + col, w);
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) w[u] = fmaf(lamTB, w[u], d[u]);
+                    }
+                    tmem_st16f(tW + lane_off + col, w);
+                    if (s == ns - 1 && owns_w_row) {
+                        float* dst = seg_slot(g) + static_cast<size_t>(wrow) * DC + col;
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            st_global_v4(dst + 4 * u, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(B_WR));
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(B_XS));
-            // W <- lambda^T_B W + dW.  The state is kept as its hi + lo bf16 pair
-            // (a 16-bit significand, ~2^-17 relative per update), which is also
-            // the next tile's MMA operand; X = A W of this tile, which read it,
-            // is done.
-            if (!wait_bar(bar(B_D), ph, abort_flag, p.status, 51)) break;
-            tc_fence_after();
+        } else {
+            // initial state of this segment, W_in(g) = f W_in(g-1) + S_{g-1} with
+            // f = lambda^(T_B n), as its hi/lo bf16 pair (zero for the first)
+            if (g > 0 && owns_w_row) {
+                const float f = static_cast<float>(
+                    exp2(static_cast<double>(kTB) * p.seg_tiles * log2(static_cast<double>(lam))));
 #pragma unroll 1
-            for (int k = 0; k < kCols / 16; ++k) {
-                float d[16];
-                const uint32_t col = c0 + k * 16;
-                tmem_ld16(tD + lane_off + col, d);
-                if (owns_w_row) {
+                for (int k = 0; k < kCols / 16; ++k) {
+                    const uint32_t col = c0 + k * 16;
+                    float w[16];
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) w[u] = 0.f;
+                    for (int gp = 0; gp < g; ++gp) {
+                        const float* src = seg_slot(gp) + static_cast<size_t>(wrow) * DC + col;
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) w[u] = fmaf(f, w[u], src[u]);
+                    }
                     const uint32_t grpo = (col >> 6) * (DA * 128);
                     const int q = (col & 63) >> 3;
-                    const uint32_t a0 = sW + grpo + sw128(wrow, q), a1 = sW + grpo + sw128(wrow, q + 1);
                     uint32_t h[8], l[8];
-                    ld_shared_v4(a0, h[0], h[1], h[2], h[3]);
-                    ld_shared_v4(a1, h[4], h[5], h[6], h[7]);
-                    ld_shared_v4(a0 + L::kWsz, l[0], l[1], l[2], l[3]);
-                    ld_shared_v4(a1 + L::kWsz, l[4], l[5], l[6], l[7]);
 #pragma unroll
-                    for (int z = 0; z < 8; ++z) {
-                        const float w0 = fmaf(lamTB, bf16lo_to_f32(h[z]) + bf16lo_to_f32(l[z]), d[2 * z]);
-                        const float w1 = fmaf(lamTB, bf16hi_to_f32(h[z]) + bf16hi_to_f32(l[z]), d[2 * z + 1]);
-                        split_pack2(w0, w1, h[z], l[z]);
-                    }
-                    st_shared_v4(a0, h[0], h[1], h[2], h[3]);
-                    st_shared_v4(a1, h[4], h[5], h[6], h[7]);
-                    st_shared_v4(a0 + L::kWsz, l[0], l[1], l[2], l[3]);
-                    st_shared_v4(a1 + L::kWsz, l[4], l[5], l[6], l[7]);
+                    for (int z = 0; z < 8; ++z) split_pack2(w[2 * z], w[2 * z + 1], h[z], l[z]);
+                    st_shared_v4(sW + grpo + sw128(wrow, q), h[0], h[1], h[2], h[3]);
+                    st_shared_v4(sW + grpo + sw128(wrow, q + 1), h[4], h[5], h[6], h[7]);
+                    st_shared_v4(sW + L::kWsz + grpo + sw128(wrow, q), l[0], l[1], l[2], l[3]);
+                    st_shared_v4(sW + L::kWsz + grpo + sw128(wrow, q + 1), l[4], l[5], l[6], l[7]);
                 }
             }
             fence_proxy_async_smem();
-            tc_fence_before();
             mbar_arrive(bar(B_WR));
-            // X of tile i, 32 columns at a time: TMEM -> registers, then an 8 x 8
-            // transpose of float4s among each group of 8 lanes (warp shuffles),
-            // after which every store instruction writes four whole 128-byte
-            // rows.  The X buffer is released once read.
-            if (!wait_bar(bar(B_PC), ph, abort_flag, p.status, 52)) break;
-            tc_fence_after();
+            float* xg = R.x + static_cast<size_t>(bh) * T * DC;
+            const int grp = lane >> 3, j = lane & 7;
+            for (int s = 0; s < ns; ++s) {
+                const uint32_t ph = s & 1;
+                const int i = tile_of(s);
+                const uint32_t xt = tX(s & 1);
+                // X row r *= w_x(r)   (the inter-tile term, still alone in X)
+                if (!wait_bar(bar(B_X), ph, abort_flag, p.status, 50)) break;
+                tc_fence_after();
 #pragma unroll 1
-            for (int b = 0; b < kCols / 32; ++b) {
-                float v[32];
-                tmem_ld16(xt + lane_off + c0 + 32 * b, *reinterpret_cast<float(*)[16]>(v));
-                tmem_ld16(xt + lane_off + c0 + 32 * b + 16, *reinterpret_cast<float(*)[16]>(v + 16));
-                if (b == kCols / 32 - 1) {
-                    tc_fence_before();
-                    mbar_arrive(bar(B_XF0 + (s & 1)));
+                for (int k = 0; k < kCols / 16; ++k) {
+                    float x[16];
+                    const uint32_t col = c0 + k * 16;
+                    tmem_ld16(xt + lane_off + col, x);
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) x[u] *= wx;
+                    tmem_st16f(xt + lane_off + col, x);
                 }
-                // lane j of a group holds chunk c (4 floats) of its row in v[4c..4c+3];
-                // afterwards it holds chunk j of row 8*grp + c in v[4c..4c+3]
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(B_XS));
+                // W <- lambda^T_B W + dW.  The state is kept as its hi + lo bf16
+                // pair (a 16-bit significand, ~2^-17 relative per update), which
+                // is also the next tile's MMA operand; X = A W of this tile, which
+                // read it, is done.
+                if (!wait_bar(bar(B_D), ph, abort_flag, p.status, 51)) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int k = 0; k < kCols / 16; ++k) {
+                    float d[16];
+                    const uint32_t col = c0 + k * 16;
+                    tmem_ld16(tD + lane_off + col, d);
+                    if (owns_w_row) {
+                        const uint32_t grpo = (col >> 6) * (DA * 128);
+                        const int q = (col & 63) >> 3;
+                        const uint32_t a0 = sW + grpo + sw128(wrow, q);
+                        const uint32_t a1 = sW + grpo + sw128(wrow, q + 1);
+                        uint32_t h[8], l[8];
+                        ld_shared_v4(a0, h[0], h[1], h[2], h[3]);
+                        ld_shared_v4(a1, h[4], h[5], h[6], h[7]);
+                        ld_shared_v4(a0 + L::kWsz, l[0], l[1], l[2], l[3]);
+                        ld_shared_v4(a1 + L::kWsz, l[4], l[5], l[6], l[7]);
 #pragma unroll
-                for (int st = 4; st >= 1; st >>= 1) {
-                    const bool up = (j & st) != 0;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        if (c & st) continue;
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float send = up ? v[4 * c + e] : v[4 * (c | st) + e];
-                            const float recv = __shfl_xor_sync(0xffffffffu, send, st);
-                            if (up) v[4 * c + e] = recv;
-                            else v[4 * (c | st) + e] = recv;
+                        for (int z = 0; z < 8; ++z) {
+                            const float w0 =
+                                fmaf(lamTB, bf16lo_to_f32(h[z]) + bf16lo_to_f32(l[z]), d[2 * z]);
+                            const float w1 =
+                                fmaf(lamTB, bf16hi_to_f32(h[z]) + bf16hi_to_f32(l[z]), d[2 * z + 1]);
+                            split_pack2(w0, w1, h[z], l[z]);
                         }
+                        st_shared_v4(a0, h[0], h[1], h[2], h[3]);
+                        st_shared_v4(a1, h[4], h[5], h[6], h[7]);
+                        st_shared_v4(a0 + L::kWsz, l[0], l[1], l[2], l[3]);
+                        st_shared_v4(a1 + L::kWsz, l[4], l[5], l[6], l[7]);
                     }
                 }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(bar(B_WR));
+                // X of tile i, 32 columns at a time: TMEM -> registers, then an
+                // 8 x 8 transpose of float4s among each group of 8 lanes (warp
+                // shuffles), after which every store instruction writes four whole
+                // 128-byte rows.  The X buffer is released once read.
+                if (!wait_bar(bar(B_PC), ph, abort_flag, p.status, 52)) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int b = 0; b < kCols / 32; ++b) {
+                    float v[32];
+                    tmem_ld16(xt + lane_off + c0 + 32 * b, *reinterpret_cast<float(*)[16]>(v));
+                    tmem_ld16(xt + lane_off + c0 + 32 * b + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+                    if (b == kCols / 32 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(bar(B_XF0 + (s & 1)));
+                    }
+                    // lane j of a group holds chunk c (4 floats) of its row in
+                    // v[4c..4c+3]; afterwards chunk j of row 8*grp + c
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const int row = i * kTB + quad * 32 + grp * 8 + c;
-                    if (row < T)
-                        st_global_v4(xg + static_cast<size_t>(row) * DC + c0 + 32 * b + 4 * j,
-                                     v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                    for (int st = 4; st >= 1; st >>= 1) {
+                        const bool up = (j & st) != 0;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            if (c & st) continue;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float send = up ? v[4 * c + e] : v[4 * (c | st) + e];
+                                const float recv = __shfl_xor_sync(0xffffffffu, send, st);
+                                if (up) v[4 * c + e] = recv;
+                                else v[4 * (c | st) + e] = recv;
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const int row = i * kTB + quad * 32 + grp * 8 + c;
+                        if (row < T)
+                            st_global_v4(xg + static_cast<size_t>(row) * DC + c0 + 32 * b + 4 * j,
+                                         v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                    }
                 }
             }
         }
@@ -469,7 +573,7 @@ la2_scan_ws(const __grid_constant__ Params p)
 
     // ---- tear-down: wait (bounded) until both issuers' MMAs are done, free TMEM
     __syncthreads();
-    if (tid == 32 && nb > 0) {
+    if (tid == 32 && ns > 0) {
         if (!mbar_wait(bar(B_FIN), 0)) atomicCAS(p.status, 0, 5 | (60 << 8));
     }
     tc_fence_before();

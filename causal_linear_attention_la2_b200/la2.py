@@ -126,8 +126,32 @@ def _stream_ptr(stream) -> int:
     return int(s.cuda_stream)
 
 
+_ws_cache: dict = {}
+
+
+def _workspace(nbytes: int, device, workspace=None):
+    """(pointer, size) of a device workspace of at least nbytes (256-byte aligned).
+
+    A caller-provided uint8 tensor is used as is; otherwise one buffer per
+    device is kept and grown on demand (torch's allocator, plumbing only).
+    """
+    if nbytes <= 0:
+        return 0, 0
+    if workspace is not None:
+        if not workspace.is_cuda or workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError(f"workspace must be a CUDA buffer of at least {nbytes} bytes")
+        return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    key = torch.device(device).index
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        _ws_cache[key] = buf
+    return buf.data_ptr(), buf.numel()
+
+
 def la2_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, decay: torch.Tensor,
-            out: torch.Tensor | None = None, block: int = 128, stream=None) -> torch.Tensor:
+            out: torch.Tensor | None = None, block: int = 128, stream=None,
+            workspace: torch.Tensor | None = None) -> torch.Tensor:
     """o[b,h,t] = sum_{s<=t} decay[h]^(t-s) (q[b,h,t] . k[b,h,s]) v[b,h,s], on q's device.
 
     q, k, v: bf16 or fp32; the output is always fp32."""
@@ -141,14 +165,16 @@ def la2_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, decay: torch.Tens
     if out is None:
         out = torch.empty((B, H, T, e), dtype=torch.float32, device=q.device)
     _check(out, "out", (B, H, T, e), torch.float32)
+    wp, wn = _workspace(la2_workspace_bytes(B, H, T, d, e, block, dt, 0), q.device, workspace)
     st = la2_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(), out.data_ptr(),
-                     B, H, T, d, e, block, dt, 0, 0, _stream_ptr(stream))
+                     B, H, T, d, e, block, dt, wp, wn, _stream_ptr(stream))
     if st != LA2_OK:
         raise LA2Error(st, "la2_fwd")
     return out
 
 
-def la2_bwd(q, k, v, decay, dout, dq=None, dk=None, dv=None, block: int = 128, stream=None):
+def la2_bwd(q, k, v, decay, dout, dq=None, dk=None, dv=None, block: int = 128, stream=None,
+            workspace: torch.Tensor | None = None):
     """(dq, dk, dv) of sum(dout * la2_fwd(q, k, v, decay)); decay is not differentiated."""
     B, H, T, d = q.shape
     e = v.shape[-1]
@@ -163,8 +189,9 @@ def la2_bwd(q, k, v, decay, dout, dq=None, dk=None, dv=None, block: int = 128, s
     dv = torch.empty((B, H, T, e), **f32) if dv is None else dv
     for t, n, shp in ((dq, "dq", (B, H, T, d)), (dk, "dk", (B, H, T, d)), (dv, "dv", (B, H, T, e))):
         _check(t, n, shp, torch.float32)
+    wp, wn = _workspace(la2_workspace_bytes(B, H, T, d, e, block, dt, 1), q.device, workspace)
     st = la2_bwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(), dout.data_ptr(),
-                     dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, T, d, e, block, dt, 0, 0,
+                     dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, T, d, e, block, dt, wp, wn,
                      _stream_ptr(stream))
     if st != LA2_OK:
         raise LA2Error(st, "la2_bwd")

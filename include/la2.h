@@ -73,10 +73,12 @@ typedef enum {
 
 /*
  * Bytes of device workspace la2_fwd (is_bwd = 0) or la2_bwd (is_bwd = 1) needs
- * for these sizes.  The value does not grow with T (the only state carried
- * along a sequence is the d x e matrix, held on chip).  0 means the call
- * accepts workspace = NULL.  Returns (size_t)-1 for arguments the call would
- * reject.
+ * for these sizes.  The state carried along a sequence (d x e) stays on chip;
+ * the workspace only holds, when there are too few sequences to fill the
+ * GPU's SMs, the fp32 end state of each segment a sequence is cut into (up to
+ * 32 segments per sequence, never more than 148 CTAs' worth in total).  The
+ * value does not depend on T.  0 means the call accepts workspace = NULL.
+ * Returns (size_t)-1 for arguments the call would reject.
  */
 size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block,
                            la2_dtype dtype, int is_bwd);
@@ -86,7 +88,9 @@ size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block,
  *
  * Supported: dtype F32 with 1 <= d, e <= 128 and any block; dtype BF16 with
  * d, e in {64, 128} and block = 128.  Anything else well-formed returns
- * LA2_ERR_UNSUPPORTED.  out must not alias an input.
+ * LA2_ERR_UNSUPPORTED.  out must not alias an input.  workspace: device
+ * memory, 256-byte aligned, of at least la2_workspace_bytes(..., 0) bytes
+ * (LA2_ERR_WORKSPACE otherwise), not used concurrently by another call.
  */
 la2_status la2_fwd(const void *q, const void *k, const void *v, const float *decay,
                    void *out, int B, int H, int T, int d, int e, int block,

@@ -110,3 +110,19 @@ def test_workspace_is_flat_in_T(lib):
              for T in (1, 1024, 65536, 1 << 20)}
     assert len(sizes) == 1
     assert la2.la2_workspace_bytes(1, 16, 1024, 128, 128, 100, la2.LA2_DTYPE_BF16, 0) == 2 ** 64 - 1
+
+
+def test_workspace_missing_or_small_is_reported(lib):
+    need = la2.la2_workspace_bytes(1, 2, 4096, 128, 128, 128, la2.LA2_DTYPE_BF16, 0)
+    assert need > 0  # two sequences: they are cut into segments
+    assert _fwd(T=4096) == la2.LA2_ERR_WORKSPACE
+    assert la2.la2_fwd_raw(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 4096, 128, 128, 128,
+                           la2.LA2_DTYPE_BF16, FAKE, need - 1) == la2.LA2_ERR_WORKSPACE
+    assert la2.la2_fwd_raw(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 4096, 128, 128, 128,
+                           la2.LA2_DTYPE_BF16, FAKE + 16, need) == la2.LA2_ERR_INVALID_ARG
+
+
+def test_no_workspace_when_the_grid_is_full(lib):
+    # 2 x 40 x 3 backward units >= 148 SMs: no segments, no workspace
+    assert la2.la2_workspace_bytes(2, 40, 6144, 128, 128, 128, la2.LA2_DTYPE_BF16, 1) == 0
+    assert la2.la2_workspace_bytes(1, 2, 512, 64, 64, 64, la2.LA2_DTYPE_F32, 1) == 0

@@ -98,6 +98,14 @@ def test_bf16_shapes_with_ragged_tails(la2mod, oracle_mod, T, d, e):
     _check(la2mod, oracle_mod, x, 128, TOL["bf16"])
 
 
+@pytest.mark.parametrize("T", [256, 300, 1000, 4000, 4100])
+@pytest.mark.parametrize("B,H,d,e", [(1, 1, 128, 128), (1, 2, 64, 64), (1, 3, 64, 128)])
+def test_bf16_segmented_sequences(la2mod, oracle_mod, B, H, T, d, e):
+    """Few sequences: each is cut into segments with a state pre-pass."""
+    x = I.make_inputs(B, H, T, d, e, "bf16", seed=T + H, decay="tnl")
+    _check(la2mod, oracle_mod, x, 128, TOL["bf16"])
+
+
 @pytest.mark.parametrize("decay", ["ones", "tiny", "tnl"])
 def test_bf16_decays(la2mod, oracle_mod, decay):
     x = I.make_inputs(1, 4, 777, 128, 128, "bf16", seed=3, decay=decay)
