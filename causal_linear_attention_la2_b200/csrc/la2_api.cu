@@ -377,3 +377,58 @@ la2_status la2_device_status(int* code, int reset) {
 int la2_last_launch_count(void) { return t_last_launches; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free forward: the segment states live in a fixed array that is
+// part of the library image on every GPU that loads it, instead of in a
+// caller-provided workspace.
+namespace {
+
+// Large enough for any forward call: the segment states of one call never
+// exceed 147 units of d x e fp32 (148 CTAs at most, and the last segment of
+// every sequence needs none), i.e. 147 * 128 * 128 * 4 bytes at d = e = 128.
+constexpr size_t kStaticScratchBytes = static_cast<size_t>(148) * 128 * 128 * 4;
+
+static __device__ __align__(256) unsigned char g_la2_static_scratch[kStaticScratchBytes];
+
+struct ScratchState {
+    std::once_flag once;
+    void* ptr = nullptr;
+    bool ok = false;
+};
+ScratchState g_scratch[kMaxDevices];
+
+// Device address of the scratch array on the current device.  The host-side
+// symbol is only a stand-in; the address must come from cudaGetSymbolAddress,
+// once per device, with that device current.
+void* static_scratch_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    ScratchState& s = g_scratch[dev];
+    std::call_once(s.once, [&s] {
+        void* ptr = nullptr;
+        s.ok = cudaGetSymbolAddress(&ptr, g_la2_static_scratch) == cudaSuccess;
+        s.ptr = ptr;
+    });
+    return s.ok ? s.ptr : nullptr;
+}
+
+}  // namespace
+
+extern "C" la2_status la2_fwd_noalloc(const void* q, const void* k, const void* v,
+                                      const float* decay, void* out, int B, int H, int T, int d,
+                                      int e, int block, la2_dtype dtype, la2_stream_t stream) {
+    t_last_launches = 0;
+    bool empty = false;
+    la2_status st = common_checks(B, H, T, d, e, block, dtype, &empty);
+    if (st != LA2_OK || empty) return st;
+    const size_t need = la2_workspace_bytes(B, H, T, d, e, block, dtype, 0);
+    if (need > kStaticScratchBytes) return LA2_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    if (need > 0) {
+        scratch = static_scratch_ptr();
+        if (!scratch) return LA2_ERR_CUDA;
+    }
+    return la2_fwd(q, k, v, decay, out, B, H, T, d, e, block, dtype, scratch,
+                   need > 0 ? kStaticScratchBytes : 0, stream);
+}

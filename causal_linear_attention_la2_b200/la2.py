@@ -27,7 +27,7 @@ LA2_DTYPE_BF16 = 1
 
 # Every entry point include/la2.h declares.
 EXPORTS = ("la2_workspace_bytes", "la2_fwd", "la2_bwd", "la2_status_str", "la2_device_status",
-           "la2_last_launch_count")
+           "la2_last_launch_count", "la2_fwd_noalloc")
 
 
 class LA2Error(RuntimeError):
@@ -61,6 +61,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la2_device_status.restype = i
     lib.la2_last_launch_count.argtypes = []
     lib.la2_last_launch_count.restype = i
+    lib.la2_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
+    lib.la2_fwd_noalloc.restype = i
     _lib = lib
     return lib
 
@@ -92,6 +94,11 @@ def la2_fwd_raw(q, k, v, decay, out, B, H, T, d, e, block, dtype, workspace=0, w
     """The C call with integer pointers; returns the status code."""
     return int(load().la2_fwd(q, k, v, decay, out, B, H, T, d, e, block, dtype, workspace,
                               ws_bytes, stream))
+
+
+def la2_fwd_noalloc_raw(q, k, v, decay, out, B, H, T, d, e, block, dtype, stream=0) -> int:
+    """The allocation-free forward (scratch built into the library); returns the status."""
+    return int(load().la2_fwd_noalloc(q, k, v, decay, out, B, H, T, d, e, block, dtype, stream))
 
 
 def la2_bwd_raw(q, k, v, decay, dout, dq, dk, dv, B, H, T, d, e, block, dtype, workspace=0,

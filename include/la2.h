@@ -127,6 +127,30 @@ la2_status la2_device_status(int *code, int reset);
  * on this host thread. */
 int la2_last_launch_count(void);
 
+/*
+ * la2_fwd without a workspace argument, for callers that cannot allocate
+ * device memory at call time: code running inside CUDA-graph capture, under a
+ * framework that owns every allocation, or in a context where cudaMalloc is
+ * not allowed.  (No counterpart in the paper; this is a deployment variant of
+ * la2_fwd.)  The inputs and the output are still the caller's; the scratch
+ * la2_fwd would take from the workspace (per-segment states, when few
+ * sequences are cut into segments) comes from an array built into the
+ * library: kStaticScratchBytes = 148 * 128 * 128 * 4 bytes (9.25 MiB), which
+ * every GPU that loads the library keeps until the process exits.  Every
+ * forward call fits in it; larger requirements would return
+ * LA2_ERR_WORKSPACE.  Nothing is allocated or freed.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call outside any stream
+ * capture.  All calls share the one array and it keeps whatever the last call
+ * left there (each call writes every value it later reads), so calls that
+ * overlap on the GPU -- on different streams, or concurrently from several
+ * threads -- race and must not be issued.  Results are those of la2_fwd.
+ */
+la2_status la2_fwd_noalloc(const void *q, const void *k, const void *v, const float *decay,
+                           void *out, int B, int H, int T, int d, int e, int block,
+                           la2_dtype dtype, la2_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
