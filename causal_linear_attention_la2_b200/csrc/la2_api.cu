@@ -43,12 +43,12 @@ EncodeTiledFn encode_fn() {
 
 template <int DA, int DC>
 bool set_ws_attrs() {
-    return cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC, false>,
+    return cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 la2::ws::Smem<DA, DC>::kBytes) == cudaSuccess &&
-           cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC, true>,
+           cudaFuncSetAttribute(la2::ws::la2_state_ws<DA, DC>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                la2::ws::Smem<DA, DC>::kBytes) == cudaSuccess;
+                                la2::ws::StateSmem<DA, DC>::kBytes) == cudaSuccess;
 }
 
 // Sequence segments for the bf16 kernel.  Each CTA takes one (sequence,
@@ -166,12 +166,12 @@ la2_status common_checks(int B, int H, int T, int d, int e, int block, la2_dtype
 
 template <int DA, int DC>
 void launch_ws(const la2::ws::Params& p, unsigned units, cudaStream_t stream) {
-    constexpr size_t smem = la2::ws::Smem<DA, DC>::kBytes;
     if (p.nseg > 1)
-        la2::ws::la2_scan_ws<DA, DC, true>
-            <<<units * static_cast<unsigned>(p.nseg - 1), la2::ws::kThreads, smem, stream>>>(p);
-    la2::ws::la2_scan_ws<DA, DC, false>
-        <<<units * static_cast<unsigned>(p.nseg), la2::ws::kThreads, smem, stream>>>(p);
+        la2::ws::la2_state_ws<DA, DC><<<units * static_cast<unsigned>(p.nseg - 1),
+                                        la2::ws::kStateThreads,
+                                        la2::ws::StateSmem<DA, DC>::kBytes, stream>>>(p);
+    la2::ws::la2_scan_ws<DA, DC><<<units * static_cast<unsigned>(p.nseg), la2::ws::kThreads,
+                                   la2::ws::Smem<DA, DC>::kBytes, stream>>>(p);
 }
 
 // Launches the warp-specialised kernel over `n` roles that share (DA, DC):

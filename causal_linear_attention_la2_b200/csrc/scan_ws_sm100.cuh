@@ -120,15 +120,11 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
 }
 
-// kState = false: the scan itself.  One CTA per (sequence, role, segment); a
-//   segment starts from the state the segments before it leave behind,
-//   W_in(g) = sum_{g' < g} lambda^(T_B n (g-1-g')) S_g' (n tiles per segment),
-//   read from seg_state.
-// kState = true: the state pre-pass.  One CTA per (sequence, role, segment
-//   but the last); it runs only the state recurrence of its segment from zero,
-//   W <- lambda^T_B W + (diag(w_s) B_i)^T C_i, and writes W (fp32) to
-//   seg_state.  Loads B and C only.
-template <int DA, int DC, bool kState>
+// The scan itself.  One CTA per (sequence, role, segment); a segment starts
+// from the state the segments before it leave behind,
+// W_in(g) = sum_{g' < g} lambda^(T_B n (g-1-g')) S_g' (n tiles per segment),
+// read from seg_state (written by la2_state_ws).
+template <int DA, int DC>
 __global__ void __launch_bounds__(kThreads, 1)
 la2_scan_ws(const __grid_constant__ Params p)
 {
@@ -147,7 +143,7 @@ la2_scan_ws(const __grid_constant__ Params p)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + L::kAbort);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int segs_in_grid = kState ? p.nseg - 1 : p.nseg;
+    const int segs_in_grid = p.nseg;
     const int g = blockIdx.x % segs_in_grid;
     const int unit = blockIdx.x / segs_in_grid;  // (sequence, role)
     const int role_id = unit % p.nroles;
@@ -173,8 +169,7 @@ la2_scan_ws(const __grid_constant__ Params p)
         tmem_relinquish();
     }
     if (tid == 0) {
-        const uint32_t counts[NBAR] = {1, 1, 1, 1, 1, 1, 1, 1, 256, 256, 256, 256, 256, 256,
-                                       kState ? 1u : 2u};
+        const uint32_t counts[NBAR] = {1, 1, 1, 1, 1, 1, 1, 1, 256, 256, 256, 256, 256, 256, 2};
         for (int b = 0; b < NBAR; ++b) mbar_init(bar(b), counts[b]);
         *abort_flag = 0;
         fence_mbar_init();
@@ -216,7 +211,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                 for (int g = 0; g < DC / 64; ++g)
                     tma_load_3d(sC + g * 16384, &R.tc, bar(FULL_C), g * 64, i * kTB, bh);
             };
-            if (!kState) load_a(tile_of(0));
+            load_a(tile_of(0));
             load_b(tile_of(0), 0);
             if (ns > 1) load_b(tile_of(1), 1);
             load_c(tile_of(0));
@@ -225,18 +220,16 @@ la2_scan_ws(const __grid_constant__ Params p)
                 // A is free once S and X = A W of tile s are done; B buffer s % 2 once
                 // dW of tile s is done; C once X += P C is done too.  Waiting in
                 // this order keeps every waiter within one phase of its barrier.
-                if (!kState) {
-                    if (!wait_bar(bar(B_S), ph, abort_flag, p.status, 13)) break;
-                    if (!wait_bar(bar(B_X), ph, abort_flag, p.status, 10)) break;
-                    if (s + 1 < ns) load_a(tile_of(s + 1));
-                }
+                if (!wait_bar(bar(B_S), ph, abort_flag, p.status, 13)) break;
+                if (!wait_bar(bar(B_X), ph, abort_flag, p.status, 10)) break;
+                if (s + 1 < ns) load_a(tile_of(s + 1));
                 if (!wait_bar(bar(B_D), ph, abort_flag, p.status, 11)) break;
                 if (s + 2 < ns) load_b(tile_of(s + 2), s & 1);
-                if (!kState && !wait_bar(bar(B_PC), ph, abort_flag, p.status, 12)) break;
+                if (!wait_bar(bar(B_PC), ph, abort_flag, p.status, 12)) break;
                 if (s + 1 < ns) load_c(tile_of(s + 1));
             }
         }
-    } else if (warp == 1 && !kState) {
+    } else if (warp == 1) {
         // ================================================= MMA issuer 1
         // S, then X += P C, tile after tile: S of the next tile overwrites the
         // P this thread's previous MMAs read, and MMAs issued by one thread
@@ -274,7 +267,7 @@ la2_scan_ws(const __grid_constant__ Params p)
         }
     } else if (warp == 2) {
         // ================================================= MMA issuer 2
-        // X = A hi(W) + A lo(W) into X buffer s % 2 (not in the state pass), then dW
+        // X = A hi(W) + A lo(W) into X buffer s % 2, then dW
         if (lane == 0) {
             constexpr uint32_t kIdX = idesc_bf16_f32(128, DC, 0, 1);
             constexpr uint32_t kIdW = idesc_bf16_f32(DA, DC, 1, 1);
@@ -282,10 +275,8 @@ la2_scan_ws(const __grid_constant__ Params p)
                 const uint32_t ph = s & 1;
                 const uint32_t sBs = sB + (s & 1) * L::kBsz;
                 // B_WR completes once when the epilogue has set the initial state
-                // (main pass) and once per tile when it has updated W and read dW
-                if (kState) {
-                    if (s > 0 && !wait_bar(bar(B_WR), ph ^ 1, abort_flag, p.status, 30)) break;
-                } else {
+                // and once per tile when it has updated W and read dW
+                {
                     if (!wait_bar(bar(B_WR), ph, abort_flag, p.status, 30)) break;
                     // X buffer s % 2 was read out after tile s-2
                     if (s > 1 &&
@@ -327,13 +318,9 @@ la2_scan_ws(const __grid_constant__ Params p)
         const float ws = dir > 0 ? pw[kTB - 1 - r] : pw[r];
         for (int s = 0; s < ns; ++s) {
             const uint32_t ph = s & 1;
-            if (kState) {  // no S in the state pass: B only has to have landed
-                if (!wait_bar(bar(FULL_B0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 42)) break;
-            } else {
-                if (!wait_bar(bar(B_S), ph, abort_flag, p.status, 40)) break;
-            }
+            if (!wait_bar(bar(B_S), ph, abort_flag, p.status, 40)) break;
             tc_fence_after();
-            if (!kState) {
+            {
             // P = decay-masked S, hi + lo bf16, over the 16 columns of S each
             // group of 16 came from: [hi (8 cols) | lo (8 cols)], the A-operand
             // layout of one K = 16 step.  Every group is loaded before it is
@@ -406,39 +393,7 @@ la2_scan_ws(const __grid_constant__ Params p)
         const float lamTB = pw[kTB];
         const bool owns_w_row = (DA == 128) || (lane < 16);
         const int wrow = (DA == 128) ? r : quad * 16 + (lane & 15);
-        if (kState) {
-            // state pass: W (fp32) lives in the first X buffer's TMEM columns
-            const uint32_t tW = tX(0);
-            for (int s = 0; s < ns; ++s) {
-                const uint32_t ph = s & 1;
-                if (!wait_bar(bar(B_D), ph, abort_flag, p.status, 56)) break;
-                tc_fence_after();
-#pragma unroll 1
-                for (int k = 0; k < kCols / 16; ++k) {
-                    float d[16], w[16];
-                    const uint32_t col = c0 + k * 16;
-                    tmem_ld16(tD + lane_off + col, d);
-                    if (s == 0) {  // TMEM starts undefined: the first update is W = dW
-#pragma unroll
-                        for (int u = 0; u < 16; ++u) w[u] = d[u];
-                    } else {
-                        tmem_ld16(tW + lane_off + col, w);
-#pragma unroll
-                        for (int u = 0; u < 16; ++u) w[u] = fmaf(lamTB, w[u], d[u]);
-                    }
-                    tmem_st16f(tW + lane_off + col, w);
-                    if (s == ns - 1 && owns_w_row) {
-                        float* dst = seg_slot(g) + static_cast<size_t>(wrow) * DC + col;
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            st_global_v4(dst + 4 * u, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-                    }
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar(B_WR));
-            }
-        } else {
+        {
             // initial state of this segment, W_in(g) = f W_in(g-1) + S_{g-1} with
             // f = lambda^(T_B n), as its hi/lo bf16 pair (zero for the first)
             if (g > 0 && owns_w_row) {
@@ -581,6 +536,192 @@ la2_scan_ws(const __grid_constant__ Params p)
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+
+// ---------------------------------------------------------------------------
+// State pre-pass for segmented sequences.  One CTA per (sequence, role,
+// segment but the last).  The state a segment of n tiles leaves behind when it
+// starts from zero is
+//
+//   S = sum_{s < n} lambda^(T_B (n-1-s)) (diag(w_s) B_s)^T C_s,
+//
+// so each tile's factor lambda^(T_B (n-1-s)) is folded into its row weights
+// and all tiles accumulate into one TMEM accumulator: no per-tile state
+// update, and B, lo(w B) and C are double-buffered.  S (fp32) goes to
+// seg_state.  Roles (12 warps): warp 0 TMA (B, C), warp 1 MMA, warps 4-11 the
+// weighted hi/lo split of B (two warps per TMEM lane quadrant, one per half
+// of a row's 16-byte chunks), then the write-out of S.
+constexpr int kStateThreads = 384;
+
+enum StateBar { SB_B0, SB_B1, SB_C0, SB_C1, SB_S0, SB_S1, SB_D0, SB_D1, SB_FIN, SB_N };
+
+template <int DA, int DC>
+struct StateSmem {
+    static constexpr uint32_t kBsz = kTB * DA * 2;
+    static constexpr uint32_t kCsz = kTB * DC * 2;
+    static constexpr uint32_t kB = 0;                     // B tiles (two), then hi(w B)
+    static constexpr uint32_t kBlo = kB + 2 * kBsz;       // lo(w B) (two)
+    static constexpr uint32_t kC = kBlo + 2 * kBsz;       // C tiles (two)
+    static constexpr uint32_t kBar = kC + 2 * kCsz;
+    static constexpr uint32_t kTmemSlot = kBar + SB_N * 8;
+    static constexpr uint32_t kAbort = kTmemSlot + 4;
+    static constexpr uint32_t kBytes = kAbort + 12;
+    static constexpr uint32_t kTmemCols = DC;             // the S accumulator
+};
+
+template <int DA, int DC>
+__global__ void __launch_bounds__(kStateThreads, 1)
+la2_state_ws(const __grid_constant__ Params p)
+{
+    using L = StateSmem<DA, DC>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t base = smem_u32(smem_raw);
+    if (base & 1023u) {
+        if (threadIdx.x == 0) atomicCAS(p.status, 0, 4);
+        return;
+    }
+    const uint32_t sB = base + L::kB, sBlo = base + L::kBlo, sC = base + L::kC;
+    auto bar = [&](int b) { return base + L::kBar + 8u * b; };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + L::kAbort);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int segs_in_grid = p.nseg - 1;
+    const int g = blockIdx.x % segs_in_grid;
+    const int unit = blockIdx.x / segs_in_grid;
+    const int role_id = unit % p.nroles;
+    const int bh = unit / p.nroles;
+    const Role& R = p.role[role_id];
+    const int dir = R.dir;
+    const int nb = (p.T + kTB - 1) / kTB;
+    const int s0 = g * p.seg_tiles;
+    const int ns = max(0, min(p.seg_tiles, nb - s0));
+    const double l2 = log2(static_cast<double>(p.decay[bh % p.H]));
+    auto tile_of = [&](int step) { return dir > 0 ? s0 + step : nb - 1 - (s0 + step); };
+
+    if (warp == 0) {
+        tmem_alloc(base + L::kTmemSlot, L::kTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        const uint32_t counts[SB_N] = {1, 1, 1, 1, 256, 256, 1, 1, 1};
+        for (int b = 0; b < SB_N; ++b) mbar_init(bar(b), counts[b]);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tD = *reinterpret_cast<volatile uint32_t*>(smem_raw + L::kTmemSlot);
+
+    if (warp == 0) {
+        // ================================================= TMA producer
+        if (lane == 0 && ns > 0) {
+            prefetch_tmap(&R.tb);
+            prefetch_tmap(&R.tc);
+            auto load = [&](int i, int slot) {
+                const uint32_t bb = bar(SB_B0 + slot), bc = bar(SB_C0 + slot);
+                mbar_arrive_expect_tx(bb, kTB * DA * 2);
+                for (int gg = 0; gg < DA / 64; ++gg)
+                    tma_load_3d(sB + slot * L::kBsz + gg * 16384, &R.tb, bb, gg * 64, i * kTB, bh);
+                mbar_arrive_expect_tx(bc, kTB * DC * 2);
+                for (int gg = 0; gg < DC / 64; ++gg)
+                    tma_load_3d(sC + slot * L::kCsz + gg * 16384, &R.tc, bc, gg * 64, i * kTB, bh);
+            };
+            load(tile_of(0), 0);
+            if (ns > 1) load(tile_of(1), 1);
+            for (int s = 0; s + 2 < ns; ++s) {
+                // buffers s % 2 are free once the MMAs of tile s are done
+                if (!wait_bar(bar(SB_D0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 70)) break;
+                load(tile_of(s + 2), s & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ================================================= MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdW = idesc_bf16_f32(DA, DC, 1, 1);
+            for (int s = 0; s < ns; ++s) {
+                const int slot = s & 1;
+                const uint32_t ph = (s >> 1) & 1;
+                if (!wait_bar(bar(SB_S0 + slot), ph, abort_flag, p.status, 71)) break;
+                if (!wait_bar(bar(SB_C0 + slot), ph, abort_flag, p.status, 72)) break;
+                tc_fence_after();
+                const uint32_t bh_ = sB + slot * L::kBsz, bl = sBlo + slot * L::kBsz;
+                const uint32_t cb = sC + slot * L::kCsz;
+#pragma unroll 1
+                for (int k = 0; k < kTB / 16; ++k) {
+                    const uint64_t cdesc = sdesc_sw128(cb + k * 2048, 16384, 1024);
+                    mma_bf16_ss(tD, sdesc_sw128(bh_ + k * 2048, 16384, 1024), cdesc, kIdW,
+                                (s > 0 || k > 0) ? 1u : 0u);
+                    mma_bf16_ss(tD, sdesc_sw128(bl + k * 2048, 16384, 1024), cdesc, kIdW, 1);
+                }
+                mma_commit(bar(SB_D0 + slot));
+            }
+            mma_commit(bar(SB_FIN));
+        }
+    } else if (warp >= 4) {
+        // ================================================= split group, then write-out
+        const int quad = warp & 3, part = (warp - 4) >> 2;
+        const int r = quad * 32 + lane;
+        for (int s = 0; s < ns; ++s) {
+            const int slot = s & 1;
+            const uint32_t ph = (s >> 1) & 1;
+            if (!wait_bar(bar(SB_B0 + slot), ph, abort_flag, p.status, 73)) break;
+            // lo(w B) buffer of this slot was read by the MMAs of tile s-2
+            if (s >= 2 && !wait_bar(bar(SB_D0 + slot), ph ^ 1, abort_flag, p.status, 74)) break;
+            // row weight lambda^(T_B (n-1-s)) w_s(r)
+            const int e = dir > 0 ? kTB * (ns - s) - 1 - r : kTB * (ns - 1 - s) + r;
+            const float wt = static_cast<float>(exp2(static_cast<double>(e) * l2));
+            const uint32_t bt = sB + slot * L::kBsz, bl = sBlo + slot * L::kBsz;
+#pragma unroll
+            for (int k = 0; k < DA / 16; ++k) {
+                const int chunk = part * (DA / 16) + k;
+                const uint32_t off = (chunk >> 3) * 16384 + sw128(r, chunk & 7);
+                uint32_t v[4], h[4], lo[4];
+                ld_shared_v4(bt + off, v[0], v[1], v[2], v[3]);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    split_pack2(bf16lo_to_f32(v[u]) * wt, bf16hi_to_f32(v[u]) * wt, h[u], lo[u]);
+                st_shared_v4(bt + off, h[0], h[1], h[2], h[3]);
+                st_shared_v4(bl + off, lo[0], lo[1], lo[2], lo[3]);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bar(SB_S0 + slot));
+        }
+        // S of this segment: TMEM -> seg_state (fp32, row-major DA x DC)
+        if (ns > 0 &&
+            wait_bar(bar(SB_D0 + ((ns - 1) & 1)), ((ns - 1) >> 1) & 1, abort_flag, p.status, 75)) {
+            tc_fence_after();
+            const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+            const bool owns_row = (DA == 128) || (lane < 16);
+            const int srow = (DA == 128) ? r : quad * 16 + (lane & 15);
+            float* dst0 = p.seg_state + (static_cast<size_t>(unit) * (p.nseg - 1) + g) * (DA * DC) +
+                          static_cast<size_t>(srow) * DC;
+#pragma unroll 1
+            for (int k = 0; k < DC / 32; ++k) {
+                const int col = part * (DC / 2) + k * 16;
+                float w[16];
+                tmem_ld16(tD + lane_off + col, w);
+                if (owns_row) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        st_global_v4(dst0 + col + 4 * u, w[4 * u], w[4 * u + 1], w[4 * u + 2],
+                                     w[4 * u + 3]);
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (tid == 32 && ns > 0) {
+        if (!mbar_wait(bar(SB_FIN), 0)) atomicCAS(p.status, 0, 5 | (76 << 8));
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tD, L::kTmemCols);
     }
 }
 
