@@ -361,7 +361,7 @@ def run_ours(args, w, world, rank, local):
         "dtype": w.dtype, "data": "synthetic", "config": workload_config(w, args),
         "tflops": tflops, "tc_frac": tflops / (tc * world), "tc_peak_tflops": tc,
         "fwd_ms": sum(fwd_ms) / len(fwd_ms), "bwd_ms": bwd_avg_ms,
-        "roofline": {"bound": "hbm", "kernel": "la2_scan_bf16_sm100 (la2_bwd launch)",
+        "roofline": {"bound": "hbm", "kernel": "la2_scan_ws (la2_bwd launch)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic,
                      "peak_kind": f"{pk_kind} hbm_gbs"},

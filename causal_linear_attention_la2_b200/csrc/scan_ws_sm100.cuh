@@ -320,48 +320,6 @@ la2_scan_ws(const __grid_constant__ Params p)
             const uint32_t ph = s & 1;
             if (!wait_bar(bar(B_S), ph, abort_flag, p.status, 40)) break;
             tc_fence_after();
-            {
-            // P = decay-masked S, hi + lo bf16, over the 16 columns of S each
-            // group of 16 came from: [hi (8 cols) | lo (8 cols)], the A-operand
-            // layout of one K = 16 step.  Every group is loaded before it is
-            // overwritten, also groups the mask zeroes entirely: storing over S
-            // columns that were not read first made the following TMEM-operand
-            // MMAs about 10x slower.
-#pragma unroll 1
-            for (int grp = part; grp < kTB / 16; grp += 2) {
-                const int lo_g = 2 * quad, hi_g = 2 * quad + 1;
-                const int kind = (grp == lo_g || grp == hi_g) ? 1 : ((dir > 0) == (grp < lo_g) ? 2 : 0);
-                uint32_t pk[16];
-                float sv[16];
-                tmem_ld16(tS + lane_off + grp * 16, sv);
-                if (kind == 2) {
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int c0 = grp * 16 + 2 * u;
-                        const float p0 = sv[2 * u] * pw[dir > 0 ? r - c0 : c0 - r];
-                        const float p1 = sv[2 * u + 1] * pw[dir > 0 ? r - c0 - 1 : c0 + 1 - r];
-                        split_pack2(p0, p1, pk[u], pk[8 + u]);
-                    }
-                } else if (kind == 1) {
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int c0 = grp * 16 + 2 * u;
-                        const int lag0 = dir > 0 ? r - c0 : c0 - r;
-                        const int lag1 = dir > 0 ? r - c0 - 1 : c0 + 1 - r;
-                        const float p0 = lag0 >= 0 ? sv[2 * u] * pw[lag0 < 0 ? 0 : lag0] : 0.f;
-                        const float p1 = lag1 >= 0 ? sv[2 * u + 1] * pw[lag1 < 0 ? 0 : lag1] : 0.f;
-                        split_pack2(p0, p1, pk[u], pk[8 + u]);
-                    }
-                } else {
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) pk[u] = 0u;
-                }
-                tmem_st16(tS + lane_off + grp * 16, pk);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(B_P));
-            }
             // row r of w_s B (S, which reads B unscaled, is done): hi in place,
             // lo into its own buffer once the previous tile's dW, its only
             // reader, is done.  Part p does the chunks of half p of the row.
@@ -381,6 +339,55 @@ la2_scan_ws(const __grid_constant__ Params p)
             }
             fence_proxy_async_smem();
             mbar_arrive(bar(B_BS));
+            {
+            // P = decay-masked S, hi + lo bf16, over the 16 columns of S each
+            // group of 16 came from: [hi (8 cols) | lo (8 cols)], the A-operand
+            // layout of one K = 16 step.  Every group is loaded before it is
+            // overwritten, also groups the mask zeroes entirely: storing over S
+            // columns that were not read first made the following TMEM-operand
+            // MMAs about 10x slower.
+            // Part p takes the 32-column pairs of groups {4k + 2p, 4k + 2p + 1},
+            // which splits the causal triangle's work about evenly.
+#pragma unroll 1
+            for (int pr = part; pr < kTB / 32; pr += 2) {
+                float sv[32];
+                tmem_ld32(tS + lane_off + pr * 32, sv);
+                uint32_t pk[32];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int grp = 2 * pr + h2;
+                    const int lo_g = 2 * quad, hi_g = 2 * quad + 1;
+                    const int kind = (grp == lo_g || grp == hi_g) ? 1 : ((dir > 0) == (grp < lo_g) ? 2 : 0);
+                    if (kind == 2) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int c0 = grp * 16 + 2 * u;
+                            const float p0 = sv[16 * h2 + 2 * u] * pw[dir > 0 ? r - c0 : c0 - r];
+                            const float p1 = sv[16 * h2 + 2 * u + 1] * pw[dir > 0 ? r - c0 - 1 : c0 + 1 - r];
+                            split_pack2(p0, p1, pk[16 * h2 + u], pk[16 * h2 + 8 + u]);
+                        }
+                    } else if (kind == 1) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int c0 = grp * 16 + 2 * u;
+                            const int lag0 = dir > 0 ? r - c0 : c0 - r;
+                            const int lag1 = dir > 0 ? r - c0 - 1 : c0 + 1 - r;
+                            const float p0 = lag0 >= 0 ? sv[16 * h2 + 2 * u] * pw[lag0 < 0 ? 0 : lag0] : 0.f;
+                            const float p1 =
+                                lag1 >= 0 ? sv[16 * h2 + 2 * u + 1] * pw[lag1 < 0 ? 0 : lag1] : 0.f;
+                            split_pack2(p0, p1, pk[16 * h2 + u], pk[16 * h2 + 8 + u]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) pk[16 * h2 + u] = 0u;
+                    }
+                }
+                tmem_st32u(tS + lane_off + pr * 32, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(B_P));
+            }
         }
     } else if (warp >= 12) {
         // ================================================= epilogue group
@@ -433,13 +440,13 @@ la2_scan_ws(const __grid_constant__ Params p)
                 if (!wait_bar(bar(B_X), ph, abort_flag, p.status, 50)) break;
                 tc_fence_after();
 #pragma unroll 1
-                for (int k = 0; k < kCols / 16; ++k) {
-                    float x[16];
-                    const uint32_t col = c0 + k * 16;
-                    tmem_ld16(xt + lane_off + col, x);
+                for (int k = 0; k < kCols / 32; ++k) {
+                    float x[32];
+                    const uint32_t col = c0 + k * 32;
+                    tmem_ld32(xt + lane_off + col, x);
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) x[u] *= wx;
-                    tmem_st16f(xt + lane_off + col, x);
+                    for (int u = 0; u < 32; ++u) x[u] *= wx;
+                    tmem_st32(xt + lane_off + col, x);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -451,32 +458,35 @@ la2_scan_ws(const __grid_constant__ Params p)
                 if (!wait_bar(bar(B_D), ph, abort_flag, p.status, 51)) break;
                 tc_fence_after();
 #pragma unroll 1
-                for (int k = 0; k < kCols / 16; ++k) {
-                    float d[16];
-                    const uint32_t col = c0 + k * 16;
-                    tmem_ld16(tD + lane_off + col, d);
+                for (int k = 0; k < kCols / 32; ++k) {
+                    float d[32];
+                    tmem_ld32(tD + lane_off + c0 + k * 32, d);
                     if (owns_w_row) {
-                        const uint32_t grpo = (col >> 6) * (DA * 128);
-                        const int q = (col & 63) >> 3;
-                        const uint32_t a0 = sW + grpo + sw128(wrow, q);
-                        const uint32_t a1 = sW + grpo + sw128(wrow, q + 1);
-                        uint32_t h[8], l[8];
-                        ld_shared_v4(a0, h[0], h[1], h[2], h[3]);
-                        ld_shared_v4(a1, h[4], h[5], h[6], h[7]);
-                        ld_shared_v4(a0 + L::kWsz, l[0], l[1], l[2], l[3]);
-                        ld_shared_v4(a1 + L::kWsz, l[4], l[5], l[6], l[7]);
 #pragma unroll
-                        for (int z = 0; z < 8; ++z) {
-                            const float w0 =
-                                fmaf(lamTB, bf16lo_to_f32(h[z]) + bf16lo_to_f32(l[z]), d[2 * z]);
-                            const float w1 =
-                                fmaf(lamTB, bf16hi_to_f32(h[z]) + bf16hi_to_f32(l[z]), d[2 * z + 1]);
-                            split_pack2(w0, w1, h[z], l[z]);
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const uint32_t col = c0 + k * 32 + hh * 16;
+                            const uint32_t grpo = (col >> 6) * (DA * 128);
+                            const int q = (col & 63) >> 3;
+                            const uint32_t a0 = sW + grpo + sw128(wrow, q);
+                            const uint32_t a1 = sW + grpo + sw128(wrow, q + 1);
+                            uint32_t h[8], l[8];
+                            ld_shared_v4(a0, h[0], h[1], h[2], h[3]);
+                            ld_shared_v4(a1, h[4], h[5], h[6], h[7]);
+                            ld_shared_v4(a0 + L::kWsz, l[0], l[1], l[2], l[3]);
+                            ld_shared_v4(a1 + L::kWsz, l[4], l[5], l[6], l[7]);
+#pragma unroll
+                            for (int z = 0; z < 8; ++z) {
+                                const float w0 = fmaf(lamTB, bf16lo_to_f32(h[z]) + bf16lo_to_f32(l[z]),
+                                                      d[16 * hh + 2 * z]);
+                                const float w1 = fmaf(lamTB, bf16hi_to_f32(h[z]) + bf16hi_to_f32(l[z]),
+                                                      d[16 * hh + 2 * z + 1]);
+                                split_pack2(w0, w1, h[z], l[z]);
+                            }
+                            st_shared_v4(a0, h[0], h[1], h[2], h[3]);
+                            st_shared_v4(a1, h[4], h[5], h[6], h[7]);
+                            st_shared_v4(a0 + L::kWsz, l[0], l[1], l[2], l[3]);
+                            st_shared_v4(a1 + L::kWsz, l[4], l[5], l[6], l[7]);
                         }
-                        st_shared_v4(a0, h[0], h[1], h[2], h[3]);
-                        st_shared_v4(a1, h[4], h[5], h[6], h[7]);
-                        st_shared_v4(a0 + L::kWsz, l[0], l[1], l[2], l[3]);
-                        st_shared_v4(a1 + L::kWsz, l[4], l[5], l[6], l[7]);
                     }
                 }
                 fence_proxy_async_smem();
@@ -491,8 +501,7 @@ la2_scan_ws(const __grid_constant__ Params p)
 #pragma unroll 1
                 for (int b = 0; b < kCols / 32; ++b) {
                     float v[32];
-                    tmem_ld16(xt + lane_off + c0 + 32 * b, *reinterpret_cast<float(*)[16]>(v));
-                    tmem_ld16(xt + lane_off + c0 + 32 * b + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+                    tmem_ld32(xt + lane_off + c0 + 32 * b, v);
                     if (b == kCols / 32 - 1) {
                         tc_fence_before();
                         mbar_arrive(bar(B_XF0 + (s & 1)));
