@@ -23,9 +23,12 @@
 //
 // Roles (20 warps):
 //   warp 0      TMA producer: A and C (one buffer each), B (two buffers)
-//   warp 1      MMA issuer 1: S, X += P C
+//   warp 3      MMA issuer 0: S (two TMEM buffers, so S of the next tile is
+//               formed while P C of this one is still pending)
+//   warp 1      MMA issuer 1: X += P C
 //   warp 2      MMA issuer 2: X = A hi(W) + A lo(W) (X double-buffered in
-//               TMEM), dW = hi(w_s B)^T C + lo(w_s B)^T C
+//               TMEM), dW = hi(w_s B)^T C + lo(w_s B)^T C (into the X buffer
+//               the next tile will use)
 //   warps 4-11  mask group (two warps per TMEM lane quadrant): P from S, then
 //               the hi/lo split of w_s B (hi in place, lo in its own buffer)
 //   warps 12-19 epilogue group (two warps per lane quadrant, one per half of
@@ -33,9 +36,8 @@
 //               memory as the hi/lo bf16 pair the next X MMA reads), X to global
 //               memory in fp32 (a warp-shuffle transpose makes every store a
 //               whole 128-byte row)
-// Tile i's epilogue overlaps tile i+1's loads, S and P; MMAs of different
-// accumulators are issued by different threads (one issuing thread sustains
-// about one MMA per 100 cycles at these shapes).
+// Tile i's epilogue overlaps tile i+1's loads, S and P; each issuer waits only
+// for the operands of its own MMAs, so no MMA queues behind an unrelated one.
 //
 // Every hand-off is an mbarrier; every wait is bounded (2 s) and a shared abort
 // flag stops all roles once one of them gives up, after which the kernel
@@ -69,8 +71,9 @@ struct Params {
 
 enum Bar {
     FULL_A, FULL_B0, FULL_B1, FULL_C,  // TMA loads landed
-    B_S, B_X, B_PC, B_D,               // MMA commits: S; X = A W; X += P C; dW
-    B_P, B_BS,                         // mask: P written, w_s B split
+    B_S0, B_S1, B_X0, B_X1, B_PC0, B_PC1, B_D,  // MMA commits: S (per S buffer); X = A W (per
+                                                // X buffer); X += P C (per S buffer); dW
+    B_P0, B_P1, B_BS,                    // mask: P written (per S buffer), w_s B split
     B_XS, B_WR, B_XF0, B_XF1,          // epilogue: X scaled; W updated (dW read); X buffer 0 / 1 read
     B_FIN, NBAR
 };
@@ -169,7 +172,8 @@ la2_scan_ws(const __grid_constant__ Params p)
         tmem_relinquish();
     }
     if (tid == 0) {
-        const uint32_t counts[NBAR] = {1, 1, 1, 1, 1, 1, 1, 1, 256, 256, 256, 256, 256, 256, 2};
+        const uint32_t counts[NBAR] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1,
+                                       256, 256, 256, 256, 256, 256, 256, 3};
         for (int b = 0; b < NBAR; ++b) mbar_init(bar(b), counts[b]);
         *abort_flag = 0;
         fence_mbar_init();
@@ -180,9 +184,11 @@ la2_scan_ws(const __grid_constant__ Params p)
     tc_fence_after();
 
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_raw + L::kTmemSlot);
-    // TMEM: S / P (128 columns), X in two buffers (DC each), dW (DC)
-    const uint32_t tS = tmem, tD = tmem + 128 + 2 * DC;
-    auto tX = [&](int b) { return tmem + 128 + static_cast<uint32_t>(b * DC); };
+    // TMEM: S / P in two buffers (128 columns each), X in two buffers (DC each).
+    // dW of tile s goes to the X buffer of tile s+1: X of tile s-1 has been read
+    // out of it, and X of tile s+1 is not issued before dW has been read.
+    auto tS = [&](int b) { return tmem + static_cast<uint32_t>(b * 128); };
+    auto tX = [&](int b) { return tmem + 256 + static_cast<uint32_t>(b * DC); };
     auto tile_of = [&](int step) { return dir > 0 ? s0 + step : nb - 1 - (s0 + step); };
     // fp32 state slot of segment gg of this (sequence, role)
     auto seg_slot = [&](int gg) {
@@ -220,54 +226,66 @@ la2_scan_ws(const __grid_constant__ Params p)
                 // A is free once S and X = A W of tile s are done; B buffer s % 2 once
                 // dW of tile s is done; C once X += P C is done too.  Waiting in
                 // this order keeps every waiter within one phase of its barrier.
-                if (!wait_bar(bar(B_S), ph, abort_flag, p.status, 13)) break;
-                if (!wait_bar(bar(B_X), ph, abort_flag, p.status, 10)) break;
+                if (!wait_bar(bar(B_S0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 13)) break;
+                if (!wait_bar(bar(B_X0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 10)) break;
                 if (s + 1 < ns) load_a(tile_of(s + 1));
                 if (!wait_bar(bar(B_D), ph, abort_flag, p.status, 11)) break;
                 if (s + 2 < ns) load_b(tile_of(s + 2), s & 1);
-                if (!wait_bar(bar(B_PC), ph, abort_flag, p.status, 12)) break;
+                if (!wait_bar(bar(B_PC0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 12)) break;
                 if (s + 1 < ns) load_c(tile_of(s + 1));
             }
         }
-    } else if (warp == 1) {
-        // ================================================= MMA issuer 1
-        // S, then X += P C, tile after tile: S of the next tile overwrites the
-        // P this thread's previous MMAs read, and MMAs issued by one thread
-        // execute in order.
+    } else if (warp == 3) {
+        // ================================================= MMA issuer 0
+        // S of tile s into S buffer s % 2, once X += P C of tile s-2, which read
+        // the P in that buffer, is done
         if (lane == 0) {
             constexpr uint32_t kIdS = idesc_bf16_f32(128, kTB, 0, 0);
-            constexpr uint32_t kIdX = idesc_bf16_f32(128, DC, 0, 1);
             for (int s = 0; s < ns; ++s) {
                 const uint32_t ph = s & 1;
                 const uint32_t sBs = sB + (s & 1) * L::kBsz;
                 if (!wait_bar(bar(FULL_A), ph, abort_flag, p.status, 20)) break;
                 if (!wait_bar(bar(FULL_B0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 21)) break;
+                if (s > 1 &&
+                    !wait_bar(bar(B_PC0 + (s & 1)), ((s - 2) >> 1) & 1, abort_flag, p.status, 22))
+                    break;
                 tc_fence_after();
+                const uint32_t st = tS(s & 1);
 #pragma unroll 1
                 for (int k = 0; k < DA / 16; ++k) {
                     const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                    mma_bf16_ss(tS, sdesc_sw128(sA + off, 16, 1024), sdesc_sw128(sBs + off, 16, 1024),
+                    mma_bf16_ss(st, sdesc_sw128(sA + off, 16, 1024), sdesc_sw128(sBs + off, 16, 1024),
                                 kIdS, k > 0);
                 }
-                mma_commit(bar(B_S));
-                if (!wait_bar(bar(B_P), ph, abort_flag, p.status, 23)) break;
+                mma_commit(bar(B_S0 + (s & 1)));
+            }
+            mma_commit(bar(B_FIN));
+        }
+    } else if (warp == 1) {
+        // ================================================= MMA issuer 1
+        // X += P C of tile s, P read from S buffer s % 2
+        if (lane == 0) {
+            constexpr uint32_t kIdX = idesc_bf16_f32(128, DC, 0, 1);
+            for (int s = 0; s < ns; ++s) {
+                const uint32_t ph = s & 1;
+                if (!wait_bar(bar(B_P0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 23)) break;
                 if (!wait_bar(bar(B_XS), ph, abort_flag, p.status, 24)) break;
                 if (!wait_bar(bar(FULL_C), ph, abort_flag, p.status, 25)) break;
                 tc_fence_after();
-                const uint32_t xt = tX(s & 1);
+                const uint32_t xt = tX(s & 1), st = tS(s & 1);
 #pragma unroll 1
                 for (int k = 0; k < kTB / 16; ++k) {
                     const uint64_t cdesc = sdesc_sw128(sC + k * 2048, 16384, 1024);
-                    mma_bf16_ts(xt, tS + k * 16, cdesc, kIdX, 1);
-                    mma_bf16_ts(xt, tS + k * 16 + 8, cdesc, kIdX, 1);
+                    mma_bf16_ts(xt, st + k * 16, cdesc, kIdX, 1);
+                    mma_bf16_ts(xt, st + k * 16 + 8, cdesc, kIdX, 1);
                 }
-                mma_commit(bar(B_PC));
+                mma_commit(bar(B_PC0 + (s & 1)));
             }
             mma_commit(bar(B_FIN));
         }
     } else if (warp == 2) {
         // ================================================= MMA issuer 2
-        // X = A hi(W) + A lo(W) into X buffer s % 2, then dW
+        // X = A hi(W) + A lo(W) into X buffer s % 2, then dW into X buffer (s+1) % 2
         if (lane == 0) {
             constexpr uint32_t kIdX = idesc_bf16_f32(128, DC, 0, 1);
             constexpr uint32_t kIdW = idesc_bf16_f32(DA, DC, 1, 1);
@@ -275,13 +293,10 @@ la2_scan_ws(const __grid_constant__ Params p)
                 const uint32_t ph = s & 1;
                 const uint32_t sBs = sB + (s & 1) * L::kBsz;
                 // B_WR completes once when the epilogue has set the initial state
-                // and once per tile when it has updated W and read dW
+                // and once per tile when it has updated W and read dW (which sat
+                // in X buffer s % 2)
                 {
                     if (!wait_bar(bar(B_WR), ph, abort_flag, p.status, 30)) break;
-                    // X buffer s % 2 was read out after tile s-2
-                    if (s > 1 &&
-                        !wait_bar(bar(B_XF0 + (s & 1)), ((s - 2) >> 1) & 1, abort_flag, p.status, 33))
-                        break;
                     if (!wait_bar(bar(FULL_A), ph, abort_flag, p.status, 34)) break;
                     tc_fence_after();
                     const uint32_t xt = tX(s & 1);
@@ -293,16 +308,21 @@ la2_scan_ws(const __grid_constant__ Params p)
                         mma_bf16_ss(xt, adesc, sdesc_sw128(sW + L::kWsz + k * 2048, DA * 128, 1024),
                                     kIdX, 1);
                     }
-                    mma_commit(bar(B_X));
+                    mma_commit(bar(B_X0 + (s & 1)));
                 }
                 if (!wait_bar(bar(B_BS), ph, abort_flag, p.status, 31)) break;
                 if (!wait_bar(bar(FULL_C), ph, abort_flag, p.status, 32)) break;
+                // X buffer (s+1) % 2 was read out after tile s-1
+                if (s > 0 &&
+                    !wait_bar(bar(B_XF0 + ((s + 1) & 1)), ((s - 1) >> 1) & 1, abort_flag, p.status, 33))
+                    break;
                 tc_fence_after();
+                const uint32_t dt = tX((s + 1) & 1);
 #pragma unroll 1
                 for (int k = 0; k < kTB / 16; ++k) {
                     const uint64_t cdesc = sdesc_sw128(sC + k * 2048, 16384, 1024);
-                    mma_bf16_ss(tD, sdesc_sw128(sBs + k * 2048, 16384, 1024), cdesc, kIdW, k > 0);
-                    mma_bf16_ss(tD, sdesc_sw128(sBlo + k * 2048, 16384, 1024), cdesc, kIdW, 1);
+                    mma_bf16_ss(dt, sdesc_sw128(sBs + k * 2048, 16384, 1024), cdesc, kIdW, k > 0);
+                    mma_bf16_ss(dt, sdesc_sw128(sBlo + k * 2048, 16384, 1024), cdesc, kIdW, 1);
                 }
                 mma_commit(bar(B_D));
             }
@@ -318,7 +338,8 @@ la2_scan_ws(const __grid_constant__ Params p)
         const float ws = dir > 0 ? pw[kTB - 1 - r] : pw[r];
         for (int s = 0; s < ns; ++s) {
             const uint32_t ph = s & 1;
-            if (!wait_bar(bar(B_S), ph, abort_flag, p.status, 40)) break;
+            if (!wait_bar(bar(B_S0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 40)) break;
+            const uint32_t st = tS(s & 1);
             tc_fence_after();
             // row r of w_s B (S, which reads B unscaled, is done): hi in place,
             // lo into its own buffer once the previous tile's dW, its only
@@ -351,7 +372,7 @@ la2_scan_ws(const __grid_constant__ Params p)
 #pragma unroll 1
             for (int pr = part; pr < kTB / 32; pr += 2) {
                 float sv[32];
-                tmem_ld32(tS + lane_off + pr * 32, sv);
+                tmem_ld32(st + lane_off + pr * 32, sv);
                 uint32_t pk[32];
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
@@ -382,11 +403,11 @@ la2_scan_ws(const __grid_constant__ Params p)
                         for (int u = 0; u < 16; ++u) pk[16 * h2 + u] = 0u;
                     }
                 }
-                tmem_st32u(tS + lane_off + pr * 32, pk);
+                tmem_st32u(st + lane_off + pr * 32, pk);
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(B_P));
+            mbar_arrive(bar(B_P0 + (s & 1)));
             }
         }
     } else if (warp >= 12) {
@@ -437,7 +458,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                 const int i = tile_of(s);
                 const uint32_t xt = tX(s & 1);
                 // X row r *= w_x(r)   (the inter-tile term, still alone in X)
-                if (!wait_bar(bar(B_X), ph, abort_flag, p.status, 50)) break;
+                if (!wait_bar(bar(B_X0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 50)) break;
                 tc_fence_after();
 #pragma unroll 1
                 for (int k = 0; k < kCols / 32; ++k) {
@@ -460,7 +481,7 @@ la2_scan_ws(const __grid_constant__ Params p)
 #pragma unroll 1
                 for (int k = 0; k < kCols / 32; ++k) {
                     float d[32];
-                    tmem_ld32(tD + lane_off + c0 + k * 32, d);
+                    tmem_ld32(tX((s + 1) & 1) + lane_off + c0 + k * 32, d);
                     if (owns_w_row) {
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
@@ -496,7 +517,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                 // 8 x 8 transpose of float4s among each group of 8 lanes (warp
                 // shuffles), after which every store instruction writes four whole
                 // 128-byte rows.  The X buffer is released once read.
-                if (!wait_bar(bar(B_PC), ph, abort_flag, p.status, 52)) break;
+                if (!wait_bar(bar(B_PC0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 52)) break;
                 tc_fence_after();
 #pragma unroll 1
                 for (int b = 0; b < kCols / 32; ++b) {
