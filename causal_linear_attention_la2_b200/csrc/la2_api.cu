@@ -376,6 +376,20 @@ la2_status la2_device_status(int* code, int reset) {
 
 int la2_last_launch_count(void) { return t_last_launches; }
 
+#ifdef LA2_TRACE
+// Debug builds only: copies (and clears) the timeline trace of la2_scan_ws.
+int la2_trace_read(void* host, size_t bytes) {
+    constexpr size_t kTraceBytes = sizeof(unsigned long long) * 2 * la2::ws::kTraceEv *
+                                   la2::ws::kTraceSteps;
+    static unsigned long long zero[kTraceBytes / 8];
+    if (bytes > kTraceBytes) bytes = kTraceBytes;
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+    if (cudaMemcpyFromSymbol(host, la2::ws::g_la2_trace, bytes) != cudaSuccess) return -1;
+    if (cudaMemcpyToSymbol(la2::ws::g_la2_trace, zero, kTraceBytes) != cudaSuccess) return -1;
+    return static_cast<int>(bytes);
+}
+#endif
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------

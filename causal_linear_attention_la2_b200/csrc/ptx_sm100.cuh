@@ -43,6 +43,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe: true once the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
 // try_wait with a suspend-time hint (ns): the thread sleeps at most that long
 // inside the instruction before it reports "not yet".
 __device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t ns) {
@@ -149,6 +160,12 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
     d |= static_cast<uint64_t>(2) << 61;  // 128-byte swizzle
     return d;
+}
+
+// The same descriptor with its start address moved by `bytes` (a multiple of
+// 16; shared-memory addresses fit the 14-bit field, so no carry leaves it).
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
+    return desc + static_cast<uint64_t>(bytes >> 4);
 }
 
 // Instruction descriptor for kind::f16 with bf16 A and B and fp32 accumulation.
@@ -335,5 +352,68 @@ __device__ __forceinline__ void st_global_v4(void* p, float a, float b, float c,
 
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
+
+}  // namespace la2
+
+namespace la2 {
+
+// Two 16x256b.x4 TMEM loads (lane bases of taddr0 and taddr1, 32 consecutive
+// columns each) and the wait for both, in one asm statement.  Register layout
+// of each load (per warp, 16 lanes x 32 columns): thread t holds, for column
+// group j = 0..3, v[4j], v[4j+1] = lane t/4, columns 8j + 2(t%4) + {0, 1}, and
+// v[4j+2], v[4j+3] = lane t/4 + 8, the same columns.
+__device__ __forceinline__ void tmem_ld16x256b_x4_pair(uint32_t taddr0, uint32_t taddr1,
+                                                       float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+          "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+          "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]),
+          "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+          "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr0), "r"(taddr1) : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void st_global_v2(void* p, float a, float b) {
+    asm volatile("st.global.v2.f32 [%0], {%1, %2};" :: "l"(p), "f"(a), "f"(b) : "memory");
+}
+
+// Packed pair arithmetic (sm_100 f32x2): (a0, a1) * (b0, b1), elementwise,
+// round to nearest.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    uint64_t x, y, z;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(b.x), "f"(b.y));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(z));
+    return r;
+}
+
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    uint64_t x, y, z;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(b.x), "f"(b.y));
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(z));
+    return r;
+}
+
+// split_pack2 on a pair, with the residual formed by one packed subtraction.
+__device__ __forceinline__ void split_pack2v(float2 x, uint32_t& hi, uint32_t& lo) {
+    hi = pack_bf16x2(x.x, x.y);
+    const float2 h = make_float2(__uint_as_float(hi << 16), __uint_as_float(hi & 0xFFFF0000u));
+    const float2 d = sub2(x, h);
+    lo = pack_bf16x2(d.x, d.y);
+}
 
 }  // namespace la2

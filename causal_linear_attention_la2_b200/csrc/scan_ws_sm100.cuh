@@ -22,26 +22,36 @@
 // w_x = lambda^(T_B-r), w_s = lambda^r for dir = -1.
 //
 // Roles (20 warps):
-//   warp 0      TMA producer: A and C (one buffer each), B (two buffers)
-//   warp 3      MMA issuer 0: S (two TMEM buffers, so S of the next tile is
-//               formed while P C of this one is still pending)
-//   warp 1      MMA issuer 1: X += P C
-//   warp 2      MMA issuer 2: X = A hi(W) + A lo(W) (X double-buffered in
-//               TMEM), dW = hi(w_s B)^T C + lo(w_s B)^T C (into the X buffer
-//               the next tile will use)
-//   warps 4-11  mask group (two warps per TMEM lane quadrant): P from S, then
-//               the hi/lo split of w_s B (hi in place, lo in its own buffer)
+//   warp 0      TMA producer and MMA issuer S, one polling loop: A, B and C
+//               each in a ring of buffers (whichever ring has a free buffer is
+//               refilled first), S = A B^T into S buffer s % 2
+//   warp 1      MMA issuer PC: X += hi(P) C + lo(P) C, P read from S buffer
+//               s % 2 as the TMEM A operand
+//   warp 2      MMA issuer XW: X = A hi(W) + A lo(W) into X buffer s % 2
+//   warp 3      MMA issuer dW: dW = hi(w_s B)^T C + lo(w_s B)^T C
+//   warps 4-11  mask group (two warps per TMEM lane quadrant): the hi/lo
+//               split of w_s B (hi in place, lo in its own ring), then P from S
 //   warps 12-19 epilogue group (two warps per lane quadrant, one per half of
 //               the columns): X = w_x X, the W update (W lives in shared
 //               memory as the hi/lo bf16 pair the next X MMA reads), X to global
 //               memory in fp32 (a warp-shuffle transpose makes every store a
 //               whole 128-byte row)
-// Tile i's epilogue overlaps tile i+1's loads, S and P; each issuer waits only
-// for the operands of its own MMAs, so no MMA queues behind an unrelated one.
+// A thread can issue one tcgen05.mma about every 126 cycles whatever its
+// shape (measured on B200), while one M = 128, N = 128 MMA keeps the tensor
+// pipe busy for 64; so the MMAs of a tile are spread over four issuing
+// threads, each issuing fully unrolled with precomputed descriptors.
+// How many buffers each operand gets depends on (DA, DC) (RingCfg): at
+// DA = DC = 64 every operand has two or three, so the only serial dependency
+// left between tiles is the state update itself; at DA = DC = 128 shared
+// memory holds one A, C and W buffer and two B buffers.  With DC = 64, dW has
+// two TMEM buffers of its own; otherwise it borrows the X buffer of the next
+// tile.
 //
-// Every hand-off is an mbarrier; every wait is bounded (2 s) and a shared abort
-// flag stops all roles once one of them gives up, after which the kernel
-// waits (bounded) for its own MMAs, frees TMEM and returns.
+// Every hand-off is an mbarrier: each buffer has a "full" barrier its
+// producer completes and an "empty" barrier its consumers complete, so a
+// waiter is never more than one phase behind.  Every wait is bounded (2 s) and
+// a shared abort flag stops all roles once one of them gives up, after which
+// the kernel waits (bounded) for its own MMAs, frees TMEM and returns.
 #pragma once
 #include "ptx_sm100.cuh"
 
@@ -69,32 +79,66 @@ struct Params {
     int seg_tiles;       // tiles per segment (the last may be shorter)
 };
 
-enum Bar {
-    FULL_A, FULL_B0, FULL_B1, FULL_C,  // TMA loads landed
-    B_S0, B_S1, B_X0, B_X1, B_PC0, B_PC1, B_D,  // MMA commits: S (per S buffer); X = A W (per
-                                                // X buffer); X += P C (per S buffer); dW
-    B_P0, B_P1, B_BS,                    // mask: P written (per S buffer), w_s B split
-    B_XS, B_WR, B_XF0, B_XF1,          // epilogue: X scaled; W updated (dW read); X buffer 0 / 1 read
-    B_FIN, NBAR
+// Buffer counts and mbarrier indices of the scan kernel for (DA, DC).
+template <int DA, int DC>
+struct RingCfg {
+    static constexpr bool kSmall = DA == 64 && DC == 64;
+    static constexpr bool kBig = DA == 128 && DC == 128;
+    static constexpr int NA = kSmall ? 3 : (kBig ? 1 : 2);  // A tiles
+    static constexpr int NB = kSmall ? 3 : 2;               // B tiles (then hi(w_s B))
+    static constexpr int NC = kSmall ? 3 : (kBig ? 1 : 2);  // C tiles
+    static constexpr int NBLO = DA == 64 ? 2 : 1;           // lo(w_s B)
+    static constexpr int NW = DA == 64 ? 2 : 1;             // W as its hi/lo pair
+    static constexpr bool kOwnD = DC == 64;                 // dW in TMEM buffers of its own
+    static constexpr int ND = kOwnD ? 2 : 1;
+    // "full": the producer has filled the buffer; "empty": its consumers are done
+    static constexpr int FULL_A = 0, EMPTY_A = FULL_A + NA;
+    static constexpr int FULL_B = EMPTY_A + NA, EMPTY_B = FULL_B + NB, BS = EMPTY_B + NB;
+    static constexpr int FULL_C = BS + NB, EMPTY_C = FULL_C + NC;
+    static constexpr int EMPTY_BLO = EMPTY_C + NC;
+    static constexpr int S_DONE = EMPTY_BLO + NBLO, EMPTY_S = S_DONE + 2, P_READY = EMPTY_S + 2;
+    static constexpr int XW_DONE = P_READY + 2, XS = XW_DONE + 2, PC_DONE = XS + 2;
+    static constexpr int EMPTY_X = PC_DONE + 2;
+    static constexpr int D_DONE = EMPTY_X + 2, EMPTY_D = D_DONE + ND;
+    static constexpr int W_READY = EMPTY_D + ND, EMPTY_W = W_READY + NW;
+    static constexpr int FIN = EMPTY_W + NW, NBARS = FIN + 1;
+
+    // arrivals that complete one phase of barrier b
+    static __device__ __forceinline__ uint32_t count(int b) {
+        if (b >= EMPTY_A && b < EMPTY_A + NA) return 2;   // S and XW commits
+        if (b >= EMPTY_C && b < EMPTY_C + NC) return 2;   // PC and dW commits
+        if (b >= BS && b < BS + NB) return 256;           // mask group
+        if (b >= P_READY && b < P_READY + 2) return 256;  // mask group
+        if (b >= XS && b < XS + 2) return 256;            // epilogue group
+        if (b >= EMPTY_X && b < EMPTY_X + 2) return 256;  // epilogue group
+        if (b >= EMPTY_D && b < EMPTY_D + ND) return 256; // epilogue group
+        if (b >= W_READY && b < W_READY + NW) return 256; // epilogue group
+        if (b == FIN) return 4;                           // the four issuers
+        return 1;                                         // TMA or one commit
+    }
 };
 
 template <int DA, int DC>
 struct Smem {
-    static constexpr uint32_t kA = 0;                        // A tile (T_B x DA)
-    static constexpr uint32_t kBsz = kTB * DA * 2;
-    static constexpr uint32_t kB = kA + kBsz;                // B tiles, two buffers, each then hi(w_s B)
-    static constexpr uint32_t kBlo = kB + 2 * kBsz;          // lo(w_s B)
-    static constexpr uint32_t kC = kBlo + kBsz;              // C tile (T_B x DC)
-    static constexpr uint32_t kWsz = DA * DC * 2;
-    static constexpr uint32_t kW = kC + kTB * DC * 2;        // hi(W), then lo(W) (DA x DC each)
-    static constexpr uint32_t kPow = kW + 2 * kWsz;          // lambda^n, n = 0..T_B
-    static constexpr uint32_t kBar = kPow + 528;
-    static constexpr uint32_t kTmemSlot = kBar + NBAR * 8;
+    using Q = RingCfg<DA, DC>;
+    static constexpr uint32_t kAsz = kTB * DA * 2;            // one A (or B) tile
+    static constexpr uint32_t kBsz = kAsz;
+    static constexpr uint32_t kCsz = kTB * DC * 2;            // one C tile
+    static constexpr uint32_t kWsz = DA * DC * 2;             // hi(W) or lo(W)
+    static constexpr uint32_t kA = 0;                         // A ring
+    static constexpr uint32_t kB = kA + Q::NA * kAsz;         // B ring, each then hi(w_s B)
+    static constexpr uint32_t kBlo = kB + Q::NB * kBsz;       // lo(w_s B) ring
+    static constexpr uint32_t kC = kBlo + Q::NBLO * kBsz;     // C ring
+    static constexpr uint32_t kW = kC + Q::NC * kCsz;         // W buffer i: hi, then lo
+    static constexpr uint32_t kPow = kW + Q::NW * 2 * kWsz;   // lambda^n, n = 0..T_B
+    static constexpr uint32_t kMuRev = kPow + 528;            // lambda^(15-n), n = 0..15
+    static constexpr uint32_t kBar = kMuRev + 64;
+    static constexpr uint32_t kTmemSlot = kBar + Q::NBARS * 8;
     static constexpr uint32_t kAbort = kTmemSlot + 4;
-    static constexpr uint32_t kEnd = kAbort + 12;
-    // Small tiles are padded so that only one CTA fits on an SM (it allocates
-    // all 512 TMEM columns).
-    static constexpr uint32_t kBytes = kEnd > 120 * 1024 ? kEnd : 120 * 1024;
+    static constexpr uint32_t kBytes = kAbort + 12;
+    static_assert(kBytes <= 232448, "shared memory over the 227 KB per-CTA limit");
+    // one CTA per SM: it allocates all 512 TMEM columns
+    static_assert(kBytes > 116 * 1024, "two CTAs would fit on an SM");
 };
 
 // Byte offset of the 16-byte chunk q (0..7) of row r inside a 128-byte
@@ -102,6 +146,21 @@ struct Smem {
 __device__ __forceinline__ uint32_t sw128(int r, int q) {
     return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((q ^ (r & 7)) << 4));
 }
+
+#ifdef LA2_TRACE
+// Timeline trace, compiled only with -DLA2_TRACE (never in the library build):
+// clock64() at fixed points of each role, per step, for two CTAs (the first
+// and the middle one of the grid), read back with la2_trace_read().
+constexpr int kTraceEv = 32, kTraceSteps = 64;
+__device__ unsigned long long g_la2_trace[2][kTraceEv][kTraceSteps];
+#define LA2_TR(ev, s)                                                                   \
+    do {                                                                                \
+        const int c_ = blockIdx.x == 0 ? 0 : (blockIdx.x == gridDim.x / 2 ? 1 : -1);   \
+        if (c_ >= 0 && (s) >= 0 && (s) < kTraceSteps) g_la2_trace[c_][ev][s] = clock64(); \
+    } while (0)
+#else
+#define LA2_TR(ev, s) ((void)0)
+#endif
 
 // Bounded wait that also gives up as soon as another role has aborted.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
@@ -123,6 +182,13 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
 }
 
+// Phase parity of the barrier of a ring of n buffers that step s waits for:
+// full_par, the fill for step s; empty_par (s >= n), the release by step s - n.
+__device__ __forceinline__ uint32_t full_par(int s, int n) { return static_cast<uint32_t>((s / n) & 1); }
+__device__ __forceinline__ uint32_t empty_par(int s, int n) {
+    return static_cast<uint32_t>(((s / n) + 1) & 1);
+}
+
 // The scan itself.  One CTA per (sequence, role, segment); a segment starts
 // from the state the segments before it leave behind,
 // W_in(g) = sum_{g' < g} lambda^(T_B n (g-1-g')) S_g' (n tiles per segment),
@@ -133,6 +199,7 @@ la2_scan_ws(const __grid_constant__ Params p)
 {
     static_assert((DA == 64 || DA == 128) && (DC == 64 || DC == 128), "DA, DC in {64, 128}");
     using L = Smem<DA, DC>;
+    using Q = RingCfg<DA, DC>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t base = smem_u32(smem_raw);
     if (base & 1023u) {  // 128-byte swizzled tiles need a 1024-byte aligned base
@@ -142,6 +209,7 @@ la2_scan_ws(const __grid_constant__ Params p)
     const uint32_t sA = base + L::kA, sB = base + L::kB, sBlo = base + L::kBlo;
     const uint32_t sC = base + L::kC, sW = base + L::kW;
     float* pw = reinterpret_cast<float*>(smem_raw + L::kPow);
+    float* murev = reinterpret_cast<float*>(smem_raw + L::kMuRev);
     auto bar = [&](int b) { return base + L::kBar + 8u * b; };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + L::kAbort);
 
@@ -160,10 +228,12 @@ la2_scan_ws(const __grid_constant__ Params p)
     const int ns = max(0, min(p.seg_tiles, nb - s0));
     const float lam = p.decay[bh % p.H];
 
-    // ---- set-up
+    if (tid == 0) LA2_TR(0, 0);
+    // ---- set-up: lambda^n table, W buffer 0 = 0, TMEM, barriers
     {
         const double l2 = log2(static_cast<double>(lam));
         for (int n = tid; n <= kTB; n += kThreads) pw[n] = static_cast<float>(exp2(n * l2));
+        if (tid < 16) murev[tid] = static_cast<float>(exp2((15 - tid) * l2));
         for (uint32_t off = tid * 16; off < 2 * L::kWsz; off += kThreads * 16)
             st_shared_v4(sW + off, 0u, 0u, 0u, 0u);
     }
@@ -172,9 +242,7 @@ la2_scan_ws(const __grid_constant__ Params p)
         tmem_relinquish();
     }
     if (tid == 0) {
-        const uint32_t counts[NBAR] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1,
-                                       256, 256, 256, 256, 256, 256, 256, 3};
-        for (int b = 0; b < NBAR; ++b) mbar_init(bar(b), counts[b]);
+        for (int b = 0; b < Q::NBARS; ++b) mbar_init(bar(b), Q::count(b));
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -183,12 +251,17 @@ la2_scan_ws(const __grid_constant__ Params p)
     __syncthreads();
     tc_fence_after();
 
+    if (tid == 0) LA2_TR(1, 0);
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_raw + L::kTmemSlot);
-    // TMEM: S / P in two buffers (128 columns each), X in two buffers (DC each).
-    // dW of tile s goes to the X buffer of tile s+1: X of tile s-1 has been read
-    // out of it, and X of tile s+1 is not issued before dW has been read.
+    // TMEM: S / P in two buffers (128 columns each), X in two buffers (DC each),
+    // then (DC = 64) two dW buffers; otherwise dW of tile s goes to the X buffer
+    // of tile s+1: X of tile s-1 has been read out of it, and X of tile s+1 is
+    // not issued before the state update has read dW.
     auto tS = [&](int b) { return tmem + static_cast<uint32_t>(b * 128); };
     auto tX = [&](int b) { return tmem + 256 + static_cast<uint32_t>(b * DC); };
+    auto tD = [&](int s) {
+        return Q::kOwnD ? tmem + 256 + static_cast<uint32_t>(2 * DC + (s & 1) * DC) : tX((s + 1) & 1);
+    };
     auto tile_of = [&](int step) { return dir > 0 ? s0 + step : nb - 1 - (s0 + step); };
     // fp32 state slot of segment gg of this (sequence, role)
     auto seg_slot = [&](int gg) {
@@ -196,156 +269,231 @@ la2_scan_ws(const __grid_constant__ Params p)
     };
 
     if (warp == 0) {
-        // ================================================= TMA producer
+        // ================================================= TMA producer + MMA issuer S
+        // One polling loop: a ring whose next buffer is free gets its load, and
+        // S of step s = A B^T (into S buffer s % 2) is issued once A and B of
+        // step s have landed and X += P C of step s-2, which read the P in that
+        // buffer, is done.  Nothing here blocks, so loads never wait behind S.
         if (lane == 0 && ns > 0) {
             prefetch_tmap(&R.ta);
             prefetch_tmap(&R.tb);
             prefetch_tmap(&R.tc);
-            auto load_a = [&](int i) {
-                mbar_arrive_expect_tx(bar(FULL_A), kTB * DA * 2);
-                for (int g = 0; g < DA / 64; ++g)
-                    tma_load_3d(sA + g * 16384, &R.ta, bar(FULL_A), g * 64, i * kTB, bh);
+            auto load_a = [&](int s) {
+                const int slot = s % Q::NA;
+                const uint32_t b = bar(Q::FULL_A + slot);
+                mbar_arrive_expect_tx(b, L::kAsz);
+                for (int gg = 0; gg < DA / 64; ++gg)
+                    tma_load_3d(sA + slot * L::kAsz + gg * 16384, &R.ta, b, gg * 64,
+                                tile_of(s) * kTB, bh);
             };
-            auto load_b = [&](int i, int slot) {
-                const uint32_t b = bar(FULL_B0 + slot);
-                mbar_arrive_expect_tx(b, kTB * DA * 2);
-                for (int g = 0; g < DA / 64; ++g)
-                    tma_load_3d(sB + slot * L::kBsz + g * 16384, &R.tb, b, g * 64, i * kTB, bh);
+            auto load_b = [&](int s) {
+                const int slot = s % Q::NB;
+                const uint32_t b = bar(Q::FULL_B + slot);
+                mbar_arrive_expect_tx(b, L::kBsz);
+                for (int gg = 0; gg < DA / 64; ++gg)
+                    tma_load_3d(sB + slot * L::kBsz + gg * 16384, &R.tb, b, gg * 64,
+                                tile_of(s) * kTB, bh);
             };
-            auto load_c = [&](int i) {
-                mbar_arrive_expect_tx(bar(FULL_C), kTB * DC * 2);
-                for (int g = 0; g < DC / 64; ++g)
-                    tma_load_3d(sC + g * 16384, &R.tc, bar(FULL_C), g * 64, i * kTB, bh);
+            auto load_c = [&](int s) {
+                const int slot = s % Q::NC;
+                const uint32_t b = bar(Q::FULL_C + slot);
+                mbar_arrive_expect_tx(b, L::kCsz);
+                for (int gg = 0; gg < DC / 64; ++gg)
+                    tma_load_3d(sC + slot * L::kCsz + gg * 16384, &R.tc, b, gg * 64,
+                                tile_of(s) * kTB, bh);
             };
-            load_a(tile_of(0));
-            load_b(tile_of(0), 0);
-            if (ns > 1) load_b(tile_of(1), 1);
-            load_c(tile_of(0));
-            for (int s = 0; s < ns; ++s) {
-                const uint32_t ph = s & 1;
-                // A is free once S and X = A W of tile s are done; B buffer s % 2 once
-                // dW of tile s is done; C once X += P C is done too.  Waiting in
-                // this order keeps every waiter within one phase of its barrier.
-                if (!wait_bar(bar(B_S0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 13)) break;
-                if (!wait_bar(bar(B_X0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 10)) break;
-                if (s + 1 < ns) load_a(tile_of(s + 1));
-                if (!wait_bar(bar(B_D), ph, abort_flag, p.status, 11)) break;
-                if (s + 2 < ns) load_b(tile_of(s + 2), s & 1);
-                if (!wait_bar(bar(B_PC0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 12)) break;
-                if (s + 1 < ns) load_c(tile_of(s + 1));
-            }
-        }
-    } else if (warp == 3) {
-        // ================================================= MMA issuer 0
-        // S of tile s into S buffer s % 2, once X += P C of tile s-2, which read
-        // the P in that buffer, is done
-        if (lane == 0) {
             constexpr uint32_t kIdS = idesc_bf16_f32(128, kTB, 0, 0);
-            for (int s = 0; s < ns; ++s) {
-                const uint32_t ph = s & 1;
-                const uint32_t sBs = sB + (s & 1) * L::kBsz;
-                if (!wait_bar(bar(FULL_A), ph, abort_flag, p.status, 20)) break;
-                if (!wait_bar(bar(FULL_B0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 21)) break;
-                if (s > 1 &&
-                    !wait_bar(bar(B_PC0 + (s & 1)), ((s - 2) >> 1) & 1, abort_flag, p.status, 22))
-                    break;
+            const uint64_t dA0 = sdesc_sw128(sA, 16, 1024), dB0 = sdesc_sw128(sB, 16, 1024);
+            auto issue_s = [&](int s) {
+                const int sa = s % Q::NA, sb = s % Q::NB;
                 tc_fence_after();
                 const uint32_t st = tS(s & 1);
-#pragma unroll 1
+                const uint64_t da = desc_add(dA0, sa * L::kAsz), db = desc_add(dB0, sb * L::kBsz);
+#pragma unroll
                 for (int k = 0; k < DA / 16; ++k) {
                     const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                    mma_bf16_ss(st, sdesc_sw128(sA + off, 16, 1024), sdesc_sw128(sBs + off, 16, 1024),
-                                kIdS, k > 0);
+                    mma_bf16_ss(st, desc_add(da, off), desc_add(db, off), kIdS, k > 0);
                 }
-                mma_commit(bar(B_S0 + (s & 1)));
+                mma_commit(bar(Q::S_DONE + (s & 1)));
+                mma_commit(bar(Q::EMPTY_A + sa));
+            };
+            // step s of a ring of n buffers may be loaded once step s - n has
+            // released its buffer
+            int ia = 0, ib = 0, ic = 0, is = 0;
+            bool idle = false;
+            uint64_t t0 = 0;
+            while (is < ns || ia < ns || ib < ns || ic < ns) {
+                bool prog = false;
+                if (ib < ns && (ib < Q::NB ||
+                                mbar_test_wait(bar(Q::EMPTY_B + ib % Q::NB), empty_par(ib, Q::NB)))) {
+                    LA2_TR(3, ib);
+                    load_b(ib++);
+                    prog = true;
+                }
+                if (ia < ns && (ia < Q::NA ||
+                                mbar_test_wait(bar(Q::EMPTY_A + ia % Q::NA), empty_par(ia, Q::NA)))) {
+                    LA2_TR(2, ia);
+                    load_a(ia++);
+                    prog = true;
+                }
+                if (ic < ns && (ic < Q::NC ||
+                                mbar_test_wait(bar(Q::EMPTY_C + ic % Q::NC), empty_par(ic, Q::NC)))) {
+                    LA2_TR(4, ic);
+                    load_c(ic++);
+                    prog = true;
+                }
+                if (is < ia && is < ib &&
+                    mbar_test_wait(bar(Q::FULL_A + is % Q::NA), full_par(is, Q::NA)) &&
+                    mbar_test_wait(bar(Q::FULL_B + is % Q::NB), full_par(is, Q::NB)) &&
+                    (is < 2 || mbar_test_wait(bar(Q::EMPTY_S + (is & 1)), empty_par(is, 2)))) {
+                    LA2_TR(5, is);
+                    issue_s(is);
+                    LA2_TR(19, is);
+                    ++is;
+                    prog = true;
+                }
+                if (prog) {
+                    idle = false;
+                    continue;
+                }
+                if (*abort_flag) break;
+                // back off briefly: this warp shares its scheduler with mask and
+                // epilogue warps, which a tight polling loop would slow down
+                __nanosleep(32);
+                const uint64_t now = global_ns();
+                if (!idle) {
+                    idle = true;
+                    t0 = now;
+                } else if (now - t0 > 2000000000ull) {
+                    *abort_flag = 1;
+                    atomicCAS(p.status, 0, 5 | ((is < ns ? 20 : 10) << 8));
+                    break;
+                }
             }
-            mma_commit(bar(B_FIN));
         }
+        if (lane == 0) mma_commit(bar(Q::FIN));
     } else if (warp == 1) {
-        // ================================================= MMA issuer 1
-        // X += P C of tile s, P read from S buffer s % 2
+        // ================================================= MMA issuer PC
+        // X += P C of tile s, P read from S buffer s % 2 (hi, then lo, per K step)
         if (lane == 0) {
             constexpr uint32_t kIdX = idesc_bf16_f32(128, DC, 0, 1);
+            const uint64_t dC0 = sdesc_sw128(sC, 16384, 1024);
             for (int s = 0; s < ns; ++s) {
-                const uint32_t ph = s & 1;
-                if (!wait_bar(bar(B_P0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 23)) break;
-                if (!wait_bar(bar(B_XS), ph, abort_flag, p.status, 24)) break;
-                if (!wait_bar(bar(FULL_C), ph, abort_flag, p.status, 25)) break;
+                const int sc = s % Q::NC;
+                if (!wait_bar(bar(Q::P_READY + (s & 1)), full_par(s, 2), abort_flag, p.status, 23)) break;
+                if (!wait_bar(bar(Q::XS + (s & 1)), full_par(s, 2), abort_flag, p.status, 24)) break;
+                if (!wait_bar(bar(Q::FULL_C + sc), full_par(s, Q::NC), abort_flag, p.status, 25)) break;
+                LA2_TR(6, s);
                 tc_fence_after();
                 const uint32_t xt = tX(s & 1), st = tS(s & 1);
-#pragma unroll 1
+                const uint64_t dc = desc_add(dC0, sc * L::kCsz);
+#pragma unroll
                 for (int k = 0; k < kTB / 16; ++k) {
-                    const uint64_t cdesc = sdesc_sw128(sC + k * 2048, 16384, 1024);
+                    const uint64_t cdesc = desc_add(dc, k * 2048);
                     mma_bf16_ts(xt, st + k * 16, cdesc, kIdX, 1);
                     mma_bf16_ts(xt, st + k * 16 + 8, cdesc, kIdX, 1);
                 }
-                mma_commit(bar(B_PC0 + (s & 1)));
+                mma_commit(bar(Q::PC_DONE + (s & 1)));
+                mma_commit(bar(Q::EMPTY_S + (s & 1)));
+                mma_commit(bar(Q::EMPTY_C + sc));
+                LA2_TR(20, s);
             }
-            mma_commit(bar(B_FIN));
+            mma_commit(bar(Q::FIN));
         }
     } else if (warp == 2) {
-        // ================================================= MMA issuer 2
-        // X = A hi(W) + A lo(W) into X buffer s % 2, then dW into X buffer (s+1) % 2
+        // ================================================= MMA issuer XW
+        // X = A hi(W) + A lo(W) into X buffer s % 2
         if (lane == 0) {
             constexpr uint32_t kIdX = idesc_bf16_f32(128, DC, 0, 1);
-            constexpr uint32_t kIdW = idesc_bf16_f32(DA, DC, 1, 1);
+            const uint64_t dA0 = sdesc_sw128(sA, 16, 1024), dW0 = sdesc_sw128(sW, DA * 128, 1024);
             for (int s = 0; s < ns; ++s) {
-                const uint32_t ph = s & 1;
-                const uint32_t sBs = sB + (s & 1) * L::kBsz;
-                // B_WR completes once when the epilogue has set the initial state
-                // and once per tile when it has updated W and read dW (which sat
-                // in X buffer s % 2)
-                {
-                    if (!wait_bar(bar(B_WR), ph, abort_flag, p.status, 30)) break;
-                    if (!wait_bar(bar(FULL_A), ph, abort_flag, p.status, 34)) break;
-                    tc_fence_after();
-                    const uint32_t xt = tX(s & 1);
-#pragma unroll 1
-                    for (int k = 0; k < DA / 16; ++k) {
-                        const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                        const uint64_t adesc = sdesc_sw128(sA + off, 16, 1024);
-                        mma_bf16_ss(xt, adesc, sdesc_sw128(sW + k * 2048, DA * 128, 1024), kIdX, k > 0);
-                        mma_bf16_ss(xt, adesc, sdesc_sw128(sW + L::kWsz + k * 2048, DA * 128, 1024),
-                                    kIdX, 1);
-                    }
-                    mma_commit(bar(B_X0 + (s & 1)));
-                }
-                if (!wait_bar(bar(B_BS), ph, abort_flag, p.status, 31)) break;
-                if (!wait_bar(bar(FULL_C), ph, abort_flag, p.status, 32)) break;
-                // X buffer (s+1) % 2 was read out after tile s-1
-                if (s > 0 &&
-                    !wait_bar(bar(B_XF0 + ((s + 1) & 1)), ((s - 1) >> 1) & 1, abort_flag, p.status, 33))
+                const int sa = s % Q::NA, sw = s % Q::NW;
+                // W_READY completes once the epilogue has set W of this step (the
+                // initial state, or the update after the previous tile, which has
+                // also read the dW that sat in this X buffer)
+                if (!wait_bar(bar(Q::W_READY + sw), full_par(s, Q::NW), abort_flag, p.status, 30)) break;
+                if (!wait_bar(bar(Q::FULL_A + sa), full_par(s, Q::NA), abort_flag, p.status, 31)) break;
+                if (s >= 2 &&
+                    !wait_bar(bar(Q::EMPTY_X + (s & 1)), empty_par(s, 2), abort_flag, p.status, 32))
                     break;
+                LA2_TR(7, s);
                 tc_fence_after();
-                const uint32_t dt = tX((s + 1) & 1);
-#pragma unroll 1
-                for (int k = 0; k < kTB / 16; ++k) {
-                    const uint64_t cdesc = sdesc_sw128(sC + k * 2048, 16384, 1024);
-                    mma_bf16_ss(dt, sdesc_sw128(sBs + k * 2048, 16384, 1024), cdesc, kIdW, k > 0);
-                    mma_bf16_ss(dt, sdesc_sw128(sBlo + k * 2048, 16384, 1024), cdesc, kIdW, 1);
+                const uint32_t xt = tX(s & 1);
+                const uint64_t da = desc_add(dA0, sa * L::kAsz), dw = desc_add(dW0, sw * 2 * L::kWsz);
+#pragma unroll
+                for (int k = 0; k < DA / 16; ++k) {
+                    const uint64_t adesc = desc_add(da, (k >> 2) * 16384 + (k & 3) * 32);
+                    mma_bf16_ss(xt, adesc, desc_add(dw, k * 2048), kIdX, k > 0);
+                    mma_bf16_ss(xt, adesc, desc_add(dw, L::kWsz + k * 2048), kIdX, 1);
                 }
-                mma_commit(bar(B_D));
+                mma_commit(bar(Q::XW_DONE + (s & 1)));
+                mma_commit(bar(Q::EMPTY_A + sa));
+                mma_commit(bar(Q::EMPTY_W + sw));
+                LA2_TR(21, s);
             }
-            mma_commit(bar(B_FIN));
+            mma_commit(bar(Q::FIN));
+        }
+    } else if (warp == 3) {
+        // ================================================= MMA issuer dW
+        // dW = hi(w_s B)^T C + lo(w_s B)^T C of tile s
+        if (lane == 0) {
+            constexpr uint32_t kIdW = idesc_bf16_f32(DA, DC, 1, 1);
+            const uint64_t dB0 = sdesc_sw128(sB, 16384, 1024), dL0 = sdesc_sw128(sBlo, 16384, 1024);
+            const uint64_t dC0 = sdesc_sw128(sC, 16384, 1024);
+            for (int s = 0; s < ns; ++s) {
+                const int sb = s % Q::NB, sc = s % Q::NC, sl = s % Q::NBLO;
+                if (!wait_bar(bar(Q::BS + sb), full_par(s, Q::NB), abort_flag, p.status, 33)) break;
+                if (!wait_bar(bar(Q::FULL_C + sc), full_par(s, Q::NC), abort_flag, p.status, 34)) break;
+                if (Q::kOwnD) {
+                    // the update after tile s-2 has read this dW buffer
+                    if (s >= 2 &&
+                        !wait_bar(bar(Q::EMPTY_D + (s & 1)), empty_par(s, 2), abort_flag, p.status, 35))
+                        break;
+                } else {
+                    // X buffer (s+1) % 2 has been read out after tile s-1
+                    if (s >= 1 && !wait_bar(bar(Q::EMPTY_X + ((s + 1) & 1)), full_par(s - 1, 2),
+                                            abort_flag, p.status, 36))
+                        break;
+                }
+                LA2_TR(8, s);
+                tc_fence_after();
+                const uint32_t dt = tD(s);
+                const uint64_t db = desc_add(dB0, sb * L::kBsz), dl = desc_add(dL0, sl * L::kBsz);
+                const uint64_t dc = desc_add(dC0, sc * L::kCsz);
+#pragma unroll
+                for (int k = 0; k < kTB / 16; ++k) {
+                    const uint64_t cdesc = desc_add(dc, k * 2048);
+                    mma_bf16_ss(dt, desc_add(db, k * 2048), cdesc, kIdW, k > 0);
+                    mma_bf16_ss(dt, desc_add(dl, k * 2048), cdesc, kIdW, 1);
+                }
+                mma_commit(bar(Q::D_DONE + (s % Q::ND)));
+                mma_commit(bar(Q::EMPTY_B + sb));
+                mma_commit(bar(Q::EMPTY_BLO + sl));
+                mma_commit(bar(Q::EMPTY_C + sc));
+                LA2_TR(22, s);
+            }
+            mma_commit(bar(Q::FIN));
         }
     } else if (warp >= 4 && warp < 12) {
         // ================================================= mask group
-        // two warps per lane quadrant; warp part p takes the 16-column groups
-        // g with g % 2 == p, which splits the causal triangle's work evenly
+        // two warps per lane quadrant; warp part p takes half of the work
         const int quad = warp & 3, part = (warp - 4) >> 2;
         const int r = quad * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const float ws = dir > 0 ? pw[kTB - 1 - r] : pw[r];
         for (int s = 0; s < ns; ++s) {
-            const uint32_t ph = s & 1;
-            if (!wait_bar(bar(B_S0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 40)) break;
+            if (!wait_bar(bar(Q::S_DONE + (s & 1)), full_par(s, 2), abort_flag, p.status, 40)) break;
+            if (tid == 128) LA2_TR(9, s);
             const uint32_t st = tS(s & 1);
             tc_fence_after();
             // row r of w_s B (S, which reads B unscaled, is done): hi in place,
-            // lo into its own buffer once the previous tile's dW, its only
-            // reader, is done.  Part p does the chunks of half p of the row.
-            if (s > 0 && !wait_bar(bar(B_D), ph ^ 1, abort_flag, p.status, 41)) break;
-            const uint32_t sBs = sB + (s & 1) * L::kBsz;
+            // lo into its own buffer once the dW that last read that buffer is
+            // done.  Part p does the chunks of half p of the row.
+            const int sl = s % Q::NBLO;
+            if (s >= Q::NBLO && !wait_bar(bar(Q::EMPTY_BLO + sl), empty_par(s, Q::NBLO), abort_flag,
+                                          p.status, 41))
+                break;
+            const uint32_t sBs = sB + (s % Q::NB) * L::kBsz, sBl = sBlo + sl * L::kBsz;
 #pragma unroll
             for (int k = 0; k < DA / 16; ++k) {
                 const int chunk = part * (DA / 16) + k;
@@ -354,13 +502,17 @@ la2_scan_ws(const __grid_constant__ Params p)
                 ld_shared_v4(sBs + off, v[0], v[1], v[2], v[3]);
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                    split_pack2(bf16lo_to_f32(v[u]) * ws, bf16hi_to_f32(v[u]) * ws, h[u], l[u]);
+                    split_pack2v(mul2(make_float2(bf16lo_to_f32(v[u]), bf16hi_to_f32(v[u])),
+                                      make_float2(ws, ws)),
+                                 h[u], l[u]);
                 st_shared_v4(sBs + off, h[0], h[1], h[2], h[3]);
-                st_shared_v4(sBlo + off, l[0], l[1], l[2], l[3]);
+                st_shared_v4(sBl + off, l[0], l[1], l[2], l[3]);
             }
+            if (tid == 128 + 96) LA2_TR(28, s);
             fence_proxy_async_smem();
-            mbar_arrive(bar(B_BS));
-            {
+            mbar_arrive(bar(Q::BS + (s % Q::NB)));
+            if (tid == 128) LA2_TR(10, s);
+            if (tid == 128 + 96) LA2_TR(29, s);
             // P = decay-masked S, hi + lo bf16, over the 16 columns of S each
             // group of 16 came from: [hi (8 cols) | lo (8 cols)], the A-operand
             // layout of one K = 16 step.  Every group is loaded before it is
@@ -380,12 +532,17 @@ la2_scan_ws(const __grid_constant__ Params p)
                     const int lo_g = 2 * quad, hi_g = 2 * quad + 1;
                     const int kind = (grp == lo_g || grp == hi_g) ? 1 : ((dir > 0) == (grp < lo_g) ? 2 : 0);
                     if (kind == 2) {
+                        // whole group on the causal side: lambda^|r-c| = alpha mu(c - 16 grp),
+                        // alpha = lambda^(r - 16 grp - 15) resp. lambda^(16 grp - r) (both
+                        // exponents in [1, 127]), mu = lambda^(15-u) resp. lambda^u
+                        const float alpha = pw[dir > 0 ? r - 16 * grp - 15 : 16 * grp - r];
+                        const float* mu = dir > 0 ? murev : pw;
 #pragma unroll
                         for (int u = 0; u < 8; ++u) {
-                            const int c0 = grp * 16 + 2 * u;
-                            const float p0 = sv[16 * h2 + 2 * u] * pw[dir > 0 ? r - c0 : c0 - r];
-                            const float p1 = sv[16 * h2 + 2 * u + 1] * pw[dir > 0 ? r - c0 - 1 : c0 + 1 - r];
-                            split_pack2(p0, p1, pk[16 * h2 + u], pk[16 * h2 + 8 + u]);
+                            const float2 m = *reinterpret_cast<const float2*>(mu + 2 * u);
+                            const float2 w = mul2(m, make_float2(alpha, alpha));
+                            split_pack2v(mul2(make_float2(sv[16 * h2 + 2 * u], sv[16 * h2 + 2 * u + 1]), w),
+                                         pk[16 * h2 + u], pk[16 * h2 + 8 + u]);
                         }
                     } else if (kind == 1) {
 #pragma unroll
@@ -404,13 +561,16 @@ la2_scan_ws(const __grid_constant__ Params p)
                     }
                 }
                 tmem_st32u(st + lane_off + pr * 32, pk);
+                if (tid == 128 + 96 && pr == part) LA2_TR(26, s);
             }
+            if (tid == 128 + 96) LA2_TR(27, s);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(B_P0 + (s & 1)));
-            }
+            mbar_arrive(bar(Q::P_READY + (s & 1)));
+            if (tid == 128) LA2_TR(11, s);
+            if (tid == 128 + 96) LA2_TR(30, s);
         }
-    } else if (warp >= 12) {
+    } else if (warp >= 12 && warp < 20) {
         // ================================================= epilogue group
         const int quad = warp & 3, half = (warp - 12) >> 2;
         const int r = quad * 32 + lane;
@@ -421,145 +581,180 @@ la2_scan_ws(const __grid_constant__ Params p)
         const float lamTB = pw[kTB];
         const bool owns_w_row = (DA == 128) || (lane < 16);
         const int wrow = (DA == 128) ? r : quad * 16 + (lane & 15);
-        {
-            // initial state of this segment, W_in(g) = f W_in(g-1) + S_{g-1} with
-            // f = lambda^(T_B n), as its hi/lo bf16 pair (zero for the first)
-            if (g > 0 && owns_w_row) {
-                const float f = static_cast<float>(
-                    exp2(static_cast<double>(kTB) * p.seg_tiles * log2(static_cast<double>(lam))));
+        // initial state of this segment, W_in(g) = f W_in(g-1) + S_{g-1} with
+        // f = lambda^(T_B n), as its hi/lo bf16 pair in W buffer 0 (zero for the
+        // first segment)
+        if (g > 0 && owns_w_row) {
+            const float f = static_cast<float>(
+                exp2(static_cast<double>(kTB) * p.seg_tiles * log2(static_cast<double>(lam))));
 #pragma unroll 1
-                for (int k = 0; k < kCols / 16; ++k) {
-                    const uint32_t col = c0 + k * 16;
-                    float w[16];
+            for (int k = 0; k < kCols / 16; ++k) {
+                const uint32_t col = c0 + k * 16;
+                float w[16];
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) w[u] = 0.f;
-                    for (int gp = 0; gp < g; ++gp) {
-                        const float* src = seg_slot(gp) + static_cast<size_t>(wrow) * DC + col;
+                for (int u = 0; u < 16; ++u) w[u] = 0.f;
+                for (int gp = 0; gp < g; ++gp) {
+                    const float* src = seg_slot(gp) + static_cast<size_t>(wrow) * DC + col;
 #pragma unroll
-                        for (int u = 0; u < 16; ++u) w[u] = fmaf(f, w[u], src[u]);
+                    for (int u = 0; u < 16; ++u) w[u] = fmaf(f, w[u], src[u]);
+                }
+                const uint32_t grpo = (col >> 6) * (DA * 128);
+                const int q = (col & 63) >> 3;
+                uint32_t h[8], l[8];
+#pragma unroll
+                for (int z = 0; z < 8; ++z) split_pack2(w[2 * z], w[2 * z + 1], h[z], l[z]);
+                st_shared_v4(sW + grpo + sw128(wrow, q), h[0], h[1], h[2], h[3]);
+                st_shared_v4(sW + grpo + sw128(wrow, q + 1), h[4], h[5], h[6], h[7]);
+                st_shared_v4(sW + L::kWsz + grpo + sw128(wrow, q), l[0], l[1], l[2], l[3]);
+                st_shared_v4(sW + L::kWsz + grpo + sw128(wrow, q + 1), l[4], l[5], l[6], l[7]);
+            }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar(Q::W_READY + 0));
+        float* xg = R.x + static_cast<size_t>(bh) * T * DC;
+
+        // X row r *= w_x(r) (the inter-tile term, still alone in X)
+        auto scale = [&](int s) -> bool {
+            if (!wait_bar(bar(Q::XW_DONE + (s & 1)), full_par(s, 2), abort_flag, p.status, 50))
+                return false;
+            if (tid == 384) LA2_TR(14, s);
+            tc_fence_after();
+            const uint32_t xt = tX(s & 1);
+#pragma unroll 1
+            for (int k = 0; k < kCols / 32; ++k) {
+                float x[32];
+                const uint32_t col = c0 + k * 32;
+                tmem_ld32(xt + lane_off + col, x);
+#pragma unroll
+                for (int u = 0; u < 32; ++u) x[u] *= wx;
+                tmem_st32(xt + lane_off + col, x);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(Q::XS + (s & 1)));
+            if (tid == 384) LA2_TR(15, s);
+            return true;
+        };
+        // W <- lambda^T_B W + dW, from W buffer s % NW into (s+1) % NW.  The
+        // state is kept as its hi + lo bf16 pair (a 16-bit significand, ~2^-17
+        // relative per update), which is also the next tile's MMA operand.
+        auto update = [&](int s) -> bool {
+            if (!wait_bar(bar(Q::D_DONE + (s % Q::ND)), full_par(s, Q::ND), abort_flag, p.status, 51))
+                return false;
+            // the X MMA that last read the W buffer written here is done
+            if (s + 1 >= Q::NW && !wait_bar(bar(Q::EMPTY_W + (s + 1) % Q::NW),
+                                            full_par(s + 1 - Q::NW, Q::NW), abort_flag, p.status, 52))
+                return false;
+            if (tid == 384) LA2_TR(12, s);
+            tc_fence_after();
+            const uint32_t wsrc = sW + (s % Q::NW) * 2 * L::kWsz;
+            const uint32_t wdst = sW + ((s + 1) % Q::NW) * 2 * L::kWsz;
+            const uint32_t dt = tD(s);
+#pragma unroll 1
+            for (int k = 0; k < kCols / 32; ++k) {
+                float d[32];
+                tmem_ld32(dt + lane_off + c0 + k * 32, d);
+                if (tid == 384 && k == 0) LA2_TR(23, s);
+                if (Q::kOwnD && k == kCols / 32 - 1) {
+                    tc_fence_before();
+                    mbar_arrive(bar(Q::EMPTY_D + (s & 1)));
+                }
+                if (owns_w_row) {
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const uint32_t col = c0 + k * 32 + hh * 16;
+                        const uint32_t o0 = (col >> 6) * (DA * 128) + sw128(wrow, (col & 63) >> 3);
+                        const uint32_t o1 = (col >> 6) * (DA * 128) + sw128(wrow, ((col & 63) >> 3) + 1);
+                        uint32_t h[8], l[8];
+                        ld_shared_v4(wsrc + o0, h[0], h[1], h[2], h[3]);
+                        ld_shared_v4(wsrc + o1, h[4], h[5], h[6], h[7]);
+                        ld_shared_v4(wsrc + L::kWsz + o0, l[0], l[1], l[2], l[3]);
+                        ld_shared_v4(wsrc + L::kWsz + o1, l[4], l[5], l[6], l[7]);
+#pragma unroll
+                        for (int z = 0; z < 8; ++z) {
+                            const float w0 = fmaf(lamTB, bf16lo_to_f32(h[z]) + bf16lo_to_f32(l[z]),
+                                                  d[16 * hh + 2 * z]);
+                            const float w1 = fmaf(lamTB, bf16hi_to_f32(h[z]) + bf16hi_to_f32(l[z]),
+                                                  d[16 * hh + 2 * z + 1]);
+                            split_pack2(w0, w1, h[z], l[z]);
+                        }
+                        st_shared_v4(wdst + o0, h[0], h[1], h[2], h[3]);
+                        st_shared_v4(wdst + o1, h[4], h[5], h[6], h[7]);
+                        st_shared_v4(wdst + L::kWsz + o0, l[0], l[1], l[2], l[3]);
+                        st_shared_v4(wdst + L::kWsz + o1, l[4], l[5], l[6], l[7]);
                     }
-                    const uint32_t grpo = (col >> 6) * (DA * 128);
-                    const int q = (col & 63) >> 3;
-                    uint32_t h[8], l[8];
-#pragma unroll
-                    for (int z = 0; z < 8; ++z) split_pack2(w[2 * z], w[2 * z + 1], h[z], l[z]);
-                    st_shared_v4(sW + grpo + sw128(wrow, q), h[0], h[1], h[2], h[3]);
-                    st_shared_v4(sW + grpo + sw128(wrow, q + 1), h[4], h[5], h[6], h[7]);
-                    st_shared_v4(sW + L::kWsz + grpo + sw128(wrow, q), l[0], l[1], l[2], l[3]);
-                    st_shared_v4(sW + L::kWsz + grpo + sw128(wrow, q + 1), l[4], l[5], l[6], l[7]);
                 }
             }
+            if (tid == 384) LA2_TR(24, s);
             fence_proxy_async_smem();
-            mbar_arrive(bar(B_WR));
-            float* xg = R.x + static_cast<size_t>(bh) * T * DC;
-            const int grp = lane >> 3, j = lane & 7;
-            for (int s = 0; s < ns; ++s) {
-                const uint32_t ph = s & 1;
-                const int i = tile_of(s);
-                const uint32_t xt = tX(s & 1);
-                // X row r *= w_x(r)   (the inter-tile term, still alone in X)
-                if (!wait_bar(bar(B_X0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 50)) break;
-                tc_fence_after();
+            if (tid == 384) LA2_TR(25, s);
+            tc_fence_before();
+            mbar_arrive(bar(Q::W_READY + (s + 1) % Q::NW));
+            if (tid == 384) LA2_TR(13, s);
+            return true;
+        };
+        // X of tile s, 32 columns at a time, read with the 16x256b TMEM shape:
+        // each group of four lanes then holds 8 consecutive floats of one row,
+        // so every float2 store of a warp fills whole 32-byte sectors (eight
+        // rows per instruction).  The X buffer is released once read.
+        auto output = [&](int s) -> bool {
+            if (!wait_bar(bar(Q::PC_DONE + (s & 1)), full_par(s, 2), abort_flag, p.status, 53))
+                return false;
+            if (tid == 384) LA2_TR(16, s);
+            tc_fence_after();
+            const int i = tile_of(s);
+            const uint32_t xt = tX(s & 1);
+            const int t4 = lane >> 2, tm = lane & 3;
+            const uint32_t l0 = static_cast<uint32_t>(quad * 32) << 16;
+            const uint32_t l1 = static_cast<uint32_t>(quad * 32 + 16) << 16;
 #pragma unroll 1
-                for (int k = 0; k < kCols / 32; ++k) {
-                    float x[32];
-                    const uint32_t col = c0 + k * 32;
-                    tmem_ld32(xt + lane_off + col, x);
-#pragma unroll
-                    for (int u = 0; u < 32; ++u) x[u] *= wx;
-                    tmem_st32(xt + lane_off + col, x);
+            for (int b = 0; b < kCols / 32; ++b) {
+                float v[32];
+                const uint32_t col = c0 + 32 * b;
+                tmem_ld16x256b_x4_pair(xt + l0 + col, xt + l1 + col, v);
+                if (b == kCols / 32 - 1) {
+                    tc_fence_before();
+                    mbar_arrive(bar(Q::EMPTY_X + (s & 1)));
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar(B_XS));
-                // W <- lambda^T_B W + dW.  The state is kept as its hi + lo bf16
-                // pair (a 16-bit significand, ~2^-17 relative per update), which
-                // is also the next tile's MMA operand; X = A W of this tile, which
-                // read it, is done.
-                if (!wait_bar(bar(B_D), ph, abort_flag, p.status, 51)) break;
-                tc_fence_after();
-#pragma unroll 1
-                for (int k = 0; k < kCols / 32; ++k) {
-                    float d[32];
-                    tmem_ld32(tX((s + 1) & 1) + lane_off + c0 + k * 32, d);
-                    if (owns_w_row) {
 #pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const uint32_t col = c0 + k * 32 + hh * 16;
-                            const uint32_t grpo = (col >> 6) * (DA * 128);
-                            const int q = (col & 63) >> 3;
-                            const uint32_t a0 = sW + grpo + sw128(wrow, q);
-                            const uint32_t a1 = sW + grpo + sw128(wrow, q + 1);
-                            uint32_t h[8], l[8];
-                            ld_shared_v4(a0, h[0], h[1], h[2], h[3]);
-                            ld_shared_v4(a1, h[4], h[5], h[6], h[7]);
-                            ld_shared_v4(a0 + L::kWsz, l[0], l[1], l[2], l[3]);
-                            ld_shared_v4(a1 + L::kWsz, l[4], l[5], l[6], l[7]);
+                for (int lh = 0; lh < 2; ++lh) {
+                    const int row = i * kTB + quad * 32 + lh * 16 + t4;
 #pragma unroll
-                            for (int z = 0; z < 8; ++z) {
-                                const float w0 = fmaf(lamTB, bf16lo_to_f32(h[z]) + bf16lo_to_f32(l[z]),
-                                                      d[16 * hh + 2 * z]);
-                                const float w1 = fmaf(lamTB, bf16hi_to_f32(h[z]) + bf16hi_to_f32(l[z]),
-                                                      d[16 * hh + 2 * z + 1]);
-                                split_pack2(w0, w1, h[z], l[z]);
-                            }
-                            st_shared_v4(a0, h[0], h[1], h[2], h[3]);
-                            st_shared_v4(a1, h[4], h[5], h[6], h[7]);
-                            st_shared_v4(a0 + L::kWsz, l[0], l[1], l[2], l[3]);
-                            st_shared_v4(a1 + L::kWsz, l[4], l[5], l[6], l[7]);
-                        }
-                    }
-                }
-                fence_proxy_async_smem();
-                tc_fence_before();
-                mbar_arrive(bar(B_WR));
-                // X of tile i, 32 columns at a time: TMEM -> registers, then an
-                // 8 x 8 transpose of float4s among each group of 8 lanes (warp
-                // shuffles), after which every store instruction writes four whole
-                // 128-byte rows.  The X buffer is released once read.
-                if (!wait_bar(bar(B_PC0 + (s & 1)), (s >> 1) & 1, abort_flag, p.status, 52)) break;
-                tc_fence_after();
-#pragma unroll 1
-                for (int b = 0; b < kCols / 32; ++b) {
-                    float v[32];
-                    tmem_ld32(xt + lane_off + c0 + 32 * b, v);
-                    if (b == kCols / 32 - 1) {
-                        tc_fence_before();
-                        mbar_arrive(bar(B_XF0 + (s & 1)));
-                    }
-                    // lane j of a group holds chunk c (4 floats) of its row in
-                    // v[4c..4c+3]; afterwards chunk j of row 8*grp + c
-#pragma unroll
-                    for (int st = 4; st >= 1; st >>= 1) {
-                        const bool up = (j & st) != 0;
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            if (c & st) continue;
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float send = up ? v[4 * c + e] : v[4 * (c | st) + e];
-                                const float recv = __shfl_xor_sync(0xffffffffu, send, st);
-                                if (up) v[4 * c + e] = recv;
-                                else v[4 * (c | st) + e] = recv;
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const int row = i * kTB + quad * 32 + grp * 8 + c;
+                    for (int j = 0; j < 4; ++j) {
+                        const int cc = static_cast<int>(col) + 8 * j + 2 * tm;
                         if (row < T)
-                            st_global_v4(xg + static_cast<size_t>(row) * DC + c0 + 32 * b + 4 * j,
-                                         v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                            st_global_v2(xg + static_cast<size_t>(row) * DC + cc, v[16 * lh + 4 * j],
+                                         v[16 * lh + 4 * j + 1]);
+                        if (row + 8 < T)
+                            st_global_v2(xg + static_cast<size_t>(row + 8) * DC + cc,
+                                         v[16 * lh + 4 * j + 2], v[16 * lh + 4 * j + 3]);
                     }
                 }
             }
+            if (tid == 384) LA2_TR(17, s);
+            return true;
+        };
+
+        if (Q::kOwnD) {
+            // dW has its own buffers, so X of a tile can be written out one step
+            // later, while X += P C of the next tile is still being issued
+            bool ok = true;
+            for (int s = 0; s < ns && ok; ++s) {
+                ok = scale(s) && update(s);
+                if (ok && s > 0) ok = output(s - 1);
+            }
+            if (ok && ns > 0) output(ns - 1);
+        } else {
+            // dW sits in the X buffer of tile s+1, which tile s-1's X must leave first
+            for (int s = 0; s < ns; ++s)
+                if (!scale(s) || !update(s) || !output(s)) break;
         }
     }
 
-    // ---- tear-down: wait (bounded) until both issuers' MMAs are done, free TMEM
+    // ---- tear-down: wait (bounded) until the issuers' MMAs are done, free TMEM
     __syncthreads();
     if (tid == 32 && ns > 0) {
-        if (!mbar_wait(bar(B_FIN), 0)) atomicCAS(p.status, 0, 5 | (60 << 8));
+        if (!mbar_wait(bar(Q::FIN), 0)) atomicCAS(p.status, 0, 5 | (60 << 8));
     }
     tc_fence_before();
     __syncthreads();
@@ -567,6 +762,7 @@ la2_scan_ws(const __grid_constant__ Params p)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    if (tid == 0) LA2_TR(18, 0);
 }
 
 
