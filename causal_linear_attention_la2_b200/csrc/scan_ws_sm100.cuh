@@ -80,37 +80,64 @@ struct Params {
 };
 
 // Buffer counts and mbarrier indices of the scan kernel for (DA, DC).
+//
+// Two operand modes.  At DA = DC = 64 (kTf32) shared memory has room for fp32
+// copies of C and of w_s B, so P (fp32 in TMEM) and w_s B enter their MMAs as
+// tf32: no hi/lo split, and w_s B is written to its own buffer, so it need
+// not wait for S.  Otherwise P and w_s B are bf16 hi + lo pairs (hi of w_s B
+// in place of B).  The state W is a bf16 hi + lo pair in both modes.
 template <int DA, int DC>
 struct RingCfg {
-    static constexpr bool kSmall = DA == 64 && DC == 64;
+    static constexpr bool kTf32 = DA == 64 && DC == 64;
     static constexpr bool kBig = DA == 128 && DC == 128;
-    static constexpr int NA = kSmall ? 3 : (kBig ? 1 : 2);  // A tiles
-    static constexpr int NB = kSmall ? 3 : 2;               // B tiles (then hi(w_s B))
-    static constexpr int NC = kSmall ? 3 : (kBig ? 1 : 2);  // C tiles
-    static constexpr int NBLO = DA == 64 ? 2 : 1;           // lo(w_s B)
-    static constexpr int NW = DA == 64 ? 2 : 1;             // W as its hi/lo pair
-    static constexpr bool kOwnD = DC == 64;                 // dW in TMEM buffers of its own
-    static constexpr int ND = kOwnD ? 2 : 1;
+    static constexpr int NA = kBig ? 1 : 2;                  // A tiles
+    static constexpr int NB = 2;                             // B tiles
+    static constexpr int NC = kBig ? 1 : 2;                  // C tiles (bf16, as loaded)
+    static constexpr int NBLO = kTf32 ? 0 : (DA == 64 ? 2 : 1);  // lo(w_s B) (bf16 mode)
+    static constexpr int NCF = kTf32 ? 2 : 0;                // fp32 C (tf32 mode)
+    static constexpr int NWB = kTf32 ? 1 : 0;                // fp32 w_s B (tf32 mode)
+    static constexpr int NW = DA == 64 ? 2 : 1;              // W as its hi/lo pair
+    // DC = 64 (kOwnD): X += P C (two TMEM buffers), X_inter = A W (one) and
+    // dW (one) are separate accumulators, and the epilogue forms
+    // w_x X_inter + X; X += P C then never waits for the state.  DC = 128: X
+    // (two buffers) holds A W, scaled by w_x in TMEM, then P C; dW borrows the
+    // X buffer of the next tile.
+    static constexpr bool kOwnD = DC == 64;
+    static constexpr int ND = 1;
+    static constexpr int NX = 2;                             // X accumulators in TMEM
+    static constexpr int NXW = kOwnD ? 1 : NX;               // XW_DONE barriers
+    static constexpr int NXS = kOwnD ? 0 : NX;               // XS barriers (scaled in TMEM)
+    static constexpr int NXI = kOwnD ? 1 : 0;                // EMPTY_XI (X_inter read out)
+    static constexpr int NBS = kTf32 ? 0 : NB;
     // "full": the producer has filled the buffer; "empty": its consumers are done
     static constexpr int FULL_A = 0, EMPTY_A = FULL_A + NA;
     static constexpr int FULL_B = EMPTY_A + NA, EMPTY_B = FULL_B + NB, BS = EMPTY_B + NB;
-    static constexpr int FULL_C = BS + NB, EMPTY_C = FULL_C + NC;
+    static constexpr int FULL_C = BS + NBS, EMPTY_C = FULL_C + NC;
     static constexpr int EMPTY_BLO = EMPTY_C + NC;
-    static constexpr int S_DONE = EMPTY_BLO + NBLO, EMPTY_S = S_DONE + 2, P_READY = EMPTY_S + 2;
-    static constexpr int XW_DONE = P_READY + 2, XS = XW_DONE + 2, PC_DONE = XS + 2;
-    static constexpr int EMPTY_X = PC_DONE + 2;
-    static constexpr int D_DONE = EMPTY_X + 2, EMPTY_D = D_DONE + ND;
+    static constexpr int CF_READY = EMPTY_BLO + NBLO, EMPTY_CF = CF_READY + NCF;
+    static constexpr int WB_READY = EMPTY_CF + NCF, EMPTY_WB = WB_READY + NWB;
+    static constexpr int S_DONE = EMPTY_WB + NWB, EMPTY_S = S_DONE + 2, P_READY = EMPTY_S + 2;
+    static constexpr int XW_DONE = P_READY + 2, XS = XW_DONE + NXW, PC_DONE = XS + NXS;
+    static constexpr int EMPTY_X = PC_DONE + NX, EMPTY_XI = EMPTY_X + NX;
+    static constexpr int D_DONE = EMPTY_XI + NXI, EMPTY_D = D_DONE + ND;
     static constexpr int W_READY = EMPTY_D + ND, EMPTY_W = W_READY + NW;
     static constexpr int FIN = EMPTY_W + NW, NBARS = FIN + 1;
 
     // arrivals that complete one phase of barrier b
     static __device__ __forceinline__ uint32_t count(int b) {
         if (b >= EMPTY_A && b < EMPTY_A + NA) return 2;   // S and XW commits
-        if (b >= EMPTY_C && b < EMPTY_C + NC) return 2;   // PC and dW commits
-        if (b >= BS && b < BS + NB) return 256;           // mask group
+        if (b >= EMPTY_B && b < EMPTY_B + NB)             // tf32: S commit + mask reads;
+            return kTf32 ? 257 : 1;                        // bf16: dW commit
+        if (b >= EMPTY_C && b < EMPTY_C + NC)             // tf32: mask (to fp32);
+            return kTf32 ? 256 : 2;                        // bf16: PC and dW commits
+        if (b >= EMPTY_CF && b < EMPTY_CF + NCF) return 2; // PC and dW commits
+        if (b >= CF_READY && b < CF_READY + NCF) return 256;
+        if (b >= WB_READY && b < WB_READY + NWB) return 256;
+        if (b >= BS && b < BS + NBS) return 256;          // mask group
         if (b >= P_READY && b < P_READY + 2) return 256;  // mask group
-        if (b >= XS && b < XS + 2) return 256;            // epilogue group
-        if (b >= EMPTY_X && b < EMPTY_X + 2) return 256;  // epilogue group
+        if (b >= XS && b < XS + NXS) return 256;          // epilogue group
+        if (b >= EMPTY_X && b < EMPTY_X + NX) return 256; // epilogue group
+        if (b >= EMPTY_XI && b < EMPTY_XI + NXI) return 256;  // epilogue group
         if (b >= EMPTY_D && b < EMPTY_D + ND) return 256; // epilogue group
         if (b >= W_READY && b < W_READY + NW) return 256; // epilogue group
         if (b == FIN) return 4;                           // the four issuers
@@ -129,10 +156,18 @@ struct Smem {
     static constexpr uint32_t kB = kA + Q::NA * kAsz;         // B ring, each then hi(w_s B)
     static constexpr uint32_t kBlo = kB + Q::NB * kBsz;       // lo(w_s B) ring
     static constexpr uint32_t kC = kBlo + Q::NBLO * kBsz;     // C ring
-    static constexpr uint32_t kW = kC + Q::NC * kCsz;         // W buffer i: hi, then lo
+    // tf32 mode: fp32 C^T and (w_s B)^T, K-major (time contiguous in 128-byte
+    // rows, one row per feature), in four 32-step groups of DC (DA) rows each
+    static constexpr uint32_t kCFsz = kTB * DC * 4;           // fp32 C^T
+    static constexpr uint32_t kWBsz = kTB * DA * 4;           // fp32 (w_s B)^T
+    static constexpr uint32_t kCF = kC + Q::NC * kCsz;        // fp32 C ring (tf32 mode)
+    static constexpr uint32_t kWB = kCF + Q::NCF * kCFsz;     // fp32 w_s B ring (tf32 mode)
+    static constexpr uint32_t kW = kWB + Q::NWB * kWBsz;      // W buffer i: hi, then lo
     static constexpr uint32_t kPow = kW + Q::NW * 2 * kWsz;   // lambda^n, n = 0..T_B
     static constexpr uint32_t kMuRev = kPow + 528;            // lambda^(15-n), n = 0..15
-    static constexpr uint32_t kBar = kMuRev + 64;
+    static constexpr uint32_t kZ = kMuRev + 64;               // diagonal-block weights, 4 shifted copies
+    static constexpr uint32_t kZstride = 72 * 4;              // bytes per copy (72 = 8 mod 32 floats)
+    static constexpr uint32_t kBar = kZ + 4 * kZstride;
     static constexpr uint32_t kTmemSlot = kBar + Q::NBARS * 8;
     static constexpr uint32_t kAbort = kTmemSlot + 4;
     static constexpr uint32_t kBytes = kAbort + 12;
@@ -208,6 +243,7 @@ la2_scan_ws(const __grid_constant__ Params p)
     }
     const uint32_t sA = base + L::kA, sB = base + L::kB, sBlo = base + L::kBlo;
     const uint32_t sC = base + L::kC, sW = base + L::kW;
+    const uint32_t sCF = base + L::kCF, sWB = base + L::kWB;
     float* pw = reinterpret_cast<float*>(smem_raw + L::kPow);
     float* murev = reinterpret_cast<float*>(smem_raw + L::kMuRev);
     auto bar = [&](int b) { return base + L::kBar + 8u * b; };
@@ -234,6 +270,14 @@ la2_scan_ws(const __grid_constant__ Params p)
         const double l2 = log2(static_cast<double>(lam));
         for (int n = tid; n <= kTB; n += kThreads) pw[n] = static_cast<float>(exp2(n * l2));
         if (tid < 16) murev[tid] = static_cast<float>(exp2((15 - tid) * l2));
+        // Z[m] = lambda^(m-31) for m >= 31, else 0 (m = 0..66); copy k holds
+        // Z[j + k] at j, so that a 32-entry window starting anywhere can be
+        // read with aligned 16-byte loads
+        for (int idx = tid; idx < 4 * 64; idx += kThreads) {
+            const int k = idx >> 6, j = idx & 63, m = j + k;
+            float* zc = reinterpret_cast<float*>(smem_raw + L::kZ + k * L::kZstride);
+            zc[j] = m >= 31 ? static_cast<float>(exp2((m - 31) * l2)) : 0.f;
+        }
         for (uint32_t off = tid * 16; off < 2 * L::kWsz; off += kThreads * 16)
             st_shared_v4(sW + off, 0u, 0u, 0u, 0u);
     }
@@ -253,15 +297,19 @@ la2_scan_ws(const __grid_constant__ Params p)
 
     if (tid == 0) LA2_TR(1, 0);
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_raw + L::kTmemSlot);
-    // TMEM: S / P in two buffers (128 columns each), X in two buffers (DC each),
-    // then (DC = 64) two dW buffers; otherwise dW of tile s goes to the X buffer
-    // of tile s+1: X of tile s-1 has been read out of it, and X of tile s+1 is
-    // not issued before the state update has read dW.
+    // TMEM: S / P in two buffers (128 columns each), X in NX buffers (DC each),
+    // then (DC = 64) a dW buffer; otherwise dW of tile s goes to the X buffer of
+    // tile s+1: X of tile s-1 has been read out of it, and X of tile s+1 is not
+    // issued before the state update has read dW.
     auto tS = [&](int b) { return tmem + static_cast<uint32_t>(b * 128); };
     auto tX = [&](int b) { return tmem + 256 + static_cast<uint32_t>(b * DC); };
+    const uint32_t tXI = tmem + 256 + static_cast<uint32_t>(Q::NX * DC);  // X_inter (DC = 64)
     auto tD = [&](int s) {
-        return Q::kOwnD ? tmem + 256 + static_cast<uint32_t>(2 * DC + (s & 1) * DC) : tX((s + 1) & 1);
+        return Q::kOwnD ? tmem + 256 + static_cast<uint32_t>((Q::NX + 1) * DC + (s % Q::ND) * DC)
+                        : tX((s + 1) % Q::NX);
     };
+    static_assert(256 + Q::NX * DC + (Q::kOwnD ? (1 + Q::ND) * DC : 0) <= static_cast<int>(kTmemCols),
+                  "TMEM columns");
     auto tile_of = [&](int step) { return dir > 0 ? s0 + step : nb - 1 - (s0 + step); };
     // fp32 state slot of segment gg of this (sequence, role)
     auto seg_slot = [&](int gg) {
@@ -316,6 +364,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                 }
                 mma_commit(bar(Q::S_DONE + (s & 1)));
                 mma_commit(bar(Q::EMPTY_A + sa));
+                if (Q::kTf32) mma_commit(bar(Q::EMPTY_B + sb));  // dW does not read B
             };
             // step s of a ring of n buffers may be loaded once step s - n has
             // released its buffer
@@ -374,28 +423,51 @@ la2_scan_ws(const __grid_constant__ Params p)
         if (lane == 0) mma_commit(bar(Q::FIN));
     } else if (warp == 1) {
         // ================================================= MMA issuer PC
-        // X += P C of tile s, P read from S buffer s % 2 (hi, then lo, per K step)
+        // X += P C of tile s, P read from S buffer s % 2: in bf16 mode its hi and
+        // lo parts per K step of 16; in tf32 mode P is fp32, K steps of 8, with
+        // the fp32 copy of C
         if (lane == 0) {
-            constexpr uint32_t kIdX = idesc_bf16_f32(128, DC, 0, 1);
-            const uint64_t dC0 = sdesc_sw128(sC, 16384, 1024);
+            constexpr uint32_t kIdX = Q::kTf32 ? idesc_tf32_f32(128, DC, 0, 0)
+                                               : idesc_bf16_f32(128, DC, 0, 1);
+            const uint64_t dC0 = Q::kTf32 ? sdesc_sw128(sCF, 16, 1024) : sdesc_sw128(sC, 16384, 1024);
             for (int s = 0; s < ns; ++s) {
-                const int sc = s % Q::NC;
+                const int sc = Q::kTf32 ? s % Q::NCF : s % Q::NC;
                 if (!wait_bar(bar(Q::P_READY + (s & 1)), full_par(s, 2), abort_flag, p.status, 23)) break;
-                if (!wait_bar(bar(Q::XS + (s & 1)), full_par(s, 2), abort_flag, p.status, 24)) break;
-                if (!wait_bar(bar(Q::FULL_C + sc), full_par(s, Q::NC), abort_flag, p.status, 25)) break;
+                if (Q::kOwnD) {
+                    // X buffer s % 2 has been read out after tile s-2
+                    if (s >= Q::NX && !wait_bar(bar(Q::EMPTY_X + s % Q::NX), empty_par(s, Q::NX),
+                                                abort_flag, p.status, 24))
+                        break;
+                } else if (!wait_bar(bar(Q::XS + s % Q::NX), full_par(s, Q::NX), abort_flag, p.status, 24)) {
+                    break;
+                }
+                if (Q::kTf32) {
+                    if (!wait_bar(bar(Q::CF_READY + sc), full_par(s, Q::NCF), abort_flag, p.status, 25))
+                        break;
+                } else if (!wait_bar(bar(Q::FULL_C + sc), full_par(s, Q::NC), abort_flag, p.status, 25)) {
+                    break;
+                }
                 LA2_TR(6, s);
                 tc_fence_after();
-                const uint32_t xt = tX(s & 1), st = tS(s & 1);
-                const uint64_t dc = desc_add(dC0, sc * L::kCsz);
+                const uint32_t xt = tX(s % Q::NX), st = tS(s & 1);
+                if constexpr (Q::kTf32) {
+                    const uint64_t dc = desc_add(dC0, sc * L::kCFsz);
 #pragma unroll
-                for (int k = 0; k < kTB / 16; ++k) {
-                    const uint64_t cdesc = desc_add(dc, k * 2048);
-                    mma_bf16_ts(xt, st + k * 16, cdesc, kIdX, 1);
-                    mma_bf16_ts(xt, st + k * 16 + 8, cdesc, kIdX, 1);
+                    for (int k = 0; k < kTB / 8; ++k)
+                        mma_tf32_ts(xt, st + k * 8, desc_add(dc, (k >> 2) * (DC * 128) + (k & 3) * 32),
+                                    kIdX, Q::kOwnD ? (k > 0) : 1);
+                } else {
+                    const uint64_t dc = desc_add(dC0, sc * L::kCsz);
+#pragma unroll
+                    for (int k = 0; k < kTB / 16; ++k) {
+                        const uint64_t cdesc = desc_add(dc, k * 2048);
+                        mma_bf16_ts(xt, st + k * 16, cdesc, kIdX, Q::kOwnD ? (k > 0) : 1);
+                        mma_bf16_ts(xt, st + k * 16 + 8, cdesc, kIdX, 1);
+                    }
                 }
-                mma_commit(bar(Q::PC_DONE + (s & 1)));
+                mma_commit(bar(Q::PC_DONE + s % Q::NX));
                 mma_commit(bar(Q::EMPTY_S + (s & 1)));
-                mma_commit(bar(Q::EMPTY_C + sc));
+                mma_commit(bar((Q::kTf32 ? Q::EMPTY_CF : Q::EMPTY_C) + sc));
                 LA2_TR(20, s);
             }
             mma_commit(bar(Q::FIN));
@@ -413,12 +485,17 @@ la2_scan_ws(const __grid_constant__ Params p)
                 // also read the dW that sat in this X buffer)
                 if (!wait_bar(bar(Q::W_READY + sw), full_par(s, Q::NW), abort_flag, p.status, 30)) break;
                 if (!wait_bar(bar(Q::FULL_A + sa), full_par(s, Q::NA), abort_flag, p.status, 31)) break;
-                if (s >= 2 &&
-                    !wait_bar(bar(Q::EMPTY_X + (s & 1)), empty_par(s, 2), abort_flag, p.status, 32))
+                if (Q::kOwnD) {
+                    // X_inter has been read out after tile s-1
+                    if (s >= 1 && !wait_bar(bar(Q::EMPTY_XI), full_par(s - 1, 1), abort_flag, p.status, 32))
+                        break;
+                } else if (s >= Q::NX && !wait_bar(bar(Q::EMPTY_X + s % Q::NX), empty_par(s, Q::NX),
+                                                   abort_flag, p.status, 32)) {
                     break;
+                }
                 LA2_TR(7, s);
                 tc_fence_after();
-                const uint32_t xt = tX(s & 1);
+                const uint32_t xt = Q::kOwnD ? tXI : tX(s % Q::NX);
                 const uint64_t da = desc_add(dA0, sa * L::kAsz), dw = desc_add(dW0, sw * 2 * L::kWsz);
 #pragma unroll
                 for (int k = 0; k < DA / 16; ++k) {
@@ -426,7 +503,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                     mma_bf16_ss(xt, adesc, desc_add(dw, k * 2048), kIdX, k > 0);
                     mma_bf16_ss(xt, adesc, desc_add(dw, L::kWsz + k * 2048), kIdX, 1);
                 }
-                mma_commit(bar(Q::XW_DONE + (s & 1)));
+                mma_commit(bar(Q::XW_DONE + s % Q::NXW));
                 mma_commit(bar(Q::EMPTY_A + sa));
                 mma_commit(bar(Q::EMPTY_W + sw));
                 LA2_TR(21, s);
@@ -435,140 +512,240 @@ la2_scan_ws(const __grid_constant__ Params p)
         }
     } else if (warp == 3) {
         // ================================================= MMA issuer dW
-        // dW = hi(w_s B)^T C + lo(w_s B)^T C of tile s
+        // dW = (w_s B)^T C of tile s: bf16 mode hi(w_s B)^T C + lo(w_s B)^T C,
+        // tf32 mode the fp32 copies of w_s B and C
         if (lane == 0) {
-            constexpr uint32_t kIdW = idesc_bf16_f32(DA, DC, 1, 1);
-            const uint64_t dB0 = sdesc_sw128(sB, 16384, 1024), dL0 = sdesc_sw128(sBlo, 16384, 1024);
-            const uint64_t dC0 = sdesc_sw128(sC, 16384, 1024);
+            constexpr uint32_t kIdW = Q::kTf32 ? idesc_tf32_f32(DA, DC, 0, 0) : idesc_bf16_f32(DA, DC, 1, 1);
+            const uint64_t dB0 = Q::kTf32 ? sdesc_sw128(sWB, 16, 1024) : sdesc_sw128(sB, 16384, 1024);
+            const uint64_t dL0 = sdesc_sw128(sBlo, 16384, 1024);
+            const uint64_t dC0 = Q::kTf32 ? sdesc_sw128(sCF, 16, 1024) : sdesc_sw128(sC, 16384, 1024);
             for (int s = 0; s < ns; ++s) {
-                const int sb = s % Q::NB, sc = s % Q::NC, sl = s % Q::NBLO;
-                if (!wait_bar(bar(Q::BS + sb), full_par(s, Q::NB), abort_flag, p.status, 33)) break;
-                if (!wait_bar(bar(Q::FULL_C + sc), full_par(s, Q::NC), abort_flag, p.status, 34)) break;
+                const int sb = Q::kTf32 ? s % Q::NWB : s % Q::NB;
+                const int sc = Q::kTf32 ? s % Q::NCF : s % Q::NC;
+                const int sl = Q::kTf32 ? 0 : s % Q::NBLO;
+                if (Q::kTf32) {
+                    if (!wait_bar(bar(Q::WB_READY + sb), full_par(s, Q::NWB), abort_flag, p.status, 33)) break;
+                    if (!wait_bar(bar(Q::CF_READY + sc), full_par(s, Q::NCF), abort_flag, p.status, 34)) break;
+                } else {
+                    if (!wait_bar(bar(Q::BS + sb), full_par(s, Q::NB), abort_flag, p.status, 33)) break;
+                    if (!wait_bar(bar(Q::FULL_C + sc), full_par(s, Q::NC), abort_flag, p.status, 34)) break;
+                }
                 if (Q::kOwnD) {
-                    // the update after tile s-2 has read this dW buffer
-                    if (s >= 2 &&
-                        !wait_bar(bar(Q::EMPTY_D + (s & 1)), empty_par(s, 2), abort_flag, p.status, 35))
+                    // the update after tile s - ND has read this dW buffer
+                    if (s >= Q::ND && !wait_bar(bar(Q::EMPTY_D + s % Q::ND), empty_par(s, Q::ND),
+                                                abort_flag, p.status, 35))
                         break;
                 } else {
                     // X buffer (s+1) % 2 has been read out after tile s-1
-                    if (s >= 1 && !wait_bar(bar(Q::EMPTY_X + ((s + 1) & 1)), full_par(s - 1, 2),
+                    static_assert(Q::kOwnD || Q::NX == 2, "dW shares the X buffers only with NX = 2");
+                    if (s >= 1 && !wait_bar(bar(Q::EMPTY_X + ((s + 1) % Q::NX)), full_par(s - 1, Q::NX),
                                             abort_flag, p.status, 36))
                         break;
                 }
                 LA2_TR(8, s);
                 tc_fence_after();
                 const uint32_t dt = tD(s);
-                const uint64_t db = desc_add(dB0, sb * L::kBsz), dl = desc_add(dL0, sl * L::kBsz);
-                const uint64_t dc = desc_add(dC0, sc * L::kCsz);
+                if constexpr (Q::kTf32) {
+                    const uint64_t db = desc_add(dB0, sb * L::kWBsz), dc = desc_add(dC0, sc * L::kCFsz);
 #pragma unroll
-                for (int k = 0; k < kTB / 16; ++k) {
-                    const uint64_t cdesc = desc_add(dc, k * 2048);
-                    mma_bf16_ss(dt, desc_add(db, k * 2048), cdesc, kIdW, k > 0);
-                    mma_bf16_ss(dt, desc_add(dl, k * 2048), cdesc, kIdW, 1);
+                    for (int k = 0; k < kTB / 8; ++k)
+                        mma_tf32_ss(dt, desc_add(db, (k >> 2) * (DA * 128) + (k & 3) * 32),
+                                    desc_add(dc, (k >> 2) * (DC * 128) + (k & 3) * 32), kIdW, k > 0);
+                    mma_commit(bar(Q::D_DONE + (s % Q::ND)));
+                    mma_commit(bar(Q::EMPTY_WB + sb));
+                    mma_commit(bar(Q::EMPTY_CF + sc));
+                } else {
+                    const uint64_t db = desc_add(dB0, sb * L::kBsz), dl = desc_add(dL0, sl * L::kBsz);
+                    const uint64_t dc = desc_add(dC0, sc * L::kCsz);
+#pragma unroll
+                    for (int k = 0; k < kTB / 16; ++k) {
+                        const uint64_t cdesc = desc_add(dc, k * 2048);
+                        mma_bf16_ss(dt, desc_add(db, k * 2048), cdesc, kIdW, k > 0);
+                        mma_bf16_ss(dt, desc_add(dl, k * 2048), cdesc, kIdW, 1);
+                    }
+                    mma_commit(bar(Q::D_DONE + (s % Q::ND)));
+                    mma_commit(bar(Q::EMPTY_B + sb));
+                    mma_commit(bar(Q::EMPTY_BLO + sl));
+                    mma_commit(bar(Q::EMPTY_C + sc));
                 }
-                mma_commit(bar(Q::D_DONE + (s % Q::ND)));
-                mma_commit(bar(Q::EMPTY_B + sb));
-                mma_commit(bar(Q::EMPTY_BLO + sl));
-                mma_commit(bar(Q::EMPTY_C + sc));
                 LA2_TR(22, s);
             }
             mma_commit(bar(Q::FIN));
         }
     } else if (warp >= 4 && warp < 12) {
         // ================================================= mask group
-        // two warps per lane quadrant; warp part p takes half of the work
+        // two warps per lane quadrant; part p of a quadrant takes half the work
         const int quad = warp & 3, part = (warp - 4) >> 2;
         const int r = quad * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const float ws = dir > 0 ? pw[kTB - 1 - r] : pw[r];
-        for (int s = 0; s < ns; ++s) {
-            if (!wait_bar(bar(Q::S_DONE + (s & 1)), full_par(s, 2), abort_flag, p.status, 40)) break;
-            if (tid == 128) LA2_TR(9, s);
-            const uint32_t st = tS(s & 1);
-            tc_fence_after();
-            // row r of w_s B (S, which reads B unscaled, is done): hi in place,
-            // lo into its own buffer once the dW that last read that buffer is
-            // done.  Part p does the chunks of half p of the row.
-            const int sl = s % Q::NBLO;
-            if (s >= Q::NBLO && !wait_bar(bar(Q::EMPTY_BLO + sl), empty_par(s, Q::NBLO), abort_flag,
-                                          p.status, 41))
-                break;
-            const uint32_t sBs = sB + (s % Q::NB) * L::kBsz, sBl = sBlo + sl * L::kBsz;
+        // diagonal 32 x 32 block of this quadrant: row `lane` reads a 32-entry
+        // window of Z (dir > 0: weight of column j = Z[lane - j + 31]; dir < 0:
+        // Z[j - lane + 31]), from the copy that makes the window 16-byte aligned
+        const int zs = dir > 0 ? lane : 31 - lane;
+        const uint32_t zwin = base + L::kZ + (zs & 3) * L::kZstride + (zs - (zs & 3)) * 4;
+        const float* mu = dir > 0 ? murev : pw;
+        // P = S * lambda^|r-c| on the causal side, 0 elsewhere, 32 columns (one
+        // pair of K = 16 groups) at a time.  pr == quad is the diagonal block;
+        // whole pairs on the causal side use lambda^|r-c| = alpha mu(c), with
+        // alpha = lambda^(r - 16 grp - 15) resp. lambda^(16 grp - r), exponents
+        // in [1, 127], and mu = lambda^(15-u) resp. lambda^u.  Every S column
+        // is loaded before it is overwritten, also columns the mask zeroes:
+        // storing over S columns that were not read first made the following
+        // TMEM-operand MMAs about 10x slower.
+        auto weigh = [&](int pr, float (&sv)[32]) {
+            const bool diag = pr == quad;
+            const bool causal = (dir > 0) == (pr < quad);
+            if (diag) {
 #pragma unroll
-            for (int k = 0; k < DA / 16; ++k) {
-                const int chunk = part * (DA / 16) + k;
-                const uint32_t off = (chunk >> 3) * 16384 + sw128(r, chunk & 7);
-                uint32_t v[4], h[4], l[4];
-                ld_shared_v4(sBs + off, v[0], v[1], v[2], v[3]);
+                for (int t4 = 0; t4 < 8; ++t4) {
+                    float z[4];
+                    ld_shared_v4f(zwin + 16 * t4, z);
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    split_pack2v(mul2(make_float2(bf16lo_to_f32(v[u]), bf16hi_to_f32(v[u])),
-                                      make_float2(ws, ws)),
-                                 h[u], l[u]);
-                st_shared_v4(sBs + off, h[0], h[1], h[2], h[3]);
-                st_shared_v4(sBl + off, l[0], l[1], l[2], l[3]);
-            }
-            if (tid == 128 + 96) LA2_TR(28, s);
-            fence_proxy_async_smem();
-            mbar_arrive(bar(Q::BS + (s % Q::NB)));
-            if (tid == 128) LA2_TR(10, s);
-            if (tid == 128 + 96) LA2_TR(29, s);
-            // P = decay-masked S, hi + lo bf16, over the 16 columns of S each
-            // group of 16 came from: [hi (8 cols) | lo (8 cols)], the A-operand
-            // layout of one K = 16 step.  Every group is loaded before it is
-            // overwritten, also groups the mask zeroes entirely: storing over S
-            // columns that were not read first made the following TMEM-operand
-            // MMAs about 10x slower.
-            // Part p takes the 32-column pairs of groups {4k + 2p, 4k + 2p + 1},
-            // which splits the causal triangle's work about evenly.
-#pragma unroll 1
-            for (int pr = part; pr < kTB / 32; pr += 2) {
-                float sv[32];
-                tmem_ld32(st + lane_off + pr * 32, sv);
-                uint32_t pk[32];
+                    for (int e = 0; e < 4; ++e) {
+                        const int t = 4 * t4 + e;           // window index
+                        const int j = dir > 0 ? 31 - t : t;  // column in the block
+                        sv[j] *= z[e];
+                    }
+                }
+            } else if (causal) {
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
                     const int grp = 2 * pr + h2;
-                    const int lo_g = 2 * quad, hi_g = 2 * quad + 1;
-                    const int kind = (grp == lo_g || grp == hi_g) ? 1 : ((dir > 0) == (grp < lo_g) ? 2 : 0);
-                    if (kind == 2) {
-                        // whole group on the causal side: lambda^|r-c| = alpha mu(c - 16 grp),
-                        // alpha = lambda^(r - 16 grp - 15) resp. lambda^(16 grp - r) (both
-                        // exponents in [1, 127]), mu = lambda^(15-u) resp. lambda^u
-                        const float alpha = pw[dir > 0 ? r - 16 * grp - 15 : 16 * grp - r];
-                        const float* mu = dir > 0 ? murev : pw;
+                    const float alpha = pw[dir > 0 ? r - 16 * grp - 15 : 16 * grp - r];
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const float2 m = *reinterpret_cast<const float2*>(mu + 2 * u);
-                            const float2 w = mul2(m, make_float2(alpha, alpha));
-                            split_pack2v(mul2(make_float2(sv[16 * h2 + 2 * u], sv[16 * h2 + 2 * u + 1]), w),
-                                         pk[16 * h2 + u], pk[16 * h2 + 8 + u]);
-                        }
-                    } else if (kind == 1) {
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const int c0 = grp * 16 + 2 * u;
-                            const int lag0 = dir > 0 ? r - c0 : c0 - r;
-                            const int lag1 = dir > 0 ? r - c0 - 1 : c0 + 1 - r;
-                            const float p0 = lag0 >= 0 ? sv[16 * h2 + 2 * u] * pw[lag0 < 0 ? 0 : lag0] : 0.f;
-                            const float p1 =
-                                lag1 >= 0 ? sv[16 * h2 + 2 * u + 1] * pw[lag1 < 0 ? 0 : lag1] : 0.f;
-                            split_pack2(p0, p1, pk[16 * h2 + u], pk[16 * h2 + 8 + u]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int u = 0; u < 16; ++u) pk[16 * h2 + u] = 0u;
+                    for (int u = 0; u < 8; ++u) {
+                        const float2 m = *reinterpret_cast<const float2*>(mu + 2 * u);
+                        const float2 w = mul2(m, make_float2(alpha, alpha));
+                        const float2 pv = mul2(make_float2(sv[16 * h2 + 2 * u], sv[16 * h2 + 2 * u + 1]), w);
+                        sv[16 * h2 + 2 * u] = pv.x;
+                        sv[16 * h2 + 2 * u + 1] = pv.y;
                     }
                 }
-                tmem_st32u(st + lane_off + pr * 32, pk);
-                if (tid == 128 + 96 && pr == part) LA2_TR(26, s);
+            } else {
+#pragma unroll
+                for (int u = 0; u < 32; ++u) sv[u] = 0.f;
             }
-            if (tid == 128 + 96) LA2_TR(27, s);
+        };
+        for (int s = 0; s < ns; ++s) {
+            if constexpr (Q::kTf32) {
+                // C -> fp32 C^T (the K-major tf32 B operand of X += P C and dW): row r
+                // of C, columns 32 part .. 32 part + 31 (bf16 chunks 4 part + k), each
+                // to word r of row n of C^T; the lanes of a warp (consecutive r) fill
+                // one whole 128-byte row, so the scalar stores meet no bank conflict
+                const int sc = s % Q::NC, scf = s % Q::NCF;
+                if (!wait_bar(bar(Q::FULL_C + sc), full_par(s, Q::NC), abort_flag, p.status, 42)) break;
+                if (s >= Q::NCF && !wait_bar(bar(Q::EMPTY_CF + scf), empty_par(s, Q::NCF), abort_flag,
+                                             p.status, 43))
+                    break;
+                {
+                    const uint32_t src = sC + sc * L::kCsz, dst = sCF + scf * L::kCFsz + quad * (DC * 128);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        uint32_t v[4];
+                        ld_shared_v4(src + sw128(r, 4 * part + k), v[0], v[1], v[2], v[3]);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int n = 32 * part + 8 * k + 2 * u;
+                            st_shared_f32(dst + sw128(n, lane >> 2) + (lane & 3) * 4, bf16lo_to_f32(v[u]));
+                            st_shared_f32(dst + sw128(n + 1, lane >> 2) + (lane & 3) * 4, bf16hi_to_f32(v[u]));
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(bar(Q::EMPTY_C + sc));
+                mbar_arrive(bar(Q::CF_READY + scf));
+                // w_s B -> fp32 (w_s B)^T (the K-major tf32 A operand of dW), laid out
+                // like C^T; B itself is left for S
+                const int sb = s % Q::NB, swb = s % Q::NWB;
+                if (!wait_bar(bar(Q::FULL_B + sb), full_par(s, Q::NB), abort_flag, p.status, 44)) break;
+                if (s >= Q::NWB && !wait_bar(bar(Q::EMPTY_WB + swb), empty_par(s, Q::NWB), abort_flag,
+                                             p.status, 45))
+                    break;
+                {
+                    const uint32_t src = sB + sb * L::kBsz, dst = sWB + swb * L::kWBsz + quad * (DA * 128);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        uint32_t v[4];
+                        ld_shared_v4(src + sw128(r, 4 * part + k), v[0], v[1], v[2], v[3]);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float2 w = mul2(make_float2(bf16lo_to_f32(v[u]), bf16hi_to_f32(v[u])),
+                                                  make_float2(ws, ws));
+                            const int n = 32 * part + 8 * k + 2 * u;
+                            st_shared_f32(dst + sw128(n, lane >> 2) + (lane & 3) * 4, w.x);
+                            st_shared_f32(dst + sw128(n + 1, lane >> 2) + (lane & 3) * 4, w.y);
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(bar(Q::EMPTY_B + sb));
+                mbar_arrive(bar(Q::WB_READY + swb));
+                if (tid == 128) LA2_TR(10, s);
+                // P in place, fp32
+                if (!wait_bar(bar(Q::S_DONE + (s & 1)), full_par(s, 2), abort_flag, p.status, 40)) break;
+                if (tid == 128) LA2_TR(9, s);
+                tc_fence_after();
+                const uint32_t st = tS(s & 1);
+#pragma unroll 1
+                for (int pr = part; pr < kTB / 32; pr += 2) {
+                    float sv[32];
+                    tmem_ld32(st + lane_off + pr * 32, sv);
+                    weigh(pr, sv);
+                    tmem_st32(st + lane_off + pr * 32, sv);
+                }
+            } else {
+                if (!wait_bar(bar(Q::S_DONE + (s & 1)), full_par(s, 2), abort_flag, p.status, 40)) break;
+                if (tid == 128) LA2_TR(9, s);
+                const uint32_t st = tS(s & 1);
+                tc_fence_after();
+                // row r of w_s B (S, which reads B unscaled, is done): hi in place,
+                // lo into its own buffer once the dW that last read that buffer is
+                // done.  Part p does the chunks of half p of the row.
+                const int sl = s % Q::NBLO;
+                if (s >= Q::NBLO && !wait_bar(bar(Q::EMPTY_BLO + sl), empty_par(s, Q::NBLO), abort_flag,
+                                              p.status, 41))
+                    break;
+                const uint32_t sBs = sB + (s % Q::NB) * L::kBsz, sBl = sBlo + sl * L::kBsz;
+#pragma unroll
+                for (int k = 0; k < DA / 16; ++k) {
+                    const int chunk = part * (DA / 16) + k;
+                    const uint32_t off = (chunk >> 3) * 16384 + sw128(r, chunk & 7);
+                    uint32_t v[4], h[4], l[4];
+                    ld_shared_v4(sBs + off, v[0], v[1], v[2], v[3]);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        split_pack2v(mul2(make_float2(bf16lo_to_f32(v[u]), bf16hi_to_f32(v[u])),
+                                          make_float2(ws, ws)),
+                                     h[u], l[u]);
+                    st_shared_v4(sBs + off, h[0], h[1], h[2], h[3]);
+                    st_shared_v4(sBl + off, l[0], l[1], l[2], l[3]);
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(bar(Q::BS + (s % Q::NB)));
+                if (tid == 128) LA2_TR(10, s);
+                // P as hi + lo bf16, over the 16 columns of S each group of 16 came
+                // from: [hi (8 cols) | lo (8 cols)], the A-operand layout of one
+                // K = 16 step
+#pragma unroll 1
+                for (int pr = part; pr < kTB / 32; pr += 2) {
+                    float sv[32];
+                    tmem_ld32(st + lane_off + pr * 32, sv);
+                    weigh(pr, sv);
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            split_pack2v(make_float2(sv[16 * h2 + 2 * u], sv[16 * h2 + 2 * u + 1]),
+                                         pk[16 * h2 + u], pk[16 * h2 + 8 + u]);
+                    tmem_st32u(st + lane_off + pr * 32, pk);
+                }
+            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(Q::P_READY + (s & 1)));
             if (tid == 128) LA2_TR(11, s);
-            if (tid == 128 + 96) LA2_TR(30, s);
         }
     } else if (warp >= 12 && warp < 20) {
         // ================================================= epilogue group
@@ -581,13 +758,20 @@ la2_scan_ws(const __grid_constant__ Params p)
         const float lamTB = pw[kTB];
         const bool owns_w_row = (DA == 128) || (lane < 16);
         const int wrow = (DA == 128) ? r : quad * 16 + (lane & 15);
+        // With 32 columns per thread (DC = 64) each owner thread keeps its part
+        // of the state in fp32 registers; the hi/lo pair in shared memory is
+        // then written, never read back.
+        constexpr bool kWReg = kCols == 32;
+        float wreg[kWReg ? 32 : 1];
+#pragma unroll
+        for (int u = 0; u < (kWReg ? 32 : 1); ++u) wreg[u] = 0.f;
         // initial state of this segment, W_in(g) = f W_in(g-1) + S_{g-1} with
         // f = lambda^(T_B n), as its hi/lo bf16 pair in W buffer 0 (zero for the
         // first segment)
         if (g > 0 && owns_w_row) {
             const float f = static_cast<float>(
                 exp2(static_cast<double>(kTB) * p.seg_tiles * log2(static_cast<double>(lam))));
-#pragma unroll 1
+#pragma unroll
             for (int k = 0; k < kCols / 16; ++k) {
                 const uint32_t col = c0 + k * 16;
                 float w[16];
@@ -597,6 +781,10 @@ la2_scan_ws(const __grid_constant__ Params p)
                     const float* src = seg_slot(gp) + static_cast<size_t>(wrow) * DC + col;
 #pragma unroll
                     for (int u = 0; u < 16; ++u) w[u] = fmaf(f, w[u], src[u]);
+                }
+                if constexpr (kWReg) {
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) wreg[16 * (k & 1) + u] = w[u];
                 }
                 const uint32_t grpo = (col >> 6) * (DA * 128);
                 const int q = (col & 63) >> 3;
@@ -615,11 +803,11 @@ la2_scan_ws(const __grid_constant__ Params p)
 
         // X row r *= w_x(r) (the inter-tile term, still alone in X)
         auto scale = [&](int s) -> bool {
-            if (!wait_bar(bar(Q::XW_DONE + (s & 1)), full_par(s, 2), abort_flag, p.status, 50))
+            if (!wait_bar(bar(Q::XW_DONE + s % Q::NXW), full_par(s, Q::NXW), abort_flag, p.status, 50))
                 return false;
             if (tid == 384) LA2_TR(14, s);
             tc_fence_after();
-            const uint32_t xt = tX(s & 1);
+            const uint32_t xt = tX(s % Q::NX);
 #pragma unroll 1
             for (int k = 0; k < kCols / 32; ++k) {
                 float x[32];
@@ -631,7 +819,7 @@ la2_scan_ws(const __grid_constant__ Params p)
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(Q::XS + (s & 1)));
+            if constexpr (Q::NXS > 0) mbar_arrive(bar(Q::XS + s % Q::NXS));
             if (tid == 384) LA2_TR(15, s);
             return true;
         };
@@ -657,9 +845,31 @@ la2_scan_ws(const __grid_constant__ Params p)
                 if (tid == 384 && k == 0) LA2_TR(23, s);
                 if (Q::kOwnD && k == kCols / 32 - 1) {
                     tc_fence_before();
-                    mbar_arrive(bar(Q::EMPTY_D + (s & 1)));
+                    mbar_arrive(bar(Q::EMPTY_D + s % Q::ND));
                 }
-                if (owns_w_row) {
+                if (kWReg && owns_w_row) {
+                    const float2 lam2 = make_float2(lamTB, lamTB);
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const uint32_t col = c0 + hh * 16;
+                        const uint32_t o0 = (col >> 6) * (DA * 128) + sw128(wrow, (col & 63) >> 3);
+                        const uint32_t o1 = (col >> 6) * (DA * 128) + sw128(wrow, ((col & 63) >> 3) + 1);
+                        uint32_t h[8], l[8];
+#pragma unroll
+                        for (int z = 0; z < 8; ++z) {
+                            const int u = 16 * hh + 2 * z;
+                            const float2 w = fma2(lam2, make_float2(wreg[u], wreg[u + 1]),
+                                                  make_float2(d[u], d[u + 1]));
+                            wreg[u] = w.x;
+                            wreg[u + 1] = w.y;
+                            split_pack2v(w, h[z], l[z]);
+                        }
+                        st_shared_v4(wdst + o0, h[0], h[1], h[2], h[3]);
+                        st_shared_v4(wdst + o1, h[4], h[5], h[6], h[7]);
+                        st_shared_v4(wdst + L::kWsz + o0, l[0], l[1], l[2], l[3]);
+                        st_shared_v4(wdst + L::kWsz + o1, l[4], l[5], l[6], l[7]);
+                    }
+                } else if (owns_w_row) {
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         const uint32_t col = c0 + k * 32 + hh * 16;
@@ -698,23 +908,51 @@ la2_scan_ws(const __grid_constant__ Params p)
         // so every float2 store of a warp fills whole 32-byte sectors (eight
         // rows per instruction).  The X buffer is released once read.
         auto output = [&](int s) -> bool {
-            if (!wait_bar(bar(Q::PC_DONE + (s & 1)), full_par(s, 2), abort_flag, p.status, 53))
+            if (!wait_bar(bar(Q::PC_DONE + s % Q::NX), full_par(s, Q::NX), abort_flag, p.status, 53))
+                return false;
+            if (Q::kOwnD &&
+                !wait_bar(bar(Q::XW_DONE + s % Q::NXW), full_par(s, Q::NXW), abort_flag, p.status, 54))
                 return false;
             if (tid == 384) LA2_TR(16, s);
             tc_fence_after();
             const int i = tile_of(s);
-            const uint32_t xt = tX(s & 1);
+            const uint32_t xt = tX(s % Q::NX);
             const int t4 = lane >> 2, tm = lane & 3;
             const uint32_t l0 = static_cast<uint32_t>(quad * 32) << 16;
             const uint32_t l1 = static_cast<uint32_t>(quad * 32 + 16) << 16;
+            // w_x of the four rows this thread holds (lane halves lh, rows +0 / +8)
+            float wxr[4];
+            if constexpr (Q::kOwnD) {
+#pragma unroll
+                for (int lh = 0; lh < 2; ++lh)
+#pragma unroll
+                    for (int h8 = 0; h8 < 2; ++h8) {
+                        const int rr = quad * 32 + lh * 16 + t4 + 8 * h8;
+                        wxr[2 * lh + h8] = dir > 0 ? pw[rr + 1] : pw[kTB - rr];
+                    }
+            }
 #pragma unroll 1
             for (int b = 0; b < kCols / 32; ++b) {
                 float v[32];
                 const uint32_t col = c0 + 32 * b;
                 tmem_ld16x256b_x4_pair(xt + l0 + col, xt + l1 + col, v);
+                if constexpr (Q::kOwnD) {
+                    float vi[32];
+                    tmem_ld16x256b_x4_pair(tXI + l0 + col, tXI + l1 + col, vi);
+#pragma unroll
+                    for (int lh = 0; lh < 2; ++lh)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int idx = 16 * lh + 4 * j + e;
+                                v[idx] = fmaf(wxr[2 * lh + (e >> 1)], vi[idx], v[idx]);
+                            }
+                }
                 if (b == kCols / 32 - 1) {
                     tc_fence_before();
-                    mbar_arrive(bar(Q::EMPTY_X + (s & 1)));
+                    mbar_arrive(bar(Q::EMPTY_X + s % Q::NX));
+                    if constexpr (Q::NXI > 0) mbar_arrive(bar(Q::EMPTY_XI));
                 }
 #pragma unroll
                 for (int lh = 0; lh < 2; ++lh) {
@@ -736,12 +974,13 @@ la2_scan_ws(const __grid_constant__ Params p)
         };
 
         if (Q::kOwnD) {
-            // dW has its own buffers, so X of a tile can be written out one step
-            // later, while X += P C of the next tile is still being issued
+            // separate accumulators, no scaling in TMEM: X of tile s-1 is
+            // written out (which frees X_inter for the next A W), then the state
+            // update of tile s
             bool ok = true;
             for (int s = 0; s < ns && ok; ++s) {
-                ok = scale(s) && update(s);
-                if (ok && s > 0) ok = output(s - 1);
+                if (s > 0) ok = output(s - 1);
+                ok = ok && update(s);
             }
             if (ok && ns > 0) output(ns - 1);
         } else {

@@ -119,8 +119,10 @@ def test_bf16_mixed_decays_in_one_launch(la2mod, oracle_mod, B, T, d, e):
     x = I.make_inputs(B, 7, T, d, e, "bf16", seed=11 + T)
     x["lam"] = torch.tensor([0.3, 0.8, 0.841, 0.843, 0.9, 0.99, 1.0], dtype=torch.float32)
     errs = _check(la2mod, oracle_mod, x, 128, TOL["bf16"])
-    # the hi/lo operand splits keep the kernel far below the bf16 bar
-    assert max(errs.values()) < 1e-3, errs
+    # Far below the bf16 bar in both operand modes: with d = e = 64 the decayed
+    # P and w_s B enter the tensor cores as tf32 (about 2^-11 relative each),
+    # otherwise as bf16 hi + lo pairs (about 2^-17)
+    assert max(errs.values()) < (4e-3 if d == e == 64 else 1e-3), errs
 
 
 def test_bf16_tiny_decay_keeps_only_diagonal(la2mod, oracle_mod):
