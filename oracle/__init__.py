@@ -54,6 +54,8 @@ def _load():
         lib.la2o_backward.argtypes = [i, i, i, i, dp, dp, dp, dp, dp, dp, dp, dp, i]
         lib.la2o_forward_blocked.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, i]
         lib.la2o_backward_blocked.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp, dp, i]
+        lib.la2o_forward_state.argtypes = [i, i, i, i, dp, dp, dp, dp, dp, dp, dp, i]
+        lib.la2o_decode_step.argtypes = [i, i, i, dp, dp, dp, dp, dp, dp]
         lib.la2o_max_threads.restype = i
         _lib = lib
     return _lib
@@ -102,6 +104,39 @@ def forward(q, k, v, lam, nthreads: int = 0) -> np.ndarray:
                          _ptr(oc), int(nthreads))
         out[a:b] = oc
     return out.reshape(*lead, T, e)
+
+
+def forward_state(q, k, v, lam, s0=None, nthreads: int = 0):
+    """(o, S_T): the forward recurrence started from the state s0 ([..., d, e];
+    None = zero) instead of zero, and the state after the last position."""
+    lib = _load()
+    lead, ns, T, d, e, lam = _prep(q, k, v, lam)
+    qc, kc, vc = (_f64(x).reshape(ns, T, -1) for x in (q, k, v))
+    out = np.empty((ns, T, e), dtype=np.float64)
+    sT = np.empty((ns, d, e), dtype=np.float64)
+    s0p = None
+    if s0 is not None:
+        s0c = _f64(s0).reshape(ns, d, e)
+        s0p = _ptr(s0c)
+    lib.la2o_forward_state(ns, T, d, e, _ptr(lam), _ptr(qc), _ptr(kc), _ptr(vc), s0p, _ptr(out),
+                           _ptr(sT), int(nthreads))
+    return out.reshape(*lead, T, e), sT.reshape(*lead, d, e)
+
+
+def decode_step(q, k, v, lam, state):
+    """(o, S'): one new token per sequence, q, k [..., d], v [..., e], state
+    [..., d, e]: S' = lam S + k v^T, o = S'^T q.  The input state is not modified."""
+    lib = _load()
+    q = _f64(q)
+    lead = tuple(q.shape[:-1])
+    d, e = int(q.shape[-1]), int(np.asarray(v).shape[-1])
+    ns = int(np.prod(lead)) if lead else 1
+    lamv = np.ascontiguousarray(np.broadcast_to(np.asarray(lam, dtype=np.float64), lead).reshape(ns))
+    qc, kc, vc = q.reshape(ns, d), _f64(k).reshape(ns, d), _f64(v).reshape(ns, e)
+    S = _f64(state).reshape(ns, d, e).copy()
+    o = np.empty((ns, e), dtype=np.float64)
+    lib.la2o_decode_step(ns, d, e, _ptr(lamv), _ptr(qc), _ptr(kc), _ptr(vc), _ptr(S), _ptr(o))
+    return o.reshape(*lead, e), S.reshape(*lead, d, e)
 
 
 def backward(q, k, v, lam, dout, nthreads: int = 0):

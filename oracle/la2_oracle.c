@@ -37,6 +37,13 @@
  *                             inter weight   lambda^(r+1) on row r
  *                             state update   KV <- lambda^TB KV
  *                                                  + sum_r lambda^(TB-1-r) k_r v_r^T
+ *   la2o_forward_state      la2o_forward from a given state: S_{-1} = S0 instead
+ *                           of 0, and the state after the last token returned
+ *                           (the state is the only thing a sequence carries,
+ *                           section 2 "Memory footprint", so a long sequence
+ *                           can be processed in consecutive pieces).
+ *   la2o_decode_step        one step of the same recurrence for one new token
+ *                           per sequence: S <- lambda S + k v^T, o = S^T q.
  *   la2o_backward_blocked   the mirrored tiling for the backward (the pages say
  *                           only that tiling covers the backward too): dq by a
  *                           forward-direction blocked scan, dk and dv by a
@@ -107,6 +114,52 @@ void la2o_forward(int NS, int T, int d, int e, const double *lam,
                 for (int j = 0; j < e; ++j) ot[j] += qt[i] * S[(size_t)i * e + j];
         }
         free(S);
+    }
+}
+
+/* ------------------------------------------------- state in / state out */
+
+void la2o_forward_state(int NS, int T, int d, int e, const double *lam,
+                        const double *q, const double *k, const double *v,
+                        const double *s0, double *o, double *sT, int nthreads)
+{
+    set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < NS; ++n) {
+        const double *qn = q + (size_t)n * T * d;
+        const double *kn = k + (size_t)n * T * d;
+        const double *vn = v + (size_t)n * T * e;
+        double *on = o + (size_t)n * T * e;
+        double *S = sT + (size_t)n * d * e; /* S[i][j], starts as S0 (or 0) */
+        if (s0) memcpy(S, s0 + (size_t)n * d * e, sizeof(double) * (size_t)d * e);
+        else memset(S, 0, sizeof(double) * (size_t)d * e);
+        const double l = lam[n];
+        for (int t = 0; t < T; ++t) {
+            const double *qt = qn + (size_t)t * d, *kt = kn + (size_t)t * d;
+            const double *vt = vn + (size_t)t * e;
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < e; ++j)
+                    S[(size_t)i * e + j] = l * S[(size_t)i * e + j] + kt[i] * vt[j];
+            double *ot = on + (size_t)t * e;
+            for (int j = 0; j < e; ++j) ot[j] = 0.0;
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < e; ++j) ot[j] += qt[i] * S[(size_t)i * e + j];
+        }
+    }
+}
+
+void la2o_decode_step(int NS, int d, int e, const double *lam, const double *q,
+                      const double *k, const double *v, double *S, double *o)
+{
+    for (int n = 0; n < NS; ++n) {
+        const double *qn = q + (size_t)n * d, *kn = k + (size_t)n * d, *vn = v + (size_t)n * e;
+        double *Sn = S + (size_t)n * d * e, *on = o + (size_t)n * e;
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < e; ++j)
+                Sn[(size_t)i * e + j] = lam[n] * Sn[(size_t)i * e + j] + kn[i] * vn[j];
+        for (int j = 0; j < e; ++j) on[j] = 0.0;
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < e; ++j) on[j] += qn[i] * Sn[(size_t)i * e + j];
     }
 }
 

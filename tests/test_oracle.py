@@ -198,3 +198,70 @@ def test_sequences_are_independent_and_use_their_own_decay(oracle_mod):
     for n in range(4):
         alone = oracle_mod.forward(q[n:n + 1], k[n:n + 1], v[n:n + 1], lam[n:n + 1])
         np.testing.assert_array_equal(together[n], alone[0])
+
+
+# ------------------------------------------------------- state in / state out
+
+def _state_closed_form(q, k, v, lam, s0):
+    """o_t = lam^(t+1) S0^T q_t + sum_{s<=t} lam^(t-s) (q_t . k_s) v_s and
+    S_T = lam^T S0 + sum_s lam^(T-1-s) k_s v_s^T, written out directly."""
+    T = q.shape[0]
+    D = _decay_matrix(T, lam)
+    t = np.arange(T)
+    o = ((q @ k.T) * D) @ v + (lam ** (t + 1))[:, None] * (q @ s0)
+    w = lam ** (T - 1 - t)
+    sT = lam ** T * s0 + (k * w[:, None]).T @ v
+    return o, sT
+
+
+@pytest.mark.parametrize("T,d,e", [(1, 3, 2), (9, 4, 5), (40, 8, 3)])
+def test_forward_state_closed_form(oracle_mod, T, d, e):
+    rng = np.random.default_rng(77 + T)
+    for lam in LAMS:
+        q, k, v = _rand(rng, T, d), _rand(rng, T, d), _rand(rng, T, e)
+        s0 = _rand(rng, d, e)
+        o, sT = oracle_mod.forward_state(q, k, v, lam, s0)
+        ro, rs = _state_closed_form(q, k, v, lam, s0)
+        assert _rel(o, ro) < 1e-12 and _rel(sT, rs) < 1e-12, lam
+        # no initial state: the plain forward, and the state from zero
+        o0, s00 = oracle_mod.forward_state(q, k, v, lam)
+        ro0, rs0 = _state_closed_form(q, k, v, lam, np.zeros((d, e)))
+        assert _rel(o0, ro0) < 1e-12 and _rel(s00, rs0) < 1e-12
+
+
+@pytest.mark.parametrize("cut", [1, 7, 13, 29])
+def test_forward_state_pieces_equal_whole(oracle_mod, cut):
+    """Processing [0, cut) and then [cut, T) from the carried state gives the
+    outputs and final state of the whole sequence (the state is all that is
+    carried)."""
+    rng = np.random.default_rng(5 + cut)
+    T, d, e = 30, 5, 4
+    q, k, v = _rand(rng, 3, T, d), _rand(rng, 3, T, d), _rand(rng, 3, T, e)
+    lam = np.array([1.0, 0.9, 0.3])
+    o1, s1 = oracle_mod.forward_state(q[:, :cut], k[:, :cut], v[:, :cut], lam)
+    o2, s2 = oracle_mod.forward_state(q[:, cut:], k[:, cut:], v[:, cut:], lam, s1)
+    o, s = oracle_mod.forward_state(q, k, v, lam)
+    assert _rel(np.concatenate([o1, o2], axis=1), o) < 1e-12
+    assert _rel(s2, s) < 1e-12
+
+
+def test_decode_steps_reproduce_the_forward(oracle_mod):
+    """T one-token decode steps from a state S0 give the forward's outputs and
+    final state from S0."""
+    rng = np.random.default_rng(11)
+    T, d, e = 12, 4, 6
+    q, k, v = _rand(rng, 2, T, d), _rand(rng, 2, T, d), _rand(rng, 2, T, e)
+    lam = np.array([0.95, 1.0])
+    s0 = _rand(rng, 2, d, e)
+    o, sT = oracle_mod.forward_state(q, k, v, lam, s0)
+    S = s0.copy()
+    outs = []
+    for t in range(T):
+        ot, S = oracle_mod.decode_step(q[:, t], k[:, t], v[:, t], lam, S)
+        outs.append(ot)
+    assert _rel(np.stack(outs, axis=1), o) < 1e-12
+    assert _rel(S, sT) < 1e-12
+    # one step by hand: S' = lam S + k v^T, o = S'^T q
+    o1, S1 = oracle_mod.decode_step(q[0, 0], k[0, 0], v[0, 0], lam[0], s0[0])
+    Sh = lam[0] * s0[0] + np.outer(k[0, 0], v[0, 0])
+    assert _rel(S1, Sh) < 1e-14 and _rel(o1, Sh.T @ q[0, 0]) < 1e-14
