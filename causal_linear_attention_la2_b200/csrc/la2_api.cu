@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "decode.cuh"
 #include "la2.h"
 #include "scan_f32.cuh"
 #include "scan_ws_sm100.cuh"
@@ -145,6 +146,8 @@ struct RoleDesc {
     const void* c;
     void* x;
     int da, dc, dir;
+    const float* init = nullptr;  // forward role only: state before position 0
+    float* fin = nullptr;         // forward role only: state after position T-1
 };
 
 la2_status common_checks(int B, int H, int T, int d, int e, int block, la2_dtype dtype,
@@ -189,6 +192,8 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
             !make_map(&p.role[r].tc, roles[r].c, BH, T, dc, false))
             return LA2_ERR_CUDA;
         p.role[r].x = static_cast<float*>(roles[r].x);
+        p.role[r].init = roles[r].init;
+        p.role[r].fin = roles[r].fin;
         p.role[r].dir = roles[r].dir;
     }
     p.decay = decay;
@@ -224,6 +229,8 @@ la2_status launch_f32(const RoleDesc* roles, int n, const float* decay, int B, i
         p.role[r].da = roles[r].da;
         p.role[r].dc = roles[r].dc;
         p.role[r].dir = roles[r].dir;
+        p.role[r].init = roles[r].init;
+        p.role[r].fin = roles[r].fin;
         da_max = roles[r].da > da_max ? roles[r].da : da_max;
         dc_max = roles[r].dc > dc_max ? roles[r].dc : dc_max;
     }
@@ -306,21 +313,44 @@ size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block, la2_dty
     return is_bwd ? bf16_workspace_bytes(bwd, 3, B, H) : bf16_workspace_bytes(fwd, 1, B, H);
 }
 
-la2_status la2_fwd(const void* q, const void* k, const void* v, const float* decay, void* out,
-                   int B, int H, int T, int d, int e, int block, la2_dtype dtype,
-                   void* workspace, size_t workspace_bytes, la2_stream_t stream) {
+la2_status la2_fwd_state(const void* q, const void* k, const void* v, const float* decay,
+                         void* out, const float* init_state, float* final_state, int B, int H,
+                         int T, int d, int e, int block, la2_dtype dtype, void* workspace,
+                         size_t workspace_bytes, la2_stream_t stream) {
     t_last_launches = 0;
     bool empty = false;
     la2_status st = common_checks(B, H, T, d, e, block, dtype, &empty);
-    if (st != LA2_OK || empty) return st;
+    if (st != LA2_OK) return st;
+    if (empty) {
+        // no position to process: the final state is the initial one (or 0)
+        if (final_state && B > 0 && H > 0) {
+            const size_t n = static_cast<size_t>(B) * H * d * e * sizeof(float);
+            const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+            const cudaError_t err =
+                init_state ? cudaMemcpyAsync(final_state, init_state, n, cudaMemcpyDeviceToDevice, cs)
+                           : cudaMemsetAsync(final_state, 0, n, cs);
+            if (err != cudaSuccess) return LA2_ERR_CUDA;
+        }
+        return LA2_OK;
+    }
     if (!q || !k || !v || !decay || !out) return LA2_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
-        (reinterpret_cast<uintptr_t>(decay) & 3u))
+        (reinterpret_cast<uintptr_t>(decay) & 3u) ||
+        (reinterpret_cast<uintptr_t>(init_state) & 3u) || (reinterpret_cast<uintptr_t>(final_state) & 3u))
         return LA2_ERR_INVALID_ARG;
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return LA2_ERR_INVALID_ARG;
-    const RoleDesc r = {q, k, v, out, d, e, +1};
+    RoleDesc r = {q, k, v, out, d, e, +1};
+    r.init = init_state;
+    r.fin = final_state;
     return run_roles(&r, 1, decay, B, H, T, block, dtype, workspace, workspace_bytes,
                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+la2_status la2_fwd(const void* q, const void* k, const void* v, const float* decay, void* out,
+                   int B, int H, int T, int d, int e, int block, la2_dtype dtype,
+                   void* workspace, size_t workspace_bytes, la2_stream_t stream) {
+    return la2_fwd_state(q, k, v, decay, out, nullptr, nullptr, B, H, T, d, e, block, dtype,
+                         workspace, workspace_bytes, stream);
 }
 
 la2_status la2_bwd(const void* q, const void* k, const void* v, const float* decay,
@@ -344,6 +374,52 @@ la2_status la2_bwd(const void* q, const void* k, const void* v, const float* dec
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return LA2_ERR_INVALID_ARG;
     return run_roles(roles, 3, decay, B, H, T, block, dtype, workspace, workspace_bytes,
                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+la2_status la2_decode(const void* q, const void* k, const void* v, const float* decay,
+                      float* state, float* out, int B, int H, int d, int e, la2_dtype dtype,
+                      la2_stream_t stream) {
+    t_last_launches = 0;
+    if (dtype != LA2_DTYPE_F32 && dtype != LA2_DTYPE_BF16) return LA2_ERR_INVALID_ARG;
+    if (B < 0 || H < 0 || d <= 0 || e <= 0) return LA2_ERR_INVALID_ARG;
+    if (B == 0 || H == 0) return LA2_OK;
+    if (d > 4096 || e > 4096) return LA2_ERR_UNSUPPORTED;
+    if (static_cast<long long>(B) * H > (1LL << 30)) return LA2_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !decay || !state || !out) return LA2_ERR_INVALID_ARG;
+    const size_t esz = dtype == LA2_DTYPE_BF16 ? 2 : 4;
+    const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                          reinterpret_cast<uintptr_t>(v);
+    if ((mis & (esz - 1)) || (reinterpret_cast<uintptr_t>(decay) & 3u) ||
+        (reinterpret_cast<uintptr_t>(state) & 3u) || (reinterpret_cast<uintptr_t>(out) & 3u))
+        return LA2_ERR_INVALID_ARG;
+    const bool vec = (e % 4 == 0) && !(reinterpret_cast<uintptr_t>(state) & 15u);
+    const dim3 grid(static_cast<unsigned>(B * H));
+    const size_t smem = la2::decode_smem_bytes(d);
+    const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == LA2_DTYPE_BF16) {
+        const auto* qb = static_cast<const __nv_bfloat16*>(q);
+        const auto* kb = static_cast<const __nv_bfloat16*>(k);
+        const auto* vb = static_cast<const __nv_bfloat16*>(v);
+        if (vec)
+            la2::la2_decode_kernel<__nv_bfloat16, true><<<grid, la2::kDecThreads, smem, cs>>>(
+                qb, kb, vb, decay, state, out, H, d, e);
+        else
+            la2::la2_decode_kernel<__nv_bfloat16, false><<<grid, la2::kDecThreads, smem, cs>>>(
+                qb, kb, vb, decay, state, out, H, d, e);
+    } else {
+        const auto* qf = static_cast<const float*>(q);
+        const auto* kf = static_cast<const float*>(k);
+        const auto* vf = static_cast<const float*>(v);
+        if (vec)
+            la2::la2_decode_kernel<float, true><<<grid, la2::kDecThreads, smem, cs>>>(
+                qf, kf, vf, decay, state, out, H, d, e);
+        else
+            la2::la2_decode_kernel<float, false><<<grid, la2::kDecThreads, smem, cs>>>(
+                qf, kf, vf, decay, state, out, H, d, e);
+    }
+    if (cudaGetLastError() != cudaSuccess) return LA2_ERR_CUDA;
+    t_last_launches = 1;
+    return LA2_OK;
 }
 
 const char* la2_status_str(la2_status s) {

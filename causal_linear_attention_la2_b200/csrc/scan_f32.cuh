@@ -19,7 +19,9 @@ struct F32Role {
     const float* b;  // [BH, T, DA]
     const float* c;  // [BH, T, DC]
     float* x;        // [BH, T, DC]
-    int da, dc, dir;
+    const float* init;  // [BH, DA, DC] state before the first position, or null (0)
+    float* fin;         // [BH, DA, DC] state after the last position, or null
+    int da, dc, dir;    // init and fin are used with dir = +1 only
 };
 
 struct F32Params {
@@ -53,7 +55,8 @@ la2_scan_f32(const __grid_constant__ F32Params p)
     const double lam = static_cast<double>(p.decay[bh % p.H]);
     const double l2 = log2(lam);
     for (int n = tid; n <= TB; n += kF32Threads) pw[n] = static_cast<float>(exp2(n * l2));
-    for (int z = tid; z < da * dc; z += kF32Threads) W[z] = 0.f;
+    for (int z = tid; z < da * dc; z += kF32Threads)
+        W[z] = R.init ? R.init[static_cast<size_t>(bh) * da * dc + z] : 0.f;
 
     const float* a = R.a + static_cast<size_t>(bh) * T * da;
     const float* b = R.b + static_cast<size_t>(bh) * T * da;
@@ -138,14 +141,18 @@ la2_scan_f32(const __grid_constant__ F32Params p)
             __syncthreads();
         }
 
-        // state update with the unmasked tile: W <- lambda^TB W + sum_c w_s(c) b_c c_c^T
-        const float lTB = pw[TB];
+        // state update with the unmasked tile: W <- lambda^TB W + sum_c w_s(c) b_c c_c^T.
+        // A forward scan's last tile may be short (len < TB rows): its exponents
+        // are taken from len, so that W is then the state after position T-1
+        // (no output reads it; the final state does).
+        const int tl = dir > 0 ? len : TB;
+        const float lTB = pw[tl];
         for (int z = tid; z < da * dc; z += kF32Threads) W[z] *= lTB;
         for (int kb = 0; kb < nsub; ++kb) {
             __syncthreads();
             for (int z = tid; z < kF32Sub * da; z += kF32Threads) {
                 const int rr = z / da, u = z % da, loc = kb * kF32Sub + rr;
-                const float ws = loc < len ? (dir > 0 ? pw[TB - 1 - loc] : pw[loc]) : 0.f;
+                const float ws = loc < len ? (dir > 0 ? pw[tl - 1 - loc] : pw[loc]) : 0.f;
                 Bs[z] = loc < len ? ws * b[static_cast<size_t>(t0 + loc) * da + u] : 0.f;
             }
             for (int z = tid; z < kF32Sub * dc; z += kF32Threads) {
@@ -162,6 +169,8 @@ la2_scan_f32(const __grid_constant__ F32Params p)
         }
         __syncthreads();
     }
+    if (R.fin)
+        for (int z = tid; z < da * dc; z += kF32Threads) R.fin[static_cast<size_t>(bh) * da * dc + z] = W[z];
 }
 
 }  // namespace la2

@@ -65,7 +65,9 @@ constexpr uint32_t kTmemCols = 512;
 struct Role {
     CUtensorMap ta, tb, tc;  // a, b: [B*H, T, DA]; c: [B*H, T, DC]; bf16, box 64 x 128
     float* x;                // [B*H, T, DC] fp32
-    int dir;                 // +1 or -1
+    const float* init;       // [B*H, DA, DC] fp32 state before the first position, or null (0)
+    float* fin;              // [B*H, DA, DC] fp32 state after the last position, or null
+    int dir;                 // +1 or -1 (init and fin are used with +1 only)
 };
 
 struct Params {
@@ -585,6 +587,15 @@ la2_scan_ws(const __grid_constant__ Params p)
         const int zs = dir > 0 ? lane : 31 - lane;
         const uint32_t zwin = base + L::kZ + (zs & 3) * L::kZstride + (zs - (zs & 3)) * 4;
         const float* mu = dir > 0 ? murev : pw;
+        // The last tile of a forward scan may hold n < T_B rows: its state
+        // update then uses lambda^(n-1-r) (and lambda^n for the old state), so
+        // that the state after it is the state after position T-1 exactly.  No
+        // output reads that state; only the final state does.
+        const int nlast = T - (nb - 1) * kTB;
+        const float ws_last = r < nlast ? pw[max(nlast - 1 - r, 0)] : 0.f;
+        auto ws_of = [&](int s) {
+            return (dir > 0 && g == p.nseg - 1 && s == ns - 1) ? ws_last : ws;
+        };
         // P = S * lambda^|r-c| on the causal side, 0 elsewhere, 32 columns (one
         // pair of K = 16 groups) at a time.  pr == quad is the diagonal block;
         // whole pairs on the causal side use lambda^|r-c| = alpha mu(c), with
@@ -663,6 +674,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                                              p.status, 45))
                     break;
                 {
+                    const float ws_s = ws_of(s);
                     const uint32_t src = sB + sb * L::kBsz, dst = sWB + swb * L::kWBsz + quad * (DA * 128);
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
@@ -671,7 +683,7 @@ la2_scan_ws(const __grid_constant__ Params p)
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             const float2 w = mul2(make_float2(bf16lo_to_f32(v[u]), bf16hi_to_f32(v[u])),
-                                                  make_float2(ws, ws));
+                                                  make_float2(ws_s, ws_s));
                             const int n = 32 * part + 8 * k + 2 * u;
                             st_shared_f32(dst + sw128(n, lane >> 2) + (lane & 3) * 4, w.x);
                             st_shared_f32(dst + sw128(n + 1, lane >> 2) + (lane & 3) * 4, w.y);
@@ -707,6 +719,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                                               p.status, 41))
                     break;
                 const uint32_t sBs = sB + (s % Q::NB) * L::kBsz, sBl = sBlo + sl * L::kBsz;
+                const float ws_s = ws_of(s);
 #pragma unroll
                 for (int k = 0; k < DA / 16; ++k) {
                     const int chunk = part * (DA / 16) + k;
@@ -716,7 +729,7 @@ la2_scan_ws(const __grid_constant__ Params p)
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
                         split_pack2v(mul2(make_float2(bf16lo_to_f32(v[u]), bf16hi_to_f32(v[u])),
-                                          make_float2(ws, ws)),
+                                          make_float2(ws_s, ws_s)),
                                      h[u], l[u]);
                     st_shared_v4(sBs + off, h[0], h[1], h[2], h[3]);
                     st_shared_v4(sBl + off, l[0], l[1], l[2], l[3]);
@@ -766,17 +779,19 @@ la2_scan_ws(const __grid_constant__ Params p)
 #pragma unroll
         for (int u = 0; u < (kWReg ? 32 : 1); ++u) wreg[u] = 0.f;
         // initial state of this segment, W_in(g) = f W_in(g-1) + S_{g-1} with
-        // f = lambda^(T_B n), as its hi/lo bf16 pair in W buffer 0 (zero for the
-        // first segment)
-        if (g > 0 && owns_w_row) {
+        // f = lambda^(T_B n) and W_in(0) the given initial state (or 0), as its
+        // hi/lo bf16 pair in W buffer 0
+        if ((g > 0 || R.init != nullptr) && owns_w_row) {
             const float f = static_cast<float>(
                 exp2(static_cast<double>(kTB) * p.seg_tiles * log2(static_cast<double>(lam))));
+            const float* w0 =
+                R.init ? R.init + static_cast<size_t>(bh) * (DA * DC) + static_cast<size_t>(wrow) * DC : nullptr;
 #pragma unroll
             for (int k = 0; k < kCols / 16; ++k) {
                 const uint32_t col = c0 + k * 16;
                 float w[16];
 #pragma unroll
-                for (int u = 0; u < 16; ++u) w[u] = 0.f;
+                for (int u = 0; u < 16; ++u) w[u] = w0 ? w0[col + u] : 0.f;
                 for (int gp = 0; gp < g; ++gp) {
                     const float* src = seg_slot(gp) + static_cast<size_t>(wrow) * DC + col;
 #pragma unroll
@@ -826,7 +841,14 @@ la2_scan_ws(const __grid_constant__ Params p)
         // W <- lambda^T_B W + dW, from W buffer s % NW into (s+1) % NW.  The
         // state is kept as its hi + lo bf16 pair (a 16-bit significand, ~2^-17
         // relative per update), which is also the next tile's MMA operand.
+        const bool has_last = dir > 0 && g == p.nseg - 1;
+        const int nlast = T - (nb - 1) * kTB;
         auto update = [&](int s) -> bool {
+            const bool last = has_last && s == ns - 1;
+            const float lam_s = last ? pw[nlast] : lamTB;
+            float* fin = (last && R.fin) ? R.fin + static_cast<size_t>(bh) * (DA * DC) +
+                                               static_cast<size_t>(wrow) * DC
+                                         : nullptr;
             if (!wait_bar(bar(Q::D_DONE + (s % Q::ND)), full_par(s, Q::ND), abort_flag, p.status, 51))
                 return false;
             // the X MMA that last read the W buffer written here is done
@@ -848,7 +870,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                     mbar_arrive(bar(Q::EMPTY_D + s % Q::ND));
                 }
                 if (kWReg && owns_w_row) {
-                    const float2 lam2 = make_float2(lamTB, lamTB);
+                    const float2 lam2 = make_float2(lam_s, lam_s);
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         const uint32_t col = c0 + hh * 16;
@@ -862,6 +884,10 @@ la2_scan_ws(const __grid_constant__ Params p)
                                                   make_float2(d[u], d[u + 1]));
                             wreg[u] = w.x;
                             wreg[u + 1] = w.y;
+                            if (fin) {
+                                fin[col + 2 * z] = w.x;
+                                fin[col + 2 * z + 1] = w.y;
+                            }
                             split_pack2v(w, h[z], l[z]);
                         }
                         st_shared_v4(wdst + o0, h[0], h[1], h[2], h[3]);
@@ -882,10 +908,14 @@ la2_scan_ws(const __grid_constant__ Params p)
                         ld_shared_v4(wsrc + L::kWsz + o1, l[4], l[5], l[6], l[7]);
 #pragma unroll
                         for (int z = 0; z < 8; ++z) {
-                            const float w0 = fmaf(lamTB, bf16lo_to_f32(h[z]) + bf16lo_to_f32(l[z]),
+                            const float w0 = fmaf(lam_s, bf16lo_to_f32(h[z]) + bf16lo_to_f32(l[z]),
                                                   d[16 * hh + 2 * z]);
-                            const float w1 = fmaf(lamTB, bf16hi_to_f32(h[z]) + bf16hi_to_f32(l[z]),
+                            const float w1 = fmaf(lam_s, bf16hi_to_f32(h[z]) + bf16hi_to_f32(l[z]),
                                                   d[16 * hh + 2 * z + 1]);
+                            if (fin) {
+                                fin[col + 2 * z] = w0;
+                                fin[col + 2 * z + 1] = w1;
+                            }
                             split_pack2(w0, w1, h[z], l[z]);
                         }
                         st_shared_v4(wdst + o0, h[0], h[1], h[2], h[3]);

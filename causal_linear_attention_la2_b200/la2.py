@@ -26,8 +26,8 @@ LA2_DTYPE_F32 = 0
 LA2_DTYPE_BF16 = 1
 
 # Every entry point include/la2.h declares.
-EXPORTS = ("la2_workspace_bytes", "la2_fwd", "la2_bwd", "la2_status_str", "la2_device_status",
-           "la2_last_launch_count", "la2_fwd_noalloc")
+EXPORTS = ("la2_workspace_bytes", "la2_fwd", "la2_fwd_state", "la2_bwd", "la2_decode",
+           "la2_status_str", "la2_device_status", "la2_last_launch_count", "la2_fwd_noalloc")
 
 
 class LA2Error(RuntimeError):
@@ -53,8 +53,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la2_workspace_bytes.restype = sz
     lib.la2_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
     lib.la2_fwd.restype = i
+    lib.la2_fwd_state.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
+    lib.la2_fwd_state.restype = i
     lib.la2_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
     lib.la2_bwd.restype = i
+    lib.la2_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+    lib.la2_decode.restype = i
     lib.la2_status_str.argtypes = [i]
     lib.la2_status_str.restype = ctypes.c_char_p
     lib.la2_device_status.argtypes = [ctypes.POINTER(ctypes.c_int), i]
@@ -177,6 +181,70 @@ def la2_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, decay: torch.Tens
                      B, H, T, d, e, block, dt, wp, wn, _stream_ptr(stream))
     if st != LA2_OK:
         raise LA2Error(st, "la2_fwd")
+    return out
+
+
+def la2_fwd_state_raw(q, k, v, decay, out, init_state, final_state, B, H, T, d, e, block, dtype,
+                      workspace=0, ws_bytes=0, stream=0) -> int:
+    """The C call with integer pointers (0 = NULL for the states); returns the status."""
+    return int(load().la2_fwd_state(q, k, v, decay, out, init_state, final_state, B, H, T, d, e,
+                                    block, dtype, workspace, ws_bytes, stream))
+
+
+def la2_fwd_state(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, decay: torch.Tensor,
+                  init_state: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                  final_state: torch.Tensor | None = None, block: int = 128, stream=None,
+                  workspace: torch.Tensor | None = None):
+    """(out, final_state): la2_fwd started from init_state ([B, H, d, e] fp32, None = 0),
+    returning the state after the last position as well."""
+    B, H, T, d = q.shape
+    e = v.shape[-1]
+    dt = _dtype_code(q)
+    _check(q, "q", (B, H, T, d), q.dtype)
+    _check(k, "k", (B, H, T, d), q.dtype)
+    _check(v, "v", (B, H, T, e), q.dtype)
+    _check(decay, "decay", (H,), torch.float32)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    out = torch.empty((B, H, T, e), **f32) if out is None else out
+    final_state = torch.empty((B, H, d, e), **f32) if final_state is None else final_state
+    _check(out, "out", (B, H, T, e), torch.float32)
+    _check(final_state, "final_state", (B, H, d, e), torch.float32)
+    ip = 0
+    if init_state is not None:
+        _check(init_state, "init_state", (B, H, d, e), torch.float32)
+        ip = init_state.data_ptr()
+    wp, wn = _workspace(la2_workspace_bytes(B, H, T, d, e, block, dt, 0), q.device, workspace)
+    st = la2_fwd_state_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(),
+                           out.data_ptr(), ip, final_state.data_ptr(), B, H, T, d, e, block, dt,
+                           wp, wn, _stream_ptr(stream))
+    if st != LA2_OK:
+        raise LA2Error(st, "la2_fwd_state")
+    return out, final_state
+
+
+def la2_decode_raw(q, k, v, decay, state, out, B, H, d, e, dtype, stream=0) -> int:
+    return int(load().la2_decode(q, k, v, decay, state, out, B, H, d, e, dtype, stream))
+
+
+def la2_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, decay: torch.Tensor,
+               state: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """One token per sequence: state <- decay state + k v^T (in place), returns state^T q.
+
+    q, k: [B, H, d], v: [B, H, e] (bf16 or fp32); state: [B, H, d, e] fp32."""
+    B, H, d = q.shape
+    e = v.shape[-1]
+    dt = _dtype_code(q)
+    _check(q, "q", (B, H, d), q.dtype)
+    _check(k, "k", (B, H, d), q.dtype)
+    _check(v, "v", (B, H, e), q.dtype)
+    _check(decay, "decay", (H,), torch.float32)
+    _check(state, "state", (B, H, d, e), torch.float32)
+    out = torch.empty((B, H, e), dtype=torch.float32, device=q.device) if out is None else out
+    _check(out, "out", (B, H, e), torch.float32)
+    st = la2_decode_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(),
+                        state.data_ptr(), out.data_ptr(), B, H, d, e, dt, _stream_ptr(stream))
+    if st != LA2_OK:
+        raise LA2Error(st, "la2_decode")
     return out
 
 

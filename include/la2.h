@@ -35,7 +35,8 @@
  *     that ran out) are recorded in a device status word that
  *     la2_device_status() reads.
  *   - B, H or T equal to 0 is an empty problem: LA2_OK, nothing is launched
- *     and no pointer is dereferenced.
+ *     and no pointer is dereferenced (except that la2_fwd_state with T = 0
+ *     still sets final_state, by a device copy or memset on `stream`).
  */
 #ifndef LA2_H_
 #define LA2_H_
@@ -98,6 +99,32 @@ la2_status la2_fwd(const void *q, const void *k, const void *v, const float *dec
                    la2_stream_t stream);
 
 /*
+ * Forward with a carried state: as la2_fwd, but the recurrence starts from
+ * init_state instead of zero and the state after the last position is written
+ * to final_state.  With S_{-1} = init_state and S_t = decay[h] S_{t-1} +
+ * k_t v_t^T (d x e), out[t] = S_t^T q_t, i.e.
+ *
+ *   out[b,h,t,:] = decay[h]^(t+1) init_state[b,h]^T q[b,h,t,:]
+ *                  + sum_{s<=t} decay[h]^(t-s) (q[b,h,t,:] . k[b,h,s,:]) v[b,h,s,:]
+ *   final_state[b,h] = S_{T-1}
+ *
+ * The state is everything a sequence carries from one position to the next
+ * ("Lightning Attention" explainer, section 2, memory footprint), so a long
+ * sequence can be processed in consecutive pieces, each starting from the
+ * final state of the one before, with the result of one call over the whole.
+ *
+ * init_state, final_state: device fp32 [B, H, d, e] contiguous (row i = key
+ * feature, column j = value feature), 4-byte aligned; either may be NULL
+ * (start from zero / do not write the state).  final_state must not alias
+ * init_state or any other argument.  With T = 0 the final state is the
+ * initial one (or zero).  Support matrix and workspace as for la2_fwd.
+ */
+la2_status la2_fwd_state(const void *q, const void *k, const void *v, const float *decay,
+                         void *out, const float *init_state, float *final_state,
+                         int B, int H, int T, int d, int e, int block, la2_dtype dtype,
+                         void *workspace, size_t workspace_bytes, la2_stream_t stream);
+
+/*
  * Backward of L = sum dout * out with respect to q, k and v (decay is not
  * differentiated):
  *   dq[t] = sum_{s<=t} lambda^(t-s) (dout_t . v_s) k_s
@@ -111,6 +138,28 @@ la2_status la2_bwd(const void *q, const void *k, const void *v, const float *dec
                    const void *dout, void *dq, void *dk, void *dv,
                    int B, int H, int T, int d, int e, int block, la2_dtype dtype,
                    void *workspace, size_t workspace_bytes, la2_stream_t stream);
+
+/*
+ * One recurrent decode step: one new token per sequence (b, h).
+ *
+ *   state[b,h] <- decay[h] state[b,h] + k[b,h,:] v[b,h,:]^T     (d x e, in place)
+ *   out[b,h,:]  = state[b,h]^T q[b,h,:]                         (with the new state)
+ *
+ * This is the prefix-sum recurrence of the "Lightning Attention" explainer
+ * (section 1) advanced by one position; starting from the final state of
+ * la2_fwd_state over a prompt, successive calls continue the same sequence at a
+ * constant cost per token (the Lightning Attention-2 abstract's constant speed).
+ *
+ * q, k: device [B, H, d] of `dtype`; v: device [B, H, e] of `dtype` (element
+ * aligned); decay: device fp32 [H]; state: device fp32 [B, H, d, e] contiguous,
+ * 4-byte aligned (16-byte aligned with e % 4 == 0 takes the vector path), read
+ * and written; out: device fp32 [B, H, e].  out must not alias state or an
+ * input.  1 <= d, e <= 4096; B = 0 or H = 0 is empty (LA2_OK, nothing
+ * launched).  Asynchronous on `stream`, one launch.
+ */
+la2_status la2_decode(const void *q, const void *k, const void *v, const float *decay,
+                      float *state, float *out, int B, int H, int d, int e, la2_dtype dtype,
+                      la2_stream_t stream);
 
 /* Static, human-readable name of a status code. */
 const char *la2_status_str(la2_status status);

@@ -127,9 +127,9 @@ def decode_step(q, k, v, lam, state):
     """(o, S'): one new token per sequence, q, k [..., d], v [..., e], state
     [..., d, e]: S' = lam S + k v^T, o = S'^T q.  The input state is not modified."""
     lib = _load()
-    q = _f64(q)
+    q, v = _f64(q), _f64(v)
     lead = tuple(q.shape[:-1])
-    d, e = int(q.shape[-1]), int(np.asarray(v).shape[-1])
+    d, e = int(q.shape[-1]), int(v.shape[-1])
     ns = int(np.prod(lead)) if lead else 1
     lamv = np.ascontiguousarray(np.broadcast_to(np.asarray(lam, dtype=np.float64), lead).reshape(ns))
     qc, kc, vc = q.reshape(ns, d), _f64(k).reshape(ns, d), _f64(v).reshape(ns, e)
