@@ -121,23 +121,24 @@ bool device_setup(int* dev_out, int** status_out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Tensor map over a contiguous [BH, T, D] tensor with 128-byte rows per box
-// (64 bf16 or 32 fp32 elements) x 128 rows x 1, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, int BH, int T, int D, bool fp32) {
+// 4-D tensor map over a contiguous bf16 tensor [B, H, T, D] (dims D, T, H, B)
+// or, with bthd, [B, T, H, D] (dims D, H, T, B), with strides increasing in
+// both cases.  Box: 64 columns (128 bytes) x 128 positions of one (b, h),
+// 128-byte swizzle; positions past T read as zero.
+bool make_map(CUtensorMap* m, const void* ptr, int B, int H, int T, int D, bool bthd) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
-    const cuuint64_t esz = fp32 ? 4 : 2;
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(T),
-                                static_cast<cuuint64_t>(BH)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * esz,
-                                   static_cast<cuuint64_t>(T) * static_cast<cuuint64_t>(D) * esz};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esz),
-                               static_cast<cuuint32_t>(la2::ws::kTB), 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-               const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    const cuuint64_t esz = 2;
+    const cuuint64_t d = static_cast<cuuint64_t>(D), t = static_cast<cuuint64_t>(T);
+    const cuuint64_t h = static_cast<cuuint64_t>(H), b = static_cast<cuuint64_t>(B);
+    const cuuint64_t dims[4] = {d, bthd ? h : t, bthd ? t : h, b};
+    const cuuint64_t strides[3] = {d * esz, (bthd ? h : t) * d * esz, t * h * d * esz};
+    const cuuint32_t box[4] = {64, bthd ? 1u : static_cast<cuuint32_t>(la2::ws::kTB),
+                               bthd ? static_cast<cuuint32_t>(la2::ws::kTB) : 1u, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 struct RoleDesc {
@@ -181,15 +182,15 @@ void launch_ws(const la2::ws::Params& p, unsigned units, cudaStream_t stream) {
 // one CTA per (sequence, role, segment), preceded by the state pre-pass when
 // sequences are split into segments.
 la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
-                          int* status, float* seg_state, cudaStream_t stream) {
+                          bool bthd, int* status, float* seg_state, cudaStream_t stream) {
     la2::ws::Params p;
     std::memset(&p, 0, sizeof(p));
     const int BH = B * H;
     const int da = roles[0].da, dc = roles[0].dc;
     for (int r = 0; r < n; ++r) {
-        if (!make_map(&p.role[r].ta, roles[r].a, BH, T, da, false) ||
-            !make_map(&p.role[r].tb, roles[r].b, BH, T, da, false) ||
-            !make_map(&p.role[r].tc, roles[r].c, BH, T, dc, false))
+        if (!make_map(&p.role[r].ta, roles[r].a, B, H, T, da, bthd) ||
+            !make_map(&p.role[r].tb, roles[r].b, B, H, T, da, bthd) ||
+            !make_map(&p.role[r].tc, roles[r].c, B, H, T, dc, bthd))
             return LA2_ERR_CUDA;
         p.role[r].x = static_cast<float*>(roles[r].x);
         p.role[r].init = roles[r].init;
@@ -201,6 +202,7 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
     p.H = H;
     p.T = T;
     p.nroles = n;
+    p.bthd = bthd ? 1 : 0;
     const SegPlan sp = plan_segments(static_cast<long long>(BH) * n, T);
     p.nseg = sp.nseg;
     p.seg_tiles = sp.seg_tiles;
@@ -217,7 +219,7 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
 }
 
 la2_status launch_f32(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
-                      int block, cudaStream_t stream) {
+                      int block, bool bthd, cudaStream_t stream) {
     la2::F32Params p;
     std::memset(&p, 0, sizeof(p));
     int da_max = 0, dc_max = 0;
@@ -239,6 +241,7 @@ la2_status launch_f32(const RoleDesc* roles, int n, const float* decay, int B, i
     p.T = T;
     p.TB = block;
     p.nroles = n;
+    p.bthd = bthd ? 1 : 0;
     const size_t smem = la2::f32_scan_smem_bytes(da_max, dc_max, block);
     const dim3 grid(static_cast<unsigned>(B * H * n));
     la2::la2_scan_f32<<<grid, la2::kF32Threads, smem, stream>>>(p);
@@ -278,7 +281,7 @@ size_t bf16_workspace_bytes(const RoleDesc* roles, int n, int B, int H) {
 }
 
 la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
-                     int block, la2_dtype dtype, void* workspace, size_t ws_bytes,
+                     int block, la2_dtype dtype, bool bthd, void* workspace, size_t ws_bytes,
                      cudaStream_t stream) {
     int dev = 0;
     int* status = nullptr;
@@ -286,13 +289,13 @@ la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, in
         (workspace == nullptr || ws_bytes < bf16_workspace_bytes(roles, n, B, H)))
         return LA2_ERR_WORKSPACE;
     if (!device_setup(&dev, &status)) return LA2_ERR_CUDA;
-    if (dtype == LA2_DTYPE_F32) return launch_f32(roles, n, decay, B, H, T, block, stream);
+    if (dtype == LA2_DTYPE_F32) return launch_f32(roles, n, decay, B, H, T, block, bthd, stream);
     size_t off = 0;
     return for_role_groups(roles, n, [&](const RoleDesc* g, int m) {
         float* seg = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) + off) : nullptr;
         off += seg_workspace_bytes(static_cast<long long>(B) * H * m, g[0].da, g[0].dc);
         off = (off + 255) & ~static_cast<size_t>(255);
-        return launch_bf16_ws(g, m, decay, B, H, T, status, seg, stream);
+        return launch_bf16_ws(g, m, decay, B, H, T, bthd, status, seg, stream);
     });
 }
 
@@ -313,11 +316,12 @@ size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block, la2_dty
     return is_bwd ? bf16_workspace_bytes(bwd, 3, B, H) : bf16_workspace_bytes(fwd, 1, B, H);
 }
 
-la2_status la2_fwd_state(const void* q, const void* k, const void* v, const float* decay,
-                         void* out, const float* init_state, float* final_state, int B, int H,
-                         int T, int d, int e, int block, la2_dtype dtype, void* workspace,
-                         size_t workspace_bytes, la2_stream_t stream) {
+la2_status la2_fwd_ex(const void* q, const void* k, const void* v, const float* decay, void* out,
+                      const float* init_state, float* final_state, int B, int H, int T, int d,
+                      int e, int block, la2_dtype dtype, la2_layout layout, void* workspace,
+                      size_t workspace_bytes, la2_stream_t stream) {
     t_last_launches = 0;
+    if (layout != LA2_LAYOUT_BHTD && layout != LA2_LAYOUT_BTHD) return LA2_ERR_INVALID_ARG;
     bool empty = false;
     la2_status st = common_checks(B, H, T, d, e, block, dtype, &empty);
     if (st != LA2_OK) return st;
@@ -342,8 +346,16 @@ la2_status la2_fwd_state(const void* q, const void* k, const void* v, const floa
     RoleDesc r = {q, k, v, out, d, e, +1};
     r.init = init_state;
     r.fin = final_state;
-    return run_roles(&r, 1, decay, B, H, T, block, dtype, workspace, workspace_bytes,
-                     reinterpret_cast<cudaStream_t>(stream));
+    return run_roles(&r, 1, decay, B, H, T, block, dtype, layout == LA2_LAYOUT_BTHD, workspace,
+                     workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+la2_status la2_fwd_state(const void* q, const void* k, const void* v, const float* decay,
+                         void* out, const float* init_state, float* final_state, int B, int H,
+                         int T, int d, int e, int block, la2_dtype dtype, void* workspace,
+                         size_t workspace_bytes, la2_stream_t stream) {
+    return la2_fwd_ex(q, k, v, decay, out, init_state, final_state, B, H, T, d, e, block, dtype,
+                      LA2_LAYOUT_BHTD, workspace, workspace_bytes, stream);
 }
 
 la2_status la2_fwd(const void* q, const void* k, const void* v, const float* decay, void* out,
@@ -357,7 +369,16 @@ la2_status la2_bwd(const void* q, const void* k, const void* v, const float* dec
                    const void* dout, void* dq, void* dk, void* dv, int B, int H, int T, int d,
                    int e, int block, la2_dtype dtype, void* workspace, size_t workspace_bytes,
                    la2_stream_t stream) {
+    return la2_bwd_ex(q, k, v, decay, dout, dq, dk, dv, B, H, T, d, e, block, dtype,
+                      LA2_LAYOUT_BHTD, workspace, workspace_bytes, stream);
+}
+
+la2_status la2_bwd_ex(const void* q, const void* k, const void* v, const float* decay,
+                      const void* dout, void* dq, void* dk, void* dv, int B, int H, int T, int d,
+                      int e, int block, la2_dtype dtype, la2_layout layout, void* workspace,
+                      size_t workspace_bytes, la2_stream_t stream) {
     t_last_launches = 0;
+    if (layout != LA2_LAYOUT_BHTD && layout != LA2_LAYOUT_BTHD) return LA2_ERR_INVALID_ARG;
     bool empty = false;
     la2_status st = common_checks(B, H, T, d, e, block, dtype, &empty);
     if (st != LA2_OK || empty) return st;
@@ -372,8 +393,8 @@ la2_status la2_bwd(const void* q, const void* k, const void* v, const float* dec
         {k, q, dout, dv, d, e, -1},
     };
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return LA2_ERR_INVALID_ARG;
-    return run_roles(roles, 3, decay, B, H, T, block, dtype, workspace, workspace_bytes,
-                     reinterpret_cast<cudaStream_t>(stream));
+    return run_roles(roles, 3, decay, B, H, T, block, dtype, layout == LA2_LAYOUT_BTHD, workspace,
+                     workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 la2_status la2_decode(const void* q, const void* k, const void* v, const float* decay,

@@ -28,6 +28,7 @@ struct F32Params {
     F32Role role[3];
     const float* decay;
     int H, T, TB, nroles;
+    int bthd;  // 0: [B, H, T, D]; 1: [B, T, H, D]
 };
 
 __host__ __device__ inline size_t f32_scan_smem_bytes(int da, int dc, int TB) {
@@ -58,10 +59,15 @@ la2_scan_f32(const __grid_constant__ F32Params p)
     for (int z = tid; z < da * dc; z += kF32Threads)
         W[z] = R.init ? R.init[static_cast<size_t>(bh) * da * dc + z] : 0.f;
 
-    const float* a = R.a + static_cast<size_t>(bh) * T * da;
-    const float* b = R.b + static_cast<size_t>(bh) * T * da;
-    const float* c = R.c + static_cast<size_t>(bh) * T * dc;
-    float* x = R.x + static_cast<size_t>(bh) * T * dc;
+    // sequence bh: base row and row stride in units of D ([B,H,T,D]: bh T, 1;
+    // [B,T,H,D]: b T H + h, H)
+    const size_t rs = p.bthd ? static_cast<size_t>(p.H) : 1;
+    const size_t r0 = p.bthd ? static_cast<size_t>(bh / p.H) * T * p.H + bh % p.H
+                             : static_cast<size_t>(bh) * T;
+    const float* a = R.a + r0 * da;
+    const float* b = R.b + r0 * da;
+    const float* c = R.c + r0 * dc;
+    float* x = R.x + r0 * dc;
 
     const int nb = (T + TB - 1) / TB;
     const int row = tid >> 2;   // 0..63: row of the 64-row sub-tile this thread accumulates
@@ -78,7 +84,7 @@ la2_scan_f32(const __grid_constant__ F32Params p)
             // query sub-tile
             for (int z = tid; z < kF32Sub * da; z += kF32Threads) {
                 const int rr = z / da, u = z % da, loc = qa * kF32Sub + rr;
-                As[z] = loc < len ? a[static_cast<size_t>(t0 + loc) * da + u] : 0.f;
+                As[z] = loc < len ? a[static_cast<size_t>(t0 + loc) * rs * da + u] : 0.f;
             }
             __syncthreads();
 
@@ -101,11 +107,11 @@ la2_scan_f32(const __grid_constant__ F32Params p)
                 __syncthreads();
                 for (int z = tid; z < kF32Sub * da; z += kF32Threads) {
                     const int rr = z / da, u = z % da, loc = kb * kF32Sub + rr;
-                    Bs[z] = loc < len ? b[static_cast<size_t>(t0 + loc) * da + u] : 0.f;
+                    Bs[z] = loc < len ? b[static_cast<size_t>(t0 + loc) * rs * da + u] : 0.f;
                 }
                 for (int z = tid; z < kF32Sub * dc; z += kF32Threads) {
                     const int rr = z / dc, j = z % dc, loc = kb * kF32Sub + rr;
-                    Cs[z] = loc < len ? c[static_cast<size_t>(t0 + loc) * dc + j] : 0.f;
+                    Cs[z] = loc < len ? c[static_cast<size_t>(t0 + loc) * rs * dc + j] : 0.f;
                 }
                 __syncthreads();
                 for (int z = tid; z < kF32Sub * kF32Sub; z += kF32Threads) {
@@ -135,7 +141,7 @@ la2_scan_f32(const __grid_constant__ F32Params p)
 #pragma unroll
                 for (int m = 0; m < 32; ++m) {
                     const int j = jc + 4 * m;
-                    if (j < dc) x[static_cast<size_t>(t0 + rloc) * dc + j] = acc[m];
+                    if (j < dc) x[static_cast<size_t>(t0 + rloc) * rs * dc + j] = acc[m];
                 }
             }
             __syncthreads();
@@ -153,11 +159,11 @@ la2_scan_f32(const __grid_constant__ F32Params p)
             for (int z = tid; z < kF32Sub * da; z += kF32Threads) {
                 const int rr = z / da, u = z % da, loc = kb * kF32Sub + rr;
                 const float ws = loc < len ? (dir > 0 ? pw[tl - 1 - loc] : pw[loc]) : 0.f;
-                Bs[z] = loc < len ? ws * b[static_cast<size_t>(t0 + loc) * da + u] : 0.f;
+                Bs[z] = loc < len ? ws * b[static_cast<size_t>(t0 + loc) * rs * da + u] : 0.f;
             }
             for (int z = tid; z < kF32Sub * dc; z += kF32Threads) {
                 const int rr = z / dc, j = z % dc, loc = kb * kF32Sub + rr;
-                Cs[z] = loc < len ? c[static_cast<size_t>(t0 + loc) * dc + j] : 0.f;
+                Cs[z] = loc < len ? c[static_cast<size_t>(t0 + loc) * rs * dc + j] : 0.f;
             }
             __syncthreads();
             for (int z = tid; z < da * dc; z += kF32Threads) {

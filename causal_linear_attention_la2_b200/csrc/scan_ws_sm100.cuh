@@ -63,7 +63,8 @@ constexpr int kThreads = 640;
 constexpr uint32_t kTmemCols = 512;
 
 struct Role {
-    CUtensorMap ta, tb, tc;  // a, b: [B*H, T, DA]; c: [B*H, T, DC]; bf16, box 64 x 128
+    CUtensorMap ta, tb, tc;  // a, b: 4-D maps of [B, H, T, DA] (or [B, T, H, DA]); c likewise
+                             // with DC; bf16, box 64 columns x 128 positions
     float* x;                // [B*H, T, DC] fp32
     const float* init;       // [B*H, DA, DC] fp32 state before the first position, or null (0)
     float* fin;              // [B*H, DA, DC] fp32 state after the last position, or null
@@ -77,6 +78,7 @@ struct Params {
     float* seg_state;    // [B*H][nroles][nseg - 1][DA][DC] fp32: local end state of each
                          // segment but the last (written by the state pass)
     int H, T, nroles;
+    int bthd;            // 0: tensors [B, H, T, D]; 1: [B, T, H, D] (rows of a sequence H*D apart)
     int nseg;            // segments per (sequence, role); 1 = no split
     int seg_tiles;       // tiles per segment (the last may be shorter)
 };
@@ -198,6 +200,15 @@ __device__ unsigned long long g_la2_trace[2][kTraceEv][kTraceSteps];
 #else
 #define LA2_TR(ev, s) ((void)0)
 #endif
+
+// TMA load of the 64-column x 128-position box at column x, position t of
+// sequence bh, from a 4-D map laid out (D, T, H, B) or, with bthd, (D, H, T, B).
+__device__ __forceinline__ void load_box(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x,
+                                         int t, int bh, int H, int bthd) {
+    const int b = bh / H, h = bh - b * H;
+    if (bthd) tma_load_4d(dst, map, bar, x, h, t, b);
+    else tma_load_4d(dst, map, bar, x, t, h, b);
+}
 
 // Bounded wait that also gives up as soon as another role has aborted.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
@@ -333,24 +344,21 @@ la2_scan_ws(const __grid_constant__ Params p)
                 const uint32_t b = bar(Q::FULL_A + slot);
                 mbar_arrive_expect_tx(b, L::kAsz);
                 for (int gg = 0; gg < DA / 64; ++gg)
-                    tma_load_3d(sA + slot * L::kAsz + gg * 16384, &R.ta, b, gg * 64,
-                                tile_of(s) * kTB, bh);
+                    load_box(sA + slot * L::kAsz + gg * 16384, &R.ta, b, gg * 64, tile_of(s) * kTB, bh, p.H, p.bthd);
             };
             auto load_b = [&](int s) {
                 const int slot = s % Q::NB;
                 const uint32_t b = bar(Q::FULL_B + slot);
                 mbar_arrive_expect_tx(b, L::kBsz);
                 for (int gg = 0; gg < DA / 64; ++gg)
-                    tma_load_3d(sB + slot * L::kBsz + gg * 16384, &R.tb, b, gg * 64,
-                                tile_of(s) * kTB, bh);
+                    load_box(sB + slot * L::kBsz + gg * 16384, &R.tb, b, gg * 64, tile_of(s) * kTB, bh, p.H, p.bthd);
             };
             auto load_c = [&](int s) {
                 const int slot = s % Q::NC;
                 const uint32_t b = bar(Q::FULL_C + slot);
                 mbar_arrive_expect_tx(b, L::kCsz);
                 for (int gg = 0; gg < DC / 64; ++gg)
-                    tma_load_3d(sC + slot * L::kCsz + gg * 16384, &R.tc, b, gg * 64,
-                                tile_of(s) * kTB, bh);
+                    load_box(sC + slot * L::kCsz + gg * 16384, &R.tc, b, gg * 64, tile_of(s) * kTB, bh, p.H, p.bthd);
             };
             constexpr uint32_t kIdS = idesc_bf16_f32(128, kTB, 0, 0);
             const uint64_t dA0 = sdesc_sw128(sA, 16, 1024), dB0 = sdesc_sw128(sB, 16, 1024);
@@ -814,7 +822,10 @@ la2_scan_ws(const __grid_constant__ Params p)
         }
         fence_proxy_async_smem();
         mbar_arrive(bar(Q::W_READY + 0));
-        float* xg = R.x + static_cast<size_t>(bh) * T * DC;
+        // output rows: [B, H, T, DC] (row stride DC) or [B, T, H, DC] (stride H DC)
+        const size_t xrs = p.bthd ? static_cast<size_t>(p.H) * DC : static_cast<size_t>(DC);
+        float* xg = R.x + (p.bthd ? (static_cast<size_t>(bh / p.H) * T * p.H + bh % p.H) * DC
+                                  : static_cast<size_t>(bh) * T * DC);
 
         // X row r *= w_x(r) (the inter-tile term, still alone in X)
         auto scale = [&](int s) -> bool {
@@ -991,10 +1002,10 @@ la2_scan_ws(const __grid_constant__ Params p)
                     for (int j = 0; j < 4; ++j) {
                         const int cc = static_cast<int>(col) + 8 * j + 2 * tm;
                         if (row < T)
-                            st_global_v2(xg + static_cast<size_t>(row) * DC + cc, v[16 * lh + 4 * j],
+                            st_global_v2(xg + static_cast<size_t>(row) * xrs + cc, v[16 * lh + 4 * j],
                                          v[16 * lh + 4 * j + 1]);
                         if (row + 8 < T)
-                            st_global_v2(xg + static_cast<size_t>(row + 8) * DC + cc,
+                            st_global_v2(xg + static_cast<size_t>(row + 8) * xrs + cc,
                                          v[16 * lh + 4 * j + 2], v[16 * lh + 4 * j + 3]);
                     }
                 }
@@ -1119,10 +1130,10 @@ la2_state_ws(const __grid_constant__ Params p)
                 const uint32_t bb = bar(SB_B0 + slot), bc = bar(SB_C0 + slot);
                 mbar_arrive_expect_tx(bb, kTB * DA * 2);
                 for (int gg = 0; gg < DA / 64; ++gg)
-                    tma_load_3d(sB + slot * L::kBsz + gg * 16384, &R.tb, bb, gg * 64, i * kTB, bh);
+                    load_box(sB + slot * L::kBsz + gg * 16384, &R.tb, bb, gg * 64, i * kTB, bh, p.H, p.bthd);
                 mbar_arrive_expect_tx(bc, kTB * DC * 2);
                 for (int gg = 0; gg < DC / 64; ++gg)
-                    tma_load_3d(sC + slot * L::kCsz + gg * 16384, &R.tc, bc, gg * 64, i * kTB, bh);
+                    load_box(sC + slot * L::kCsz + gg * 16384, &R.tc, bc, gg * 64, i * kTB, bh, p.H, p.bthd);
             };
             load(tile_of(0), 0);
             if (ns > 1) load(tile_of(1), 1);

@@ -26,8 +26,13 @@ LA2_DTYPE_F32 = 0
 LA2_DTYPE_BF16 = 1
 
 # Every entry point include/la2.h declares.
-EXPORTS = ("la2_workspace_bytes", "la2_fwd", "la2_fwd_state", "la2_bwd", "la2_decode",
-           "la2_status_str", "la2_device_status", "la2_last_launch_count", "la2_fwd_noalloc")
+EXPORTS = ("la2_workspace_bytes", "la2_fwd", "la2_fwd_state", "la2_fwd_ex", "la2_bwd", "la2_bwd_ex",
+           "la2_decode", "la2_status_str", "la2_device_status", "la2_last_launch_count",
+           "la2_fwd_noalloc")
+
+LA2_LAYOUT_BHTD = 0
+LA2_LAYOUT_BTHD = 1
+_LAYOUTS = {"bhtd": LA2_LAYOUT_BHTD, "bthd": LA2_LAYOUT_BTHD}
 
 
 class LA2Error(RuntimeError):
@@ -57,6 +62,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la2_fwd_state.restype = i
     lib.la2_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
     lib.la2_bwd.restype = i
+    lib.la2_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, sz, vp]
+    lib.la2_fwd_ex.restype = i
+    lib.la2_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, sz, vp]
+    lib.la2_bwd_ex.restype = i
     lib.la2_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
     lib.la2_decode.restype = i
     lib.la2_status_str.argtypes = [i]
@@ -220,6 +229,77 @@ def la2_fwd_state(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, decay: torc
     if st != LA2_OK:
         raise LA2Error(st, "la2_fwd_state")
     return out, final_state
+
+
+def _dims(q, v, layout):
+    """(B, H, T, d, e) from q's and v's shapes in the given layout."""
+    if layout == "bhtd":
+        B, H, T, d = q.shape
+    elif layout == "bthd":
+        B, T, H, d = q.shape
+    else:
+        raise ValueError(f"unknown layout {layout!r}; expected 'bhtd' or 'bthd'")
+    return B, H, T, d, v.shape[-1]
+
+
+def _shape(layout, B, H, T, D):
+    return (B, H, T, D) if layout == "bhtd" else (B, T, H, D)
+
+
+def la2_fwd_ex(q, k, v, decay, layout: str = "bhtd", init_state=None, out=None, final_state=None,
+               want_final: bool = False, block: int = 128, stream=None, workspace=None):
+    """la2_fwd_state for q, k, v (and out) laid out [B, H, T, D] ('bhtd') or
+    [B, T, H, D] ('bthd').  Returns out, or (out, final_state) with want_final
+    or a final_state buffer given."""
+    B, H, T, d, e = _dims(q, v, layout)
+    dt = _dtype_code(q)
+    _check(q, "q", _shape(layout, B, H, T, d), q.dtype)
+    _check(k, "k", _shape(layout, B, H, T, d), q.dtype)
+    _check(v, "v", _shape(layout, B, H, T, e), q.dtype)
+    _check(decay, "decay", (H,), torch.float32)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    out = torch.empty(_shape(layout, B, H, T, e), **f32) if out is None else out
+    _check(out, "out", _shape(layout, B, H, T, e), torch.float32)
+    if final_state is None and want_final:
+        final_state = torch.empty((B, H, d, e), **f32)
+    fp = 0
+    if final_state is not None:
+        _check(final_state, "final_state", (B, H, d, e), torch.float32)
+        fp = final_state.data_ptr()
+    ip = 0
+    if init_state is not None:
+        _check(init_state, "init_state", (B, H, d, e), torch.float32)
+        ip = init_state.data_ptr()
+    wp, wn = _workspace(la2_workspace_bytes(B, H, T, d, e, block, dt, 0), q.device, workspace)
+    st = int(load().la2_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(),
+                               out.data_ptr(), ip, fp, B, H, T, d, e, block, dt, _LAYOUTS[layout],
+                               wp, wn, _stream_ptr(stream)))
+    if st != LA2_OK:
+        raise LA2Error(st, "la2_fwd_ex")
+    return (out, final_state) if final_state is not None else out
+
+
+def la2_bwd_ex(q, k, v, decay, dout, layout: str = "bhtd", dq=None, dk=None, dv=None,
+               block: int = 128, stream=None, workspace=None):
+    """la2_bwd for tensors laid out [B, H, T, D] ('bhtd') or [B, T, H, D] ('bthd')."""
+    B, H, T, d, e = _dims(q, v, layout)
+    dt = _dtype_code(q)
+    for t, n, D in ((q, "q", d), (k, "k", d), (v, "v", e), (dout, "dout", e)):
+        _check(t, n, _shape(layout, B, H, T, D), q.dtype)
+    _check(decay, "decay", (H,), torch.float32)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty(_shape(layout, B, H, T, d), **f32) if dq is None else dq
+    dk = torch.empty(_shape(layout, B, H, T, d), **f32) if dk is None else dk
+    dv = torch.empty(_shape(layout, B, H, T, e), **f32) if dv is None else dv
+    for t, n, D in ((dq, "dq", d), (dk, "dk", d), (dv, "dv", e)):
+        _check(t, n, _shape(layout, B, H, T, D), torch.float32)
+    wp, wn = _workspace(la2_workspace_bytes(B, H, T, d, e, block, dt, 1), q.device, workspace)
+    st = int(load().la2_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(),
+                               dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, T,
+                               d, e, block, dt, _LAYOUTS[layout], wp, wn, _stream_ptr(stream)))
+    if st != LA2_OK:
+        raise LA2Error(st, "la2_bwd_ex")
+    return dq, dk, dv
 
 
 def la2_decode_raw(q, k, v, decay, state, out, B, H, d, e, dtype, stream=0) -> int:

@@ -73,6 +73,19 @@ typedef enum {
 } la2_dtype;
 
 /*
+ * Memory layout of the [.., T, ..] tensors (q, k, v, out, dout, dq, dk, dv):
+ * LA2_LAYOUT_BHTD is [B, H, T, D] (each sequence contiguous, the layout of the
+ * "Lightning Attention" explainer's section 3 sketch, and of every entry point
+ * without a layout argument); LA2_LAYOUT_BTHD is [B, T, H, D], the layout a
+ * model's projections produce (positions of one sequence H*D elements apart).
+ * States (init_state, final_state, decode state) are [B, H, d, e] in both.
+ */
+typedef enum {
+    LA2_LAYOUT_BHTD = 0,
+    LA2_LAYOUT_BTHD = 1
+} la2_layout;
+
+/*
  * Bytes of device workspace la2_fwd (is_bwd = 0) or la2_bwd (is_bwd = 1) needs
  * for these sizes.  The state carried along a sequence (d x e) stays on chip;
  * the workspace only holds, when there are too few sequences to fill the
@@ -125,6 +138,16 @@ la2_status la2_fwd_state(const void *q, const void *k, const void *v, const floa
                          void *workspace, size_t workspace_bytes, la2_stream_t stream);
 
 /*
+ * la2_fwd_state with an explicit layout of q, k, v and out (see la2_layout);
+ * everything else as la2_fwd_state.  An unknown layout is LA2_ERR_INVALID_ARG.
+ */
+la2_status la2_fwd_ex(const void *q, const void *k, const void *v, const float *decay,
+                      void *out, const float *init_state, float *final_state,
+                      int B, int H, int T, int d, int e, int block, la2_dtype dtype,
+                      la2_layout layout, void *workspace, size_t workspace_bytes,
+                      la2_stream_t stream);
+
+/*
  * Backward of L = sum dout * out with respect to q, k and v (decay is not
  * differentiated):
  *   dq[t] = sum_{s<=t} lambda^(t-s) (dout_t . v_s) k_s
@@ -159,6 +182,16 @@ la2_status la2_bwd(const void *q, const void *k, const void *v, const float *dec
  */
 la2_status la2_decode(const void *q, const void *k, const void *v, const float *decay,
                       float *state, float *out, int B, int H, int d, int e, la2_dtype dtype,
+                      la2_stream_t stream);
+
+/*
+ * la2_bwd with an explicit layout of q, k, v, dout, dq, dk and dv (see
+ * la2_layout); everything else as la2_bwd.
+ */
+la2_status la2_bwd_ex(const void *q, const void *k, const void *v, const float *decay,
+                      const void *dout, void *dq, void *dk, void *dv,
+                      int B, int H, int T, int d, int e, int block, la2_dtype dtype,
+                      la2_layout layout, void *workspace, size_t workspace_bytes,
                       la2_stream_t stream);
 
 /* Static, human-readable name of a status code. */
