@@ -646,6 +646,14 @@ la2_scan_ws(const __grid_constant__ Params p)
                 for (int u = 0; u < 32; ++u) sv[u] = 0.f;
             }
         };
+        // tf32 mode: transposed stores go to row n = 32 part + 8 k + j, word
+        // `lane` of a 128-byte row; the part of the swizzled address that depends
+        // on j and the lane is fixed per thread, the rest ((4 part + k) * 1024) is
+        // an immediate
+        uint32_t toff[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            toff[j] = static_cast<uint32_t>(part * 4096 + j * 128 + (((lane >> 2) ^ j) << 4) + (lane & 3) * 4);
         for (int s = 0; s < ns; ++s) {
             if constexpr (Q::kTf32) {
                 // C -> fp32 C^T (the K-major tf32 B operand of X += P C and dW): row r
@@ -665,9 +673,8 @@ la2_scan_ws(const __grid_constant__ Params p)
                         ld_shared_v4(src + sw128(r, 4 * part + k), v[0], v[1], v[2], v[3]);
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
-                            const int n = 32 * part + 8 * k + 2 * u;
-                            st_shared_f32(dst + sw128(n, lane >> 2) + (lane & 3) * 4, bf16lo_to_f32(v[u]));
-                            st_shared_f32(dst + sw128(n + 1, lane >> 2) + (lane & 3) * 4, bf16hi_to_f32(v[u]));
+                            st_shared_f32(dst + toff[2 * u] + k * 1024, bf16lo_to_f32(v[u]));
+                            st_shared_f32(dst + toff[2 * u + 1] + k * 1024, bf16hi_to_f32(v[u]));
                         }
                     }
                 }
@@ -692,9 +699,8 @@ la2_scan_ws(const __grid_constant__ Params p)
                         for (int u = 0; u < 4; ++u) {
                             const float2 w = mul2(make_float2(bf16lo_to_f32(v[u]), bf16hi_to_f32(v[u])),
                                                   make_float2(ws_s, ws_s));
-                            const int n = 32 * part + 8 * k + 2 * u;
-                            st_shared_f32(dst + sw128(n, lane >> 2) + (lane & 3) * 4, w.x);
-                            st_shared_f32(dst + sw128(n + 1, lane >> 2) + (lane & 3) * 4, w.y);
+                            st_shared_f32(dst + toff[2 * u] + k * 1024, w.x);
+                            st_shared_f32(dst + toff[2 * u + 1] + k * 1024, w.y);
                         }
                     }
                 }
@@ -857,9 +863,6 @@ la2_scan_ws(const __grid_constant__ Params p)
         auto update = [&](int s) -> bool {
             const bool last = has_last && s == ns - 1;
             const float lam_s = last ? pw[nlast] : lamTB;
-            float* fin = (last && R.fin) ? R.fin + static_cast<size_t>(bh) * (DA * DC) +
-                                               static_cast<size_t>(wrow) * DC
-                                         : nullptr;
             if (!wait_bar(bar(Q::D_DONE + (s % Q::ND)), full_par(s, Q::ND), abort_flag, p.status, 51))
                 return false;
             // the X MMA that last read the W buffer written here is done
@@ -895,10 +898,6 @@ la2_scan_ws(const __grid_constant__ Params p)
                                                   make_float2(d[u], d[u + 1]));
                             wreg[u] = w.x;
                             wreg[u + 1] = w.y;
-                            if (fin) {
-                                fin[col + 2 * z] = w.x;
-                                fin[col + 2 * z + 1] = w.y;
-                            }
                             split_pack2v(w, h[z], l[z]);
                         }
                         st_shared_v4(wdst + o0, h[0], h[1], h[2], h[3]);
@@ -923,16 +922,35 @@ la2_scan_ws(const __grid_constant__ Params p)
                                                   d[16 * hh + 2 * z]);
                             const float w1 = fmaf(lam_s, bf16hi_to_f32(h[z]) + bf16hi_to_f32(l[z]),
                                                   d[16 * hh + 2 * z + 1]);
-                            if (fin) {
-                                fin[col + 2 * z] = w0;
-                                fin[col + 2 * z + 1] = w1;
-                            }
                             split_pack2(w0, w1, h[z], l[z]);
                         }
                         st_shared_v4(wdst + o0, h[0], h[1], h[2], h[3]);
                         st_shared_v4(wdst + o1, h[4], h[5], h[6], h[7]);
                         st_shared_v4(wdst + L::kWsz + o0, l[0], l[1], l[2], l[3]);
                         st_shared_v4(wdst + L::kWsz + o1, l[4], l[5], l[6], l[7]);
+                    }
+                }
+            }
+            if (last && R.fin && owns_w_row) {
+                // the state after position T-1: fp32 from registers (32 columns per
+                // thread), else from the hi + lo pair just written
+                float* fin = R.fin + static_cast<size_t>(bh) * (DA * DC) + static_cast<size_t>(wrow) * DC;
+                if constexpr (kWReg) {
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) fin[c0 + u] = wreg[u];
+                } else {
+#pragma unroll 1
+                    for (int cc = 0; cc < kCols; cc += 8) {
+                        const uint32_t col = c0 + cc;
+                        const uint32_t o = (col >> 6) * (DA * 128) + sw128(wrow, (col & 63) >> 3);
+                        uint32_t h[4], l[4];
+                        ld_shared_v4(wdst + o, h[0], h[1], h[2], h[3]);
+                        ld_shared_v4(wdst + L::kWsz + o, l[0], l[1], l[2], l[3]);
+#pragma unroll
+                        for (int z = 0; z < 4; ++z) {
+                            fin[col + 2 * z] = bf16lo_to_f32(h[z]) + bf16lo_to_f32(l[z]);
+                            fin[col + 2 * z + 1] = bf16hi_to_f32(h[z]) + bf16hi_to_f32(l[z]);
+                        }
                     }
                 }
             }
