@@ -247,9 +247,112 @@ def run_reference(args, w, world, rank):
 
 def workload_config(w, args):
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "e": w.e,
-            "block": w.block, "global_batch": w.B * args.gpus, "seq_len": w.T,
+            "block": w.block, "layout": getattr(args, "layout", "bhtd"),
+            "global_batch": w.B * args.gpus, "seq_len": w.T,
             "parallelism": f"replicas{args.gpus}",
             "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"}
+
+
+def run_decode(args, world, rank, local):
+    """One recurrent decode step (la2_decode) per timed step: one new token for
+    each of B*H sequences, state [B, H, d, e] fp32 read and written in place.
+    Roofline: HBM, with the state's read and write plus q, k, v in and o out."""
+    from causal_linear_attention_la2_b200 import la2
+    la2.load()
+    dw = I.DECODE_WORKLOADS[args.decode_workload]
+    B, H, d, e = dw.B, dw.H, dw.d, dw.e
+    dev = torch.device("cuda", local)
+    g = torch.Generator().manual_seed(args.seed)
+    x = I.make_inputs(B, H, args.steps + args.warmup + 2, d, e, dw.dtype, seed=args.seed)
+    lam = x["lam"].to(dev)
+    state = (torch.randn(B, H, d, e, generator=g) * 0.1).to(dev)
+    tok = [{n: x[n][:, :, t].contiguous().to(dev) for n in ("q", "k", "v")}
+           for t in range(args.steps + args.warmup + 2)]
+    out = torch.empty(B, H, e, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for t in range(args.warmup):
+        flush.fill_(0.0)
+        la2.la2_decode(tok[t]["q"], tok[t]["k"], tok[t]["v"], lam, state, out=out)
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    launches = 0
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        t = args.warmup + i
+        s, e_ = ev[i]
+        s.record(stream)
+        la2.la2_decode(tok[t]["q"], tok[t]["k"], tok[t]["v"], lam, state, out=out)
+        launches += la2.la2_last_launch_count()
+        e_.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop() if clocks else None
+    step_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / len(ev), world)
+    # end to end: q, k, v of the token from pinned host memory in, o back out
+    hq = {n: tok[0][n].cpu().pin_memory() for n in ("q", "k", "v")}
+    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(5):
+        dq_, dk_, dv_ = (hq[n].to(dev, non_blocking=True) for n in ("q", "k", "v"))
+        la2.la2_decode(dq_, dk_, dv_, lam, state, out=out)
+        hout.copy_(out, non_blocking=True)
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1) / 5, world)
+    if rank != 0:
+        return 0
+    pk, pk_kind = peaks()
+    hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    esz = 2 if dw.dtype == "bf16" else 4
+    step_bytes = B * H * (2 * d * e * 4 + (2 * d + e) * esz + e * 4)
+    achieved = step_bytes / (step_ms * 1e-3) / 1e9
+    value = B * world / (step_ms * 1e-3)
+    line = {
+        "metric": "decode tokens/s (one new token per sequence, all heads, per la2_decode step)",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": dw.dtype, "data": "synthetic",
+        "config": {"workload": dw.name, "B": B, "H": H, "d": d, "e": e,
+                   "state_bytes": B * H * d * e * 4, "parallelism": f"replicas{args.gpus}",
+                   "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"},
+        "token_heads_per_s": value * H,
+        "roofline": {"bound": "hbm", "kernel": "la2_decode_kernel", "achieved": achieved,
+                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                     "peak_kind": f"{pk_kind} hbm_gbs"},
+        "e2e": {"value": B * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hq.values()),
+                "d2h_bytes_per_step": hout.numel() * hout.element_size()},
+        "gpu_launches": launches, "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        n = max(1, min(B * H, 256))
+        qs = tok[0]["q"].reshape(B * H, d)[:n].float().cpu().numpy()
+        ks = tok[0]["k"].reshape(B * H, d)[:n].float().cpu().numpy()
+        vs = tok[0]["v"].reshape(B * H, e)[:n].float().cpu().numpy()
+        st = state.reshape(B * H, d, e)[:n].cpu().numpy().astype(np.float64)
+        lam_n = np.resize(x["lam"].numpy().astype(np.float64), n)
+        reps, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < min(args.ref_seconds, 5.0):
+            oracle.decode_step(qs, ks, vs, lam_n, st)
+            reps += 1
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": reps * n / H / dt, "unit": "tokens/s", "cores": 1,
+                                "kind": "oracle",
+                                "sample": f"{reps} decode steps of {n} sequences (b, h), d={d}, "
+                                          f"e={e}, in {dt:.2f} s"}
+    print(json.dumps(line), flush=True)
+    return 0
 
 
 def run_ours(args, w, world, rank, local):
@@ -257,6 +360,9 @@ def run_ours(args, w, world, rank, local):
     la2.load()
     dev = torch.device("cuda", local)
     x = I.make_workload_inputs(w, seed=args.seed)
+    lay = args.layout
+    if lay == "bthd":  # [B, T, H, D]: the model-native layout
+        x = dict(x, **{n: x[n].transpose(1, 2).contiguous() for n in ("q", "k", "v", "do")})
     q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
     lam = x["lam"].to(dev)
     f32 = dict(dtype=torch.float32, device=dev)
@@ -265,13 +371,19 @@ def run_ours(args, w, world, rank, local):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    def fwd(qq, kk, vv):
+        la2.la2_fwd_ex(qq, kk, vv, lam, lay, out=out, block=w.block)
+
+    def bwd(qq, kk, vv, dd):
+        la2.la2_bwd_ex(qq, kk, vv, lam, dd, lay, dq=dq, dk=dk, dv=dv, block=w.block)
+
     launches = 0
 
     def step():
         nonlocal launches
-        la2.la2_fwd(q, k, v, lam, out=out, block=w.block)
+        fwd(q, k, v)
         launches += la2.la2_last_launch_count()
-        la2.la2_bwd(q, k, v, lam, do, dq=dq, dk=dk, dv=dv, block=w.block)
+        bwd(q, k, v, do)
         launches += la2.la2_last_launch_count()
 
     for _ in range(args.warmup):
@@ -293,10 +405,10 @@ def run_ours(args, w, world, rank, local):
         flush.fill_(float(i))
         s, m, e = ev[i]
         s.record(stream)
-        la2.la2_fwd(q, k, v, lam, out=out, block=w.block)
+        fwd(q, k, v)
         launches += la2.la2_last_launch_count()
         m.record(stream)
-        la2.la2_bwd(q, k, v, lam, do, dq=dq, dk=dk, dv=dv, block=w.block)
+        bwd(q, k, v, do)
         launches += la2.la2_last_launch_count()
         e.record(stream)
     torch.cuda.synchronize(dev)
@@ -317,8 +429,8 @@ def run_ours(args, w, world, rank, local):
 
     def e2e_step():
         qd, kd, vd, dd = (hosts[n].to(dev, non_blocking=True) for n in ("q", "k", "v", "do"))
-        la2.la2_fwd(qd, kd, vd, lam, out=out, block=w.block)
-        la2.la2_bwd(qd, kd, vd, lam, dd, dq=dq, dk=dk, dv=dv, block=w.block)
+        fwd(qd, kd, vd)
+        bwd(qd, kd, vd, dd)
         for h, dsrc in zip(houts, (out, dq, dk, dv)):
             h.copy_(dsrc, non_blocking=True)
 
@@ -386,6 +498,11 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--ref-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layout", default="bhtd", choices=["bhtd", "bthd"],
+                    help="tensor layout of the fwd+bwd step: [B,H,T,D] or [B,T,H,D]")
+    ap.add_argument("--mode", default="train", choices=["train", "decode"],
+                    help="train: la2_fwd + la2_bwd (the default line); decode: la2_decode steps")
+    ap.add_argument("--decode-workload", default="decode_tnl15b", choices=sorted(I.DECODE_WORKLOADS))
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be at least 3")
@@ -394,6 +511,8 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             return run_reference(args, w, world, rank)
+        if args.mode == "decode":
+            return run_decode(args, world, rank, local)
         return run_ours(args, w, world, rank, local)
     finally:
         if world > 1:

@@ -93,6 +93,17 @@ for _T in SWEEP_T:
         WORKLOADS[_w.name] = _w
 
 
+# Decode-step shapes: one new token for each of B sequences of H heads, the
+# heads of the TNL-15B and TNL-400M layers at serving batch sizes (the fp32
+# states, 168 MB and 33.5 MB, are larger than or comparable to the L2).
+DECODE_WORKLOADS = {
+    "decode_tnl15b": Workload("decode_tnl15b", 64, 40, 1, 128, 128, 128, "bf16", "tnl",
+                              "decode step, TNL-15B heads, batch 64"),
+    "decode_tnl400m": Workload("decode_tnl400m", 128, 16, 1, 64, 64, 128, "bf16", "tnl",
+                               "decode step, TNL-400M heads, batch 128"),
+}
+
+
 def make_inputs(B: int, H: int, T: int, d: int, e: int, dtype: str = "bf16",
                 seed: int = 0, decay: str = "tnl"):
     """Return dict(q, k, v, do, lam) as CPU tensors (lam: float32 [H])."""
