@@ -210,10 +210,30 @@ __device__ __forceinline__ void load_box(uint32_t dst, const CUtensorMap* map, u
     else tma_load_4d(dst, map, bar, x, t, h, b);
 }
 
-// Bounded wait that also gives up as soon as another role has aborted.
+// Bounded wait that also gives up as soon as another role has aborted.  The
+// loop is kept out of line (one copy for every call site) to keep each role's
+// code small; the first probe is inline.
+__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                           int* status, int where) {
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait_hint(bar, parity, 64)) return true;
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > 2000000000ull) {
+            *abort_flag = 1;
+            atomicCAS(status, 0, 5 | (where << 8));
+            return false;
+        }
+    }
+}
+
+// kOutline: the retry loop out of line (measured faster where instruction
+// fetch limits the kernel, d = 64) or inline (d = 128).
+template <bool kOutline = false>
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          int* status, int where) {
     if (mbar_try_wait_hint(bar, parity, 64)) return true;
+    if constexpr (kOutline) return wait_bar_slow(bar, parity, abort_flag, status, where);
     const uint64_t t0 = global_ns();
     while (true) {
         if (mbar_try_wait_hint(bar, parity, 64)) return true;
@@ -442,19 +462,19 @@ la2_scan_ws(const __grid_constant__ Params p)
             const uint64_t dC0 = Q::kTf32 ? sdesc_sw128(sCF, 16, 1024) : sdesc_sw128(sC, 16384, 1024);
             for (int s = 0; s < ns; ++s) {
                 const int sc = Q::kTf32 ? s % Q::NCF : s % Q::NC;
-                if (!wait_bar(bar(Q::P_READY + (s & 1)), full_par(s, 2), abort_flag, p.status, 23)) break;
+                if (!wait_bar<Q::kTf32>(bar(Q::P_READY + (s & 1)), full_par(s, 2), abort_flag, p.status, 23)) break;
                 if (Q::kOwnD) {
                     // X buffer s % 2 has been read out after tile s-2
-                    if (s >= Q::NX && !wait_bar(bar(Q::EMPTY_X + s % Q::NX), empty_par(s, Q::NX),
+                    if (s >= Q::NX && !wait_bar<Q::kTf32>(bar(Q::EMPTY_X + s % Q::NX), empty_par(s, Q::NX),
                                                 abort_flag, p.status, 24))
                         break;
-                } else if (!wait_bar(bar(Q::XS + s % Q::NX), full_par(s, Q::NX), abort_flag, p.status, 24)) {
+                } else if (!wait_bar<Q::kTf32>(bar(Q::XS + s % Q::NX), full_par(s, Q::NX), abort_flag, p.status, 24)) {
                     break;
                 }
                 if (Q::kTf32) {
-                    if (!wait_bar(bar(Q::CF_READY + sc), full_par(s, Q::NCF), abort_flag, p.status, 25))
+                    if (!wait_bar<Q::kTf32>(bar(Q::CF_READY + sc), full_par(s, Q::NCF), abort_flag, p.status, 25))
                         break;
-                } else if (!wait_bar(bar(Q::FULL_C + sc), full_par(s, Q::NC), abort_flag, p.status, 25)) {
+                } else if (!wait_bar<Q::kTf32>(bar(Q::FULL_C + sc), full_par(s, Q::NC), abort_flag, p.status, 25)) {
                     break;
                 }
                 LA2_TR(6, s);
@@ -493,13 +513,13 @@ la2_scan_ws(const __grid_constant__ Params p)
                 // W_READY completes once the epilogue has set W of this step (the
                 // initial state, or the update after the previous tile, which has
                 // also read the dW that sat in this X buffer)
-                if (!wait_bar(bar(Q::W_READY + sw), full_par(s, Q::NW), abort_flag, p.status, 30)) break;
-                if (!wait_bar(bar(Q::FULL_A + sa), full_par(s, Q::NA), abort_flag, p.status, 31)) break;
+                if (!wait_bar<Q::kTf32>(bar(Q::W_READY + sw), full_par(s, Q::NW), abort_flag, p.status, 30)) break;
+                if (!wait_bar<Q::kTf32>(bar(Q::FULL_A + sa), full_par(s, Q::NA), abort_flag, p.status, 31)) break;
                 if (Q::kOwnD) {
                     // X_inter has been read out after tile s-1
-                    if (s >= 1 && !wait_bar(bar(Q::EMPTY_XI), full_par(s - 1, 1), abort_flag, p.status, 32))
+                    if (s >= 1 && !wait_bar<Q::kTf32>(bar(Q::EMPTY_XI), full_par(s - 1, 1), abort_flag, p.status, 32))
                         break;
-                } else if (s >= Q::NX && !wait_bar(bar(Q::EMPTY_X + s % Q::NX), empty_par(s, Q::NX),
+                } else if (s >= Q::NX && !wait_bar<Q::kTf32>(bar(Q::EMPTY_X + s % Q::NX), empty_par(s, Q::NX),
                                                    abort_flag, p.status, 32)) {
                     break;
                 }
@@ -534,21 +554,21 @@ la2_scan_ws(const __grid_constant__ Params p)
                 const int sc = Q::kTf32 ? s % Q::NCF : s % Q::NC;
                 const int sl = Q::kTf32 ? 0 : s % Q::NBLO;
                 if (Q::kTf32) {
-                    if (!wait_bar(bar(Q::WB_READY + sb), full_par(s, Q::NWB), abort_flag, p.status, 33)) break;
-                    if (!wait_bar(bar(Q::CF_READY + sc), full_par(s, Q::NCF), abort_flag, p.status, 34)) break;
+                    if (!wait_bar<Q::kTf32>(bar(Q::WB_READY + sb), full_par(s, Q::NWB), abort_flag, p.status, 33)) break;
+                    if (!wait_bar<Q::kTf32>(bar(Q::CF_READY + sc), full_par(s, Q::NCF), abort_flag, p.status, 34)) break;
                 } else {
-                    if (!wait_bar(bar(Q::BS + sb), full_par(s, Q::NB), abort_flag, p.status, 33)) break;
-                    if (!wait_bar(bar(Q::FULL_C + sc), full_par(s, Q::NC), abort_flag, p.status, 34)) break;
+                    if (!wait_bar<Q::kTf32>(bar(Q::BS + sb), full_par(s, Q::NB), abort_flag, p.status, 33)) break;
+                    if (!wait_bar<Q::kTf32>(bar(Q::FULL_C + sc), full_par(s, Q::NC), abort_flag, p.status, 34)) break;
                 }
                 if (Q::kOwnD) {
                     // the update after tile s - ND has read this dW buffer
-                    if (s >= Q::ND && !wait_bar(bar(Q::EMPTY_D + s % Q::ND), empty_par(s, Q::ND),
+                    if (s >= Q::ND && !wait_bar<Q::kTf32>(bar(Q::EMPTY_D + s % Q::ND), empty_par(s, Q::ND),
                                                 abort_flag, p.status, 35))
                         break;
                 } else {
                     // X buffer (s+1) % 2 has been read out after tile s-1
                     static_assert(Q::kOwnD || Q::NX == 2, "dW shares the X buffers only with NX = 2");
-                    if (s >= 1 && !wait_bar(bar(Q::EMPTY_X + ((s + 1) % Q::NX)), full_par(s - 1, Q::NX),
+                    if (s >= 1 && !wait_bar<Q::kTf32>(bar(Q::EMPTY_X + ((s + 1) % Q::NX)), full_par(s - 1, Q::NX),
                                             abort_flag, p.status, 36))
                         break;
                 }
@@ -661,8 +681,8 @@ la2_scan_ws(const __grid_constant__ Params p)
                 // to word r of row n of C^T; the lanes of a warp (consecutive r) fill
                 // one whole 128-byte row, so the scalar stores meet no bank conflict
                 const int sc = s % Q::NC, scf = s % Q::NCF;
-                if (!wait_bar(bar(Q::FULL_C + sc), full_par(s, Q::NC), abort_flag, p.status, 42)) break;
-                if (s >= Q::NCF && !wait_bar(bar(Q::EMPTY_CF + scf), empty_par(s, Q::NCF), abort_flag,
+                if (!wait_bar<Q::kTf32>(bar(Q::FULL_C + sc), full_par(s, Q::NC), abort_flag, p.status, 42)) break;
+                if (s >= Q::NCF && !wait_bar<Q::kTf32>(bar(Q::EMPTY_CF + scf), empty_par(s, Q::NCF), abort_flag,
                                              p.status, 43))
                     break;
                 {
@@ -684,8 +704,8 @@ la2_scan_ws(const __grid_constant__ Params p)
                 // w_s B -> fp32 (w_s B)^T (the K-major tf32 A operand of dW), laid out
                 // like C^T; B itself is left for S
                 const int sb = s % Q::NB, swb = s % Q::NWB;
-                if (!wait_bar(bar(Q::FULL_B + sb), full_par(s, Q::NB), abort_flag, p.status, 44)) break;
-                if (s >= Q::NWB && !wait_bar(bar(Q::EMPTY_WB + swb), empty_par(s, Q::NWB), abort_flag,
+                if (!wait_bar<Q::kTf32>(bar(Q::FULL_B + sb), full_par(s, Q::NB), abort_flag, p.status, 44)) break;
+                if (s >= Q::NWB && !wait_bar<Q::kTf32>(bar(Q::EMPTY_WB + swb), empty_par(s, Q::NWB), abort_flag,
                                              p.status, 45))
                     break;
                 {
@@ -709,7 +729,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                 mbar_arrive(bar(Q::WB_READY + swb));
                 if (tid == 128) LA2_TR(10, s);
                 // P in place, fp32
-                if (!wait_bar(bar(Q::S_DONE + (s & 1)), full_par(s, 2), abort_flag, p.status, 40)) break;
+                if (!wait_bar<Q::kTf32>(bar(Q::S_DONE + (s & 1)), full_par(s, 2), abort_flag, p.status, 40)) break;
                 if (tid == 128) LA2_TR(9, s);
                 tc_fence_after();
                 const uint32_t st = tS(s & 1);
@@ -721,7 +741,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                     tmem_st32(st + lane_off + pr * 32, sv);
                 }
             } else {
-                if (!wait_bar(bar(Q::S_DONE + (s & 1)), full_par(s, 2), abort_flag, p.status, 40)) break;
+                if (!wait_bar<Q::kTf32>(bar(Q::S_DONE + (s & 1)), full_par(s, 2), abort_flag, p.status, 40)) break;
                 if (tid == 128) LA2_TR(9, s);
                 const uint32_t st = tS(s & 1);
                 tc_fence_after();
@@ -729,7 +749,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                 // lo into its own buffer once the dW that last read that buffer is
                 // done.  Part p does the chunks of half p of the row.
                 const int sl = s % Q::NBLO;
-                if (s >= Q::NBLO && !wait_bar(bar(Q::EMPTY_BLO + sl), empty_par(s, Q::NBLO), abort_flag,
+                if (s >= Q::NBLO && !wait_bar<Q::kTf32>(bar(Q::EMPTY_BLO + sl), empty_par(s, Q::NBLO), abort_flag,
                                               p.status, 41))
                     break;
                 const uint32_t sBs = sB + (s % Q::NB) * L::kBsz, sBl = sBlo + sl * L::kBsz;
@@ -835,7 +855,7 @@ la2_scan_ws(const __grid_constant__ Params p)
 
         // X row r *= w_x(r) (the inter-tile term, still alone in X)
         auto scale = [&](int s) -> bool {
-            if (!wait_bar(bar(Q::XW_DONE + s % Q::NXW), full_par(s, Q::NXW), abort_flag, p.status, 50))
+            if (!wait_bar<Q::kTf32>(bar(Q::XW_DONE + s % Q::NXW), full_par(s, Q::NXW), abort_flag, p.status, 50))
                 return false;
             if (tid == 384) LA2_TR(14, s);
             tc_fence_after();
@@ -863,10 +883,10 @@ la2_scan_ws(const __grid_constant__ Params p)
         auto update = [&](int s) -> bool {
             const bool last = has_last && s == ns - 1;
             const float lam_s = last ? pw[nlast] : lamTB;
-            if (!wait_bar(bar(Q::D_DONE + (s % Q::ND)), full_par(s, Q::ND), abort_flag, p.status, 51))
+            if (!wait_bar<Q::kTf32>(bar(Q::D_DONE + (s % Q::ND)), full_par(s, Q::ND), abort_flag, p.status, 51))
                 return false;
             // the X MMA that last read the W buffer written here is done
-            if (s + 1 >= Q::NW && !wait_bar(bar(Q::EMPTY_W + (s + 1) % Q::NW),
+            if (s + 1 >= Q::NW && !wait_bar<Q::kTf32>(bar(Q::EMPTY_W + (s + 1) % Q::NW),
                                             full_par(s + 1 - Q::NW, Q::NW), abort_flag, p.status, 52))
                 return false;
             if (tid == 384) LA2_TR(12, s);
@@ -967,10 +987,10 @@ la2_scan_ws(const __grid_constant__ Params p)
         // so every float2 store of a warp fills whole 32-byte sectors (eight
         // rows per instruction).  The X buffer is released once read.
         auto output = [&](int s) -> bool {
-            if (!wait_bar(bar(Q::PC_DONE + s % Q::NX), full_par(s, Q::NX), abort_flag, p.status, 53))
+            if (!wait_bar<Q::kTf32>(bar(Q::PC_DONE + s % Q::NX), full_par(s, Q::NX), abort_flag, p.status, 53))
                 return false;
             if (Q::kOwnD &&
-                !wait_bar(bar(Q::XW_DONE + s % Q::NXW), full_par(s, Q::NXW), abort_flag, p.status, 54))
+                !wait_bar<Q::kTf32>(bar(Q::XW_DONE + s % Q::NXW), full_par(s, Q::NXW), abort_flag, p.status, 54))
                 return false;
             if (tid == 384) LA2_TR(16, s);
             tc_fence_after();
