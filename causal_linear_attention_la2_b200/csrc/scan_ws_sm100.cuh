@@ -482,7 +482,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                 const uint32_t xt = tX(s % Q::NX), st = tS(s & 1);
                 if constexpr (Q::kTf32) {
                     const uint64_t dc = desc_add(dC0, sc * L::kCFsz);
-#pragma unroll
+#pragma unroll 4
                     for (int k = 0; k < kTB / 8; ++k)
                         mma_tf32_ts(xt, st + k * 8, desc_add(dc, (k >> 2) * (DC * 128) + (k & 3) * 32),
                                     kIdX, Q::kOwnD ? (k > 0) : 1);
@@ -577,7 +577,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                 const uint32_t dt = tD(s);
                 if constexpr (Q::kTf32) {
                     const uint64_t db = desc_add(dB0, sb * L::kWBsz), dc = desc_add(dC0, sc * L::kCFsz);
-#pragma unroll
+#pragma unroll 4
                     for (int k = 0; k < kTB / 8; ++k)
                         mma_tf32_ss(dt, desc_add(db, (k >> 2) * (DA * 128) + (k & 3) * 32),
                                     desc_add(dc, (k >> 2) * (DC * 128) + (k & 3) * 32), kIdW, k > 0);
