@@ -298,22 +298,9 @@ la2_scan_ws(const __grid_constant__ Params p)
     const float lam = p.decay[bh % p.H];
 
     if (tid == 0) LA2_TR(0, 0);
-    // ---- set-up: lambda^n table, W buffer 0 = 0, TMEM, barriers
-    {
-        const double l2 = log2(static_cast<double>(lam));
-        for (int n = tid; n <= kTB; n += kThreads) pw[n] = static_cast<float>(exp2(n * l2));
-        if (tid < 16) murev[tid] = static_cast<float>(exp2((15 - tid) * l2));
-        // Z[m] = lambda^(m-31) for m >= 31, else 0 (m = 0..66); copy k holds
-        // Z[j + k] at j, so that a 32-entry window starting anywhere can be
-        // read with aligned 16-byte loads
-        for (int idx = tid; idx < 4 * 64; idx += kThreads) {
-            const int k = idx >> 6, j = idx & 63, m = j + k;
-            float* zc = reinterpret_cast<float*>(smem_raw + L::kZ + k * L::kZstride);
-            zc[j] = m >= 31 ? static_cast<float>(exp2((m - 31) * l2)) : 0.f;
-        }
-        for (uint32_t off = tid * 16; off < 2 * L::kWsz; off += kThreads * 16)
-            st_shared_v4(sW + off, 0u, 0u, 0u, 0u);
-    }
+    // ---- set-up: TMEM and barriers here; the decay tables and W buffer 0 are
+    // made below by the mask and epilogue warps (the only ones that read them),
+    // while the producer's first loads are already in flight
     if (warp == 0) {
         tmem_alloc(base + L::kTmemSlot, kTmemCols);
         tmem_relinquish();
@@ -330,6 +317,26 @@ la2_scan_ws(const __grid_constant__ Params p)
 
     if (tid == 0) LA2_TR(1, 0);
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_raw + L::kTmemSlot);
+    if (warp >= 4) {
+        // lambda^n (n = 0..T_B), lambda^(15-n), the diagonal-block table
+        // Z[m] = lambda^(m-31) for m >= 31, else 0 (m = 0..66; copy k holds
+        // Z[j + k] at j, so that a 32-entry window starting anywhere can be read
+        // with aligned 16-byte loads), and W buffer 0 = 0; then a barrier among
+        // the 16 warps that use them
+        const int t = tid - 128;
+        const double l2 = log2(static_cast<double>(lam));
+        for (int n = t; n <= kTB; n += kThreads - 128) pw[n] = static_cast<float>(exp2(n * l2));
+        if (t < 16) murev[t] = static_cast<float>(exp2((15 - t) * l2));
+        for (int idx = t; idx < 4 * 64; idx += kThreads - 128) {
+            const int k = idx >> 6, j = idx & 63, m = j + k;
+            float* zc = reinterpret_cast<float*>(smem_raw + L::kZ + k * L::kZstride);
+            zc[j] = m >= 31 ? static_cast<float>(exp2((m - 31) * l2)) : 0.f;
+        }
+        for (uint32_t off = t * 16; off < 2 * L::kWsz; off += (kThreads - 128) * 16)
+            st_shared_v4(sW + off, 0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
+        named_barrier_sync(1, kThreads - 128);
+    }
     // TMEM: S / P in two buffers (128 columns each), X in NX buffers (DC each),
     // then (DC = 64) a dW buffer; otherwise dW of tile s goes to the X buffer of
     // tile s+1: X of tile s-1 has been read out of it, and X of tile s+1 is not
