@@ -101,14 +101,15 @@ struct RingCfg {
     static constexpr int NCF = kTf32 ? 2 : 0;                // fp32 C (tf32 mode)
     static constexpr int NWB = kTf32 ? 1 : 0;                // fp32 w_s B (tf32 mode)
     static constexpr int NW = DA == 64 ? 2 : 1;              // W as its hi/lo pair
-    // DC = 64 (kOwnD): X += P C (two TMEM buffers), X_inter = A W (one) and
-    // dW (one) are separate accumulators, and the epilogue forms
-    // w_x X_inter + X; X += P C then never waits for the state.  DC = 128: X
-    // (two buffers) holds A W, scaled by w_x in TMEM, then P C; dW borrows the
-    // X buffer of the next tile.
+    // DC = 64 (kOwnD): X += P C (one TMEM buffer), X_inter = A W (one) and
+    // dW (two) are separate accumulators, and the epilogue forms
+    // w_x X_inter + X; X += P C then never waits for the state, and dW of
+    // tile s+1 never waits for the update after tile s.  DC = 128: X (two
+    // buffers) holds A W, scaled by w_x in TMEM, then P C; dW borrows the X
+    // buffer of the next tile.
     static constexpr bool kOwnD = DC == 64;
-    static constexpr int ND = 1;
-    static constexpr int NX = 2;                             // X accumulators in TMEM
+    static constexpr int ND = kOwnD ? 2 : 1;                 // dW accumulators (own-D)
+    static constexpr int NX = kOwnD ? 1 : 2;                 // X accumulators in TMEM
     static constexpr int NXW = kOwnD ? 1 : NX;               // XW_DONE barriers
     static constexpr int NXS = kOwnD ? 0 : NX;               // XS barriers (scaled in TMEM)
     static constexpr int NXI = kOwnD ? 1 : 0;                // EMPTY_XI (X_inter read out)
@@ -208,6 +209,11 @@ __device__ __forceinline__ void load_box(uint32_t dst, const CUtensorMap* map, u
     const int b = bh / H, h = bh - b * H;
     if (bthd) tma_load_4d(dst, map, bar, x, h, t, b);
     else tma_load_4d(dst, map, bar, x, t, h, b);
+}
+__device__ __forceinline__ void prefetch_box(const CUtensorMap* map, int x, int t, int bh, int H, int bthd) {
+    const int b = bh / H, h = bh - b * H;
+    if (bthd) tma_prefetch_4d(map, x, h, t, b);
+    else tma_prefetch_4d(map, x, t, h, b);
 }
 
 // Bounded wait that also gives up as soon as another role has aborted.  The
@@ -338,7 +344,7 @@ la2_scan_ws(const __grid_constant__ Params p)
         named_barrier_sync(1, kThreads - 128);
     }
     // TMEM: S / P in two buffers (128 columns each), X in NX buffers (DC each),
-    // then (DC = 64) a dW buffer; otherwise dW of tile s goes to the X buffer of
+    // then (DC = 64) X_inter and ND dW buffers; otherwise dW of tile s goes to the X buffer of
     // tile s+1: X of tile s-1 has been read out of it, and X of tile s+1 is not
     // issued before the state update has read dW.
     auto tS = [&](int b) { return tmem + static_cast<uint32_t>(b * 128); };
@@ -373,12 +379,18 @@ la2_scan_ws(const __grid_constant__ Params p)
                 for (int gg = 0; gg < DA / 64; ++gg)
                     load_box(sA + slot * L::kAsz + gg * 16384, &R.ta, b, gg * 64, tile_of(s) * kTB, bh, p.H, p.bthd);
             };
+            // A of step s is also read by X_inter = A W, which waits for the
+            // state, so its buffer comes free late; an L2 prefetch of it, made
+            // when B of step s is loaded, takes the HBM latency off that load
             auto load_b = [&](int s) {
                 const int slot = s % Q::NB;
                 const uint32_t b = bar(Q::FULL_B + slot);
                 mbar_arrive_expect_tx(b, L::kBsz);
                 for (int gg = 0; gg < DA / 64; ++gg)
                     load_box(sB + slot * L::kBsz + gg * 16384, &R.tb, b, gg * 64, tile_of(s) * kTB, bh, p.H, p.bthd);
+                if (s >= Q::NA)
+                    for (int gg = 0; gg < DA / 64; ++gg)
+                        prefetch_box(&R.ta, gg * 64, tile_of(s) * kTB, bh, p.H, p.bthd);
             };
             auto load_c = [&](int s) {
                 const int slot = s % Q::NC;
