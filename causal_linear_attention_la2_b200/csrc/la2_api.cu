@@ -7,6 +7,7 @@
 
 #include <cstdint>
 #include <cstdlib>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -44,7 +45,10 @@ EncodeTiledFn encode_fn() {
 
 template <int DA, int DC>
 bool set_ws_attrs() {
-    return cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC>,
+    return cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC, false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                la2::ws::Smem<DA, DC>::kBytes) == cudaSuccess &&
+           cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC, true>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 la2::ws::Smem<DA, DC>::kBytes) == cudaSuccess &&
            cudaFuncSetAttribute(la2::ws::la2_state_ws<DA, DC>,
@@ -52,15 +56,28 @@ bool set_ws_attrs() {
                                 la2::ws::StateSmem<DA, DC>::kBytes) == cudaSuccess;
 }
 
-// Sequence segments for the bf16 kernel.  Each CTA takes one (sequence,
-// role, segment) and fills one SM; when there are fewer (sequence, role)
-// units than the B200's 148 SMs, each sequence is cut into segments so that
-// the grid fills the GPU (a state pre-pass hands each segment its incoming
-// state).  The count depends on the number of units only, never on T, so the
-// workspace it needs is flat in T; per call it is further capped so that a
-// segment holds at least two tiles.
+// How the bf16 kernel spreads its (sequence, role) units over CTAs.  Each CTA
+// fills one SM (148 on a B200).  Two plans:
+//
+// - uniform: each unit is cut into g equal segments, one CTA each; g > 1 only
+//   when there are fewer units than SMs, and depends on the number of units
+//   only (the workspace is flat in T);
+// - balanced: the units' tiles are laid end to end and CTA c takes tiles
+//   [c L, (c+1) L), L = ceil(total / 148): one wave, every SM the same work,
+//   a CTA running the end of one unit and the start of the next one after the
+//   other.  At most 147 segments end inside a unit, so the workspace is flat
+//   in T as well.
+//
+// A segment that does not start its unit gets its incoming state from the
+// state pre-pass, which reads that unit's B and C up to the segment.  The plan
+// with the lower modelled time is taken, in units of one tile of the scan:
+// kFill per segment a CTA runs (pipeline fill and drain) and kPreTile per
+// tile of the pre-pass, plus kPreFill per pre-pass CTA.
 constexpr int kTargetCTAs = 148;
 constexpr int kMaxSegments = 32;
+constexpr double kFill = 1.5, kPreTile = 0.4, kPreFill = 0.5;
+
+std::atomic<int> g_schedule{LA2_SCHEDULE_AUTO};
 
 int max_segments(long long units) {
     if (units <= 0 || units >= kTargetCTAs) return 1;
@@ -69,24 +86,64 @@ int max_segments(long long units) {
 }
 
 struct SegPlan {
-    int nseg, seg_tiles;
+    int balanced = 0;
+    int nseg = 1;        // uniform: segments per unit
+    int seg_tiles = 1;   // L
+    long long nctas = 0, npre = 0;  // scan and pre-pass grids
+    long long slots = 0;            // fp32 DA x DC states in the workspace
+    double cost = 0;
 };
 
-SegPlan plan_segments(long long units, int T) {
-    const int nb = (T + la2::ws::kTB - 1) / la2::ws::kTB;
+long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+SegPlan uniform_plan(long long units, int nb) {
     int g = max_segments(units);
     const int cap = nb / 2 > 1 ? nb / 2 : 1;
     if (g > cap) g = cap;
     SegPlan sp;
-    sp.seg_tiles = (nb + g - 1) / g;
-    sp.nseg = (nb + sp.seg_tiles - 1) / sp.seg_tiles;
+    sp.seg_tiles = static_cast<int>(cdiv(nb, g));
+    sp.nseg = static_cast<int>(cdiv(nb, sp.seg_tiles));
+    sp.nctas = units * sp.nseg;
+    sp.npre = units * (sp.nseg - 1);
+    sp.slots = sp.npre;
+    sp.cost = cdiv(sp.nctas, kTargetCTAs) * (sp.seg_tiles + kFill) +
+              (sp.npre > 0 ? cdiv(sp.npre, kTargetCTAs) * (sp.seg_tiles * kPreTile + kPreFill) : 0.0);
     return sp;
 }
 
+// Returns false when the balanced plan does not apply (segment length out of
+// the kernel's int range).
+bool balanced_plan(long long units, int nb, SegPlan* out) {
+    const long long total = units * nb;
+    const long long L = cdiv(total, kTargetCTAs);
+    if (L < 1 || L > (1LL << 28)) return false;
+    SegPlan sp;
+    sp.balanced = 1;
+    sp.seg_tiles = static_cast<int>(L);
+    sp.nctas = cdiv(total, L);
+    const bool split = L % nb != 0;  // some CTA boundary falls inside a unit
+    sp.npre = split ? sp.nctas - 1 : 0;
+    sp.slots = sp.npre;
+    const long long items = (L + nb - 2) / nb + 1;  // segments one CTA may run
+    sp.cost = L + kFill * items + (split ? (L < nb - 1 ? L : nb - 1) * kPreTile + kPreFill : 0.0);
+    *out = sp;
+    return true;
+}
+
+SegPlan plan_segments(long long units, int T) {
+    const int nb = (T + la2::ws::kTB - 1) / la2::ws::kTB;
+    const SegPlan u = uniform_plan(units, nb);
+    SegPlan b;
+    const int mode = g_schedule.load();
+    if (mode == LA2_SCHEDULE_UNIFORM || !balanced_plan(units, nb, &b)) return u;
+    if (mode == LA2_SCHEDULE_BALANCED) return b;
+    return b.cost < 0.95 * u.cost ? b : u;
+}
+
 // Workspace bytes of one bf16 launch over `units` (sequence, role) units.
-size_t seg_workspace_bytes(long long units, int da, int dc) {
-    return static_cast<size_t>(max_segments(units) - 1) * static_cast<size_t>(units) *
-           static_cast<size_t>(da) * static_cast<size_t>(dc) * sizeof(float);
+size_t seg_workspace_bytes(long long units, int T, int da, int dc) {
+    return static_cast<size_t>(plan_segments(units, T).slots) * static_cast<size_t>(da) *
+           static_cast<size_t>(dc) * sizeof(float);
 }
 
 struct DeviceState {
@@ -169,18 +226,21 @@ la2_status common_checks(int B, int H, int T, int d, int e, int block, la2_dtype
 }
 
 template <int DA, int DC>
-void launch_ws(const la2::ws::Params& p, unsigned units, cudaStream_t stream) {
-    if (p.nseg > 1)
-        la2::ws::la2_state_ws<DA, DC><<<units * static_cast<unsigned>(p.nseg - 1),
-                                        la2::ws::kStateThreads,
+void launch_ws(const la2::ws::Params& p, const SegPlan& sp, cudaStream_t stream) {
+    if (sp.npre > 0)
+        la2::ws::la2_state_ws<DA, DC><<<static_cast<unsigned>(sp.npre), la2::ws::kStateThreads,
                                         la2::ws::StateSmem<DA, DC>::kBytes, stream>>>(p);
-    la2::ws::la2_scan_ws<DA, DC><<<units * static_cast<unsigned>(p.nseg), la2::ws::kThreads,
-                                   la2::ws::Smem<DA, DC>::kBytes, stream>>>(p);
+    if (sp.balanced)
+        la2::ws::la2_scan_ws<DA, DC, true><<<static_cast<unsigned>(sp.nctas), la2::ws::kThreads,
+                                             la2::ws::Smem<DA, DC>::kBytes, stream>>>(p);
+    else
+        la2::ws::la2_scan_ws<DA, DC, false><<<static_cast<unsigned>(sp.nctas), la2::ws::kThreads,
+                                              la2::ws::Smem<DA, DC>::kBytes, stream>>>(p);
 }
 
-// Launches the warp-specialised kernel over `n` roles that share (DA, DC):
-// one CTA per (sequence, role, segment), preceded by the state pre-pass when
-// sequences are split into segments.
+// Launches the warp-specialised kernel over `n` roles that share (DA, DC),
+// with the CTAs of plan_segments, preceded by the state pre-pass when some
+// segment starts inside its unit.
 la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
                           bool bthd, int* status, float* seg_state, cudaStream_t stream) {
     la2::ws::Params p;
@@ -204,17 +264,19 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
     p.nroles = n;
     p.bthd = bthd ? 1 : 0;
     const SegPlan sp = plan_segments(static_cast<long long>(BH) * n, T);
+    p.nunits = BH * n;
     p.nseg = sp.nseg;
     p.seg_tiles = sp.seg_tiles;
+    p.balanced = sp.balanced;
     p.seg_state = seg_state;
-    if (sp.nseg > 1 && !seg_state) return LA2_ERR_WORKSPACE;
-    const unsigned units = static_cast<unsigned>(BH * n);
-    if (da == 128 && dc == 128) launch_ws<128, 128>(p, units, stream);
-    else if (da == 128) launch_ws<128, 64>(p, units, stream);
-    else if (dc == 128) launch_ws<64, 128>(p, units, stream);
-    else launch_ws<64, 64>(p, units, stream);
+    if (sp.slots > 0 && !seg_state) return LA2_ERR_WORKSPACE;
+    if (sp.nctas > 0x7fffffffLL) return LA2_ERR_UNSUPPORTED;
+    if (da == 128 && dc == 128) launch_ws<128, 128>(p, sp, stream);
+    else if (da == 128) launch_ws<128, 64>(p, sp, stream);
+    else if (dc == 128) launch_ws<64, 128>(p, sp, stream);
+    else launch_ws<64, 64>(p, sp, stream);
     if (cudaGetLastError() != cudaSuccess) return LA2_ERR_CUDA;
-    t_last_launches += sp.nseg > 1 ? 2 : 1;
+    t_last_launches += sp.npre > 0 ? 2 : 1;
     return LA2_OK;
 }
 
@@ -270,10 +332,10 @@ la2_status for_role_groups(const RoleDesc* roles, int n, F&& f) {
     return LA2_OK;
 }
 
-size_t bf16_workspace_bytes(const RoleDesc* roles, int n, int B, int H) {
+size_t bf16_workspace_bytes(const RoleDesc* roles, int n, int B, int H, int T) {
     size_t total = 0;
     for_role_groups(roles, n, [&](const RoleDesc* g, int m) {
-        total += seg_workspace_bytes(static_cast<long long>(B) * H * m, g[0].da, g[0].dc);
+        total += seg_workspace_bytes(static_cast<long long>(B) * H * m, T, g[0].da, g[0].dc);
         total = (total + 255) & ~static_cast<size_t>(255);
         return LA2_OK;
     });
@@ -285,15 +347,15 @@ la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, in
                      cudaStream_t stream) {
     int dev = 0;
     int* status = nullptr;
-    if (dtype == LA2_DTYPE_BF16 && bf16_workspace_bytes(roles, n, B, H) > 0 &&
-        (workspace == nullptr || ws_bytes < bf16_workspace_bytes(roles, n, B, H)))
+    if (dtype == LA2_DTYPE_BF16 && bf16_workspace_bytes(roles, n, B, H, T) > 0 &&
+        (workspace == nullptr || ws_bytes < bf16_workspace_bytes(roles, n, B, H, T)))
         return LA2_ERR_WORKSPACE;
     if (!device_setup(&dev, &status)) return LA2_ERR_CUDA;
     if (dtype == LA2_DTYPE_F32) return launch_f32(roles, n, decay, B, H, T, block, bthd, stream);
     size_t off = 0;
     return for_role_groups(roles, n, [&](const RoleDesc* g, int m) {
         float* seg = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) + off) : nullptr;
-        off += seg_workspace_bytes(static_cast<long long>(B) * H * m, g[0].da, g[0].dc);
+        off += seg_workspace_bytes(static_cast<long long>(B) * H * m, T, g[0].da, g[0].dc);
         off = (off + 255) & ~static_cast<size_t>(255);
         return launch_bf16_ws(g, m, decay, B, H, T, bthd, status, seg, stream);
     });
@@ -313,7 +375,14 @@ size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block, la2_dty
     const RoleDesc bwd[3] = {{nullptr, nullptr, nullptr, nullptr, e, d, +1},
                              {nullptr, nullptr, nullptr, nullptr, e, d, -1},
                              {nullptr, nullptr, nullptr, nullptr, d, e, -1}};
-    return is_bwd ? bf16_workspace_bytes(bwd, 3, B, H) : bf16_workspace_bytes(fwd, 1, B, H);
+    return is_bwd ? bf16_workspace_bytes(bwd, 3, B, H, T) : bf16_workspace_bytes(fwd, 1, B, H, T);
+}
+
+la2_schedule la2_set_schedule(la2_schedule schedule) {
+    if (schedule != LA2_SCHEDULE_AUTO && schedule != LA2_SCHEDULE_UNIFORM &&
+        schedule != LA2_SCHEDULE_BALANCED)
+        return static_cast<la2_schedule>(g_schedule.load());
+    return static_cast<la2_schedule>(g_schedule.exchange(schedule));
 }
 
 la2_status la2_fwd_ex(const void* q, const void* k, const void* v, const float* decay, void* out,

@@ -75,13 +75,37 @@ struct Params {
     Role role[3];
     const float* decay;  // [H]
     int* status;         // device status word
-    float* seg_state;    // [B*H][nroles][nseg - 1][DA][DC] fp32: local end state of each
-                         // segment but the last (written by the state pass)
+    float* seg_state;    // [slots][DA][DC] fp32: local end state of each segment but the
+                         // last of its unit (written by the state pass), see seg_slot_index
     int H, T, nroles;
     int bthd;            // 0: tensors [B, H, T, D]; 1: [B, T, H, D] (rows of a sequence H*D apart)
-    int nseg;            // segments per (sequence, role); 1 = no split
-    int seg_tiles;       // tiles per segment (the last may be shorter)
+    int nunits;          // (sequence, role) units, unit u = (sequence u / nroles, role u % nroles)
+    int seg_tiles;       // L: segment length in tiles
+    int balanced;        // 0: every unit is cut into nseg segments [j L, (j+1) L), one CTA
+                         //    each (CTA c: unit c / nseg, segment c % nseg);
+                         // 1: the units' steps laid end to end, CTA c takes global steps
+                         //    [c L, (c+1) L), i.e. the ends of some units and the starts
+                         //    of others, one after the other
+    int nseg;            // balanced = 0: segments per unit (1 = no split)
 };
+
+// Segments of unit u (nb tiles, in scan order).  Boundary j >= 1 sits at step
+// j L - ph(u), where ph(u) = (u nb) mod L in the balanced plan (the boundaries
+// are the CTA boundaries of the global step axis) and 0 otherwise.
+// (`balanced` is p.balanced, passed separately so that a kernel that knows it
+// at compile time drops the other branch.)
+__device__ __forceinline__ int seg_phase(const Params& p, bool balanced, int u, int nb) {
+    return balanced ? static_cast<int>((static_cast<long long>(u) * nb) % p.seg_tiles) : 0;
+}
+__device__ __forceinline__ int seg_begin(const Params& p, bool balanced, int u, int j, int nb) {
+    return j == 0 ? 0 : min(nb, j * p.seg_tiles - seg_phase(p, balanced, u, nb));
+}
+// Slot in seg_state of segment j (not the unit's last): balanced, the index of
+// the CTA boundary that ends it, minus one; otherwise u (nseg - 1) + j.
+__device__ __forceinline__ long long seg_slot_index(const Params& p, bool balanced, int u, int j, int nb) {
+    return balanced ? static_cast<long long>(u) * nb / p.seg_tiles + j
+                    : static_cast<long long>(u) * (p.nseg - 1) + j;
+}
 
 // Buffer counts and mbarrier indices of the scan kernel for (DA, DC).
 //
@@ -173,7 +197,7 @@ struct Smem {
     static constexpr uint32_t kZ = kMuRev + 64;               // diagonal-block weights, 4 shifted copies
     static constexpr uint32_t kZstride = 72 * 4;              // bytes per copy (72 = 8 mod 32 floats)
     static constexpr uint32_t kBar = kZ + 4 * kZstride;
-    static constexpr uint32_t kTmemSlot = kBar + Q::NBARS * 8;
+    static constexpr uint32_t kTmemSlot = kBar + 2 * Q::NBARS * 8;  // two barrier sets
     static constexpr uint32_t kAbort = kTmemSlot + 4;
     static constexpr uint32_t kBytes = kAbort + 12;
     static_assert(kBytes <= 232448, "shared memory over the 227 KB per-CTA limit");
@@ -267,7 +291,10 @@ __device__ __forceinline__ uint32_t empty_par(int s, int n) {
 // from the state the segments before it leave behind,
 // W_in(g) = sum_{g' < g} lambda^(T_B n (g-1-g')) S_g' (n tiles per segment),
 // read from seg_state (written by la2_state_ws).
-template <int DA, int DC>
+// kMulti: the balanced plan's CTAs, which may run several segments (a
+// separate instantiation, so that the one-segment kernel carries no loop
+// state in its registers).
+template <int DA, int DC, bool kMulti>
 __global__ void __launch_bounds__(kThreads, 1)
 la2_scan_ws(const __grid_constant__ Params p)
 {
@@ -285,23 +312,16 @@ la2_scan_ws(const __grid_constant__ Params p)
     const uint32_t sCF = base + L::kCF, sWB = base + L::kWB;
     float* pw = reinterpret_cast<float*>(smem_raw + L::kPow);
     float* murev = reinterpret_cast<float*>(smem_raw + L::kMuRev);
-    auto bar = [&](int b) { return base + L::kBar + 8u * b; };
+    // Two sets of barriers: segment i of a CTA uses set i % 2, so that a set
+    // is initialised again only after a whole segment has run since its last
+    // use (no arrival of a finished segment can still be on its way then).
+    uint32_t bar_set = base + L::kBar;
+    auto bar = [&](int b) { return bar_set + 8u * b; };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + L::kAbort);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int segs_in_grid = p.nseg;
-    const int g = blockIdx.x % segs_in_grid;
-    const int unit = blockIdx.x / segs_in_grid;  // (sequence, role)
-    const int role_id = unit % p.nroles;
-    const int bh = unit / p.nroles;
-    const Role& R = p.role[role_id];
-    const int dir = R.dir;
     const int T = p.T;
     const int nb = (T + kTB - 1) / kTB;
-    // this CTA's steps (in scan order): [s0, s0 + ns)
-    const int s0 = g * p.seg_tiles;
-    const int ns = max(0, min(p.seg_tiles, nb - s0));
-    const float lam = p.decay[bh % p.H];
 
     if (tid == 0) LA2_TR(0, 0);
     // ---- set-up: TMEM and barriers here; the decay tables and W buffer 0 are
@@ -312,7 +332,7 @@ la2_scan_ws(const __grid_constant__ Params p)
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int b = 0; b < Q::NBARS; ++b) mbar_init(bar(b), Q::count(b));
+        for (int b = 0; b < (kMulti ? 2 : 1) * Q::NBARS; ++b) mbar_init(bar(b), Q::count(b % Q::NBARS));
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -323,6 +343,46 @@ la2_scan_ws(const __grid_constant__ Params p)
 
     if (tid == 0) LA2_TR(1, 0);
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_raw + L::kTmemSlot);
+
+    // ---- the CTA's segments, one after the other: one in the uniform plan;
+    // in the balanced plan the pieces of the units its global steps cover
+    for (int item = 0; item < (kMulti ? 0x7fffffff : 1); ++item) {
+    int unit, sj, s0, ns;  // (sequence, role), segment, its steps [s0, s0 + ns)
+    if (!kMulti) {
+        unit = blockIdx.x / p.nseg;
+        sj = blockIdx.x % p.nseg;
+        s0 = seg_begin(p, kMulti, unit, sj, nb);
+        ns = max(0, seg_begin(p, kMulti, unit, sj + 1, nb) - s0);
+    } else {
+        // global steps [c0, c1) of this CTA; item i is the piece of unit
+        // c0 / nb + i they cover
+        const long long c0 = static_cast<long long>(blockIdx.x) * p.seg_tiles;
+        const long long c1 = min(c0 + p.seg_tiles, static_cast<long long>(p.nunits) * nb);
+        unit = static_cast<int>(c0 / nb) + item;
+        const long long ub = static_cast<long long>(unit) * nb;
+        if (ub >= c1) break;
+        s0 = static_cast<int>(max(c0 - ub, 0LL));
+        ns = static_cast<int>(min(static_cast<long long>(nb), c1 - ub)) - s0;
+        sj = (s0 + seg_phase(p, kMulti, unit, nb)) / p.seg_tiles;
+    }
+    bar_set = base + L::kBar + static_cast<uint32_t>(item & 1) * (Q::NBARS * 8);
+    if (item > 1) {
+        // set item % 2 was last used two segments ago: fresh barriers
+        if (tid == 0) {
+            for (int b = 0; b < Q::NBARS; ++b) {
+                mbar_inval(bar(b));
+                mbar_init(bar(b), Q::count(b));
+            }
+            fence_mbar_init();
+        }
+        __syncthreads();
+    }
+    const int role_id = unit % p.nroles;
+    const int bh = unit / p.nroles;
+    const Role& R = p.role[role_id];
+    const int dir = R.dir;
+    const bool unit_end = s0 + ns == nb;  // the segment holds the unit's last step
+    const float lam = p.decay[bh % p.H];
     if (warp >= 4) {
         // lambda^n (n = 0..T_B), lambda^(15-n), the diagonal-block table
         // Z[m] = lambda^(m-31) for m >= 31, else 0 (m = 0..66; copy k holds
@@ -359,7 +419,7 @@ la2_scan_ws(const __grid_constant__ Params p)
     auto tile_of = [&](int step) { return dir > 0 ? s0 + step : nb - 1 - (s0 + step); };
     // fp32 state slot of segment gg of this (sequence, role)
     auto seg_slot = [&](int gg) {
-        return p.seg_state + (static_cast<size_t>(unit) * (p.nseg - 1) + gg) * (DA * DC);
+        return p.seg_state + static_cast<size_t>(seg_slot_index(p, kMulti, unit, gg, nb)) * (DA * DC);
     };
 
     if (warp == 0) {
@@ -641,7 +701,7 @@ la2_scan_ws(const __grid_constant__ Params p)
         const int nlast = T - (nb - 1) * kTB;
         const float ws_last = r < nlast ? pw[max(nlast - 1 - r, 0)] : 0.f;
         auto ws_of = [&](int s) {
-            return (dir > 0 && g == p.nseg - 1 && s == ns - 1) ? ws_last : ws;
+            return (dir > 0 && unit_end && s == ns - 1) ? ws_last : ws;
         };
         // P = S * lambda^|r-c| on the causal side, 0 elsewhere, 32 columns (one
         // pair of K = 16 groups) at a time.  pr == quad is the diagonal block;
@@ -831,12 +891,15 @@ la2_scan_ws(const __grid_constant__ Params p)
         float wreg[kWReg ? 32 : 1];
 #pragma unroll
         for (int u = 0; u < (kWReg ? 32 : 1); ++u) wreg[u] = 0.f;
-        // initial state of this segment, W_in(g) = f W_in(g-1) + S_{g-1} with
-        // f = lambda^(T_B n) and W_in(0) the given initial state (or 0), as its
-        // hi/lo bf16 pair in W buffer 0
-        if ((g > 0 || R.init != nullptr) && owns_w_row) {
-            const float f = static_cast<float>(
-                exp2(static_cast<double>(kTB) * p.seg_tiles * log2(static_cast<double>(lam))));
+        // initial state of this segment, W_in(j) = f_{j-1} W_in(j-1) + S_{j-1}
+        // with f_i = lambda^(T_B n_i) (n_i tiles in segment i: L, except for
+        // segment 0, which ends at step L - ph) and W_in(0) the given initial
+        // state (or 0), as its hi/lo bf16 pair in W buffer 0
+        if ((sj > 0 || R.init != nullptr) && owns_w_row) {
+            const double l2 = log2(static_cast<double>(lam));
+            const float fL = static_cast<float>(exp2(static_cast<double>(kTB) * p.seg_tiles * l2));
+            const float f0 = static_cast<float>(
+                exp2(static_cast<double>(kTB) * (p.seg_tiles - seg_phase(p, kMulti, unit, nb)) * l2));
             const float* w0 =
                 R.init ? R.init + static_cast<size_t>(bh) * (DA * DC) + static_cast<size_t>(wrow) * DC : nullptr;
 #pragma unroll
@@ -845,7 +908,8 @@ la2_scan_ws(const __grid_constant__ Params p)
                 float w[16];
 #pragma unroll
                 for (int u = 0; u < 16; ++u) w[u] = w0 ? w0[col + u] : 0.f;
-                for (int gp = 0; gp < g; ++gp) {
+                for (int gp = 0; gp < sj; ++gp) {
+                    const float f = gp == 0 ? f0 : fL;
                     const float* src = seg_slot(gp) + static_cast<size_t>(wrow) * DC + col;
 #pragma unroll
                     for (int u = 0; u < 16; ++u) w[u] = fmaf(f, w[u], src[u]);
@@ -897,7 +961,7 @@ la2_scan_ws(const __grid_constant__ Params p)
         // W <- lambda^T_B W + dW, from W buffer s % NW into (s+1) % NW.  The
         // state is kept as its hi + lo bf16 pair (a 16-bit significand, ~2^-17
         // relative per update), which is also the next tile's MMA operand.
-        const bool has_last = dir > 0 && g == p.nseg - 1;
+        const bool has_last = dir > 0 && unit_end;
         const int nlast = T - (nb - 1) * kTB;
         auto update = [&](int s) -> bool {
             const bool last = has_last && s == ns - 1;
@@ -1088,13 +1152,21 @@ la2_scan_ws(const __grid_constant__ Params p)
         }
     }
 
-    // ---- tear-down: wait (bounded) until the issuers' MMAs are done, free TMEM
+    // ---- end of the segment: wait (bounded) until the issuers' MMAs are done
     __syncthreads();
     if (tid == 32 && ns > 0) {
-        if (!mbar_wait(bar(Q::FIN), 0)) atomicCAS(p.status, 0, 5 | (60 << 8));
+        if (!mbar_wait(bar(Q::FIN), 0)) {
+            *abort_flag = 1;
+            atomicCAS(p.status, 0, 5 | (60 << 8));
+        }
     }
     tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    if (*abort_flag) break;
+    }  // segments
+
+    // ---- tear-down: free TMEM
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
@@ -1150,16 +1222,32 @@ la2_state_ws(const __grid_constant__ Params p)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + L::kAbort);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int segs_in_grid = p.nseg - 1;
-    const int g = blockIdx.x % segs_in_grid;
-    const int unit = blockIdx.x / segs_in_grid;
+    const int nb = (p.T + kTB - 1) / kTB;
+    int unit, s0, ns;  // (sequence, role) and the segment's steps [s0, s0 + ns)
+    long long slot;    // its slot in seg_state
+    if (!p.balanced) {
+        const int sj = blockIdx.x % (p.nseg - 1);
+        unit = blockIdx.x / (p.nseg - 1);
+        s0 = seg_begin(p, false, unit, sj, nb);
+        ns = max(0, seg_begin(p, false, unit, sj + 1, nb) - s0);
+        slot = seg_slot_index(p, false, unit, sj, nb);
+    } else {
+        // the segment that ends at boundary blockIdx.x + 1 of the scan's CTAs,
+        // if that boundary falls inside a unit
+        const long long gend = (static_cast<long long>(blockIdx.x) + 1) * p.seg_tiles;
+        if (gend >= static_cast<long long>(p.nunits) * nb) return;
+        unit = static_cast<int>(gend / nb);
+        const int eloc = static_cast<int>(gend - static_cast<long long>(unit) * nb);
+        if (eloc == 0) return;
+        s0 = static_cast<int>(max(gend - p.seg_tiles, static_cast<long long>(unit) * nb) -
+                              static_cast<long long>(unit) * nb);
+        ns = eloc - s0;
+        slot = blockIdx.x;
+    }
     const int role_id = unit % p.nroles;
     const int bh = unit / p.nroles;
     const Role& R = p.role[role_id];
     const int dir = R.dir;
-    const int nb = (p.T + kTB - 1) / kTB;
-    const int s0 = g * p.seg_tiles;
-    const int ns = max(0, min(p.seg_tiles, nb - s0));
     const double l2 = log2(static_cast<double>(p.decay[bh % p.H]));
     auto tile_of = [&](int step) { return dir > 0 ? s0 + step : nb - 1 - (s0 + step); };
 
@@ -1259,8 +1347,7 @@ la2_state_ws(const __grid_constant__ Params p)
             const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
             const bool owns_row = (DA == 128) || (lane < 16);
             const int srow = (DA == 128) ? r : quad * 16 + (lane & 15);
-            float* dst0 = p.seg_state + (static_cast<size_t>(unit) * (p.nseg - 1) + g) * (DA * DC) +
-                          static_cast<size_t>(srow) * DC;
+            float* dst0 = p.seg_state + static_cast<size_t>(slot) * (DA * DC) + static_cast<size_t>(srow) * DC;
 #pragma unroll 1
             for (int k = 0; k < DC / 32; ++k) {
                 const int col = part * (DC / 2) + k * 16;

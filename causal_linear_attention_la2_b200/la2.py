@@ -28,11 +28,16 @@ LA2_DTYPE_BF16 = 1
 # Every entry point include/la2.h declares.
 EXPORTS = ("la2_workspace_bytes", "la2_fwd", "la2_fwd_state", "la2_fwd_ex", "la2_bwd", "la2_bwd_ex",
            "la2_decode", "la2_status_str", "la2_device_status", "la2_last_launch_count",
-           "la2_fwd_noalloc")
+           "la2_fwd_noalloc", "la2_set_schedule")
 
 LA2_LAYOUT_BHTD = 0
 LA2_LAYOUT_BTHD = 1
 _LAYOUTS = {"bhtd": LA2_LAYOUT_BHTD, "bthd": LA2_LAYOUT_BTHD}
+
+LA2_SCHEDULE_AUTO = 0
+LA2_SCHEDULE_UNIFORM = 1
+LA2_SCHEDULE_BALANCED = 2
+_SCHEDULES = {"auto": LA2_SCHEDULE_AUTO, "uniform": LA2_SCHEDULE_UNIFORM, "balanced": LA2_SCHEDULE_BALANCED}
 
 
 class LA2Error(RuntimeError):
@@ -76,6 +81,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la2_last_launch_count.restype = i
     lib.la2_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
     lib.la2_fwd_noalloc.restype = i
+    lib.la2_set_schedule.argtypes = [i]
+    lib.la2_set_schedule.restype = i
     _lib = lib
     return lib
 
@@ -98,6 +105,13 @@ def la2_device_status(reset: bool = True) -> int:
 
 def la2_last_launch_count() -> int:
     return int(load().la2_last_launch_count())
+
+
+def la2_set_schedule(schedule: str) -> str:
+    """Sets how the bf16 kernels spread their work over CTAs ("auto",
+    "uniform" or "balanced"); returns the previous setting."""
+    prev = int(load().la2_set_schedule(_SCHEDULES[schedule]))
+    return {v: k for k, v in _SCHEDULES.items()}[prev]
 
 
 # ---------------------------------------------------------------- raw C calls

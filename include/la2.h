@@ -88,14 +88,39 @@ typedef enum {
 /*
  * Bytes of device workspace la2_fwd (is_bwd = 0) or la2_bwd (is_bwd = 1) needs
  * for these sizes.  The state carried along a sequence (d x e) stays on chip;
- * the workspace only holds, when there are too few sequences to fill the
- * GPU's SMs, the fp32 end state of each segment a sequence is cut into (up to
- * 32 segments per sequence, never more than 148 CTAs' worth in total).  The
- * value does not depend on T.  0 means the call accepts workspace = NULL.
- * Returns (size_t)-1 for arguments the call would reject.
+ * the workspace only holds the fp32 end state of each segment that a sequence
+ * is cut into so that the work fills the GPU's 148 SMs (see la2_schedule): at
+ * most 148 states of d x e floats per group of roles with the same (d, e),
+ * whatever T is.  0 means the call accepts workspace = NULL.  Returns
+ * (size_t)-1 for arguments the call would reject.  The value depends on the
+ * schedule setting in force (la2_set_schedule).
  */
 size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block,
                            la2_dtype dtype, int is_bwd);
+
+/*
+ * How the bf16 kernels spread the (sequence, role) units of a call over CTAs,
+ * one CTA per SM (the scan of each unit is sequential in T):
+ *   UNIFORM  each unit is cut into equal segments, one CTA each, when there
+ *            are fewer units than SMs (otherwise one CTA per unit, in waves);
+ *   BALANCED the units' 128-position tiles are laid end to end and cut into
+ *            148 equal runs, one CTA each, which processes the pieces of
+ *            units its run covers one after the other (one wave, equal work);
+ *   AUTO     (default) whichever of the two a cost model of the kernel's
+ *            per-tile time, pipeline fill and state pre-pass rates as faster.
+ * A segment that starts inside its unit receives its incoming state from a
+ * pre-pass over the unit's earlier positions.  Results agree between the
+ * schedules to rounding (the sum is grouped differently).  Process-wide;
+ * returns the previous setting, or leaves it and returns it for an unknown
+ * value.  Change it only between calls; la2_workspace_bytes follows it.
+ */
+typedef enum {
+    LA2_SCHEDULE_AUTO = 0,
+    LA2_SCHEDULE_UNIFORM = 1,
+    LA2_SCHEDULE_BALANCED = 2
+} la2_schedule;
+
+la2_schedule la2_set_schedule(la2_schedule schedule);
 
 /*
  * Forward: out[b,h,t,:] = sum_{s<=t} decay[h]^(t-s) (q[b,h,t,:] . k[b,h,s,:]) v[b,h,s,:].
