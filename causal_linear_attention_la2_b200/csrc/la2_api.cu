@@ -69,13 +69,16 @@ bool set_ws_attrs() {
 //   in T as well.
 //
 // A segment that does not start its unit gets its incoming state from the
-// state pre-pass, which reads that unit's B and C up to the segment.  The plan
-// with the lower modelled time is taken, in units of one tile of the scan:
-// kFill per segment a CTA runs (pipeline fill and drain) and kPreTile per
-// tile of the pre-pass, plus kPreFill per pre-pass CTA.
+// state pre-pass, which reads that unit's B and C up to the segment.  Both
+// plans are modelled in units of one tile of the scan: kFill per segment a
+// CTA runs (pipeline fill and drain) and kPreTile per tile of the pre-pass,
+// plus kPreFill per pre-pass CTA.  The model does not see that a tile takes
+// longer when every SM is busy (measured: 20-40% at d = 128, where the scan
+// approaches the memory system's limit) nor that partial waves run faster, so
+// the balanced plan is taken only when it models kBalancedGain times faster.
 constexpr int kTargetCTAs = 148;
 constexpr int kMaxSegments = 32;
-constexpr double kFill = 1.5, kPreTile = 0.4, kPreFill = 0.5;
+constexpr double kFill = 1.5, kPreTile = 0.4, kPreFill = 0.5, kBalancedGain = 1.0 / 0.75;
 
 std::atomic<int> g_schedule{LA2_SCHEDULE_AUTO};
 
@@ -137,7 +140,7 @@ SegPlan plan_segments(long long units, int T) {
     const int mode = g_schedule.load();
     if (mode == LA2_SCHEDULE_UNIFORM || !balanced_plan(units, nb, &b)) return u;
     if (mode == LA2_SCHEDULE_BALANCED) return b;
-    return b.cost < 0.95 * u.cost ? b : u;
+    return b.cost * kBalancedGain < u.cost ? b : u;
 }
 
 // Workspace bytes of one bf16 launch over `units` (sequence, role) units.

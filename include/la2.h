@@ -106,8 +106,10 @@ size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block,
  *   BALANCED the units' 128-position tiles are laid end to end and cut into
  *            148 equal runs, one CTA each, which processes the pieces of
  *            units its run covers one after the other (one wave, equal work);
- *   AUTO     (default) whichever of the two a cost model of the kernel's
- *            per-tile time, pipeline fill and state pre-pass rates as faster.
+ *   AUTO     (default) UNIFORM, unless a cost model of the kernel's per-tile
+ *            time, pipeline fill and state pre-pass rates BALANCED at least
+ *            4/3 times faster (on a B200 a busier GPU slows every tile, so
+ *            smaller modelled gains did not materialise).
  * A segment that starts inside its unit receives its incoming state from a
  * pre-pass over the unit's earlier positions.  Results agree between the
  * schedules to rounding (the sum is grouped differently).  Process-wide;

@@ -123,3 +123,29 @@ def test_balanced_and_uniform_agree(la2mod):
         a, b = a.float(), b.float()
         rms = a.pow(2).mean().sqrt()
         assert ((a - b).abs().max() / rms).item() < 2e-3
+
+
+@pytest.mark.parametrize("schedule", ["balanced"], indirect=True)
+@pytest.mark.parametrize("name", ["tnl15b", "sweep_T131072_blk128"])
+def test_balanced_full_size_sampled_sequences(la2mod, oracle_mod, schedule, name):
+    """The full-size workloads under the balanced schedule (148 CTAs, runs of
+    26 to 665 tiles, pieces cut inside units), checked on whole sampled
+    sequences: the first, a middle and the last (b, h)."""
+    w = I.WORKLOADS[name]
+    x = I.make_workload_inputs(w, seed=0)
+    dev = torch.device("cuda")
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    lam = x["lam"].to(dev)
+    o = la2mod.la2_fwd(q, k, v, lam)
+    dq, dk, dv = la2mod.la2_bwd(q, k, v, lam, do)
+    torch.cuda.synchronize()
+    assert la2mod.la2_device_status(reset=True) == 0
+    bi = np.array([0, w.B // 2, w.B - 1])
+    hi = np.array([0, w.H // 2, w.H - 1])
+    tb, th = torch.from_numpy(bi), torch.from_numpy(hi)
+    sub = {n: x[n][tb, th] for n in ("q", "k", "v", "do")}
+    lam_s = x["lam"].numpy().astype(np.float64)[hi]
+    ro = oracle_mod.forward(sub["q"], sub["k"], sub["v"], lam_s)
+    rdq, rdk, rdv = oracle_mod.backward(sub["q"], sub["k"], sub["v"], lam_s, sub["do"])
+    errs = [_err(t[tb.to(dev), th.to(dev)], r) for t, r in zip((o, dq, dk, dv), (ro, rdq, rdk, rdv))]
+    assert max(errs) <= TOL, errs
