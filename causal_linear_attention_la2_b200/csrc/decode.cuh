@@ -17,10 +17,10 @@
 
 namespace la2 {
 
-constexpr int kDecThreads = 256;
-
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+constexpr int kDecThreads = 256;
 
 // Shared memory: q and k of the sequence (d floats each) and one partial sum
 // of 4 floats per thread.
@@ -61,26 +61,48 @@ la2_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
             acc[w] = 0.f;
             vv[w] = to_f32(vn[col + w]);
         }
+        // rows rg, rg + rgn, ...: kRows of them loaded before any is stored,
+        // so that the loads of one thread are in flight together
+        auto update_row = [&](int i, float (&sv)[W]) {
+            const float ki = ks[i], qi = qs[i];
+#pragma unroll
+            for (int w = 0; w < W; ++w) {
+                sv[w] = fmaf(lam, sv[w], ki * vv[w]);
+                acc[w] = fmaf(sv[w], qi, acc[w]);
+            }
+        };
+        auto load_row = [&](int i, float (&sv)[W]) {
+            const float* row = S + static_cast<size_t>(i) * e + col;
+            if constexpr (kVec) {
+                const float4 s4 = *reinterpret_cast<const float4*>(row);
+                sv[0] = s4.x; sv[1] = s4.y; sv[2] = s4.z; sv[3] = s4.w;
+            } else {
+                sv[0] = row[0];
+            }
+        };
+        auto store_row = [&](int i, const float (&sv)[W]) {
+            float* row = S + static_cast<size_t>(i) * e + col;
+            if constexpr (kVec) *reinterpret_cast<float4*>(row) = make_float4(sv[0], sv[1], sv[2], sv[3]);
+            else row[0] = sv[0];
+        };
         if (rg < rgn) {
-            for (int i = rg; i < d; i += rgn) {
-                float* row = S + static_cast<size_t>(i) * e + col;
-                const float ki = ks[i], qi = qs[i];
-                if constexpr (kVec) {
-                    float4 s4 = *reinterpret_cast<const float4*>(row);
-                    s4.x = fmaf(lam, s4.x, ki * vv[0]);
-                    s4.y = fmaf(lam, s4.y, ki * vv[1]);
-                    s4.z = fmaf(lam, s4.z, ki * vv[2]);
-                    s4.w = fmaf(lam, s4.w, ki * vv[3]);
-                    *reinterpret_cast<float4*>(row) = s4;
-                    acc[0] = fmaf(s4.x, qi, acc[0]);
-                    acc[1] = fmaf(s4.y, qi, acc[1]);
-                    acc[2] = fmaf(s4.z, qi, acc[2]);
-                    acc[3] = fmaf(s4.w, qi, acc[3]);
-                } else {
-                    const float s1 = fmaf(lam, row[0], ki * vv[0]);
-                    row[0] = s1;
-                    acc[0] = fmaf(s1, qi, acc[0]);
+            constexpr int kRows = 4;
+            int i = rg;
+            for (; i + (kRows - 1) * rgn < d; i += kRows * rgn) {
+                float sv[kRows][W];
+#pragma unroll
+                for (int b = 0; b < kRows; ++b) load_row(i + b * rgn, sv[b]);
+#pragma unroll
+                for (int b = 0; b < kRows; ++b) {
+                    update_row(i + b * rgn, sv[b]);
+                    store_row(i + b * rgn, sv[b]);
                 }
+            }
+            for (; i < d; i += rgn) {
+                float sv[W];
+                load_row(i, sv);
+                update_row(i, sv);
+                store_row(i, sv);
             }
         }
 #pragma unroll

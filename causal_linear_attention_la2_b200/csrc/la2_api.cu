@@ -10,6 +10,7 @@
 #include <atomic>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "decode.cuh"
 #include "la2.h"
@@ -489,26 +490,21 @@ la2_status la2_decode(const void* q, const void* k, const void* v, const float* 
     const dim3 grid(static_cast<unsigned>(B * H));
     const size_t smem = la2::decode_smem_bytes(d);
     const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    auto run = [&](auto tin_tag, auto vec_tag) {
+        using Tin = decltype(tin_tag);
+        constexpr bool kV = decltype(vec_tag)::value;
+        const auto* qt = static_cast<const Tin*>(q);
+        const auto* kt = static_cast<const Tin*>(k);
+        const auto* vt = static_cast<const Tin*>(v);
+        la2::la2_decode_kernel<Tin, kV><<<grid, la2::kDecThreads, smem, cs>>>(qt, kt, vt, decay, state, out, H, d,
+                                                                          e);
+    };
     if (dtype == LA2_DTYPE_BF16) {
-        const auto* qb = static_cast<const __nv_bfloat16*>(q);
-        const auto* kb = static_cast<const __nv_bfloat16*>(k);
-        const auto* vb = static_cast<const __nv_bfloat16*>(v);
-        if (vec)
-            la2::la2_decode_kernel<__nv_bfloat16, true><<<grid, la2::kDecThreads, smem, cs>>>(
-                qb, kb, vb, decay, state, out, H, d, e);
-        else
-            la2::la2_decode_kernel<__nv_bfloat16, false><<<grid, la2::kDecThreads, smem, cs>>>(
-                qb, kb, vb, decay, state, out, H, d, e);
+        if (vec) run(__nv_bfloat16(), std::true_type());
+        else run(__nv_bfloat16(), std::false_type());
     } else {
-        const auto* qf = static_cast<const float*>(q);
-        const auto* kf = static_cast<const float*>(k);
-        const auto* vf = static_cast<const float*>(v);
-        if (vec)
-            la2::la2_decode_kernel<float, true><<<grid, la2::kDecThreads, smem, cs>>>(
-                qf, kf, vf, decay, state, out, H, d, e);
-        else
-            la2::la2_decode_kernel<float, false><<<grid, la2::kDecThreads, smem, cs>>>(
-                qf, kf, vf, decay, state, out, H, d, e);
+        if (vec) run(float(), std::true_type());
+        else run(float(), std::false_type());
     }
     if (cudaGetLastError() != cudaSuccess) return LA2_ERR_CUDA;
     t_last_launches = 1;
