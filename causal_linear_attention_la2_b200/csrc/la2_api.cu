@@ -60,26 +60,25 @@ bool set_ws_attrs() {
 // How the bf16 kernel spreads its (sequence, role) units over CTAs.  Each CTA
 // fills one SM (148 on a B200).  Two plans:
 //
-// - uniform: each unit is cut into g equal segments, one CTA each; g > 1 only
-//   when there are fewer units than SMs, and depends on the number of units
-//   only (the workspace is flat in T);
-// - balanced: the units' tiles are laid end to end and CTA c takes tiles
-//   [c L, (c+1) L), L = ceil(total / 148): one wave, every SM the same work,
-//   a CTA running the end of one unit and the start of the next one after the
-//   other.  At most 147 segments end inside a unit, so the workspace is flat
-//   in T as well.
+// - uniform (the default): each unit is cut into g equal segments, one CTA
+//   each; g > 1 only when there are fewer units than SMs;
+// - balanced (on request, la2_set_schedule): the units' tiles are laid end to
+//   end and CTA c takes tiles [c L, (c+1) L), L = ceil(total / 148): one wave,
+//   every SM the same work, a CTA running the end of one unit and the start of
+//   the next one after the other.
 //
 // A segment that does not start its unit gets its incoming state from the
-// state pre-pass, which reads that unit's B and C up to the segment.  Both
-// plans are modelled in units of one tile of the scan: kFill per segment a
-// CTA runs (pipeline fill and drain) and kPreTile per tile of the pre-pass,
-// plus kPreFill per pre-pass CTA.  The model does not see that a tile takes
-// longer when every SM is busy (measured: 20-40% at d = 128, where the scan
-// approaches the memory system's limit) nor that partial waves run faster, so
-// the balanced plan is taken only when it models kBalancedGain times faster.
+// state pre-pass, which reads that unit's B and C up to the segment.  On a
+// B200 the balanced plan measured no faster on any benchmark shape: a tile
+// takes 20-40% longer once every SM runs the scan (at d = 128 the scan then
+// nears what the memory system delivers), a partial last wave runs faster, and
+// the pre-pass re-reads B and C.
+//
+// Workspace, flat in T in both plans: uniform, (g - 1) states per unit with g
+// from the number of units alone (a short sequence may use fewer); balanced,
+// one state per CTA boundary, at most 147.
 constexpr int kTargetCTAs = 148;
 constexpr int kMaxSegments = 32;
-constexpr double kFill = 1.5, kPreTile = 0.4, kPreFill = 0.5, kBalancedGain = 1.0 / 0.75;
 
 std::atomic<int> g_schedule{LA2_SCHEDULE_AUTO};
 
@@ -94,8 +93,6 @@ struct SegPlan {
     int nseg = 1;        // uniform: segments per unit
     int seg_tiles = 1;   // L
     long long nctas = 0, npre = 0;  // scan and pre-pass grids
-    long long slots = 0;            // fp32 DA x DC states in the workspace
-    double cost = 0;
 };
 
 long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
@@ -109,9 +106,6 @@ SegPlan uniform_plan(long long units, int nb) {
     sp.nseg = static_cast<int>(cdiv(nb, sp.seg_tiles));
     sp.nctas = units * sp.nseg;
     sp.npre = units * (sp.nseg - 1);
-    sp.slots = sp.npre;
-    sp.cost = cdiv(sp.nctas, kTargetCTAs) * (sp.seg_tiles + kFill) +
-              (sp.npre > 0 ? cdiv(sp.npre, kTargetCTAs) * (sp.seg_tiles * kPreTile + kPreFill) : 0.0);
     return sp;
 }
 
@@ -125,29 +119,23 @@ bool balanced_plan(long long units, int nb, SegPlan* out) {
     sp.balanced = 1;
     sp.seg_tiles = static_cast<int>(L);
     sp.nctas = cdiv(total, L);
-    const bool split = L % nb != 0;  // some CTA boundary falls inside a unit
-    sp.npre = split ? sp.nctas - 1 : 0;
-    sp.slots = sp.npre;
-    const long long items = (L + nb - 2) / nb + 1;  // segments one CTA may run
-    sp.cost = L + kFill * items + (split ? (L < nb - 1 ? L : nb - 1) * kPreTile + kPreFill : 0.0);
+    sp.npre = L % nb != 0 ? sp.nctas - 1 : 0;  // some CTA boundary falls inside a unit
     *out = sp;
     return true;
 }
 
 SegPlan plan_segments(long long units, int T) {
     const int nb = (T + la2::ws::kTB - 1) / la2::ws::kTB;
-    const SegPlan u = uniform_plan(units, nb);
     SegPlan b;
-    const int mode = g_schedule.load();
-    if (mode == LA2_SCHEDULE_UNIFORM || !balanced_plan(units, nb, &b)) return u;
-    if (mode == LA2_SCHEDULE_BALANCED) return b;
-    return b.cost * kBalancedGain < u.cost ? b : u;
+    if (g_schedule.load() == LA2_SCHEDULE_BALANCED && balanced_plan(units, nb, &b)) return b;
+    return uniform_plan(units, nb);
 }
 
 // Workspace bytes of one bf16 launch over `units` (sequence, role) units.
 size_t seg_workspace_bytes(long long units, int T, int da, int dc) {
-    return static_cast<size_t>(plan_segments(units, T).slots) * static_cast<size_t>(da) *
-           static_cast<size_t>(dc) * sizeof(float);
+    const size_t state = static_cast<size_t>(da) * static_cast<size_t>(dc) * sizeof(float);
+    if (plan_segments(units, T).balanced) return static_cast<size_t>(kTargetCTAs - 1) * state;
+    return static_cast<size_t>(max_segments(units) - 1) * static_cast<size_t>(units) * state;
 }
 
 struct DeviceState {
@@ -273,7 +261,7 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
     p.seg_tiles = sp.seg_tiles;
     p.balanced = sp.balanced;
     p.seg_state = seg_state;
-    if (sp.slots > 0 && !seg_state) return LA2_ERR_WORKSPACE;
+    if (sp.npre > 0 && !seg_state) return LA2_ERR_WORKSPACE;
     if (sp.nctas > 0x7fffffffLL) return LA2_ERR_UNSUPPORTED;
     if (da == 128 && dc == 128) launch_ws<128, 128>(p, sp, stream);
     else if (da == 128) launch_ws<128, 64>(p, sp, stream);

@@ -90,10 +90,10 @@ typedef enum {
  * for these sizes.  The state carried along a sequence (d x e) stays on chip;
  * the workspace only holds the fp32 end state of each segment that a sequence
  * is cut into so that the work fills the GPU's 148 SMs (see la2_schedule): at
- * most 148 states of d x e floats per group of roles with the same (d, e),
- * whatever T is.  0 means the call accepts workspace = NULL.  Returns
- * (size_t)-1 for arguments the call would reject.  The value depends on the
- * schedule setting in force (la2_set_schedule).
+ * most 147 states of d x e floats per group of roles with the same (d, e).
+ * The value does not depend on T; it depends on the schedule setting in force
+ * (la2_set_schedule).  0 means the call accepts workspace = NULL.  Returns
+ * (size_t)-1 for arguments the call would reject.
  */
 size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block,
                            la2_dtype dtype, int is_bwd);
@@ -106,10 +106,10 @@ size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block,
  *   BALANCED the units' 128-position tiles are laid end to end and cut into
  *            148 equal runs, one CTA each, which processes the pieces of
  *            units its run covers one after the other (one wave, equal work);
- *   AUTO     (default) UNIFORM, unless a cost model of the kernel's per-tile
- *            time, pipeline fill and state pre-pass rates BALANCED at least
- *            4/3 times faster (on a B200 a busier GPU slows every tile, so
- *            smaller modelled gains did not materialise).
+ *   AUTO     (default) the library's choice: UNIFORM, which measured as fast
+ *            or faster on every benchmark shape on a B200 (with every SM busy
+ *            each tile takes longer, and BALANCED re-reads inputs for its
+ *            pre-pass).
  * A segment that starts inside its unit receives its incoming state from a
  * pre-pass over the unit's earlier positions.  Results agree between the
  * schedules to rounding (the sum is grouped differently).  Process-wide;

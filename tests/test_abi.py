@@ -106,18 +106,20 @@ def test_empty_problem_is_ok_and_touches_nothing(lib, kw):
 
 
 @pytest.mark.parametrize("schedule", ["auto", "uniform", "balanced"])
-def test_workspace_is_bounded_in_T(lib, schedule):
-    # at most 148 fp32 d x e segment states per group of roles with one (d, e),
-    # whatever T is
+def test_workspace_is_flat_in_T_and_bounded(lib, schedule):
+    # the same size for every T, and at most 147 fp32 d x e segment states per
+    # group of roles with one (d, e)
     prev = la2.la2_set_schedule(schedule)
     try:
         for B, H in ((1, 16), (1, 1), (3, 7), (64, 64)):
-            for T in (1, 129, 1024, 65536, 1 << 20):
-                for d, e in ((64, 64), (128, 128), (64, 128)):
-                    groups = 1 if d == e else 2
-                    for is_bwd in (0, 1):
-                        n = la2.la2_workspace_bytes(B, H, T, d, e, 128, la2.LA2_DTYPE_BF16, is_bwd)
-                        assert 0 <= n <= groups * (148 * d * e * 4 + 256), (B, H, T, d, e, is_bwd, n)
+            for d, e in ((64, 64), (128, 128), (64, 128)):
+                groups = 1 if d == e else 2
+                for is_bwd in (0, 1):
+                    sizes = {la2.la2_workspace_bytes(B, H, T, d, e, 128, la2.LA2_DTYPE_BF16, is_bwd)
+                             for T in (1, 129, 1024, 65536, 1 << 20)}
+                    assert len(sizes) == 1, (B, H, d, e, is_bwd, sizes)
+                    n = sizes.pop()
+                    assert 0 <= n <= groups * (147 * d * e * 4 + 256), (B, H, d, e, is_bwd, n)
     finally:
         la2.la2_set_schedule(prev)
     assert la2.la2_workspace_bytes(1, 16, 1024, 128, 128, 100, la2.LA2_DTYPE_BF16, 0) == 2 ** 64 - 1
@@ -133,16 +135,6 @@ def test_schedule_setting_round_trips(lib):
         assert la2.la2_set_schedule("auto") == "auto"
     finally:
         la2.la2_set_schedule(prev)
-
-
-def test_uniform_workspace_is_flat_in_T(lib):
-    prev = la2.la2_set_schedule("uniform")
-    try:
-        sizes = {la2.la2_workspace_bytes(1, 16, T, 128, 128, 128, la2.LA2_DTYPE_BF16, 1)
-                 for T in (1024, 65536, 1 << 20)}
-    finally:
-        la2.la2_set_schedule(prev)
-    assert len(sizes) == 1
 
 
 def test_workspace_missing_or_small_is_reported(lib):
