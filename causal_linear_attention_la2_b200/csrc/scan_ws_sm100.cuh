@@ -535,7 +535,11 @@ la2_scan_ws(const __grid_constant__ Params p)
         // X += P C of tile s, P read from S buffer s % 2: in bf16 mode its hi and
         // lo parts per K step of 16; in tf32 mode P is fp32, K steps of 8, with
         // the fp32 copy of C
-        if (lane == 0) {
+        if (Q::kTf32 || lane == 0) {
+            // d = 64: the whole warp runs the issuing loop and lane 0 issues
+            // (warp-uniform descriptor arithmetic measured +4% there); d = 128:
+            // lane 0 alone
+            const uint32_t leader = Q::kTf32 ? lane == 0 : 1;
             constexpr uint32_t kIdX = Q::kTf32 ? idesc_tf32_f32(128, DC, 0, 0)
                                                : idesc_bf16_f32(128, DC, 0, 1);
             const uint64_t dC0 = Q::kTf32 ? sdesc_sw128(sCF, 16, 1024) : sdesc_sw128(sC, 16384, 1024);
@@ -563,28 +567,29 @@ la2_scan_ws(const __grid_constant__ Params p)
                     const uint64_t dc = desc_add(dC0, sc * L::kCFsz);
 #pragma unroll 4
                     for (int k = 0; k < kTB / 8; ++k)
-                        mma_tf32_ts(xt, st + k * 8, desc_add(dc, (k >> 2) * (DC * 128) + (k & 3) * 32),
-                                    kIdX, Q::kOwnD ? (k > 0) : 1);
+                        mma_tf32_ts_w(xt, st + k * 8, desc_add(dc, (k >> 2) * (DC * 128) + (k & 3) * 32),
+                                    kIdX, Q::kOwnD ? (k > 0) : 1, leader);
                 } else {
                     const uint64_t dc = desc_add(dC0, sc * L::kCsz);
 #pragma unroll
                     for (int k = 0; k < kTB / 16; ++k) {
                         const uint64_t cdesc = desc_add(dc, k * 2048);
-                        mma_bf16_ts(xt, st + k * 16, cdesc, kIdX, Q::kOwnD ? (k > 0) : 1);
-                        mma_bf16_ts(xt, st + k * 16 + 8, cdesc, kIdX, 1);
+                        mma_bf16_ts_w(xt, st + k * 16, cdesc, kIdX, Q::kOwnD ? (k > 0) : 1, leader);
+                        mma_bf16_ts_w(xt, st + k * 16 + 8, cdesc, kIdX, 1, leader);
                     }
                 }
-                mma_commit(bar(Q::PC_DONE + s % Q::NX));
-                mma_commit(bar(Q::EMPTY_S + (s & 1)));
-                mma_commit(bar((Q::kTf32 ? Q::EMPTY_CF : Q::EMPTY_C) + sc));
+                mma_commit_w(bar(Q::PC_DONE + s % Q::NX), leader);
+                mma_commit_w(bar(Q::EMPTY_S + (s & 1)), leader);
+                mma_commit_w(bar((Q::kTf32 ? Q::EMPTY_CF : Q::EMPTY_C) + sc), leader);
                 LA2_TR(20, s);
             }
-            mma_commit(bar(Q::FIN));
+            mma_commit_w(bar(Q::FIN), leader);
         }
     } else if (warp == 2) {
         // ================================================= MMA issuer XW
         // X = A hi(W) + A lo(W) into X buffer s % 2
-        if (lane == 0) {
+        if (Q::kTf32 || lane == 0) {
+            const uint32_t leader = Q::kTf32 ? lane == 0 : 1;
             constexpr uint32_t kIdX = idesc_bf16_f32(128, DC, 0, 1);
             const uint64_t dA0 = sdesc_sw128(sA, 16, 1024), dW0 = sdesc_sw128(sW, DA * 128, 1024);
             for (int s = 0; s < ns; ++s) {
@@ -609,21 +614,22 @@ la2_scan_ws(const __grid_constant__ Params p)
 #pragma unroll
                 for (int k = 0; k < DA / 16; ++k) {
                     const uint64_t adesc = desc_add(da, (k >> 2) * 16384 + (k & 3) * 32);
-                    mma_bf16_ss(xt, adesc, desc_add(dw, k * 2048), kIdX, k > 0);
-                    mma_bf16_ss(xt, adesc, desc_add(dw, L::kWsz + k * 2048), kIdX, 1);
+                    mma_bf16_ss_w(xt, adesc, desc_add(dw, k * 2048), kIdX, k > 0, leader);
+                    mma_bf16_ss_w(xt, adesc, desc_add(dw, L::kWsz + k * 2048), kIdX, 1, leader);
                 }
-                mma_commit(bar(Q::XW_DONE + s % Q::NXW));
-                mma_commit(bar(Q::EMPTY_A + sa));
-                mma_commit(bar(Q::EMPTY_W + sw));
+                mma_commit_w(bar(Q::XW_DONE + s % Q::NXW), leader);
+                mma_commit_w(bar(Q::EMPTY_A + sa), leader);
+                mma_commit_w(bar(Q::EMPTY_W + sw), leader);
                 LA2_TR(21, s);
             }
-            mma_commit(bar(Q::FIN));
+            mma_commit_w(bar(Q::FIN), leader);
         }
     } else if (warp == 3) {
         // ================================================= MMA issuer dW
         // dW = (w_s B)^T C of tile s: bf16 mode hi(w_s B)^T C + lo(w_s B)^T C,
         // tf32 mode the fp32 copies of w_s B and C
-        if (lane == 0) {
+        if (Q::kTf32 || lane == 0) {
+            const uint32_t leader = Q::kTf32 ? lane == 0 : 1;
             constexpr uint32_t kIdW = Q::kTf32 ? idesc_tf32_f32(DA, DC, 0, 0) : idesc_bf16_f32(DA, DC, 1, 1);
             const uint64_t dB0 = Q::kTf32 ? sdesc_sw128(sWB, 16, 1024) : sdesc_sw128(sB, 16384, 1024);
             const uint64_t dL0 = sdesc_sw128(sBlo, 16384, 1024);
@@ -658,28 +664,28 @@ la2_scan_ws(const __grid_constant__ Params p)
                     const uint64_t db = desc_add(dB0, sb * L::kWBsz), dc = desc_add(dC0, sc * L::kCFsz);
 #pragma unroll 4
                     for (int k = 0; k < kTB / 8; ++k)
-                        mma_tf32_ss(dt, desc_add(db, (k >> 2) * (DA * 128) + (k & 3) * 32),
-                                    desc_add(dc, (k >> 2) * (DC * 128) + (k & 3) * 32), kIdW, k > 0);
-                    mma_commit(bar(Q::D_DONE + (s % Q::ND)));
-                    mma_commit(bar(Q::EMPTY_WB + sb));
-                    mma_commit(bar(Q::EMPTY_CF + sc));
+                        mma_tf32_ss_w(dt, desc_add(db, (k >> 2) * (DA * 128) + (k & 3) * 32),
+                                    desc_add(dc, (k >> 2) * (DC * 128) + (k & 3) * 32), kIdW, k > 0, leader);
+                    mma_commit_w(bar(Q::D_DONE + (s % Q::ND)), leader);
+                    mma_commit_w(bar(Q::EMPTY_WB + sb), leader);
+                    mma_commit_w(bar(Q::EMPTY_CF + sc), leader);
                 } else {
                     const uint64_t db = desc_add(dB0, sb * L::kBsz), dl = desc_add(dL0, sl * L::kBsz);
                     const uint64_t dc = desc_add(dC0, sc * L::kCsz);
 #pragma unroll
                     for (int k = 0; k < kTB / 16; ++k) {
                         const uint64_t cdesc = desc_add(dc, k * 2048);
-                        mma_bf16_ss(dt, desc_add(db, k * 2048), cdesc, kIdW, k > 0);
-                        mma_bf16_ss(dt, desc_add(dl, k * 2048), cdesc, kIdW, 1);
+                        mma_bf16_ss_w(dt, desc_add(db, k * 2048), cdesc, kIdW, k > 0, leader);
+                        mma_bf16_ss_w(dt, desc_add(dl, k * 2048), cdesc, kIdW, 1, leader);
                     }
-                    mma_commit(bar(Q::D_DONE + (s % Q::ND)));
-                    mma_commit(bar(Q::EMPTY_B + sb));
-                    mma_commit(bar(Q::EMPTY_BLO + sl));
-                    mma_commit(bar(Q::EMPTY_C + sc));
+                    mma_commit_w(bar(Q::D_DONE + (s % Q::ND)), leader);
+                    mma_commit_w(bar(Q::EMPTY_B + sb), leader);
+                    mma_commit_w(bar(Q::EMPTY_BLO + sl), leader);
+                    mma_commit_w(bar(Q::EMPTY_C + sc), leader);
                 }
                 LA2_TR(22, s);
             }
-            mma_commit(bar(Q::FIN));
+            mma_commit_w(bar(Q::FIN), leader);
         }
     } else if (warp >= 4 && warp < 12) {
         // ================================================= mask group
