@@ -106,10 +106,10 @@ size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block,
  *   BALANCED the units' 128-position tiles are laid end to end and cut into
  *            148 equal runs, one CTA each, which processes the pieces of
  *            units its run covers one after the other (one wave, equal work);
- *   AUTO     (default) the library's choice: UNIFORM, which measured as fast
- *            or faster on every benchmark shape on a B200 (with every SM busy
- *            each tile takes longer, and BALANCED re-reads inputs for its
- *            pre-pass).
+ *   AUTO     (default) the library's choice: UNIFORM.  On a B200 BALANCED
+ *            was at best 3% faster on the benchmark shapes and up to 11%
+ *            slower: with every SM busy each tile takes longer, and its
+ *            pre-pass re-reads inputs.
  * A segment that starts inside its unit receives its incoming state from a
  * pre-pass over the unit's earlier positions.  Results agree between the
  * schedules to rounding (the sum is grouped differently).  Process-wide;
