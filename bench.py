@@ -482,6 +482,10 @@ def run_ours(args, w, world, rank, local):
         "gpu_launches": launches,
         "clocks": clk,
     }
+    if w.dtype == "bf16":
+        # the launch plans the two calls ran (schedule, segments, CTAs, pre-pass)
+        line["plan"] = {"fwd": la2.la2_plan_info(w.B, w.H, w.T, w.d, w.e, w.block),
+                        "bwd": la2.la2_plan_info(w.B, w.H, w.T, w.d, w.e, w.block, is_bwd=True)}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_rate(w, x, target_s=args.ref_seconds)
     print(json.dumps(line), flush=True)

@@ -377,6 +377,36 @@ la2_schedule la2_set_schedule(la2_schedule schedule) {
     return static_cast<la2_schedule>(g_schedule.exchange(schedule));
 }
 
+int la2_plan_info(int B, int H, int T, int d, int e, int block, la2_dtype dtype, int is_bwd,
+                  la2_plan* out, int max_out) {
+    bool empty = false;
+    if (common_checks(B, H, T, d, e, block, dtype, &empty) != LA2_OK) return -1;
+    if (empty || dtype != LA2_DTYPE_BF16) return 0;
+    const RoleDesc fwd[1] = {{nullptr, nullptr, nullptr, nullptr, d, e, +1}};
+    const RoleDesc bwd[3] = {{nullptr, nullptr, nullptr, nullptr, e, d, +1},
+                             {nullptr, nullptr, nullptr, nullptr, e, d, -1},
+                             {nullptr, nullptr, nullptr, nullptr, d, e, -1}};
+    int n = 0;
+    for_role_groups(is_bwd ? bwd : fwd, is_bwd ? 3 : 1, [&](const RoleDesc* g, int m) {
+        if (out && n < max_out) {
+            const long long units = static_cast<long long>(B) * H * m;
+            const SegPlan sp = plan_segments(units, T);
+            la2_plan& o = out[n];
+            o.d = g[0].da;
+            o.e = g[0].dc;
+            o.schedule = sp.balanced ? LA2_SCHEDULE_BALANCED : LA2_SCHEDULE_UNIFORM;
+            o.units = units;
+            o.segments = sp.balanced ? 0 : sp.nseg;
+            o.tiles_per_cta = sp.seg_tiles;
+            o.ctas = sp.nctas;
+            o.prepass_ctas = sp.npre;
+        }
+        ++n;
+        return LA2_OK;
+    });
+    return n;
+}
+
 la2_status la2_fwd_ex(const void* q, const void* k, const void* v, const float* decay, void* out,
                       const float* init_state, float* final_state, int B, int H, int T, int d,
                       int e, int block, la2_dtype dtype, la2_layout layout, void* workspace,

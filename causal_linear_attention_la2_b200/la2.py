@@ -28,7 +28,7 @@ LA2_DTYPE_BF16 = 1
 # Every entry point include/la2.h declares.
 EXPORTS = ("la2_workspace_bytes", "la2_fwd", "la2_fwd_state", "la2_fwd_ex", "la2_bwd", "la2_bwd_ex",
            "la2_decode", "la2_status_str", "la2_device_status", "la2_last_launch_count",
-           "la2_fwd_noalloc", "la2_set_schedule")
+           "la2_fwd_noalloc", "la2_set_schedule", "la2_plan_info")
 
 LA2_LAYOUT_BHTD = 0
 LA2_LAYOUT_BTHD = 1
@@ -83,6 +83,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la2_fwd_noalloc.restype = i
     lib.la2_set_schedule.argtypes = [i]
     lib.la2_set_schedule.restype = i
+    lib.la2_plan_info.argtypes = [i, i, i, i, i, i, i, i, ctypes.POINTER(LA2Plan), i]
+    lib.la2_plan_info.restype = i
     _lib = lib
     return lib
 
@@ -105,6 +107,26 @@ def la2_device_status(reset: bool = True) -> int:
 
 def la2_last_launch_count() -> int:
     return int(load().la2_last_launch_count())
+
+
+class LA2Plan(ctypes.Structure):
+    """la2_plan of include/la2.h."""
+    _fields_ = [("d", ctypes.c_int), ("e", ctypes.c_int), ("schedule", ctypes.c_int),
+                ("units", ctypes.c_longlong), ("segments", ctypes.c_int), ("tiles_per_cta", ctypes.c_int),
+                ("ctas", ctypes.c_longlong), ("prepass_ctas", ctypes.c_longlong)]
+
+
+def la2_plan_info(B, H, T, d, e, block=128, dtype=LA2_DTYPE_BF16, is_bwd=False) -> list:
+    """The launch plan(s) of a bf16 call of these sizes, as dicts (one per
+    launch group); [] for an empty problem or fp32 inputs."""
+    plans = (LA2Plan * 2)()
+    n = int(load().la2_plan_info(B, H, T, d, e, block, dtype, int(is_bwd), plans, 2))
+    if n < 0:
+        raise LA2Error(LA2_ERR_INVALID_ARG, "la2_plan_info")
+    names = {LA2_SCHEDULE_UNIFORM: "uniform", LA2_SCHEDULE_BALANCED: "balanced"}
+    return [{"d": p.d, "e": p.e, "schedule": names[p.schedule], "units": p.units, "segments": p.segments,
+             "tiles_per_cta": p.tiles_per_cta, "ctas": p.ctas, "prepass_ctas": p.prepass_ctas}
+            for p in plans[:n]]
 
 
 def la2_set_schedule(schedule: str) -> str:

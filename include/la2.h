@@ -125,6 +125,29 @@ typedef enum {
 la2_schedule la2_set_schedule(la2_schedule schedule);
 
 /*
+ * The launch plan a bf16 la2_fwd (is_bwd = 0) or la2_bwd (is_bwd = 1) call of
+ * these sizes would run under the schedule setting in force: one entry per
+ * launch group (roles sharing (d, e) run in one launch; the backward with
+ * d != e has two groups).  Host-only, launches nothing.  Fills up to max_out
+ * entries of `out` (which may be NULL) and returns the number of groups, 0
+ * for an empty problem or fp32 inputs (one SIMT launch, no plan), or -1 for
+ * arguments the calls would reject.
+ */
+typedef struct {
+    int d, e;                  /* operand widths of the group's roles (a, b: d; c: e) */
+    int schedule;              /* LA2_SCHEDULE_UNIFORM or LA2_SCHEDULE_BALANCED */
+    long long units;           /* (sequence, role) units: B * H * roles in the group */
+    int segments;              /* UNIFORM: segments each unit is cut into; BALANCED: 0 */
+    int tiles_per_cta;         /* 128-position tiles of a segment (UNIFORM, the last may be
+                                  shorter) or of a CTA's run (BALANCED) */
+    long long ctas;            /* CTAs of the scan launch */
+    long long prepass_ctas;    /* CTAs of the state pre-pass launch (0: no pre-pass) */
+} la2_plan;
+
+int la2_plan_info(int B, int H, int T, int d, int e, int block, la2_dtype dtype, int is_bwd,
+                  la2_plan *out, int max_out);
+
+/*
  * Forward: out[b,h,t,:] = sum_{s<=t} decay[h]^(t-s) (q[b,h,t,:] . k[b,h,s,:]) v[b,h,s,:].
  *
  * Supported: dtype F32 with 1 <= d, e <= 128 and any block; dtype BF16 with

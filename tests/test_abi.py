@@ -151,3 +151,31 @@ def test_no_workspace_when_the_grid_is_full(lib):
     # 2 x 40 x 3 backward units >= 148 SMs: no segments, no workspace
     assert la2.la2_workspace_bytes(2, 40, 6144, 128, 128, 128, la2.LA2_DTYPE_BF16, 1) == 0
     assert la2.la2_workspace_bytes(1, 2, 512, 64, 64, 64, la2.LA2_DTYPE_F32, 1) == 0
+
+
+def test_plan_info(lib):
+    # long-context forward: 16 units of 512 tiles, cut into 9 segments of 57 tiles
+    assert la2.la2_plan_info(1, 16, 65536, 128, 128) == [
+        {"d": 128, "e": 128, "schedule": "uniform", "units": 16, "segments": 9, "tiles_per_cta": 57,
+         "ctas": 144, "prepass_ctas": 128}]
+    # its backward: 48 units in 3 segments of 171 tiles
+    assert la2.la2_plan_info(1, 16, 65536, 128, 128, is_bwd=True)[0]["segments"] == 3
+    # 15B backward: 240 units fill the GPU, no segments, no pre-pass
+    p = la2.la2_plan_info(2, 40, 6144, 128, 128, is_bwd=True)
+    assert len(p) == 1 and p[0]["units"] == 240 and p[0]["ctas"] == 240 and p[0]["prepass_ctas"] == 0
+    # d != e backward: dq and dk (a, b of width e) in one launch, dv in another
+    p = la2.la2_plan_info(2, 3, 1000, 64, 128, is_bwd=True)
+    assert [(g["d"], g["e"], g["units"]) for g in p] == [(128, 64, 12), (64, 128, 6)]
+    # fp32 inputs and empty problems have no plan; bad arguments are rejected
+    assert la2.la2_plan_info(1, 2, 512, 64, 64, 64, la2.LA2_DTYPE_F32) == []
+    assert la2.la2_plan_info(0, 2, 512, 64, 64) == []
+    with pytest.raises(la2.LA2Error):
+        la2.la2_plan_info(1, 2, 512, 64, 64, 100)
+    prev = la2.la2_set_schedule("balanced")
+    try:
+        # 80 units x 48 tiles laid end to end: runs of 26 tiles on 148 CTAs
+        assert la2.la2_plan_info(2, 40, 6144, 128, 128) == [
+            {"d": 128, "e": 128, "schedule": "balanced", "units": 80, "segments": 0, "tiles_per_cta": 26,
+             "ctas": 148, "prepass_ctas": 147}]
+    finally:
+        la2.la2_set_schedule(prev)
