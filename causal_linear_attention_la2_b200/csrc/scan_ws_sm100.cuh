@@ -1,6 +1,8 @@
 // scan_ws_sm100.cuh -- warp-specialised bf16-input tcgen05 kernel of the
-// Lightning Attention-2 hot path: one CTA per SM and per (sequence, role),
-// the whole value width (DC = 64 or 128) in one CTA, tiles of T_B = 128 rows.
+// Lightning Attention-2 hot path: one CTA per SM, running one segment of one
+// (sequence, role) unit (or, in the balanced schedule, the pieces of several
+// units one after the other), the whole value width (DC = 64 or 128) in one
+// CTA, tiles of T_B = 128 rows.
 //
 // It computes the same decayed scan as the forward and backward roles of the
 // library (see la2_api.cu):
@@ -13,39 +15,43 @@
 // in.  Per tile i (local row r, column c):
 //
 //   S   = A_i B_i^T                                 (tcgen05, TMEM)
-//   P   = S * lambda^|r-c| on the causal side, else 0 (registers -> TMEM, hi + lo bf16)
+//   P   = S * lambda^|r-c| on the causal side, else 0 (registers -> TMEM)
 //   X   = diag(w_x) A_i W + P C_i                   (tcgen05, TMEM, fp32)
-//   dW  = (diag(w_s) B_i)^T C_i                     (tcgen05, TMEM; hi + lo of w_s B)
-//   W  <- lambda^T_B W + dW                         (fp32 arithmetic; W kept as hi + lo bf16)
+//   dW  = (diag(w_s) B_i)^T C_i                     (tcgen05, TMEM)
+//   W  <- lambda^T_B W + dW                         (fp32 arithmetic)
 //
 // with w_x = lambda^(r+1), w_s = lambda^(T_B-1-r) for dir = +1 and
-// w_x = lambda^(T_B-r), w_s = lambda^r for dir = -1.
+// w_x = lambda^(T_B-r), w_s = lambda^r for dir = -1.  Operand precision: at
+// DA = DC = 64, P and w_s B enter their MMAs as tf32 (P stays fp32 in TMEM;
+// the mask warps write fp32 copies of C and w_s B, transposed so that they are
+// K-major); otherwise P and w_s B are split into bf16 hi + lo pairs.  The
+// state W is always kept as its bf16 hi + lo pair in shared memory (the X
+// MMA's operand), and in fp32 registers as well at DC = 64.
 //
 // Roles (20 warps):
 //   warp 0      TMA producer and MMA issuer S, one polling loop: A, B and C
 //               each in a ring of buffers (whichever ring has a free buffer is
 //               refilled first), S = A B^T into S buffer s % 2
-//   warp 1      MMA issuer PC: X += hi(P) C + lo(P) C, P read from S buffer
-//               s % 2 as the TMEM A operand
-//   warp 2      MMA issuer XW: X = A hi(W) + A lo(W) into X buffer s % 2
-//   warp 3      MMA issuer dW: dW = hi(w_s B)^T C + lo(w_s B)^T C
-//   warps 4-11  mask group (two warps per TMEM lane quadrant): the hi/lo
-//               split of w_s B (hi in place, lo in its own ring), then P from S
+//   warp 1      MMA issuer PC: X += P C, P read from S buffer s % 2 as the
+//               TMEM A operand
+//   warp 2      MMA issuer XW: A W, into X_inter (DC = 64) or into X (DC = 128)
+//   warp 3      MMA issuer dW
+//   warps 4-11  mask group (two warps per TMEM lane quadrant): the operand
+//               copies or hi/lo splits of C and w_s B, then P from S
 //   warps 12-19 epilogue group (two warps per lane quadrant, one per half of
-//               the columns): X = w_x X, the W update (W lives in shared
-//               memory as the hi/lo bf16 pair the next X MMA reads), X to global
-//               memory in fp32 (a warp-shuffle transpose makes every store a
-//               whole 128-byte row)
-// A thread can issue one tcgen05.mma about every 126 cycles whatever its
-// shape (measured on B200), while one M = 128, N = 128 MMA keeps the tensor
-// pipe busy for 64; so the MMAs of a tile are spread over four issuing
-// threads, each issuing fully unrolled with precomputed descriptors.
-// How many buffers each operand gets depends on (DA, DC) (RingCfg): at
-// DA = DC = 64 every operand has two or three, so the only serial dependency
-// left between tiles is the state update itself; at DA = DC = 128 shared
-// memory holds one A, C and W buffer and two B buffers.  With DC = 64, dW has
-// two TMEM buffers of its own; otherwise it borrows the X buffer of the next
-// tile.
+//               the columns): the W update, and the output: X (+ w_x X_inter
+//               at DC = 64) read with the 16x256b TMEM shape, so that float2
+//               stores of a warp fill whole 32-byte sectors
+// The tensor core takes one N = 64 MMA about every 45 cycles and one N = 128
+// MMA every 64, but a single issuing thread is slower than that once it also
+// computes descriptors and waits, so the MMAs of a tile are spread over four
+// issuing threads; at d = 64 those warps run their loops warp-converged (lane
+// 0 issues through predicated instructions).
+// How many buffers each operand gets depends on (DA, DC) (RingCfg): shared
+// memory holds two of most rings, and at DA = DC = 128 one A, C and W buffer
+// and two B buffers.  With DC = 64, X += P C, X_inter and dW (two buffers)
+// are separate TMEM accumulators; otherwise A W is scaled in place by w_x
+// before P C adds to it, and dW borrows the X buffer of the next tile.
 //
 // Every hand-off is an mbarrier: each buffer has a "full" barrier its
 // producer completes and an "empty" barrier its consumers complete, so a
@@ -287,10 +293,11 @@ __device__ __forceinline__ uint32_t empty_par(int s, int n) {
     return static_cast<uint32_t>(((s / n) + 1) & 1);
 }
 
-// The scan itself.  One CTA per (sequence, role, segment); a segment starts
-// from the state the segments before it leave behind,
-// W_in(g) = sum_{g' < g} lambda^(T_B n (g-1-g')) S_g' (n tiles per segment),
-// read from seg_state (written by la2_state_ws).
+// The scan itself.  A segment j of a (sequence, role) unit starts from the
+// state the segments before it leave behind, W_in(j) = f_{j-1} W_in(j-1) +
+// S_{j-1} with f_i = lambda^(T_B n_i) (n_i tiles in segment i) and W_in(0) the
+// given initial state or 0; the S_i are read from seg_state (written by
+// la2_state_ws).
 // kMulti: the balanced plan's CTAs, which may run several segments (a
 // separate instantiation, so that the one-segment kernel carries no loop
 // state in its registers).
@@ -1182,9 +1189,9 @@ la2_scan_ws(const __grid_constant__ Params p)
 
 
 // ---------------------------------------------------------------------------
-// State pre-pass for segmented sequences.  One CTA per (sequence, role,
-// segment but the last).  The state a segment of n tiles leaves behind when it
-// starts from zero is
+// State pre-pass for segmented sequences.  One CTA per segment that ends
+// inside its (sequence, role) unit.  The state a segment of n tiles leaves
+// behind when it starts from zero is
 //
 //   S = sum_{s < n} lambda^(T_B (n-1-s)) (diag(w_s) B_s)^T C_s,
 //
