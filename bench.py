@@ -4,7 +4,11 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 One step = la2_fwd + la2_bwd over one batch of the named workload (default:
-the TNL-400M-shaped layer), inputs resident in HBM.  Prints one JSON line.
+the length-sweep point T = 131,072, B = 1, H = 32, d = e = 128, block 128),
+inputs resident in HBM.  Prints one JSON line.  With a sweep workload the line
+also carries `sweep`: tokens/s and TFLOP/s of the same step at every sweep
+length and at the TNL-15B layer, timed in the same process, so one run shows
+how flat the throughput is in T.
 Under torchrun (N > 1) every rank runs its own replica (the path has no
 exchange step), the timed region is bracketed by a barrier and device
 synchronisation on every rank, and the slowest rank's time is reported.
@@ -71,7 +75,14 @@ def elem_bytes(w: I.Workload) -> int:
 
 
 def bwd_algorithmic_bytes(w: I.Workload) -> float:
-    """la2_bwd reads q, k, v, dO and writes fp32 dq, dk, dv, each once."""
+    """la2_bwd reads q, k, v, dO and writes dq, dk, dv, each once, every tensor
+    counted at the input element width (the per-token-head bytes of the
+    measurement plan: w (2d + 2e) in, w (2d + e) out)."""
+    return float(w.sequences) * w.T * elem_bytes(w) * (4 * w.d + 3 * w.e)
+
+
+def bwd_written_bytes(w: I.Workload) -> float:
+    """The same with the outputs at the fp32 width the kernel writes."""
     return float(w.sequences) * w.T * (elem_bytes(w) * (2 * w.d + 2 * w.e) + 4 * (2 * w.d + w.e))
 
 
@@ -137,10 +148,13 @@ class ClockSampler:
 # --------------------------------------------------------------- CPU oracle
 
 class OracleSample:
-    """Fwd+bwd of the fp64 oracle on a sample of whole sequences of a workload.
+    """Fwd+bwd of the fp64 oracle on a bounded sample of a workload.
 
-    A sequence is one (b, h); H of them carry the per-head work of w.T tokens,
-    so a sample of n sequences stands for n * T / H tokens of the metric.
+    The sample is n sequences (b, h), each its first P positions (P = T when
+    whole sequences fit the time budget).  A sequence carries the per-head work
+    of its positions, so n sequences of P positions stand for n * P / H tokens
+    of the metric; the oracle's cost per position does not depend on T (it is a
+    linear-time recurrence), so a prefix measures the same rate.
     """
 
     def __init__(self, w: I.Workload, x, target_s: float):
@@ -154,17 +168,23 @@ class OracleSample:
                                    (B, H)).reshape(-1)
         self.q, self.k, self.v, self.do = (x[n].reshape(B * H, w.T, -1)
                                            for n in ("q", "k", "v", "do"))
-        n = self.cores
-        dt = self.run(n)
-        if dt < target_s / 2:
-            n = min(64 * self.cores, max(n, int(n * target_s / max(dt, 1e-3))))
-        self.n = n
+        # calibrate on one sequence per core and a short prefix, then size the
+        # sample (positions first, then sequences) to about target_s
+        n, P = self.cores, min(w.T, 1024)
+        dt = self.run(n, P)
+        per_pos = max(dt, 1e-4) / (n * P)
+        want = max(1, int(target_s / per_pos))
+        P = min(w.T, max(P, want // n))
+        if P == w.T:
+            n = min(64 * self.cores, max(n, want // w.T))
+        self.n, self.P = n, P
 
-    def run(self, n=None):
+    def run(self, n=None, P=None):
         n = self.n if n is None else n
+        P = self.P if P is None else P
         idx = np.arange(n) % (self.w.B * self.w.H)
         t = torch.from_numpy(idx)
-        qs, ks, vs, ds = self.q[t], self.k[t], self.v[t], self.do[t]
+        qs, ks, vs, ds = (z[t, :P] for z in (self.q, self.k, self.v, self.do))
         t0 = time.perf_counter()
         self.oracle.forward(qs, ks, vs, self.lam[idx], nthreads=self.cores)
         self.oracle.backward(qs, ks, vs, self.lam[idx], ds, nthreads=self.cores)
@@ -172,10 +192,11 @@ class OracleSample:
 
     def rate(self):
         dt = self.run()
-        tokens = self.n * self.w.T / self.w.H
+        tokens = self.n * self.P / self.w.H
+        what = "whole sequences" if self.P == self.w.T else f"sequences, first {self.P} positions each,"
         return {"value": tokens / dt, "unit": "tokens/s", "cores": self.cores, "kind": "oracle",
-                "sample": f"{self.n} whole sequences (b,h) of T={self.w.T}, d={self.w.d}, "
-                          f"e={self.w.e}: {tokens:.0f} token-equivalents in {dt:.2f} s"}
+                "sample": f"{self.n} {what} (b,h) of T={self.w.T}, d={self.w.d}, e={self.w.e}: "
+                          f"{tokens:.0f} token-equivalents in {dt:.2f} s"}
 
 
 def oracle_rate(w: I.Workload, x, target_s: float = 12.0):
@@ -355,6 +376,78 @@ def run_decode(args, world, rank, local):
     return 0
 
 
+def time_steps(la2, fwd, bwd, stream, flush, steps, warmup):
+    """CUDA-event times of `steps` fwd and bwd calls after `warmup` untimed
+    ones, the L2 flushed (outside the events) before each; returns the per-step
+    fwd and bwd times in ms and the kernels launched in the timed steps."""
+    for _ in range(warmup):
+        flush.fill_(0.0)
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    assert la2.la2_device_status(reset=True) == 0, "kernel reported a device fault in warm-up"
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    launches = 0
+    for i in range(steps):
+        flush.fill_(float(i))
+        s, m, e = ev[i]
+        s.record(stream)
+        fwd()
+        launches += la2.la2_last_launch_count()
+        m.record(stream)
+        bwd()
+        launches += la2.la2_last_launch_count()
+        e.record(stream)
+    torch.cuda.synchronize()
+    assert la2.la2_device_status(reset=True) == 0, "kernel reported a device fault"
+    return [s.elapsed_time(m) for s, m, _ in ev], [m.elapsed_time(e) for _, m, e in ev], launches
+
+
+def step_line(w, fwd_ms, bwd_ms, tc, hbm, world=1):
+    """tokens/s, credited TFLOP/s and roofline figures of one workload's step."""
+    f = sum(fwd_ms) / len(fwd_ms)
+    b = sum(bwd_ms) / len(bwd_ms)
+    step_ms = f + b
+    tflops = flops_per_token_head(w) * w.T * w.sequences * world / (step_ms * 1e-3) / 1e12
+    return {"tokens_per_s": w.tokens * world / (step_ms * 1e-3), "ms_per_step": step_ms,
+            "fwd_ms": f, "bwd_ms": b, "tflops": tflops, "tc_frac": tflops / (tc * world),
+            "bwd_hbm_frac": bwd_algorithmic_bytes(w) / (b * 1e-3) / 1e9 / hbm,
+            "bwd_hbm_frac_fp32_out": bwd_written_bytes(w) / (b * 1e-3) / 1e9 / hbm}
+
+
+def sweep_lines(la2, w, dev_in, dev_out, lam_sweep, dev, stream, flush, args, tc, hbm):
+    """The same fwd+bwd step at every sweep length (and at the TNL-15B layer),
+    on views of the resident inputs: every sweep point has B T = 131,072, and
+    its inputs drawn by the recipe are the same flat buffers reshaped (T =
+    92,160, B = 1, and the 15B layer take a prefix of them)."""
+    lines = []
+    cases = [I.sweep_workload(T, w.block) for T in I.SWEEP_T] + [I.WORKLOADS["tnl15b"]]
+    for ws in cases:
+        if ws.d != w.d or ws.e != w.e:
+            continue
+        nq, nv = ws.sequences * ws.T * ws.d, ws.sequences * ws.T * ws.e
+        shp_q, shp_v = (ws.B, ws.H, ws.T, ws.d), (ws.B, ws.H, ws.T, ws.e)
+        q, k = (t.reshape(-1)[:nq].view(shp_q) for t in dev_in[:2])
+        v, do = (t.reshape(-1)[:nv].view(shp_v) for t in dev_in[2:])
+        out = dev_out[0].reshape(-1)[:nv].view(shp_v)
+        dq, dk = (t.reshape(-1)[:nq].view(shp_q) for t in dev_out[1:3])
+        dv = dev_out[3].reshape(-1)[:nv].view(shp_v)
+        lam = lam_sweep if ws.H == w.H else torch.from_numpy(ws.decays().copy()).to(dev)
+
+        def fwd():
+            la2.la2_fwd(q, k, v, lam, out=out, block=ws.block)
+
+        def bwd():
+            la2.la2_bwd(q, k, v, lam, do, dq=dq, dk=dk, dv=dv, block=ws.block)
+
+        fm, bm, _ = time_steps(la2, fwd, bwd, stream, flush, args.sweep_steps, 3)
+        ent = {"workload": ws.name, "B": ws.B, "T": ws.T, "H": ws.H, "block": ws.block}
+        ent.update(step_line(ws, fm, bm, tc, hbm))
+        lines.append(ent)
+    return lines
+
+
 def run_ours(args, w, world, rank, local):
     from causal_linear_attention_la2_b200 import la2
     la2.load()
@@ -371,68 +464,46 @@ def run_ours(args, w, world, rank, local):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def fwd(qq, kk, vv):
+    def fwd(qq=q, kk=k, vv=v):
         la2.la2_fwd_ex(qq, kk, vv, lam, lay, out=out, block=w.block)
 
-    def bwd(qq, kk, vv, dd):
+    def bwd(qq=q, kk=k, vv=v, dd=do):
         la2.la2_bwd_ex(qq, kk, vv, lam, dd, lay, dq=dq, dk=dk, dv=dv, block=w.block)
-
-    launches = 0
-
-    def step():
-        nonlocal launches
-        fwd(q, k, v)
-        launches += la2.la2_last_launch_count()
-        bwd(q, k, v, do)
-        launches += la2.la2_last_launch_count()
 
     for _ in range(args.warmup):
         flush.fill_(0.0)
-        step()
+        fwd()
+        bwd()
     torch.cuda.synchronize(dev)
     assert la2.la2_device_status(reset=True) == 0, "kernel reported a device fault in warm-up"
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if clocks:
         clocks.start()
         time.sleep(0.3)
-    launches = 0
     barrier(world)
     torch.cuda.synchronize(dev)
-    for i in range(args.steps):
-        flush.fill_(float(i))
-        s, m, e = ev[i]
-        s.record(stream)
-        fwd(q, k, v)
-        launches += la2.la2_last_launch_count()
-        m.record(stream)
-        bwd(q, k, v, do)
-        launches += la2.la2_last_launch_count()
-        e.record(stream)
-    torch.cuda.synchronize(dev)
+    fwd_ms, bwd_ms, launches = time_steps(la2, fwd, bwd, stream, flush, args.steps, 0)
     barrier(world)
     clk = clocks.stop() if clocks else None
-    fwd_ms = [s.elapsed_time(m) for s, m, _ in ev]
-    bwd_ms = [m.elapsed_time(e) for _, m, e in ev]
-    step_ms = sum(fwd_ms) / len(fwd_ms) + sum(bwd_ms) / len(bwd_ms)
-    step_ms = max_over_ranks(step_ms, world)
-    assert la2.la2_device_status(reset=True) == 0, "kernel reported a device fault"
+    step_ms = max_over_ranks(sum(fwd_ms) / len(fwd_ms) + sum(bwd_ms) / len(bwd_ms), world)
 
-    # end to end through the public API: pinned host in -> device -> host out
+    # end to end through the public API: pinned host in -> device -> host out.
+    # The four outputs are read back into one pinned buffer, one after the
+    # other (every byte still crosses PCIe; the host copy is not kept).
     hosts = {n: x[n].pin_memory() for n in ("q", "k", "v", "do")}
-    houts = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (out, dq, dk, dv)]
+    hout = torch.empty(max(t.numel() for t in (out, dq, dk, dv)), dtype=torch.float32,
+                       pin_memory=True)
     h2d = sum(t.numel() * t.element_size() for t in hosts.values())
-    d2h = sum(t.numel() * t.element_size() for t in houts)
+    d2h = sum(t.numel() * t.element_size() for t in (out, dq, dk, dv))
     e2e_steps = max(2, min(args.steps, 5))
 
     def e2e_step():
         qd, kd, vd, dd = (hosts[n].to(dev, non_blocking=True) for n in ("q", "k", "v", "do"))
         fwd(qd, kd, vd)
         bwd(qd, kd, vd, dd)
-        for h, dsrc in zip(houts, (out, dq, dk, dv)):
-            h.copy_(dsrc, non_blocking=True)
+        for dsrc in (out, dq, dk, dv):
+            hout[:dsrc.numel()].copy_(dsrc.reshape(-1), non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize(dev)
@@ -445,6 +516,7 @@ def run_ours(args, w, world, rank, local):
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(s0.elapsed_time(s1) / e2e_steps, world)
     barrier(world)
+    del hosts, hout
 
     if rank != 0:
         return 0
@@ -456,6 +528,7 @@ def run_ours(args, w, world, rank, local):
     value = tokens_per_step / (step_ms * 1e-3)
     bwd_avg_ms = sum(bwd_ms) / len(bwd_ms)
     achieved = bwd_algorithmic_bytes(w) / (bwd_avg_ms * 1e-3) / 1e9
+    written = bwd_written_bytes(w) / (bwd_avg_ms * 1e-3) / 1e9
     traffic = None
     try:
         with open(PROFILE_TRAFFIC) as f:
@@ -476,7 +549,9 @@ def run_ours(args, w, world, rank, local):
         "roofline": {"bound": "hbm", "kernel": "la2_scan_ws (la2_bwd launch)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic,
-                     "peak_kind": f"{pk_kind} hbm_gbs"},
+                     "peak_kind": f"{pk_kind} hbm_gbs",
+                     "bytes": "q, k, v, dO in and dq, dk, dv out, each once at the input width",
+                     "achieved_fp32_out": written, "frac_fp32_out": written / hbm},
         "e2e": {"value": tokens_per_step / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
@@ -486,6 +561,10 @@ def run_ours(args, w, world, rank, local):
         # the launch plans the two calls ran (schedule, segments, CTAs, pre-pass)
         line["plan"] = {"fwd": la2.la2_plan_info(w.B, w.H, w.T, w.d, w.e, w.block),
                         "bwd": la2.la2_plan_info(w.B, w.H, w.T, w.d, w.e, w.block, is_bwd=True)}
+    if (world == 1 and lay == "bhtd" and w.name.startswith("sweep_") and args.sweep_steps > 0
+            and w.B * w.T == 131072):
+        line["sweep"] = sweep_lines(la2, w, (q, k, v, do), (out, dq, dk, dv), lam, dev, stream,
+                                    flush, args, tc, hbm)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_rate(w, x, target_s=args.ref_seconds)
     print(json.dumps(line), flush=True)
@@ -497,7 +576,9 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="tnl400m", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--workload", default="sweep_T131072_blk128", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--sweep-steps", type=int, default=5,
+                    help="timed steps per entry of the sweep object (0: leave it out)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--ref-seconds", type=float, default=12.0)

@@ -20,6 +20,7 @@
 namespace {
 
 __device__ int g_la2_status = 0;  // device status word (see la2_device_status)
+__device__ int g_la2_never_set = 0;  // la2_selftest_timeout's flag: nothing ever writes it
 
 thread_local int t_last_launches = 0;
 
@@ -124,23 +125,27 @@ bool balanced_plan(long long units, int nb, SegPlan* out) {
     return true;
 }
 
-SegPlan plan_segments(long long units, int T) {
+// `sched` is the schedule setting read once at the top of the entry point, so
+// that one call sizes its workspace and launches with the same plan even if
+// another thread changes the setting meanwhile.
+SegPlan plan_segments(long long units, int T, int sched) {
     const int nb = (T + la2::ws::kTB - 1) / la2::ws::kTB;
     SegPlan b;
-    if (g_schedule.load() == LA2_SCHEDULE_BALANCED && balanced_plan(units, nb, &b)) return b;
+    if (sched == LA2_SCHEDULE_BALANCED && balanced_plan(units, nb, &b)) return b;
     return uniform_plan(units, nb);
 }
 
 // Workspace bytes of one bf16 launch over `units` (sequence, role) units.
-size_t seg_workspace_bytes(long long units, int T, int da, int dc) {
+size_t seg_workspace_bytes(long long units, int T, int da, int dc, int sched) {
     const size_t state = static_cast<size_t>(da) * static_cast<size_t>(dc) * sizeof(float);
-    if (plan_segments(units, T).balanced) return static_cast<size_t>(kTargetCTAs - 1) * state;
+    if (plan_segments(units, T, sched).balanced) return static_cast<size_t>(kTargetCTAs - 1) * state;
     return static_cast<size_t>(max_segments(units) - 1) * static_cast<size_t>(units) * state;
 }
 
 struct DeviceState {
     std::once_flag once;
     int* status = nullptr;
+    int* never_set = nullptr;
     bool ok = false;
 };
 DeviceState g_dev[kMaxDevices];
@@ -154,6 +159,9 @@ bool device_setup(int* dev_out, int** status_out) {
         void* p = nullptr;
         bool ok = cudaGetSymbolAddress(&p, g_la2_status) == cudaSuccess;
         s.status = static_cast<int*>(p);
+        void* f = nullptr;
+        ok = ok && cudaGetSymbolAddress(&f, g_la2_never_set) == cudaSuccess;
+        s.never_set = static_cast<int*>(f);
         ok = ok && set_ws_attrs<64, 64>() && set_ws_attrs<64, 128>() && set_ws_attrs<128, 64>() &&
              set_ws_attrs<128, 128>();
         ok = ok && cudaFuncSetAttribute(la2::la2_scan_f32,
@@ -166,6 +174,12 @@ bool device_setup(int* dev_out, int** status_out) {
     *dev_out = dev;
     *status_out = s.status;
     return true;
+}
+
+int* never_set_flag() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    return g_dev[dev].ok ? g_dev[dev].never_set : nullptr;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -198,6 +212,13 @@ struct RoleDesc {
     int da, dc, dir;
     const float* init = nullptr;  // forward role only: state before position 0
     float* fin = nullptr;         // forward role only: state after position T-1
+};
+
+// Self-test only (la2_selftest_timeout): a device flag that nothing sets, which
+// the scan kernel's producer waits on, bounded by `ns`, before its first load.
+struct Hold {
+    const int* flag = nullptr;
+    unsigned long long ns = 0;
 };
 
 la2_status common_checks(int B, int H, int T, int d, int e, int block, la2_dtype dtype,
@@ -234,7 +255,8 @@ void launch_ws(const la2::ws::Params& p, const SegPlan& sp, cudaStream_t stream)
 // with the CTAs of plan_segments, preceded by the state pre-pass when some
 // segment starts inside its unit.
 la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
-                          bool bthd, int* status, float* seg_state, cudaStream_t stream) {
+                          bool bthd, int sched, int* status, float* seg_state, const Hold& hold,
+                          cudaStream_t stream) {
     la2::ws::Params p;
     std::memset(&p, 0, sizeof(p));
     const int BH = B * H;
@@ -255,7 +277,9 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
     p.T = T;
     p.nroles = n;
     p.bthd = bthd ? 1 : 0;
-    const SegPlan sp = plan_segments(static_cast<long long>(BH) * n, T);
+    p.hold = hold.flag;
+    p.hold_ns = hold.ns;
+    const SegPlan sp = plan_segments(static_cast<long long>(BH) * n, T, sched);
     p.nunits = BH * n;
     p.nseg = sp.nseg;
     p.seg_tiles = sp.seg_tiles;
@@ -324,10 +348,10 @@ la2_status for_role_groups(const RoleDesc* roles, int n, F&& f) {
     return LA2_OK;
 }
 
-size_t bf16_workspace_bytes(const RoleDesc* roles, int n, int B, int H, int T) {
+size_t bf16_workspace_bytes(const RoleDesc* roles, int n, int B, int H, int T, int sched) {
     size_t total = 0;
     for_role_groups(roles, n, [&](const RoleDesc* g, int m) {
-        total += seg_workspace_bytes(static_cast<long long>(B) * H * m, T, g[0].da, g[0].dc);
+        total += seg_workspace_bytes(static_cast<long long>(B) * H * m, T, g[0].da, g[0].dc, sched);
         total = (total + 255) & ~static_cast<size_t>(255);
         return LA2_OK;
     });
@@ -335,21 +359,22 @@ size_t bf16_workspace_bytes(const RoleDesc* roles, int n, int B, int H, int T) {
 }
 
 la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
-                     int block, la2_dtype dtype, bool bthd, void* workspace, size_t ws_bytes,
-                     cudaStream_t stream) {
+                     int block, la2_dtype dtype, bool bthd, int sched, void* workspace,
+                     size_t ws_bytes, cudaStream_t stream, const Hold& hold = Hold()) {
     int dev = 0;
     int* status = nullptr;
-    if (dtype == LA2_DTYPE_BF16 && bf16_workspace_bytes(roles, n, B, H, T) > 0 &&
-        (workspace == nullptr || ws_bytes < bf16_workspace_bytes(roles, n, B, H, T)))
-        return LA2_ERR_WORKSPACE;
+    if (dtype == LA2_DTYPE_BF16) {
+        const size_t need = bf16_workspace_bytes(roles, n, B, H, T, sched);
+        if (need > 0 && (workspace == nullptr || ws_bytes < need)) return LA2_ERR_WORKSPACE;
+    }
     if (!device_setup(&dev, &status)) return LA2_ERR_CUDA;
     if (dtype == LA2_DTYPE_F32) return launch_f32(roles, n, decay, B, H, T, block, bthd, stream);
     size_t off = 0;
     return for_role_groups(roles, n, [&](const RoleDesc* g, int m) {
         float* seg = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) + off) : nullptr;
-        off += seg_workspace_bytes(static_cast<long long>(B) * H * m, T, g[0].da, g[0].dc);
+        off += seg_workspace_bytes(static_cast<long long>(B) * H * m, T, g[0].da, g[0].dc, sched);
         off = (off + 255) & ~static_cast<size_t>(255);
-        return launch_bf16_ws(g, m, decay, B, H, T, bthd, status, seg, stream);
+        return launch_bf16_ws(g, m, decay, B, H, T, bthd, sched, status, seg, hold, stream);
     });
 }
 
@@ -367,7 +392,8 @@ size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block, la2_dty
     const RoleDesc bwd[3] = {{nullptr, nullptr, nullptr, nullptr, e, d, +1},
                              {nullptr, nullptr, nullptr, nullptr, e, d, -1},
                              {nullptr, nullptr, nullptr, nullptr, d, e, -1}};
-    return is_bwd ? bf16_workspace_bytes(bwd, 3, B, H, T) : bf16_workspace_bytes(fwd, 1, B, H, T);
+    const int sched = g_schedule.load();
+    return is_bwd ? bf16_workspace_bytes(bwd, 3, B, H, T, sched) : bf16_workspace_bytes(fwd, 1, B, H, T, sched);
 }
 
 la2_schedule la2_set_schedule(la2_schedule schedule) {
@@ -387,10 +413,11 @@ int la2_plan_info(int B, int H, int T, int d, int e, int block, la2_dtype dtype,
                              {nullptr, nullptr, nullptr, nullptr, e, d, -1},
                              {nullptr, nullptr, nullptr, nullptr, d, e, -1}};
     int n = 0;
+    const int sched = g_schedule.load();
     for_role_groups(is_bwd ? bwd : fwd, is_bwd ? 3 : 1, [&](const RoleDesc* g, int m) {
         if (out && n < max_out) {
             const long long units = static_cast<long long>(B) * H * m;
-            const SegPlan sp = plan_segments(units, T);
+            const SegPlan sp = plan_segments(units, T, sched);
             la2_plan& o = out[n];
             o.d = g[0].da;
             o.e = g[0].dc;
@@ -437,8 +464,9 @@ la2_status la2_fwd_ex(const void* q, const void* k, const void* v, const float* 
     RoleDesc r = {q, k, v, out, d, e, +1};
     r.init = init_state;
     r.fin = final_state;
-    return run_roles(&r, 1, decay, B, H, T, block, dtype, layout == LA2_LAYOUT_BTHD, workspace,
-                     workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+    return run_roles(&r, 1, decay, B, H, T, block, dtype, layout == LA2_LAYOUT_BTHD,
+                     g_schedule.load(), workspace, workspace_bytes,
+                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 la2_status la2_fwd_state(const void* q, const void* k, const void* v, const float* decay,
@@ -484,8 +512,9 @@ la2_status la2_bwd_ex(const void* q, const void* k, const void* v, const float* 
         {k, q, dout, dv, d, e, -1},
     };
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return LA2_ERR_INVALID_ARG;
-    return run_roles(roles, 3, decay, B, H, T, block, dtype, layout == LA2_LAYOUT_BTHD, workspace,
-                     workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+    return run_roles(roles, 3, decay, B, H, T, block, dtype, layout == LA2_LAYOUT_BTHD,
+                     g_schedule.load(), workspace, workspace_bytes,
+                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 la2_status la2_decode(const void* q, const void* k, const void* v, const float* decay,
@@ -527,6 +556,32 @@ la2_status la2_decode(const void* q, const void* k, const void* v, const float* 
     if (cudaGetLastError() != cudaSuccess) return LA2_ERR_CUDA;
     t_last_launches = 1;
     return LA2_OK;
+}
+
+la2_status la2_selftest_timeout(const void* q, const void* k, const void* v, const float* decay,
+                                void* out, int T, int d, int e, unsigned limit_us,
+                                la2_stream_t stream) {
+    t_last_launches = 0;
+    if (T < 1 || T > 2 * la2::ws::kTB || limit_us == 0 || limit_us > 1000000u)
+        return LA2_ERR_INVALID_ARG;
+    bool empty = false;
+    const la2_status st = common_checks(1, 1, T, d, e, la2::ws::kTB, LA2_DTYPE_BF16, &empty);
+    if (st != LA2_OK) return st;
+    if (!q || !k || !v || !decay || !out) return LA2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(decay) & 3u))
+        return LA2_ERR_INVALID_ARG;
+    int dev = 0;
+    int* status = nullptr;
+    if (!device_setup(&dev, &status)) return LA2_ERR_CUDA;
+    Hold hold;
+    hold.flag = never_set_flag();
+    hold.ns = static_cast<unsigned long long>(limit_us) * 1000ull;
+    if (!hold.flag) return LA2_ERR_CUDA;
+    // one sequence of at most two tiles: one segment, no workspace
+    const RoleDesc r = {q, k, v, out, d, e, +1};
+    return run_roles(&r, 1, decay, 1, 1, T, la2::ws::kTB, LA2_DTYPE_BF16, false,
+                     LA2_SCHEDULE_UNIFORM, nullptr, 0, reinterpret_cast<cudaStream_t>(stream), hold);
 }
 
 const char* la2_status_str(la2_status s) {

@@ -93,7 +93,16 @@ struct Params {
                          //    [c L, (c+1) L), i.e. the ends of some units and the starts
                          //    of others, one after the other
     int nseg;            // balanced = 0: segments per unit (1 = no split)
+    const int* hold;     // null, except in the failure-path self-test: a device flag that
+                         // nothing sets, which the producer waits on (bounded by hold_ns)
+                         // before its first load, so that the wait runs out
+    unsigned long long hold_ns;
 };
+
+// Status code a kernel records when a bounded wait runs out: LA2_ERR_TIMEOUT
+// (5) in the low byte, the site of the wait above it.
+constexpr int kTimeoutCode = 5;
+constexpr int kSiteHold = 90;  // the self-test's wait on p.hold
 
 // Segments of unit u (nb tiles, in scan order).  Boundary j >= 1 sits at step
 // j L - ph(u), where ph(u) = (u nb) mod L in the balanced plan (the boundaries
@@ -435,7 +444,21 @@ la2_scan_ws(const __grid_constant__ Params p)
         // S of step s = A B^T (into S buffer s % 2) is issued once A and B of
         // step s have landed and X += P C of step s-2, which read the P in that
         // buffer, is done.  Nothing here blocks, so loads never wait behind S.
-        if (lane == 0 && ns > 0) {
+        if (lane == 0 && ns > 0 && p.hold != nullptr) {
+            // failure-path self-test: wait for a flag that is never set; the
+            // wait runs out before any load is issued, and every role then
+            // leaves through the abort flag
+            const uint64_t t0 = global_ns();
+            while (*reinterpret_cast<const volatile int*>(p.hold) == 0) {
+                if (global_ns() - t0 > p.hold_ns) {
+                    *abort_flag = 1;
+                    atomicCAS(p.status, 0, kTimeoutCode | (kSiteHold << 8));
+                    break;
+                }
+                __nanosleep(1000);
+            }
+        }
+        if (lane == 0 && ns > 0 && !*abort_flag) {
             prefetch_tmap(&R.ta);
             prefetch_tmap(&R.tb);
             prefetch_tmap(&R.tc);

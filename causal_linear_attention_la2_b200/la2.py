@@ -28,7 +28,7 @@ LA2_DTYPE_BF16 = 1
 # Every entry point include/la2.h declares.
 EXPORTS = ("la2_workspace_bytes", "la2_fwd", "la2_fwd_state", "la2_fwd_ex", "la2_bwd", "la2_bwd_ex",
            "la2_decode", "la2_status_str", "la2_device_status", "la2_last_launch_count",
-           "la2_fwd_noalloc", "la2_set_schedule", "la2_plan_info")
+           "la2_fwd_noalloc", "la2_set_schedule", "la2_plan_info", "la2_selftest_timeout")
 
 LA2_LAYOUT_BHTD = 0
 LA2_LAYOUT_BTHD = 1
@@ -85,6 +85,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la2_set_schedule.restype = i
     lib.la2_plan_info.argtypes = [i, i, i, i, i, i, i, i, ctypes.POINTER(LA2Plan), i]
     lib.la2_plan_info.restype = i
+    lib.la2_selftest_timeout.argtypes = [vp, vp, vp, vp, vp, i, i, i, ctypes.c_uint, vp]
+    lib.la2_selftest_timeout.restype = i
     _lib = lib
     return lib
 
@@ -137,6 +139,13 @@ def la2_set_schedule(schedule: str) -> str:
 
 
 # ---------------------------------------------------------------- raw C calls
+
+def la2_selftest_timeout_raw(q, k, v, decay, out, T, d, e, limit_us, stream=0) -> int:
+    """Failure-path self-test: the bf16 forward kernel waits, bounded by
+    limit_us, on a flag nothing sets and records LA2_ERR_TIMEOUT; returns the
+    launch status (read the recorded code with la2_device_status)."""
+    return int(load().la2_selftest_timeout(q, k, v, decay, out, T, d, e, limit_us, stream))
+
 
 def la2_fwd_raw(q, k, v, decay, out, B, H, T, d, e, block, dtype, workspace=0, ws_bytes=0,
                 stream=0) -> int:

@@ -260,6 +260,22 @@ la2_status la2_device_status(int *code, int reset);
 int la2_last_launch_count(void);
 
 /*
+ * Self-test of the failure path of the bf16 scan kernel (no counterpart in
+ * the paper).  Launches the forward kernel once on one sequence (B = H = 1,
+ * 1 <= T <= 256, d, e in {64, 128}, block 128, bf16, [B, H, T, D]) with its
+ * producer first waiting on a device flag that nothing ever sets, bounded by
+ * limit_us microseconds (1 .. 1,000,000).  The wait runs out before any load
+ * is issued; the kernel records LA2_ERR_TIMEOUT | (90 << 8) in the device
+ * status word, every role leaves its loop through the CTA's abort flag, the
+ * kernel frees its TMEM and returns, and the context stays usable.  `out` is
+ * not written.  Returns LA2_OK once the launch is queued; read the recorded
+ * code with la2_device_status.  Nothing traps, faults or hangs.
+ */
+la2_status la2_selftest_timeout(const void *q, const void *k, const void *v, const float *decay,
+                                void *out, int T, int d, int e, unsigned limit_us,
+                                la2_stream_t stream);
+
+/*
  * la2_fwd without a workspace argument, for callers that cannot allocate
  * device memory at call time: code running inside CUDA-graph capture, under a
  * framework that owns every allocation, or in a context where cudaMalloc is

@@ -179,3 +179,14 @@ def test_plan_info(lib):
              "ctas": 148, "prepass_ctas": 147}]
     finally:
         la2.la2_set_schedule(prev)
+
+
+def test_selftest_timeout_rejects_bad_arguments(lib):
+    fake = FAKE
+    for T, lim in ((0, 100), (257, 100), (100, 0), (100, 2_000_000)):
+        assert la2.la2_selftest_timeout_raw(fake, fake, fake, fake, fake, T, 128, 128, lim) == \
+            la2.LA2_ERR_INVALID_ARG
+    assert la2.la2_selftest_timeout_raw(0, fake, fake, fake, fake, 100, 128, 128, 100) == \
+        la2.LA2_ERR_INVALID_ARG
+    assert la2.la2_selftest_timeout_raw(fake, fake, fake, fake, fake, 100, 96, 128, 100) == \
+        la2.LA2_ERR_UNSUPPORTED

@@ -166,16 +166,50 @@ def test_outputs_do_not_write_past_their_end(la2mod):
 
 # -------------------------------------------------- full-size named workloads
 
+_FLAT = {}
+
+
+def _workload_inputs(w):
+    """make_workload_inputs(w, seed=0), drawn once for the whole length sweep:
+    every sweep point has B T = 131,072, so the recipe's draws are the same flat
+    buffers for every T, and each point is a reshape of them."""
+    if not (w.name.startswith("sweep_") and w.B * w.T == 131072):
+        return I.make_workload_inputs(w, seed=0)
+    key = (w.H, w.d, w.e, w.dtype, w.decay)
+    if key not in _FLAT:
+        _FLAT.clear()
+        _FLAT[key] = I.make_inputs(1, w.H, 131072, w.d, w.e, w.dtype, seed=0, decay=w.decay)
+    base = _FLAT[key]
+    x = {n: base[n].reshape(w.B, w.H, w.T, base[n].shape[-1]) for n in ("q", "k", "v", "do")}
+    x["lam"] = base["lam"]
+    return x
+
+
 FULL = ["tnl400m", "tnl15b", "tnl15b_nodecay", "long", "sweep_T1024_blk128",
-        "sweep_T131072_blk128", "sweep_T92160_blk128"]
+        "sweep_T4096_blk128", "sweep_T16384_blk128", "sweep_T32768_blk128",
+        "sweep_T65536_blk128", "sweep_T131072_blk128", "sweep_T92160_blk128"]
+
+
+def _sampled(la2mod, oracle_mod, w, x):
+    B, H = w.B, w.H
+    # first and last sequence (smallest and largest decay) and one in the middle
+    bi = np.array([0, B // 2, B - 1])
+    hi = np.array([0, H // 2, H - 1])
+    return _check(la2mod, oracle_mod, x, w.block, TOL[w.dtype], heads=(bi, hi))
 
 
 @pytest.mark.parametrize("name", FULL)
 def test_full_size_workload_sampled_sequences(la2mod, oracle_mod, name):
     w = I.WORKLOADS[name]
-    x = I.make_workload_inputs(w, seed=0)
-    B, H = w.B, w.H
-    # first and last sequence (smallest and largest decay) and one in the middle
-    bi = np.array([0, B // 2, B - 1])
-    hi = np.array([0, H // 2, H - 1])
-    _check(la2mod, oracle_mod, x, w.block, TOL[w.dtype], heads=(bi, hi))
+    _sampled(la2mod, oracle_mod, w, _workload_inputs(w))
+
+
+def test_sweep_longest_no_decay(la2mod, oracle_mod):
+    """lambda = 1 at T = 131,072, d = e = 128: nothing in the carried state is
+    ever decayed away, so every rounding of the state update stays in it; the
+    longest sweep sequence is the worst case for the state's precision."""
+    w = I.WORKLOADS["sweep_T131072_blk128"]
+    x = dict(_workload_inputs(w))
+    x["lam"] = torch.ones(w.H, dtype=torch.float32)
+    errs = _sampled(la2mod, oracle_mod, w, x)
+    assert max(errs.values()) < 2e-3, errs
