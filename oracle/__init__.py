@@ -56,6 +56,8 @@ def _load():
         lib.la2o_backward_blocked.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp, dp, i]
         lib.la2o_forward_state.argtypes = [i, i, i, i, dp, dp, dp, dp, dp, dp, dp, i]
         lib.la2o_decode_step.argtypes = [i, i, i, dp, dp, dp, dp, dp, dp]
+        lib.la2o_backward_state.argtypes = [i, i, i, i, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp,
+                                            dp, i]
         lib.la2o_max_threads.restype = i
         _lib = lib
     return _lib
@@ -153,6 +155,25 @@ def backward(q, k, v, lam, dout, nthreads: int = 0):
                           _ptr(dqc), _ptr(dkc), _ptr(dvc), int(nthreads))
         dq[a:b], dk[a:b], dv[a:b] = dqc, dkc, dvc
     return dq.reshape(*lead, T, d), dk.reshape(*lead, T, d), dv.reshape(*lead, T, e)
+
+
+def backward_state(q, k, v, lam, dout, s0=None, dsT=None, nthreads: int = 0):
+    """(dq, dk, dv, dS0) of L = sum_t dout_t . o_t + <dsT, S_{T-1}> for the
+    forward started from the state s0 ([..., d, e]; None = zero); dsT is the
+    gradient arriving at the final state (None = zero)."""
+    lib = _load()
+    lead, ns, T, d, e, lam = _prep(q, k, v, lam)
+    qc, kc, vc, gc = (_f64(x).reshape(ns, T, w) for x, w in ((q, d), (k, d), (v, e), (dout, e)))
+    dq = np.empty((ns, T, d)); dk = np.empty((ns, T, d)); dv = np.empty((ns, T, e))
+    ds0 = np.empty((ns, d, e))
+    s0a = _f64(s0).reshape(ns, d, e) if s0 is not None else None
+    gTa = _f64(dsT).reshape(ns, d, e) if dsT is not None else None
+    lib.la2o_backward_state(ns, T, d, e, _ptr(lam), _ptr(qc), _ptr(kc), _ptr(vc), _ptr(gc),
+                            _ptr(s0a) if s0a is not None else None,
+                            _ptr(gTa) if gTa is not None else None,
+                            _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds0), int(nthreads))
+    return (dq.reshape(*lead, T, d), dk.reshape(*lead, T, d), dv.reshape(*lead, T, e),
+            ds0.reshape(*lead, d, e))
 
 
 def forward_blocked(q, k, v, lam, block: int, nthreads: int = 0) -> np.ndarray:

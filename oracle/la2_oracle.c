@@ -42,6 +42,16 @@
  *                           (the state is the only thing a sequence carries,
  *                           section 2 "Memory footprint", so a long sequence
  *                           can be processed in consecutive pieces).
+ *   la2o_backward_state     gradients of L = sum_t do_t . o_t + <G, S_{T-1}>
+ *                           for the forward from a given state S_{-1} = S0:
+ *                           dq, dk, dv, and dS0.  G (the gradient arriving at
+ *                           the final state) enters the reverse sweep at the
+ *                           last position: R_{T-1} = q_{T-1} do_{T-1}^T + G,
+ *                           R_t = lambda R_{t+1} + q_t do_t^T; dq_t = S_t do_t
+ *                           with S_t started from S0; dS0 = lambda R_0 (G
+ *                           when T = 0).  This is what a sequence trained in
+ *                           consecutive pieces needs (section 2, "Memory
+ *                           footprint": the state is all a piece carries).
  *   la2o_decode_step        one step of the same recurrence for one new token
  *                           per sequence: S <- lambda S + k v^T, o = S^T q.
  *   la2o_backward_blocked   the mirrored tiling for the backward (the pages say
@@ -218,6 +228,74 @@ void la2o_backward(int NS, int T, int d, int e, const double *lam,
             for (int i = 0; i < d; ++i)
                 for (int j = 0; j < e; ++j) dvt[j] += R[(size_t)i * e + j] * kt[i];
         }
+        free(S);
+    }
+}
+
+/* ------------------------------------------- backward with carried state */
+
+void la2o_backward_state(int NS, int T, int d, int e, const double *lam,
+                         const double *q, const double *k, const double *v,
+                         const double *dout, const double *s0, const double *dsT,
+                         double *dq, double *dk, double *dv, double *ds0,
+                         int nthreads)
+{
+    set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < NS; ++n) {
+        const double *qn = q + (size_t)n * T * d;
+        const double *kn = k + (size_t)n * T * d;
+        const double *vn = v + (size_t)n * T * e;
+        const double *gn = dout + (size_t)n * T * e;
+        double *dqn = dq + (size_t)n * T * d;
+        double *dkn = dk + (size_t)n * T * d;
+        double *dvn = dv + (size_t)n * T * e;
+        double *S = (double *)calloc((size_t)d * e, sizeof(double));
+        const double l = lam[n];
+
+        /* forward sweep from S_{-1} = S0: dq_t = S_t do_t */
+        if (s0) memcpy(S, s0 + (size_t)n * d * e, sizeof(double) * (size_t)d * e);
+        for (int t = 0; t < T; ++t) {
+            const double *kt = kn + (size_t)t * d, *vt = vn + (size_t)t * e;
+            const double *gt = gn + (size_t)t * e;
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < e; ++j)
+                    S[(size_t)i * e + j] = l * S[(size_t)i * e + j] + kt[i] * vt[j];
+            double *dqt = dqn + (size_t)t * d;
+            for (int i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < e; ++j) acc += S[(size_t)i * e + j] * gt[j];
+                dqt[i] = acc;
+            }
+        }
+
+        /* reverse sweep: R starts as G at the last position (no decay there),
+           R_t = lambda R_{t+1} + q_t do_t^T before it; dk_t = R_t v_t,
+           dv_t = R_t^T k_t */
+        double *R = S;
+        if (dsT) memcpy(R, dsT + (size_t)n * d * e, sizeof(double) * (size_t)d * e);
+        else memset(R, 0, sizeof(double) * (size_t)d * e);
+        for (int t = T - 1; t >= 0; --t) {
+            const double *qt = qn + (size_t)t * d, *kt = kn + (size_t)t * d;
+            const double *vt = vn + (size_t)t * e, *gt = gn + (size_t)t * e;
+            const double f = (t == T - 1) ? 1.0 : l;
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < e; ++j)
+                    R[(size_t)i * e + j] = f * R[(size_t)i * e + j] + qt[i] * gt[j];
+            double *dkt = dkn + (size_t)t * d, *dvt = dvn + (size_t)t * e;
+            for (int i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < e; ++j) acc += R[(size_t)i * e + j] * vt[j];
+                dkt[i] = acc;
+            }
+            for (int j = 0; j < e; ++j) dvt[j] = 0.0;
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < e; ++j) dvt[j] += R[(size_t)i * e + j] * kt[i];
+        }
+        /* S_0 = lambda S_{-1} + k_0 v_0^T, so dS_{-1} = lambda R_0; with no
+           position at all, S_{T-1} is S_{-1} itself */
+        double *g0 = ds0 + (size_t)n * d * e;
+        for (size_t z = 0; z < (size_t)d * e; ++z) g0[z] = T > 0 ? l * R[z] : R[z];
         free(S);
     }
 }

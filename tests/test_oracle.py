@@ -265,3 +265,103 @@ def test_decode_steps_reproduce_the_forward(oracle_mod):
     o1, S1 = oracle_mod.decode_step(q[0, 0], k[0, 0], v[0, 0], lam[0], s0[0])
     Sh = lam[0] * s0[0] + np.outer(k[0, 0], v[0, 0])
     assert _rel(S1, Sh) < 1e-14 and _rel(o1, Sh.T @ q[0, 0]) < 1e-14
+
+
+# ------------------------------------------------ backward with carried state
+
+def _bwd_state_closed_form(q, k, v, do, lam, s0, g):
+    """Gradients of L = sum_t do_t . o_t + <G, S_{T-1}> with S_{-1} = S0,
+    written out as matrices:
+      dq_t = sum_{s<=t} lam^(t-s) (do_t . v_s) k_s + lam^(t+1) S0 do_t
+      dk_s = sum_{t>=s} lam^(t-s) (do_t . v_s) q_t + lam^(T-1-s) G v_s
+      dv_s = sum_{t>=s} lam^(t-s) (q_t . k_s) do_t + lam^(T-1-s) G^T k_s
+      dS0  = sum_t lam^(t+1) q_t do_t^T + lam^T G
+    """
+    T = q.shape[0]
+    _, dq, dk, dv = _brute(q, k, v, do, lam)
+    t = np.arange(T)
+    wq = lam ** (t + 1)
+    wk = lam ** (T - 1 - t)
+    dq = dq + wq[:, None] * (do @ s0.T)
+    dk = dk + wk[:, None] * (v @ g.T)
+    dv = dv + wk[:, None] * (k @ g)
+    ds0 = (q * wq[:, None]).T @ do + lam ** T * g
+    return dq, dk, dv, ds0
+
+
+@pytest.mark.parametrize("T,d,e", [(1, 3, 2), (9, 4, 5), (40, 8, 3)])
+def test_backward_state_closed_form(oracle_mod, T, d, e):
+    rng = np.random.default_rng(91 + T)
+    for lam in LAMS:
+        q, k, v, do = _rand(rng, T, d), _rand(rng, T, d), _rand(rng, T, e), _rand(rng, T, e)
+        s0, g = _rand(rng, d, e), _rand(rng, d, e)
+        got = oracle_mod.backward_state(q, k, v, lam, do, s0, g)
+        want = _bwd_state_closed_form(q, k, v, do, lam, s0, g)
+        for a, b in zip(got, want):
+            assert _rel(a, b) < 1e-12, lam
+        # no states: the plain backward (and dS0 of the plain forward)
+        got0 = oracle_mod.backward_state(q, k, v, lam, do)
+        want0 = _bwd_state_closed_form(q, k, v, do, lam, np.zeros((d, e)), np.zeros((d, e)))
+        for a, b in zip(got0, want0):
+            assert _rel(a, b) < 1e-12
+
+
+@pytest.mark.parametrize("lam", [1.0, 0.9])
+def test_backward_state_finite_differences(oracle_mod, lam):
+    """Central differences of L = sum do * o + <G, S_T> through forward_state
+    (pinned on its own) in every coordinate of S0, q, k and v: L is linear in
+    each single coordinate, so the differences are exact up to rounding."""
+    rng = np.random.default_rng(8)
+    T, d, e = 6, 3, 2
+    q, k, v, do = _rand(rng, T, d), _rand(rng, T, d), _rand(rng, T, e), _rand(rng, T, e)
+    s0, g = _rand(rng, d, e), _rand(rng, d, e)
+
+    def loss(qq, kk, vv, ss):
+        o, sT = oracle_mod.forward_state(qq, kk, vv, lam, ss)
+        return float(np.sum(do * o) + np.sum(g * sT))
+
+    dq, dk, dv, ds0 = oracle_mod.backward_state(q, k, v, lam, do, s0, g)
+    h = 0.5
+    for arr, grad, idx in ((q, dq, 0), (k, dk, 1), (v, dv, 2), (s0, ds0, 3)):
+        for pos in np.ndindex(arr.shape):
+            args = [q, k, v, s0]
+            up, dn = arr.copy(), arr.copy()
+            up[pos] += h
+            dn[pos] -= h
+            args[idx] = up
+            lu = loss(*args)
+            args[idx] = dn
+            ld = loss(*args)
+            assert abs((lu - ld) / (2 * h) - grad[pos]) <= 1e-10 * max(1.0, abs(grad[pos]))
+
+
+@pytest.mark.parametrize("cut", [1, 7, 13, 29])
+def test_backward_state_pieces_equal_whole(oracle_mod, cut):
+    """A sequence trained in two pieces: the forward of piece 1 gives the state
+    S_mid; the backward of piece 2 from S_mid returns dS_mid, which enters the
+    backward of piece 1 as the gradient at its final state.  The gradients of
+    the pieces, concatenated, and dS0 equal those of the whole sequence."""
+    rng = np.random.default_rng(40 + cut)
+    T, d, e = 30, 5, 4
+    q, k, v, do = (_rand(rng, 3, T, w) for w in (d, d, e, e))
+    lam = np.array([1.0, 0.9, 0.3])
+    s0, g = _rand(rng, 3, d, e), _rand(rng, 3, d, e)
+    _, smid = oracle_mod.forward_state(q[:, :cut], k[:, :cut], v[:, :cut], lam, s0)
+    dq2, dk2, dv2, dsmid = oracle_mod.backward_state(q[:, cut:], k[:, cut:], v[:, cut:], lam,
+                                                     do[:, cut:], smid, g)
+    dq1, dk1, dv1, ds0 = oracle_mod.backward_state(q[:, :cut], k[:, :cut], v[:, :cut], lam,
+                                                   do[:, :cut], s0, dsmid)
+    whole = oracle_mod.backward_state(q, k, v, lam, do, s0, g)
+    for a, b in zip((np.concatenate([dq1, dq2], 1), np.concatenate([dk1, dk2], 1),
+                     np.concatenate([dv1, dv2], 1), ds0), whole):
+        assert _rel(a, b) < 1e-12
+
+
+def test_backward_state_empty_sequence(oracle_mod):
+    """With no position the final state is S0 itself, so dS0 = G."""
+    rng = np.random.default_rng(3)
+    d, e = 4, 3
+    g = _rand(rng, 2, d, e)
+    z = np.zeros((2, 0, d)), np.zeros((2, 0, e))
+    out = oracle_mod.backward_state(z[0], z[0], z[1], [0.9, 1.0], z[1], _rand(rng, 2, d, e), g)
+    np.testing.assert_array_equal(out[3], g)
