@@ -169,14 +169,17 @@ class OracleSample:
         self.q, self.k, self.v, self.do = (x[n].reshape(B * H, w.T, -1)
                                            for n in ("q", "k", "v", "do"))
         # calibrate on one sequence per core and a short prefix, then size the
-        # sample (positions first, then sequences) to about target_s
+        # sample (positions first, then sequences) to about target_s.  The
+        # oracle hands its threads sequences in chunks of about 1 GiB of
+        # float64, so a prefix is kept short enough that every chunk still
+        # holds a sequence for each core.
         n, P = self.cores, min(w.T, 1024)
         dt = self.run(n, P)
         per_pos = max(dt, 1e-4) / (n * P)
         want = max(1, int(target_s / per_pos))
-        P = min(w.T, max(P, want // n))
-        if P == w.T:
-            n = min(64 * self.cores, max(n, want // w.T))
+        p_cap = max(1024, (1 << 30) // (8 * self.cores * 4 * (w.d + w.e)))
+        P = min(w.T, p_cap, max(P, want // n))
+        n = min(64 * self.cores, max(n, want // P))
         self.n, self.P = n, P
 
     def run(self, n=None, P=None):

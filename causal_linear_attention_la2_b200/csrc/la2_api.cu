@@ -210,8 +210,9 @@ struct RoleDesc {
     const void* c;
     void* x;
     int da, dc, dir;
-    const float* init = nullptr;  // forward role only: state before position 0
-    float* fin = nullptr;         // forward role only: state after position T-1
+    const float* init = nullptr;  // state the scan starts from (see la2::ws::Role)
+    float* fin = nullptr;         // state the scan ends with
+    int init_t = 0;               // init stored transposed ([DC][DA])
 };
 
 // Self-test only (la2_selftest_timeout): a device flag that nothing sets, which
@@ -270,6 +271,7 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
         p.role[r].init = roles[r].init;
         p.role[r].fin = roles[r].fin;
         p.role[r].dir = roles[r].dir;
+        p.role[r].init_t = roles[r].init_t;
     }
     p.decay = decay;
     p.status = status;
@@ -311,6 +313,7 @@ la2_status launch_f32(const RoleDesc* roles, int n, const float* decay, int B, i
         p.role[r].dir = roles[r].dir;
         p.role[r].init = roles[r].init;
         p.role[r].fin = roles[r].fin;
+        p.role[r].init_t = roles[r].init_t;
         da_max = roles[r].da > da_max ? roles[r].da : da_max;
         dc_max = roles[r].dc > dc_max ? roles[r].dc : dc_max;
     }
@@ -496,21 +499,58 @@ la2_status la2_bwd_ex(const void* q, const void* k, const void* v, const float* 
                       const void* dout, void* dq, void* dk, void* dv, int B, int H, int T, int d,
                       int e, int block, la2_dtype dtype, la2_layout layout, void* workspace,
                       size_t workspace_bytes, la2_stream_t stream) {
+    return la2_bwd_state(q, k, v, decay, dout, nullptr, nullptr, dq, dk, dv, nullptr, B, H, T, d,
+                         e, block, dtype, layout, workspace, workspace_bytes, stream);
+}
+
+la2_status la2_bwd_state(const void* q, const void* k, const void* v, const float* decay,
+                         const void* dout, const float* init_state, const float* d_final_state,
+                         void* dq, void* dk, void* dv, float* d_init_state, int B, int H, int T,
+                         int d, int e, int block, la2_dtype dtype, la2_layout layout,
+                         void* workspace, size_t workspace_bytes, la2_stream_t stream) {
     t_last_launches = 0;
     if (layout != LA2_LAYOUT_BHTD && layout != LA2_LAYOUT_BTHD) return LA2_ERR_INVALID_ARG;
     bool empty = false;
     la2_status st = common_checks(B, H, T, d, e, block, dtype, &empty);
-    if (st != LA2_OK || empty) return st;
+    if (st != LA2_OK) return st;
+    const uintptr_t smis = reinterpret_cast<uintptr_t>(init_state) |
+                           reinterpret_cast<uintptr_t>(d_final_state) |
+                           reinterpret_cast<uintptr_t>(d_init_state);
+    if (smis & 3u) return LA2_ERR_INVALID_ARG;
+    if (empty) {
+        // no position: the final state is the initial one, so its gradient
+        // passes through unchanged (or is 0)
+        if (d_init_state && B > 0 && H > 0) {
+            const size_t n = static_cast<size_t>(B) * H * d * e * sizeof(float);
+            const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+            const cudaError_t err =
+                d_final_state
+                    ? cudaMemcpyAsync(d_init_state, d_final_state, n, cudaMemcpyDeviceToDevice, cs)
+                    : cudaMemsetAsync(d_init_state, 0, n, cs);
+            if (err != cudaSuccess) return LA2_ERR_CUDA;
+        }
+        return LA2_OK;
+    }
     if (!q || !k || !v || !decay || !dout || !dq || !dk || !dv) return LA2_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
         !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(decay) & 3u))
         return LA2_ERR_INVALID_ARG;
-    // dq = scan(+1; dO, v, k), dk = scan(-1; v, dO, q), dv = scan(-1; k, q, dO)
-    const RoleDesc roles[3] = {
+    // dq = scan(+1; dO, v, k), dk = scan(-1; v, dO, q), dv = scan(-1; k, q, dO).
+    // The carried states enter as the scans' initial states: S0^T for dq (a
+    // state before position 0), G^T for dk and G for dv (a state entering at
+    // position T-1); dS0 is the dv scan's final state (lambda times its state
+    // at position 0, which is sum_t lambda^(t+1) q_t dO_t^T + lambda^T G).
+    RoleDesc roles[3] = {
         {dout, v, k, dq, e, d, +1},
         {v, dout, q, dk, e, d, -1},
         {k, q, dout, dv, d, e, -1},
     };
+    roles[0].init = init_state;
+    roles[0].init_t = 1;
+    roles[1].init = d_final_state;
+    roles[1].init_t = 1;
+    roles[2].init = d_final_state;
+    roles[2].fin = d_init_state;
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return LA2_ERR_INVALID_ARG;
     return run_roles(roles, 3, decay, B, H, T, block, dtype, layout == LA2_LAYOUT_BTHD,
                      g_schedule.load(), workspace, workspace_bytes,
@@ -578,10 +618,12 @@ la2_status la2_selftest_timeout(const void* q, const void* k, const void* v, con
     hold.flag = never_set_flag();
     hold.ns = static_cast<unsigned long long>(limit_us) * 1000ull;
     if (!hold.flag) return LA2_ERR_CUDA;
-    // one sequence of at most two tiles: one segment, no workspace
+    // one sequence of at most two tiles: the uniform plan runs it as one
+    // segment, so the scan needs no pre-pass and no workspace (launch_bf16_ws
+    // refuses a plan with a pre-pass when it gets none)
     const RoleDesc r = {q, k, v, out, d, e, +1};
-    return run_roles(&r, 1, decay, 1, 1, T, la2::ws::kTB, LA2_DTYPE_BF16, false,
-                     LA2_SCHEDULE_UNIFORM, nullptr, 0, reinterpret_cast<cudaStream_t>(stream), hold);
+    return launch_bf16_ws(&r, 1, decay, 1, 1, T, false, LA2_SCHEDULE_UNIFORM, status, nullptr, hold,
+                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 const char* la2_status_str(la2_status s) {

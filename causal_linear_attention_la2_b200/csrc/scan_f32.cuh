@@ -19,9 +19,14 @@ struct F32Role {
     const float* b;  // [BH, T, DA]
     const float* c;  // [BH, T, DC]
     float* x;        // [BH, T, DC]
-    const float* init;  // [BH, DA, DC] state before the first position, or null (0)
-    float* fin;         // [BH, DA, DC] state after the last position, or null
-    int da, dc, dir;    // init and fin are used with dir = +1 only
+    const float* init;  // [BH, DA, DC] state the scan starts from, or null (0); with
+                        // init_t, [BH, DC, DA] read transposed
+    float* fin;         // [BH, DA, DC] state the scan ends with, or null
+    int da, dc, dir;
+    int init_t;
+    // dir = +1: init is the state before position 0, fin the state after
+    // position T-1.  dir = -1: init enters at position T-1 (row t weighs it by
+    // lambda^(T-1-t)), and fin is lambda times the state at position 0.
 };
 
 struct F32Params {
@@ -56,8 +61,12 @@ la2_scan_f32(const __grid_constant__ F32Params p)
     const double lam = static_cast<double>(p.decay[bh % p.H]);
     const double l2 = log2(lam);
     for (int n = tid; n <= TB; n += kF32Threads) pw[n] = static_cast<float>(exp2(n * l2));
-    for (int z = tid; z < da * dc; z += kF32Threads)
-        W[z] = R.init ? R.init[static_cast<size_t>(bh) * da * dc + z] : 0.f;
+    for (int z = tid; z < da * dc; z += kF32Threads) {
+        const int u = z / dc, j = z % dc;
+        W[z] = R.init ? R.init[static_cast<size_t>(bh) * da * dc +
+                               (R.init_t ? static_cast<size_t>(j) * da + u : static_cast<size_t>(z))]
+                      : 0.f;
+    }
 
     // sequence bh: base row and row stride in units of D ([B,H,T,D]: bh T, 1;
     // [B,T,H,D]: b T H + h, H)
@@ -91,7 +100,10 @@ la2_scan_f32(const __grid_constant__ F32Params p)
             // inter-tile term: w_x(r) * a_r^T W
             float acc[32];
             const int rloc = qa * kF32Sub + row;
-            const float wx = dir > 0 ? pw[min(rloc + 1, TB)] : pw[max(TB - rloc, 0)];
+            // the reverse scan's first tile (the sequence's last) takes the
+            // entering state at position T-1: lambda^(len-1-r)
+            const float wx = dir > 0 ? pw[min(rloc + 1, TB)]
+                                     : (step == 0 ? pw[max(len - 1 - rloc, 0)] : pw[max(TB - rloc, 0)]);
 #pragma unroll
             for (int m = 0; m < 32; ++m) {
                 const int j = jc + 4 * m;
@@ -151,8 +163,9 @@ la2_scan_f32(const __grid_constant__ F32Params p)
         // A forward scan's last tile may be short (len < TB rows): its exponents
         // are taken from len, so that W is then the state after position T-1
         // (no output reads it; the final state does).
+        // A reverse scan's first tile decays the entering state by lambda^(len-1).
         const int tl = dir > 0 ? len : TB;
-        const float lTB = pw[tl];
+        const float lTB = (dir < 0 && step == 0) ? pw[len - 1] : pw[tl];
         for (int z = tid; z < da * dc; z += kF32Threads) W[z] *= lTB;
         for (int kb = 0; kb < nsub; ++kb) {
             __syncthreads();
@@ -175,8 +188,11 @@ la2_scan_f32(const __grid_constant__ F32Params p)
         }
         __syncthreads();
     }
-    if (R.fin)
-        for (int z = tid; z < da * dc; z += kF32Threads) R.fin[static_cast<size_t>(bh) * da * dc + z] = W[z];
+    if (R.fin) {
+        const float fs = dir > 0 ? 1.f : static_cast<float>(lam);
+        for (int z = tid; z < da * dc; z += kF32Threads)
+            R.fin[static_cast<size_t>(bh) * da * dc + z] = fs * W[z];
+    }
 }
 
 }  // namespace la2

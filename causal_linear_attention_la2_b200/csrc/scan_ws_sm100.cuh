@@ -72,9 +72,16 @@ struct Role {
     CUtensorMap ta, tb, tc;  // a, b: 4-D maps of [B, H, T, DA] (or [B, T, H, DA]); c likewise
                              // with DC; bf16, box 64 columns x 128 positions
     float* x;                // [B*H, T, DC] fp32
-    const float* init;       // [B*H, DA, DC] fp32 state before the first position, or null (0)
-    float* fin;              // [B*H, DA, DC] fp32 state after the last position, or null
-    int dir;                 // +1 or -1 (init and fin are used with +1 only)
+    const float* init;       // [B*H, DA, DC] fp32 state the scan starts from, or null (0);
+                             // with init_t, [B*H, DC, DA] read transposed
+    float* fin;              // [B*H, DA, DC] fp32 state the scan ends with, or null
+    int dir;                 // +1 or -1
+    int init_t;              // 1: init is stored transposed
+    // dir = +1: init is the state before position 0 (row t of the output gets
+    // lambda^(t+1) a_t^T init) and fin the state after position T-1.
+    // dir = -1: init is a state entering at position T-1 (row t gets
+    // lambda^(T-1-t) a_t^T init), and fin is lambda times the state at
+    // position 0, i.e. the state the scan would carry past the first position.
 };
 
 struct Params {
@@ -918,6 +925,12 @@ la2_scan_ws(const __grid_constant__ Params p)
         const int c0 = half * kCols;
         const float wx = dir > 0 ? pw[r + 1] : pw[kTB - r];
         const float lamTB = pw[kTB];
+        // The reverse scan's first tile (the sequence's last, n = nlast rows)
+        // takes a given state as entering at position T-1: its rows weigh it
+        // by lambda^(n-1-r) and it decays by lambda^(n-1) across the tile.
+        const int nlast = T - (nb - 1) * kTB;
+        const bool first_rev = dir < 0 && s0 == 0;
+        const float wx_first = r < nlast ? pw[nlast - 1 - r] : 0.f;
         const bool owns_w_row = (DA == 128) || (lane < 16);
         const int wrow = (DA == 128) ? r : quad * 16 + (lane & 15);
         // With 32 columns per thread (DC = 64) each owner thread keeps its part
@@ -934,16 +947,24 @@ la2_scan_ws(const __grid_constant__ Params p)
         if ((sj > 0 || R.init != nullptr) && owns_w_row) {
             const double l2 = log2(static_cast<double>(lam));
             const float fL = static_cast<float>(exp2(static_cast<double>(kTB) * p.seg_tiles * l2));
-            const float f0 = static_cast<float>(
-                exp2(static_cast<double>(kTB) * (p.seg_tiles - seg_phase(p, kMulti, unit, nb)) * l2));
-            const float* w0 =
-                R.init ? R.init + static_cast<size_t>(bh) * (DA * DC) + static_cast<size_t>(wrow) * DC : nullptr;
+            // segment 0 has n0 tiles; in the reverse direction its first tile
+            // decays an entering state by lambda^(nlast-1) instead of lambda^T_B
+            const int n0 = p.seg_tiles - seg_phase(p, kMulti, unit, nb);
+            const double e0 = dir > 0 ? static_cast<double>(kTB) * n0
+                                      : static_cast<double>(kTB) * (n0 - 1) + (nlast - 1);
+            const float f0 = static_cast<float>(exp2(e0 * l2));
+            const float* w0 = R.init ? R.init + static_cast<size_t>(bh) * (DA * DC) : nullptr;
 #pragma unroll
             for (int k = 0; k < kCols / 16; ++k) {
                 const uint32_t col = c0 + k * 16;
                 float w[16];
+                if (w0 && R.init_t) {
 #pragma unroll
-                for (int u = 0; u < 16; ++u) w[u] = w0 ? w0[col + u] : 0.f;
+                    for (int u = 0; u < 16; ++u) w[u] = w0[static_cast<size_t>(col + u) * DA + wrow];
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) w[u] = w0 ? w0[static_cast<size_t>(wrow) * DC + col + u] : 0.f;
+                }
                 for (int gp = 0; gp < sj; ++gp) {
                     const float f = gp == 0 ? f0 : fL;
                     const float* src = seg_slot(gp) + static_cast<size_t>(wrow) * DC + col;
@@ -979,13 +1000,14 @@ la2_scan_ws(const __grid_constant__ Params p)
             if (tid == 384) LA2_TR(14, s);
             tc_fence_after();
             const uint32_t xt = tX(s % Q::NX);
+            const float wxs = (first_rev && s == 0) ? wx_first : wx;
 #pragma unroll 1
             for (int k = 0; k < kCols / 32; ++k) {
                 float x[32];
                 const uint32_t col = c0 + k * 32;
                 tmem_ld32(xt + lane_off + col, x);
 #pragma unroll
-                for (int u = 0; u < 32; ++u) x[u] *= wx;
+                for (int u = 0; u < 32; ++u) x[u] *= wxs;
                 tmem_st32(xt + lane_off + col, x);
             }
             tmem_wait_st();
@@ -998,10 +1020,9 @@ la2_scan_ws(const __grid_constant__ Params p)
         // state is kept as its hi + lo bf16 pair (a 16-bit significand, ~2^-17
         // relative per update), which is also the next tile's MMA operand.
         const bool has_last = dir > 0 && unit_end;
-        const int nlast = T - (nb - 1) * kTB;
         auto update = [&](int s) -> bool {
             const bool last = has_last && s == ns - 1;
-            const float lam_s = last ? pw[nlast] : lamTB;
+            const float lam_s = last ? pw[nlast] : ((first_rev && s == 0) ? pw[nlast - 1] : lamTB);
             if (!wait_bar<Q::kTf32>(bar(Q::D_DONE + (s % Q::ND)), full_par(s, Q::ND), abort_flag, p.status, 51))
                 return false;
             // the X MMA that last read the W buffer written here is done
@@ -1070,13 +1091,15 @@ la2_scan_ws(const __grid_constant__ Params p)
                     }
                 }
             }
-            if (last && R.fin && owns_w_row) {
-                // the state after position T-1: fp32 from registers (32 columns per
-                // thread), else from the hi + lo pair just written
+            if (unit_end && s == ns - 1 && R.fin && owns_w_row) {
+                // the final state: fp32 from registers (32 columns per thread),
+                // else from the hi + lo pair just written; a reverse scan hands
+                // on lambda times its state at position 0
                 float* fin = R.fin + static_cast<size_t>(bh) * (DA * DC) + static_cast<size_t>(wrow) * DC;
+                const float fs = dir > 0 ? 1.f : lam;
                 if constexpr (kWReg) {
 #pragma unroll
-                    for (int u = 0; u < 32; ++u) fin[c0 + u] = wreg[u];
+                    for (int u = 0; u < 32; ++u) fin[c0 + u] = fs * wreg[u];
                 } else {
 #pragma unroll 1
                     for (int cc = 0; cc < kCols; cc += 8) {
@@ -1087,8 +1110,8 @@ la2_scan_ws(const __grid_constant__ Params p)
                         ld_shared_v4(wdst + L::kWsz + o, l[0], l[1], l[2], l[3]);
 #pragma unroll
                         for (int z = 0; z < 4; ++z) {
-                            fin[col + 2 * z] = bf16lo_to_f32(h[z]) + bf16lo_to_f32(l[z]);
-                            fin[col + 2 * z + 1] = bf16hi_to_f32(h[z]) + bf16hi_to_f32(l[z]);
+                            fin[col + 2 * z] = fs * (bf16lo_to_f32(h[z]) + bf16lo_to_f32(l[z]));
+                            fin[col + 2 * z + 1] = fs * (bf16hi_to_f32(h[z]) + bf16hi_to_f32(l[z]));
                         }
                     }
                 }
@@ -1126,7 +1149,9 @@ la2_scan_ws(const __grid_constant__ Params p)
 #pragma unroll
                     for (int h8 = 0; h8 < 2; ++h8) {
                         const int rr = quad * 32 + lh * 16 + t4 + 8 * h8;
-                        wxr[2 * lh + h8] = dir > 0 ? pw[rr + 1] : pw[kTB - rr];
+                        wxr[2 * lh + h8] = (first_rev && s == 0)
+                                               ? (rr < nlast ? pw[nlast - 1 - rr] : 0.f)
+                                               : (dir > 0 ? pw[rr + 1] : pw[kTB - rr]);
                     }
             }
 #pragma unroll 1

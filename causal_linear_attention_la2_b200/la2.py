@@ -28,7 +28,8 @@ LA2_DTYPE_BF16 = 1
 # Every entry point include/la2.h declares.
 EXPORTS = ("la2_workspace_bytes", "la2_fwd", "la2_fwd_state", "la2_fwd_ex", "la2_bwd", "la2_bwd_ex",
            "la2_decode", "la2_status_str", "la2_device_status", "la2_last_launch_count",
-           "la2_fwd_noalloc", "la2_set_schedule", "la2_plan_info", "la2_selftest_timeout")
+           "la2_fwd_noalloc", "la2_set_schedule", "la2_plan_info", "la2_selftest_timeout",
+           "la2_bwd_state")
 
 LA2_LAYOUT_BHTD = 0
 LA2_LAYOUT_BTHD = 1
@@ -87,6 +88,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la2_plan_info.restype = i
     lib.la2_selftest_timeout.argtypes = [vp, vp, vp, vp, vp, i, i, i, ctypes.c_uint, vp]
     lib.la2_selftest_timeout.restype = i
+    lib.la2_bwd_state.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i,
+                                  i, vp, sz, vp]
+    lib.la2_bwd_state.restype = i
     _lib = lib
     return lib
 
@@ -345,6 +349,41 @@ def la2_bwd_ex(q, k, v, decay, dout, layout: str = "bhtd", dq=None, dk=None, dv=
     if st != LA2_OK:
         raise LA2Error(st, "la2_bwd_ex")
     return dq, dk, dv
+
+
+def la2_bwd_state(q, k, v, decay, dout, init_state=None, d_final_state=None, layout: str = "bhtd",
+                  dq=None, dk=None, dv=None, d_init_state=None, want_d_init: bool = True,
+                  block: int = 128, stream=None, workspace=None):
+    """(dq, dk, dv, d_init_state) of sum(dout * out) + sum(d_final_state * final_state) for
+    the forward la2_fwd_ex(q, k, v, decay, layout, init_state); states [B, H, d, e] fp32
+    (None = zero).  d_init_state is None unless want_d_init or a buffer is given."""
+    B, H, T, d, e = _dims(q, v, layout)
+    dt = _dtype_code(q)
+    for t, n, D in ((q, "q", d), (k, "k", d), (v, "v", e), (dout, "dout", e)):
+        _check(t, n, _shape(layout, B, H, T, D), q.dtype)
+    _check(decay, "decay", (H,), torch.float32)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty(_shape(layout, B, H, T, d), **f32) if dq is None else dq
+    dk = torch.empty(_shape(layout, B, H, T, d), **f32) if dk is None else dk
+    dv = torch.empty(_shape(layout, B, H, T, e), **f32) if dv is None else dv
+    for t, n, D in ((dq, "dq", d), (dk, "dk", d), (dv, "dv", e)):
+        _check(t, n, _shape(layout, B, H, T, D), torch.float32)
+    if d_init_state is None and want_d_init:
+        d_init_state = torch.empty((B, H, d, e), **f32)
+    ptrs = []
+    for t, n in ((init_state, "init_state"), (d_final_state, "d_final_state"),
+                 (d_init_state, "d_init_state")):
+        if t is not None:
+            _check(t, n, (B, H, d, e), torch.float32)
+        ptrs.append(0 if t is None else t.data_ptr())
+    wp, wn = _workspace(la2_workspace_bytes(B, H, T, d, e, block, dt, 1), q.device, workspace)
+    st = int(load().la2_bwd_state(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(),
+                                  dout.data_ptr(), ptrs[0], ptrs[1], dq.data_ptr(), dk.data_ptr(),
+                                  dv.data_ptr(), ptrs[2], B, H, T, d, e, block, dt,
+                                  _LAYOUTS[layout], wp, wn, _stream_ptr(stream)))
+    if st != LA2_OK:
+        raise LA2Error(st, "la2_bwd_state")
+    return dq, dk, dv, d_init_state
 
 
 def la2_decode_raw(q, k, v, decay, state, out, B, H, d, e, dtype, stream=0) -> int:

@@ -244,6 +244,39 @@ la2_status la2_bwd_ex(const void *q, const void *k, const void *v, const float *
                       la2_layout layout, void *workspace, size_t workspace_bytes,
                       la2_stream_t stream);
 
+/*
+ * Backward with carried states: the gradients of
+ *
+ *     L = sum_t dout_t . out_t + <d_final_state, S_{T-1}>
+ *
+ * for the forward of la2_fwd_state started from init_state (S_{-1}), with
+ * respect to q, k, v and init_state.  d_final_state is the gradient arriving
+ * at the forward's final state from what follows (the next piece of a
+ * sequence trained in pieces).  With S0 = init_state and G = d_final_state:
+ *
+ *   dq[t]  = sum_{s<=t} lambda^(t-s) (dout_t . v_s) k_s + lambda^(t+1) S0 dout_t
+ *   dk[s]  = sum_{t>=s} lambda^(t-s) (v_s . dout_t) q_t + lambda^(T-1-s) G v_s
+ *   dv[s]  = sum_{t>=s} lambda^(t-s) (k_s . q_t) dout_t + lambda^(T-1-s) G^T k_s
+ *   d_init_state = sum_t lambda^(t+1) q_t dout_t^T + lambda^T G
+ *
+ * The state is all a piece of a sequence carries ("Lightning Attention"
+ * explainer, section 2, memory footprint): the backward of the last piece
+ * from the incoming state, then of each earlier piece with the d_init_state
+ * of the one after it as its d_final_state, gives the gradients of the whole.
+ *
+ * init_state, d_final_state: device fp32 [B, H, d, e], or NULL (zero);
+ * d_init_state: device fp32 [B, H, d, e], or NULL (not computed); all 4-byte
+ * aligned, d_init_state aliasing nothing else.  With T = 0, d_init_state =
+ * d_final_state.  Layout, support matrix and workspace as la2_bwd_ex (the
+ * same size with or without states).
+ */
+la2_status la2_bwd_state(const void *q, const void *k, const void *v, const float *decay,
+                         const void *dout, const float *init_state, const float *d_final_state,
+                         void *dq, void *dk, void *dv, float *d_init_state,
+                         int B, int H, int T, int d, int e, int block, la2_dtype dtype,
+                         la2_layout layout, void *workspace, size_t workspace_bytes,
+                         la2_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 const char *la2_status_str(la2_status status);
 

@@ -58,6 +58,7 @@ def _load():
         lib.la2o_decode_step.argtypes = [i, i, i, dp, dp, dp, dp, dp, dp]
         lib.la2o_backward_state.argtypes = [i, i, i, i, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp,
                                             dp, i]
+        lib.la2o_dlambda.argtypes = [i, i, i, i, dp, dp, dp, dp, dp, dp, dp, dp, i]
         lib.la2o_max_threads.restype = i
         _lib = lib
     return _lib
@@ -174,6 +175,21 @@ def backward_state(q, k, v, lam, dout, s0=None, dsT=None, nthreads: int = 0):
                             _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds0), int(nthreads))
     return (dq.reshape(*lead, T, d), dk.reshape(*lead, T, d), dv.reshape(*lead, T, e),
             ds0.reshape(*lead, d, e))
+
+
+def dlambda(q, k, v, lam, dout, s0=None, dsT=None, nthreads: int = 0):
+    """dL/dlam per sequence ([...]) for L = sum_t dout_t . o_t + <dsT, S_{T-1}>,
+    the forward started from s0 (None = zero, dsT None = zero)."""
+    lib = _load()
+    lead, ns, T, d, e, lam = _prep(q, k, v, lam)
+    qc, kc, vc, gc = (_f64(x).reshape(ns, T, w) for x, w in ((q, d), (k, d), (v, e), (dout, e)))
+    s0a = _f64(s0).reshape(ns, d, e) if s0 is not None else None
+    gTa = _f64(dsT).reshape(ns, d, e) if dsT is not None else None
+    out = np.empty(ns)
+    lib.la2o_dlambda(ns, T, d, e, _ptr(lam), _ptr(qc), _ptr(kc), _ptr(vc), _ptr(gc),
+                     _ptr(s0a) if s0a is not None else None,
+                     _ptr(gTa) if gTa is not None else None, _ptr(out), int(nthreads))
+    return out.reshape(lead)
 
 
 def forward_blocked(q, k, v, lam, block: int, nthreads: int = 0) -> np.ndarray:

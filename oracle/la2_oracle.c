@@ -52,6 +52,11 @@
  *                           when T = 0).  This is what a sequence trained in
  *                           consecutive pieces needs (section 2, "Memory
  *                           footprint": the state is all a piece carries).
+ *   la2o_dlambda            the gradient of the same L with respect to lambda
+ *                           (one scalar per sequence), by differentiating the
+ *                           recurrence: U_t = dS_t/dlambda obeys
+ *                           U_t = lambda U_{t-1} + S_{t-1} (U_{-1} = 0), and
+ *                           dL/dlambda = sum_t q_t^T U_t do_t + <G, U_{T-1}>.
  *   la2o_decode_step        one step of the same recurrence for one new token
  *                           per sequence: S <- lambda S + k v^T, o = S^T q.
  *   la2o_backward_blocked   the mirrored tiling for the backward (the pages say
@@ -297,6 +302,50 @@ void la2o_backward_state(int NS, int T, int d, int e, const double *lam,
         double *g0 = ds0 + (size_t)n * d * e;
         for (size_t z = 0; z < (size_t)d * e; ++z) g0[z] = T > 0 ? l * R[z] : R[z];
         free(S);
+    }
+}
+
+/* ------------------------------------------------- gradient in lambda */
+
+void la2o_dlambda(int NS, int T, int d, int e, const double *lam,
+                  const double *q, const double *k, const double *v,
+                  const double *dout, const double *s0, const double *dsT,
+                  double *dlam, int nthreads)
+{
+    set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < NS; ++n) {
+        const double *qn = q + (size_t)n * T * d;
+        const double *kn = k + (size_t)n * T * d;
+        const double *vn = v + (size_t)n * T * e;
+        const double *gn = dout + (size_t)n * T * e;
+        double *S = (double *)calloc((size_t)d * e, sizeof(double));
+        double *U = (double *)calloc((size_t)d * e, sizeof(double));
+        const double l = lam[n];
+        if (s0) memcpy(S, s0 + (size_t)n * d * e, sizeof(double) * (size_t)d * e);
+        double acc = 0.0;
+        for (int t = 0; t < T; ++t) {
+            const double *qt = qn + (size_t)t * d, *kt = kn + (size_t)t * d;
+            const double *vt = vn + (size_t)t * e, *gt = gn + (size_t)t * e;
+            /* U_t = lambda U_{t-1} + S_{t-1}, then S_t = lambda S_{t-1} + k_t v_t^T */
+            for (size_t z = 0; z < (size_t)d * e; ++z) U[z] = l * U[z] + S[z];
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < e; ++j)
+                    S[(size_t)i * e + j] = l * S[(size_t)i * e + j] + kt[i] * vt[j];
+            /* q_t^T U_t do_t */
+            for (int i = 0; i < d; ++i) {
+                double r = 0.0;
+                for (int j = 0; j < e; ++j) r += U[(size_t)i * e + j] * gt[j];
+                acc += qt[i] * r;
+            }
+        }
+        if (dsT && T > 0) {
+            const double *g = dsT + (size_t)n * d * e;
+            for (size_t z = 0; z < (size_t)d * e; ++z) acc += g[z] * U[z];
+        }
+        dlam[n] = acc;
+        free(S);
+        free(U);
     }
 }
 

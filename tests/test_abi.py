@@ -190,3 +190,13 @@ def test_selftest_timeout_rejects_bad_arguments(lib):
         la2.LA2_ERR_INVALID_ARG
     assert la2.la2_selftest_timeout_raw(fake, fake, fake, fake, fake, 100, 96, 128, 100) == \
         la2.LA2_ERR_UNSUPPORTED
+
+
+def test_bwd_state_rejects_misaligned_states(lib):
+    for pos in range(3):
+        st = [0, 0, 0]
+        st[pos] = FAKE + 2
+        r = la2.load().la2_bwd_state(FAKE, FAKE, FAKE, FAKE, FAKE, st[0], st[1], FAKE, FAKE, FAKE,
+                                     st[2], 1, 2, 256, 128, 128, 128, la2.LA2_DTYPE_BF16,
+                                     la2.LA2_LAYOUT_BHTD, 0, 0, 0)
+        assert r == la2.LA2_ERR_INVALID_ARG

@@ -365,3 +365,74 @@ def test_backward_state_empty_sequence(oracle_mod):
     z = np.zeros((2, 0, d)), np.zeros((2, 0, e))
     out = oracle_mod.backward_state(z[0], z[0], z[1], [0.9, 1.0], z[1], _rand(rng, 2, d, e), g)
     np.testing.assert_array_equal(out[3], g)
+
+
+# -------------------------------------------------------- gradient in lambda
+
+def _dlambda_closed_form(q, k, v, do, lam, s0, g):
+    """dL/dlam for L = sum_t do_t . o_t + <G, S_{T-1}>, written out:
+      sum_{s<t} (t-s) lam^(t-s-1) (q_t . k_s)(do_t . v_s)
+      + sum_t (t+1) lam^t q_t^T S0 do_t
+      + <G, T lam^(T-1) S0 + sum_s (T-1-s) lam^(T-2-s) k_s v_s^T>
+    (every power with a zero factor in front taken as 0)."""
+    T = q.shape[0]
+    t = np.arange(T)
+    lag = t[:, None] - t[None, :]
+    lagp = np.maximum(lag - 1, 0).astype(np.float64)
+    M = np.where(lag >= 1, lag * np.power(lam, lagp), 0.0)
+    val = np.sum(M * (q @ k.T) * (do @ v.T))
+    val += np.sum((t + 1) * lam ** t * np.einsum("ti,ij,tj->t", q, s0, do))
+    w = T - 1 - t
+    ws = np.where(w >= 1, w * np.power(lam, np.maximum(w - 1, 0).astype(np.float64)), 0.0)
+    dsT = (T * lam ** (T - 1) if T >= 1 else 0.0) * s0 + (k * ws[:, None]).T @ v
+    return val + np.sum(g * dsT)
+
+
+@pytest.mark.parametrize("T,d,e", [(1, 3, 2), (2, 2, 2), (9, 4, 5), (40, 8, 3)])
+def test_dlambda_closed_form(oracle_mod, T, d, e):
+    rng = np.random.default_rng(300 + T)
+    for lam in LAMS:
+        q, k, v, do = _rand(rng, T, d), _rand(rng, T, d), _rand(rng, T, e), _rand(rng, T, e)
+        s0, g = _rand(rng, d, e), _rand(rng, d, e)
+        got = oracle_mod.dlambda(q, k, v, lam, do, s0, g)
+        want = _dlambda_closed_form(q, k, v, do, lam, s0, g)
+        assert abs(got - want) <= 1e-11 * max(1.0, abs(want)), (lam, got, want)
+        got0 = oracle_mod.dlambda(q, k, v, lam, do)
+        want0 = _dlambda_closed_form(q, k, v, do, lam, np.zeros((d, e)), np.zeros((d, e)))
+        assert abs(got0 - want0) <= 1e-11 * max(1.0, abs(want0))
+
+
+@pytest.mark.parametrize("lam", [1.0, 0.9, 0.5])
+def test_dlambda_central_differences(oracle_mod, lam):
+    """Richardson-extrapolated central differences of L(lam) through
+    forward_state (pinned on its own): the step-h and step-h/2 estimates
+    combined cancel the h^2 term, leaving O(h^4)."""
+    rng = np.random.default_rng(9)
+    T, d, e = 7, 3, 2
+    q, k, v, do = _rand(rng, T, d), _rand(rng, T, d), _rand(rng, T, e), _rand(rng, T, e)
+    s0, g = _rand(rng, d, e), _rand(rng, d, e)
+
+    def loss(lm):
+        o, sT = oracle_mod.forward_state(q, k, v, lm, s0)
+        return float(np.sum(do * o) + np.sum(g * sT))
+
+    def cd(h):
+        return (loss(lam + h) - loss(lam - h)) / (2 * h)
+
+    h = 1e-3
+    est = (4 * cd(h / 2) - cd(h)) / 3
+    got = float(oracle_mod.dlambda(q, k, v, lam, do, s0, g))
+    assert abs(est - got) <= 1e-8 * max(1.0, abs(got)), (est, got)
+
+
+def test_dlambda_zero_decay_keeps_lag_one(oracle_mod):
+    """At lam = 0 only lag-1 terms survive: sum_t (q_t . k_{t-1})(do_t . v_{t-1})
+    + q_0^T S0 do_0 (+ <G, k_{T-2} v_{T-2}^T> from the state)."""
+    rng = np.random.default_rng(5)
+    T, d, e = 6, 3, 4
+    q, k, v, do = _rand(rng, T, d), _rand(rng, T, d), _rand(rng, T, e), _rand(rng, T, e)
+    s0, g = _rand(rng, d, e), _rand(rng, d, e)
+    want = sum(float(q[t] @ k[t - 1]) * float(do[t] @ v[t - 1]) for t in range(1, T))
+    want += float(q[0] @ s0 @ do[0]) + float(np.sum(g * np.outer(k[T - 2], v[T - 2])))
+    got = float(oracle_mod.dlambda(q, k, v, 0.0, do, s0, g))
+    assert abs(got - want) <= 1e-12 * max(1.0, abs(want))
