@@ -13,6 +13,7 @@
 #include <type_traits>
 
 #include "decode.cuh"
+#include "dlambda.cuh"
 #include "la2.h"
 #include "scan_f32.cuh"
 #include "scan_ws_sm100.cuh"
@@ -142,6 +143,35 @@ size_t seg_workspace_bytes(long long units, int T, int da, int dc, int sched) {
     return static_cast<size_t>(max_segments(units) - 1) * static_cast<size_t>(units) * state;
 }
 
+// The gradient in lambda (dlambda.cuh): each sequence is cut into g segments
+// of a multiple of 32 rows, g = min(32, 148 / sequences) (at least 1), so that
+// few sequences still fill the SMs.  Workspace, flat in T: one fp64 partial
+// sum per (sequence, segment) and the fp32 (W, U) pair at the end of every
+// segment but the last.
+struct DlPlan {
+    int g = 1;         // segments the workspace is sized for
+    int nseg = 1;      // segments of this T (<= g)
+    int seg_rows = 0;  // rows per segment
+};
+
+DlPlan dl_plan(long long seqs, int T) {
+    DlPlan pl;
+    pl.g = static_cast<int>(seqs >= kTargetCTAs ? 1 : (kTargetCTAs / seqs < kMaxSegments ? kTargetCTAs / seqs
+                                                                                          : kMaxSegments));
+    if (pl.g < 1) pl.g = 1;
+    const long long per = cdiv(T > 0 ? T : 1, pl.g);
+    pl.seg_rows = static_cast<int>(cdiv(per, la2::kDlRows) * la2::kDlRows);
+    pl.nseg = static_cast<int>(cdiv(T > 0 ? T : 1, pl.seg_rows));
+    return pl;
+}
+
+size_t dl_workspace_bytes(long long seqs, int T, int d, int e) {
+    const DlPlan pl = dl_plan(seqs, T);
+    size_t partial = static_cast<size_t>(seqs) * pl.g * sizeof(double);
+    partial = (partial + 255) & ~static_cast<size_t>(255);
+    return partial + static_cast<size_t>(seqs) * (pl.g - 1) * 2 * d * e * sizeof(float);
+}
+
 struct DeviceState {
     std::once_flag once;
     int* status = nullptr;
@@ -164,6 +194,12 @@ bool device_setup(int* dev_out, int** status_out) {
         s.never_set = static_cast<int*>(f);
         ok = ok && set_ws_attrs<64, 64>() && set_ws_attrs<64, 128>() && set_ws_attrs<128, 64>() &&
              set_ws_attrs<128, 128>();
+        ok = ok &&
+             cudaFuncSetAttribute(la2::la2_dlam_scan<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(la2::dl_scan_smem_bytes())) == cudaSuccess &&
+             cudaFuncSetAttribute(la2::la2_dlam_scan<__nv_bfloat16>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(la2::dl_scan_smem_bytes())) == cudaSuccess;
         ok = ok && cudaFuncSetAttribute(la2::la2_scan_f32,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         static_cast<int>(la2::f32_scan_smem_bytes(128, 128, 256))) ==
@@ -624,6 +660,96 @@ la2_status la2_selftest_timeout(const void* q, const void* k, const void* v, con
     const RoleDesc r = {q, k, v, out, d, e, +1};
     return launch_bf16_ws(&r, 1, decay, 1, 1, T, false, LA2_SCHEDULE_UNIFORM, status, nullptr, hold,
                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t la2_dlambda_workspace_bytes(int B, int H, int T, int d, int e, la2_dtype dtype) {
+    if (dtype != LA2_DTYPE_F32 && dtype != LA2_DTYPE_BF16) return static_cast<size_t>(-1);
+    if (B < 0 || H < 0 || T < 0 || d <= 0 || e <= 0) return static_cast<size_t>(-1);
+    if (d > 128 || e > 128 || static_cast<long long>(B) * H > (1LL << 24)) return static_cast<size_t>(-1);
+    if (B == 0 || H == 0 || T == 0) return 0;
+    return dl_workspace_bytes(static_cast<long long>(B) * H, T, d, e);
+}
+
+la2_status la2_dlambda(const void* q, const void* k, const void* v, const float* decay,
+                       const void* dout, const float* init_state, const float* d_final_state,
+                       float* d_decay, int B, int H, int T, int d, int e, la2_dtype dtype,
+                       la2_layout layout, void* workspace, size_t workspace_bytes,
+                       la2_stream_t stream) {
+    t_last_launches = 0;
+    if (dtype != LA2_DTYPE_F32 && dtype != LA2_DTYPE_BF16) return LA2_ERR_INVALID_ARG;
+    if (layout != LA2_LAYOUT_BHTD && layout != LA2_LAYOUT_BTHD) return LA2_ERR_INVALID_ARG;
+    if (B < 0 || H < 0 || T < 0 || d <= 0 || e <= 0) return LA2_ERR_INVALID_ARG;
+    if (d > 128 || e > 128 || static_cast<long long>(B) * H > (1LL << 24)) return LA2_ERR_UNSUPPORTED;
+    if (H == 0) return LA2_OK;
+    if (!d_decay || (reinterpret_cast<uintptr_t>(d_decay) & 3u)) return LA2_ERR_INVALID_ARG;
+    const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (B == 0 || T == 0) {
+        // no position: L does not depend on lambda
+        return cudaMemsetAsync(d_decay, 0, static_cast<size_t>(H) * sizeof(float), cs) == cudaSuccess
+                   ? LA2_OK
+                   : LA2_ERR_CUDA;
+    }
+    if (!q || !k || !v || !decay || !dout) return LA2_ERR_INVALID_ARG;
+    const size_t esz = dtype == LA2_DTYPE_BF16 ? 2 : 4;
+    const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                          reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(dout);
+    const uintptr_t smis = reinterpret_cast<uintptr_t>(decay) | reinterpret_cast<uintptr_t>(init_state) |
+                           reinterpret_cast<uintptr_t>(d_final_state);
+    if ((mis & (esz - 1)) || (smis & 3u)) return LA2_ERR_INVALID_ARG;
+    const long long seqs = static_cast<long long>(B) * H;
+    const size_t need = dl_workspace_bytes(seqs, T, d, e);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) ? LA2_ERR_INVALID_ARG
+                                                                               : LA2_ERR_WORKSPACE;
+    int dev = 0;
+    int* status = nullptr;
+    if (!device_setup(&dev, &status)) return LA2_ERR_CUDA;
+    const DlPlan pl = dl_plan(seqs, T);
+    la2::DlParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.g = dout;
+    p.decay = decay;
+    p.init = init_state;
+    p.dfin = d_final_state;
+    size_t poff = static_cast<size_t>(seqs) * pl.g * sizeof(double);
+    poff = (poff + 255) & ~static_cast<size_t>(255);
+    p.partial = static_cast<double*>(workspace);
+    p.seg_state = reinterpret_cast<float*>(static_cast<char*>(workspace) + poff);
+    p.d_decay = d_decay;
+    p.B = B;
+    p.H = H;
+    p.T = T;
+    p.d = d;
+    p.e = e;
+    p.bthd = layout == LA2_LAYOUT_BTHD ? 1 : 0;
+    p.nseg = pl.nseg;
+    p.seg_rows = pl.seg_rows;
+    // 16-byte vector staging when every row starts on a 16-byte boundary
+    const int vel = static_cast<int>(16 / esz);
+    p.vec = (d % vel == 0 && e % vel == 0 && !(mis & 15u)) ? 1 : 0;
+    const bool bf = dtype == LA2_DTYPE_BF16;
+    int launches = 0;
+    if (pl.nseg > 1) {
+        const unsigned grid = static_cast<unsigned>(seqs * (pl.nseg - 1));
+        if (bf)
+            la2::la2_dlam_prepass<__nv_bfloat16><<<grid, la2::kDlThreads, la2::dl_prepass_smem_bytes(), cs>>>(p);
+        else
+            la2::la2_dlam_prepass<float><<<grid, la2::kDlThreads, la2::dl_prepass_smem_bytes(), cs>>>(p);
+        ++launches;
+    }
+    const unsigned grid = static_cast<unsigned>(seqs * pl.nseg);
+    if (bf)
+        la2::la2_dlam_scan<__nv_bfloat16><<<grid, la2::kDlThreads, la2::dl_scan_smem_bytes(), cs>>>(p);
+    else
+        la2::la2_dlam_scan<float><<<grid, la2::kDlThreads, la2::dl_scan_smem_bytes(), cs>>>(p);
+    la2::la2_dlam_reduce<<<static_cast<unsigned>((H + 255) / 256), 256, 0, cs>>>(p);
+    launches += 2;
+    if (cudaGetLastError() != cudaSuccess) return LA2_ERR_CUDA;
+    t_last_launches = launches;
+    return LA2_OK;
 }
 
 const char* la2_status_str(la2_status s) {

@@ -29,7 +29,7 @@ LA2_DTYPE_BF16 = 1
 EXPORTS = ("la2_workspace_bytes", "la2_fwd", "la2_fwd_state", "la2_fwd_ex", "la2_bwd", "la2_bwd_ex",
            "la2_decode", "la2_status_str", "la2_device_status", "la2_last_launch_count",
            "la2_fwd_noalloc", "la2_set_schedule", "la2_plan_info", "la2_selftest_timeout",
-           "la2_bwd_state")
+           "la2_bwd_state", "la2_dlambda", "la2_dlambda_workspace_bytes")
 
 LA2_LAYOUT_BHTD = 0
 LA2_LAYOUT_BTHD = 1
@@ -91,6 +91,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la2_bwd_state.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i,
                                   i, vp, sz, vp]
     lib.la2_bwd_state.restype = i
+    lib.la2_dlambda_workspace_bytes.argtypes = [i, i, i, i, i, i]
+    lib.la2_dlambda_workspace_bytes.restype = sz
+    lib.la2_dlambda.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
+    lib.la2_dlambda.restype = i
     _lib = lib
     return lib
 
@@ -384,6 +388,35 @@ def la2_bwd_state(q, k, v, decay, dout, init_state=None, d_final_state=None, lay
     if st != LA2_OK:
         raise LA2Error(st, "la2_bwd_state")
     return dq, dk, dv, d_init_state
+
+
+def la2_dlambda_workspace_bytes(B, H, T, d, e, dtype) -> int:
+    return int(load().la2_dlambda_workspace_bytes(B, H, T, d, e, dtype))
+
+
+def la2_dlambda(q, k, v, decay, dout, init_state=None, d_final_state=None, layout: str = "bhtd",
+                d_decay=None, stream=None, workspace=None):
+    """dL/d(decay) [H] (summed over the batch) for L = sum(dout * out) + sum(d_final_state *
+    final_state), the forward la2_fwd_ex(q, k, v, decay, layout, init_state)."""
+    B, H, T, d, e = _dims(q, v, layout)
+    dt = _dtype_code(q)
+    for t, n, D in ((q, "q", d), (k, "k", d), (v, "v", e), (dout, "dout", e)):
+        _check(t, n, _shape(layout, B, H, T, D), q.dtype)
+    _check(decay, "decay", (H,), torch.float32)
+    d_decay = torch.empty((H,), dtype=torch.float32, device=q.device) if d_decay is None else d_decay
+    _check(d_decay, "d_decay", (H,), torch.float32)
+    ptrs = []
+    for t, n in ((init_state, "init_state"), (d_final_state, "d_final_state")):
+        if t is not None:
+            _check(t, n, (B, H, d, e), torch.float32)
+        ptrs.append(0 if t is None else t.data_ptr())
+    wp, wn = _workspace(la2_dlambda_workspace_bytes(B, H, T, d, e, dt), q.device, workspace)
+    st = int(load().la2_dlambda(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(),
+                                dout.data_ptr(), ptrs[0], ptrs[1], d_decay.data_ptr(), B, H, T, d, e,
+                                dt, _LAYOUTS[layout], wp, wn, _stream_ptr(stream)))
+    if st != LA2_OK:
+        raise LA2Error(st, "la2_dlambda")
+    return d_decay
 
 
 def la2_decode_raw(q, k, v, decay, state, out, B, H, d, e, dtype, stream=0) -> int:

@@ -277,6 +277,37 @@ la2_status la2_bwd_state(const void *q, const void *k, const void *v, const floa
                          la2_layout layout, void *workspace, size_t workspace_bytes,
                          la2_stream_t stream);
 
+/*
+ * Gradient with respect to the decay: d_decay[h] = sum over the batch of
+ * dL/dlambda_h, for the same L as la2_bwd_state (the forward from init_state,
+ * d_final_state the gradient arriving at its final state; NULL = zero):
+ *
+ *   dL/dlambda = sum_{s<t} (t-s) lambda^(t-s-1) (q_t . k_s)(dout_t . v_s)
+ *                + sum_t (t+1) lambda^t q_t^T S0 dout_t + <G, dS_{T-1}/dlambda>
+ *
+ * i.e. the recurrence of the "Lightning Attention" explainer (section 1) with
+ * its decay differentiated: U_t = dS_t/dlambda = lambda U_{t-1} + S_{t-1}, and
+ * dL/dlambda = sum_t q_t^T U_t dout_t + <G, U_{T-1}>.  The pages print no
+ * gradient in lambda; this is the derivative of the definition.
+ *
+ * Inputs as la2_bwd_state (dtype F32 or BF16, any 1 <= d, e <= 128, both
+ * layouts, element-aligned pointers); d_decay: device fp32 [H], overwritten.
+ * Computed in fp32 SIMT arithmetic with the scalar accumulated in fp64, in 32-
+ * row sub-tiles, each sequence cut into up to 32 segments (a pre-pass gives
+ * each segment its incoming states); the batch is summed in a fixed order, so
+ * the result is deterministic.  workspace: device memory of at least
+ * la2_dlambda_workspace_bytes() bytes, 256-byte aligned (LA2_ERR_WORKSPACE if
+ * missing or short), flat in T.  B = 0 or T = 0 writes zeros.  Asynchronous on
+ * `stream`; two or three launches.
+ */
+size_t la2_dlambda_workspace_bytes(int B, int H, int T, int d, int e, la2_dtype dtype);
+
+la2_status la2_dlambda(const void *q, const void *k, const void *v, const float *decay,
+                       const void *dout, const float *init_state, const float *d_final_state,
+                       float *d_decay, int B, int H, int T, int d, int e, la2_dtype dtype,
+                       la2_layout layout, void *workspace, size_t workspace_bytes,
+                       la2_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 const char *la2_status_str(la2_status status);
 

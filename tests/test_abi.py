@@ -200,3 +200,25 @@ def test_bwd_state_rejects_misaligned_states(lib):
                                      st[2], 1, 2, 256, 128, 128, 128, la2.LA2_DTYPE_BF16,
                                      la2.LA2_LAYOUT_BHTD, 0, 0, 0)
         assert r == la2.LA2_ERR_INVALID_ARG
+
+
+def test_dlambda_workspace_flat_in_T_and_arguments(lib):
+    sizes = {la2.la2_dlambda_workspace_bytes(1, 16, T, 128, 128, la2.LA2_DTYPE_BF16)
+             for T in (1000, 65536, 1 << 20)}
+    assert len(sizes) == 1 and sizes.pop() > 0
+    assert la2.la2_dlambda_workspace_bytes(1, 2, 100, 129, 64, la2.LA2_DTYPE_F32) == 2 ** 64 - 1
+    assert la2.la2_dlambda_workspace_bytes(1, 2, 0, 64, 64, la2.LA2_DTYPE_F32) == 0
+    f = la2.load().la2_dlambda
+    ok = dict(B=1, H=2, T=100, d=64, e=64)
+    # misaligned element pointer, NULL input, missing workspace, bad layout
+    assert f(FAKE + 1, FAKE, FAKE, FAKE, FAKE, 0, 0, FAKE, 1, 2, 100, 64, 64, la2.LA2_DTYPE_BF16, 0,
+             FAKE, 1 << 30, 0) == la2.LA2_ERR_INVALID_ARG
+    assert f(0, FAKE, FAKE, FAKE, FAKE, 0, 0, FAKE, 1, 2, 100, 64, 64, la2.LA2_DTYPE_BF16, 0,
+             FAKE, 1 << 30, 0) == la2.LA2_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0, FAKE, 1, 2, 100, 64, 64, la2.LA2_DTYPE_BF16, 0,
+             0, 0, 0) == la2.LA2_ERR_WORKSPACE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0, FAKE, 1, 2, 100, 64, 64, la2.LA2_DTYPE_BF16, 7,
+             FAKE, 1 << 30, 0) == la2.LA2_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0, FAKE, 1, 2, 100, 200, 64, la2.LA2_DTYPE_BF16, 0,
+             FAKE, 1 << 30, 0) == la2.LA2_ERR_UNSUPPORTED
+    del ok
