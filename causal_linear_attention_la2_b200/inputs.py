@@ -92,6 +92,14 @@ for _T in SWEEP_T:
         _w = sweep_workload(_T, _blk)
         WORKLOADS[_w.name] = _w
 
+# The launch plan of the T = 131,072 sweep point (32 sequences: a forward in
+# four segments with a state pre-pass, a backward of 96 one-segment units) at
+# an eighth of its length, so that a full profiler capture holds about 1.7 GB
+# on the device; per-launch DRAM traffic scales to the full length by 8.
+WORKLOADS["sweep_plan_T16384"] = Workload(
+    "sweep_plan_T16384", 1, 32, 16384, 128, 128, 128, "bf16", "tnl",
+    "profiling shape: the T = 131,072 sweep point's launch plan at 1/8 of its length")
+
 
 # Decode-step shapes: one new token for each of B sequences of H heads, the
 # heads of the TNL-15B and TNL-400M layers at serving batch sizes (the fp32

@@ -59,6 +59,8 @@ def _load():
         lib.la2o_backward_state.argtypes = [i, i, i, i, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp,
                                             dp, i]
         lib.la2o_dlambda.argtypes = [i, i, i, i, dp, dp, dp, dp, dp, dp, dp, dp, i]
+        lib.la2o_forward_norm.argtypes = [i, i, i, i, dp, dp, dp, dp, dp, dp, i]
+        lib.la2o_backward_norm.argtypes = [i, i, i, i, dp, dp, dp, dp, dp, dp, dp, dp, i]
         lib.la2o_max_threads.restype = i
         _lib = lib
     return _lib
@@ -190,6 +192,30 @@ def dlambda(q, k, v, lam, dout, s0=None, dsT=None, nthreads: int = 0):
                      _ptr(s0a) if s0a is not None else None,
                      _ptr(gTa) if gTa is not None else None, _ptr(out), int(nthreads))
     return out.reshape(lead)
+
+
+def forward_norm(q, k, v, lam, nthreads: int = 0):
+    """(y, den): the normalised form y_t = (S_t^T q_t) / (q_t . z_t) with
+    z_t = lam z_{t-1} + k_t (identity feature map)."""
+    lib = _load()
+    lead, ns, T, d, e, lam = _prep(q, k, v, lam)
+    qc, kc, vc = (_f64(x).reshape(ns, T, w) for x, w in ((q, d), (k, d), (v, e)))
+    y = np.empty((ns, T, e))
+    den = np.empty((ns, T))
+    lib.la2o_forward_norm(ns, T, d, e, _ptr(lam), _ptr(qc), _ptr(kc), _ptr(vc), _ptr(y), _ptr(den),
+                          int(nthreads))
+    return y.reshape(*lead, T, e), den.reshape(*lead, T)
+
+
+def backward_norm(q, k, v, lam, dy, nthreads: int = 0):
+    """(dq, dk, dv) of L = sum_t dy_t . y_t for y = forward_norm(...)[0]."""
+    lib = _load()
+    lead, ns, T, d, e, lam = _prep(q, k, v, lam)
+    qc, kc, vc, gc = (_f64(x).reshape(ns, T, w) for x, w in ((q, d), (k, d), (v, e), (dy, e)))
+    dq = np.empty((ns, T, d)); dk = np.empty((ns, T, d)); dv = np.empty((ns, T, e))
+    lib.la2o_backward_norm(ns, T, d, e, _ptr(lam), _ptr(qc), _ptr(kc), _ptr(vc), _ptr(gc),
+                           _ptr(dq), _ptr(dk), _ptr(dv), int(nthreads))
+    return dq.reshape(*lead, T, d), dk.reshape(*lead, T, d), dv.reshape(*lead, T, e)
 
 
 def forward_blocked(q, k, v, lam, block: int, nthreads: int = 0) -> np.ndarray:

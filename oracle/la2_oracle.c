@@ -57,6 +57,18 @@
  *                           recurrence: U_t = dS_t/dlambda obeys
  *                           U_t = lambda U_{t-1} + S_{t-1} (U_{-1} = 0), and
  *                           dL/dlambda = sum_t q_t^T U_t do_t + <G, U_{T-1}>.
+ *   la2o_forward_norm       the normalised form of section 1 (feature map
+ *                           identity, as section 2 says the default is; any
+ *                           other phi is applied to q and k beforehand), with
+ *                           the same decay on the denominator's running sum:
+ *                           z_t = lambda z_{t-1} + k_t, den_t = q_t . z_t,
+ *                           y_t = (S_t^T q_t) / den_t.
+ *   la2o_backward_norm      gradients of L = sum_t dy_t . y_t through it:
+ *                           dnum_t = dy_t / den_t, dden_t = -(dy_t . num_t) / den_t^2,
+ *                           dq_t = S_t dnum_t + dden_t z_t; reverse sweep
+ *                           R_t = lambda R_{t+1} + q_t dnum_t^T,
+ *                           r_t = lambda r_{t+1} + dden_t q_t,
+ *                           dk_t = R_t v_t + r_t, dv_t = R_t^T k_t.
  *   la2o_decode_step        one step of the same recurrence for one new token
  *                           per sequence: S <- lambda S + k v^T, o = S^T q.
  *   la2o_backward_blocked   the mirrored tiling for the backward (the pages say
@@ -346,6 +358,115 @@ void la2o_dlambda(int NS, int T, int d, int e, const double *lam,
         dlam[n] = acc;
         free(S);
         free(U);
+    }
+}
+
+/* ------------------------------------------------- normalised variant */
+
+void la2o_forward_norm(int NS, int T, int d, int e, const double *lam,
+                       const double *q, const double *k, const double *v,
+                       double *y, double *den, int nthreads)
+{
+    set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < NS; ++n) {
+        const double *qn = q + (size_t)n * T * d, *kn = k + (size_t)n * T * d;
+        const double *vn = v + (size_t)n * T * e;
+        double *yn = y + (size_t)n * T * e, *dn = den + (size_t)n * T;
+        double *S = (double *)calloc((size_t)d * e, sizeof(double));
+        double *z = (double *)calloc((size_t)d, sizeof(double));
+        const double l = lam[n];
+        for (int t = 0; t < T; ++t) {
+            const double *qt = qn + (size_t)t * d, *kt = kn + (size_t)t * d;
+            const double *vt = vn + (size_t)t * e;
+            for (int i = 0; i < d; ++i) {
+                z[i] = l * z[i] + kt[i];
+                for (int j = 0; j < e; ++j)
+                    S[(size_t)i * e + j] = l * S[(size_t)i * e + j] + kt[i] * vt[j];
+            }
+            double dd = 0.0;
+            for (int i = 0; i < d; ++i) dd += qt[i] * z[i];
+            dn[t] = dd;
+            double *yt = yn + (size_t)t * e;
+            for (int j = 0; j < e; ++j) yt[j] = 0.0;
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < e; ++j) yt[j] += qt[i] * S[(size_t)i * e + j];
+            for (int j = 0; j < e; ++j) yt[j] /= dd;
+        }
+        free(S);
+        free(z);
+    }
+}
+
+void la2o_backward_norm(int NS, int T, int d, int e, const double *lam,
+                        const double *q, const double *k, const double *v,
+                        const double *dy, double *dq, double *dk, double *dv,
+                        int nthreads)
+{
+    set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < NS; ++n) {
+        const double *qn = q + (size_t)n * T * d, *kn = k + (size_t)n * T * d;
+        const double *vn = v + (size_t)n * T * e, *gn = dy + (size_t)n * T * e;
+        double *dqn = dq + (size_t)n * T * d, *dkn = dk + (size_t)n * T * d;
+        double *dvn = dv + (size_t)n * T * e;
+        double *S = (double *)calloc((size_t)d * e, sizeof(double));
+        double *z = (double *)calloc((size_t)d, sizeof(double));
+        double *dnum = (double *)malloc(sizeof(double) * ((size_t)T * e + 1));
+        double *dden = (double *)malloc(sizeof(double) * ((size_t)T + 1));
+        const double l = lam[n];
+        /* forward sweep: S_t, z_t, num_t, den_t; dq_t = S_t dnum_t + dden_t z_t */
+        for (int t = 0; t < T; ++t) {
+            const double *qt = qn + (size_t)t * d, *kt = kn + (size_t)t * d;
+            const double *vt = vn + (size_t)t * e, *gt = gn + (size_t)t * e;
+            for (int i = 0; i < d; ++i) {
+                z[i] = l * z[i] + kt[i];
+                for (int j = 0; j < e; ++j)
+                    S[(size_t)i * e + j] = l * S[(size_t)i * e + j] + kt[i] * vt[j];
+            }
+            double den = 0.0;
+            for (int i = 0; i < d; ++i) den += qt[i] * z[i];
+            double gnum = 0.0;
+            for (int j = 0; j < e; ++j) {
+                double num = 0.0;
+                for (int i = 0; i < d; ++i) num += qt[i] * S[(size_t)i * e + j];
+                gnum += gt[j] * num;
+                dnum[(size_t)t * e + j] = gt[j] / den;
+            }
+            dden[t] = -gnum / (den * den);
+            double *dqt = dqn + (size_t)t * d;
+            for (int i = 0; i < d; ++i) {
+                double acc = dden[t] * z[i];
+                for (int j = 0; j < e; ++j) acc += S[(size_t)i * e + j] * dnum[(size_t)t * e + j];
+                dqt[i] = acc;
+            }
+        }
+        /* reverse sweep: R_t = lambda R_{t+1} + q_t dnum_t^T, r_t = lambda r_{t+1} + dden_t q_t */
+        double *R = S, *r = z;
+        memset(R, 0, sizeof(double) * (size_t)d * e);
+        memset(r, 0, sizeof(double) * (size_t)d);
+        for (int t = T - 1; t >= 0; --t) {
+            const double *qt = qn + (size_t)t * d, *kt = kn + (size_t)t * d;
+            const double *vt = vn + (size_t)t * e;
+            for (int i = 0; i < d; ++i) {
+                r[i] = l * r[i] + dden[t] * qt[i];
+                for (int j = 0; j < e; ++j)
+                    R[(size_t)i * e + j] = l * R[(size_t)i * e + j] + qt[i] * dnum[(size_t)t * e + j];
+            }
+            double *dkt = dkn + (size_t)t * d, *dvt = dvn + (size_t)t * e;
+            for (int i = 0; i < d; ++i) {
+                double acc = r[i];
+                for (int j = 0; j < e; ++j) acc += R[(size_t)i * e + j] * vt[j];
+                dkt[i] = acc;
+            }
+            for (int j = 0; j < e; ++j) dvt[j] = 0.0;
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < e; ++j) dvt[j] += R[(size_t)i * e + j] * kt[i];
+        }
+        free(S);
+        free(z);
+        free(dnum);
+        free(dden);
     }
 }
 

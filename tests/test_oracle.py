@@ -436,3 +436,96 @@ def test_dlambda_zero_decay_keeps_lag_one(oracle_mod):
     want += float(q[0] @ s0 @ do[0]) + float(np.sum(g * np.outer(k[T - 2], v[T - 2])))
     got = float(oracle_mod.dlambda(q, k, v, 0.0, do, s0, g))
     assert abs(got - want) <= 1e-12 * max(1.0, abs(want))
+
+
+# ------------------------------------------------------ normalised variant
+
+def _norm_closed_form(q, k, v, dy, lam):
+    """The normalised form and its gradients as matrices, D_ts = lam^(t-s) [s<=t]:
+      num = ((Q K^T) * D) V,  z = D K,  den = rowsum(Q * z),  y = num / den
+      dnum = dy / den,  dden = -rowsum(dy * num) / den^2
+      dQ = ((dnum V^T) * D) K + dden z
+      dK = ((dnum V^T) * D)^T Q + D^T (dden Q)
+      dV = ((Q K^T) * D)^T dnum"""
+    D = _decay_matrix(q.shape[0], lam)
+    A = (q @ k.T) * D
+    num = A @ v
+    z = D @ k
+    den = np.sum(q * z, axis=1)
+    y = num / den[:, None]
+    dnum = dy / den[:, None]
+    dden = -np.sum(dy * num, axis=1) / den ** 2
+    G = (dnum @ v.T) * D
+    dq1, dq2 = G @ k, dden[:, None] * z
+    dk1, dk2 = G.T @ q, D.T @ (dden[:, None] * q)
+    dv = A.T @ dnum
+    # the two parts of dq (and of dk) cancel where y hardly depends on q (k),
+    # e.g. T = 1 or a tiny decay; compare those against the parts' size
+    scale = (None, None, max(np.max(np.abs(dq1)), np.max(np.abs(dq2))),
+             max(np.max(np.abs(dk1)), np.max(np.abs(dk2))), None)
+    return (y, den, dq1 + dq2, dk1 + dk2, dv), scale
+
+
+def _positive(rng, *shape):
+    return np.abs(rng.standard_normal(shape)) + 0.1
+
+
+@pytest.mark.parametrize("T,d,e", [(1, 3, 2), (9, 4, 5), (40, 8, 3)])
+def test_norm_closed_form(oracle_mod, T, d, e):
+    rng = np.random.default_rng(500 + T)
+    for lam in LAMS:
+        q, k = _positive(rng, T, d), _positive(rng, T, d)
+        v, dy = _rand(rng, T, e), _rand(rng, T, e)
+        y, den = oracle_mod.forward_norm(q, k, v, lam)
+        grads = oracle_mod.backward_norm(q, k, v, lam, dy)
+        want, scale = _norm_closed_form(q, k, v, dy, lam)
+        for a, b, sc in zip((y, den) + tuple(grads), want, scale):
+            ref = np.max(np.abs(b)) if sc is None else max(sc, np.max(np.abs(b)))
+            assert np.max(np.abs(a - b)) <= 1e-12 * ref, lam
+
+
+def test_norm_single_position_returns_v(oracle_mod):
+    """T = 1: y = (q.k) v / (q.k) = v whatever q and k, so dq = dk = 0, dv = dy."""
+    rng = np.random.default_rng(2)
+    q, k, v, dy = _positive(rng, 1, 4), _positive(rng, 1, 4), _rand(rng, 1, 3), _rand(rng, 1, 3)
+    y, _ = oracle_mod.forward_norm(q, k, v, 0.7)
+    dq, dk, dv = oracle_mod.backward_norm(q, k, v, 0.7, dy)
+    assert _rel(y, v) < 1e-15 and np.max(np.abs(dq)) < 1e-15 and np.max(np.abs(dk)) < 1e-15
+    assert _rel(dv, dy) < 1e-15
+
+
+def test_norm_scale_invariance(oracle_mod):
+    """y does not change when q or k is scaled by a positive constant."""
+    rng = np.random.default_rng(3)
+    q, k, v = _positive(rng, 2, 20, 4), _positive(rng, 2, 20, 4), _rand(rng, 2, 20, 3)
+    lam = np.array([0.9, 1.0])
+    y, _ = oracle_mod.forward_norm(q, k, v, lam)
+    assert _rel(oracle_mod.forward_norm(3.0 * q, k, v, lam)[0], y) < 1e-13
+    assert _rel(oracle_mod.forward_norm(q, 0.25 * k, v, lam)[0], y) < 1e-13
+
+
+def test_norm_central_differences(oracle_mod):
+    """Richardson-extrapolated central differences of L = sum dy * y in every
+    coordinate of q, k and v (y is not linear in q or k, so plain differences
+    would carry an h^2 error)."""
+    rng = np.random.default_rng(4)
+    T, d, e, lam = 5, 3, 2, 0.9
+    q, k, v, dy = _positive(rng, T, d), _positive(rng, T, d), _rand(rng, T, e), _rand(rng, T, e)
+    grads = oracle_mod.backward_norm(q, k, v, lam, dy)
+
+    def loss(args):
+        return float(np.sum(dy * oracle_mod.forward_norm(*args, lam)[0]))
+
+    for idx, (arr, g) in enumerate(zip((q, k, v), grads)):
+        for pos in np.ndindex(arr.shape):
+            def cd(h):
+                args = [q, k, v]
+                up, dn = arr.copy(), arr.copy()
+                up[pos] += h
+                dn[pos] -= h
+                args[idx] = up
+                lu = loss(args)
+                args[idx] = dn
+                return (lu - loss(args)) / (2 * h)
+            est = (4 * cd(1e-3) - cd(2e-3)) / 3
+            assert abs(est - g[pos]) <= 1e-8 * max(1.0, abs(g[pos])), (idx, pos, est, g[pos])
