@@ -54,10 +54,15 @@ def peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+SCAN_SOURCES = ("ptx_sm100.cuh", "scan_ws_sm100.cuh")  # the files that define la2_scan_ws
+
+
 def kernel_source_hash() -> str:
+    """Hash of the scan kernel's sources: recorded DRAM traffic is used only
+    while the kernel is the one that was profiled."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "causal_linear_attention_la2_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(SCAN_SOURCES):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
