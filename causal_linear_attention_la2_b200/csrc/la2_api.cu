@@ -15,6 +15,7 @@
 #include "decode.cuh"
 #include "dlambda.cuh"
 #include "la2.h"
+#include "normalize.cuh"
 #include "scan_f32.cuh"
 #include "scan_ws_sm100.cuh"
 
@@ -46,14 +47,14 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-template <int DA, int DC>
+template <int DA, int DC, bool kNorm = false>
 bool set_ws_attrs() {
-    return cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC, false>,
+    return cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC, false, kNorm>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                la2::ws::Smem<DA, DC>::kBytes) == cudaSuccess &&
-           cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC, true>,
+                                la2::ws::Smem<DA, DC, kNorm>::kBytes) == cudaSuccess &&
+           cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC, true, kNorm>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                la2::ws::Smem<DA, DC>::kBytes) == cudaSuccess &&
+                                la2::ws::Smem<DA, DC, kNorm>::kBytes) == cudaSuccess &&
            cudaFuncSetAttribute(la2::ws::la2_state_ws<DA, DC>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 la2::ws::StateSmem<DA, DC>::kBytes) == cudaSuccess;
@@ -172,6 +173,31 @@ size_t dl_workspace_bytes(long long seqs, int T, int d, int e) {
     return partial + static_cast<size_t>(seqs) * (pl.g - 1) * 2 * d * e * sizeof(float);
 }
 
+// The normalised form (normalize.cuh): each sequence is cut into chunks of a
+// multiple of 32 rows, g = min(64, ceil(8 * 148 / sequences)) (at least 1), the
+// 128-thread scans then filling the SMs several CTAs deep.  Chunk end states
+// (one d-vector each but the last) sit in the workspace, flat in T.
+struct NzPlan {
+    int g = 1, nchunk = 1, rows = 0;
+};
+
+NzPlan nz_plan(long long seqs, int T) {
+    NzPlan pl;
+    const long long want = cdiv(8LL * kTargetCTAs, seqs > 0 ? seqs : 1);
+    pl.g = static_cast<int>(want < 1 ? 1 : (want > 64 ? 64 : want));
+    const long long per = cdiv(T > 0 ? T : 1, pl.g);
+    pl.rows = static_cast<int>(cdiv(per, la2::kNzRows) * la2::kNzRows);
+    pl.nchunk = static_cast<int>(cdiv(T > 0 ? T : 1, pl.rows));
+    return pl;
+}
+
+size_t nz_chunk_bytes(long long seqs, int T, int d) {
+    const NzPlan pl = nz_plan(seqs, T);
+    return static_cast<size_t>(seqs) * (pl.g - 1) * d * sizeof(float);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
 struct DeviceState {
     std::once_flag once;
     int* status = nullptr;
@@ -193,7 +219,8 @@ bool device_setup(int* dev_out, int** status_out) {
         ok = ok && cudaGetSymbolAddress(&f, g_la2_never_set) == cudaSuccess;
         s.never_set = static_cast<int*>(f);
         ok = ok && set_ws_attrs<64, 64>() && set_ws_attrs<64, 128>() && set_ws_attrs<128, 64>() &&
-             set_ws_attrs<128, 128>();
+             set_ws_attrs<128, 128>() && set_ws_attrs<64, 64, true>() && set_ws_attrs<64, 128, true>() &&
+             set_ws_attrs<128, 64, true>() && set_ws_attrs<128, 128, true>();
         ok = ok &&
              cudaFuncSetAttribute(la2::la2_dlam_scan<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(la2::dl_scan_smem_bytes())) == cudaSuccess &&
@@ -249,6 +276,7 @@ struct RoleDesc {
     const float* init = nullptr;  // state the scan starts from (see la2::ws::Role)
     float* fin = nullptr;         // state the scan ends with
     int init_t = 0;               // init stored transposed ([DC][DA])
+    const float* colf = nullptr;  // per-position factor on the summed index ([B*H, T])
 };
 
 // Self-test only (la2_selftest_timeout): a device flag that nothing sets, which
@@ -275,17 +303,17 @@ la2_status common_checks(int B, int H, int T, int d, int e, int block, la2_dtype
     return LA2_OK;
 }
 
-template <int DA, int DC>
+template <int DA, int DC, bool kNorm = false>
 void launch_ws(const la2::ws::Params& p, const SegPlan& sp, cudaStream_t stream) {
     if (sp.npre > 0)
         la2::ws::la2_state_ws<DA, DC><<<static_cast<unsigned>(sp.npre), la2::ws::kStateThreads,
                                         la2::ws::StateSmem<DA, DC>::kBytes, stream>>>(p);
     if (sp.balanced)
-        la2::ws::la2_scan_ws<DA, DC, true><<<static_cast<unsigned>(sp.nctas), la2::ws::kThreads,
-                                             la2::ws::Smem<DA, DC>::kBytes, stream>>>(p);
+        la2::ws::la2_scan_ws<DA, DC, true, kNorm><<<static_cast<unsigned>(sp.nctas), la2::ws::kThreads,
+                                                    la2::ws::Smem<DA, DC, kNorm>::kBytes, stream>>>(p);
     else
-        la2::ws::la2_scan_ws<DA, DC, false><<<static_cast<unsigned>(sp.nctas), la2::ws::kThreads,
-                                              la2::ws::Smem<DA, DC>::kBytes, stream>>>(p);
+        la2::ws::la2_scan_ws<DA, DC, false, kNorm><<<static_cast<unsigned>(sp.nctas), la2::ws::kThreads,
+                                                     la2::ws::Smem<DA, DC, kNorm>::kBytes, stream>>>(p);
 }
 
 // Launches the warp-specialised kernel over `n` roles that share (DA, DC),
@@ -293,7 +321,7 @@ void launch_ws(const la2::ws::Params& p, const SegPlan& sp, cudaStream_t stream)
 // segment starts inside its unit.
 la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
                           bool bthd, int sched, int* status, float* seg_state, const Hold& hold,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, bool norm = false) {
     la2::ws::Params p;
     std::memset(&p, 0, sizeof(p));
     const int BH = B * H;
@@ -308,6 +336,7 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
         p.role[r].fin = roles[r].fin;
         p.role[r].dir = roles[r].dir;
         p.role[r].init_t = roles[r].init_t;
+        p.role[r].colf = roles[r].colf;
     }
     p.decay = decay;
     p.status = status;
@@ -325,10 +354,17 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
     p.seg_state = seg_state;
     if (sp.npre > 0 && !seg_state) return LA2_ERR_WORKSPACE;
     if (sp.nctas > 0x7fffffffLL) return LA2_ERR_UNSUPPORTED;
-    if (da == 128 && dc == 128) launch_ws<128, 128>(p, sp, stream);
-    else if (da == 128) launch_ws<128, 64>(p, sp, stream);
-    else if (dc == 128) launch_ws<64, 128>(p, sp, stream);
-    else launch_ws<64, 64>(p, sp, stream);
+    if (norm) {
+        if (da == 128 && dc == 128) launch_ws<128, 128, true>(p, sp, stream);
+        else if (da == 128) launch_ws<128, 64, true>(p, sp, stream);
+        else if (dc == 128) launch_ws<64, 128, true>(p, sp, stream);
+        else launch_ws<64, 64, true>(p, sp, stream);
+    } else {
+        if (da == 128 && dc == 128) launch_ws<128, 128>(p, sp, stream);
+        else if (da == 128) launch_ws<128, 64>(p, sp, stream);
+        else if (dc == 128) launch_ws<64, 128>(p, sp, stream);
+        else launch_ws<64, 64>(p, sp, stream);
+    }
     if (cudaGetLastError() != cudaSuccess) return LA2_ERR_CUDA;
     t_last_launches += sp.npre > 0 ? 2 : 1;
     return LA2_OK;
@@ -350,6 +386,7 @@ la2_status launch_f32(const RoleDesc* roles, int n, const float* decay, int B, i
         p.role[r].init = roles[r].init;
         p.role[r].fin = roles[r].fin;
         p.role[r].init_t = roles[r].init_t;
+        p.role[r].colf = roles[r].colf;
         da_max = roles[r].da > da_max ? roles[r].da : da_max;
         dc_max = roles[r].dc > dc_max ? roles[r].dc : dc_max;
     }
@@ -399,7 +436,8 @@ size_t bf16_workspace_bytes(const RoleDesc* roles, int n, int B, int H, int T, i
 
 la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
                      int block, la2_dtype dtype, bool bthd, int sched, void* workspace,
-                     size_t ws_bytes, cudaStream_t stream, const Hold& hold = Hold()) {
+                     size_t ws_bytes, cudaStream_t stream, const Hold& hold = Hold(),
+                     bool norm = false) {
     int dev = 0;
     int* status = nullptr;
     if (dtype == LA2_DTYPE_BF16) {
@@ -413,8 +451,46 @@ la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, in
         float* seg = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) + off) : nullptr;
         off += seg_workspace_bytes(static_cast<long long>(B) * H * m, T, g[0].da, g[0].dc, sched);
         off = (off + 255) & ~static_cast<size_t>(255);
-        return launch_bf16_ws(g, m, decay, B, H, T, bthd, sched, status, seg, hold, stream);
+        return launch_bf16_ws(g, m, decay, B, H, T, bthd, sched, status, seg, hold, stream, norm);
     });
+}
+
+
+template <typename Tin>
+void nz_launch(const la2::NzParams& p, long long seqs, cudaStream_t cs, int* launches) {
+    if (p.nchunk > 1) {
+        la2::la2_nz_prepass<Tin><<<static_cast<unsigned>(seqs * (p.nchunk - 1)), la2::kNzThreads, 0, cs>>>(p);
+        ++*launches;
+    }
+    la2::la2_nz_scan<Tin><<<static_cast<unsigned>(seqs * p.nchunk), la2::kNzThreads, 0, cs>>>(p);
+    ++*launches;
+}
+
+la2::NzParams nz_params(int B, int H, int T, int d, int e, bool bthd, const float* decay, float* chunk) {
+    la2::NzParams p;
+    std::memset(&p, 0, sizeof(p));
+    const NzPlan pl = nz_plan(static_cast<long long>(B) * H, T);
+    p.decay = decay;
+    p.chunk = chunk;
+    p.B = B;
+    p.H = H;
+    p.T = T;
+    p.d = d;
+    p.e = e;
+    p.bthd = bthd ? 1 : 0;
+    p.nchunk = pl.nchunk;
+    p.chunk_rows = pl.rows;
+    return p;
+}
+
+la2_status norm_checks(const void* q, const void* k, const void* v, const float* decay, int B, int H,
+                       int T, int d, int e, int block, la2_dtype dtype, la2_layout layout, bool* empty) {
+    if (layout != LA2_LAYOUT_BHTD && layout != LA2_LAYOUT_BTHD) return LA2_ERR_INVALID_ARG;
+    const la2_status st = common_checks(B, H, T, d, e, block, dtype, empty);
+    if (st != LA2_OK || *empty) return st;
+    if (d > 128) return LA2_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !decay) return LA2_ERR_INVALID_ARG;
+    return LA2_OK;
 }
 
 }  // namespace
@@ -747,6 +823,140 @@ la2_status la2_dlambda(const void* q, const void* k, const void* v, const float*
         la2::la2_dlam_scan<float><<<grid, la2::kDlThreads, la2::dl_scan_smem_bytes(), cs>>>(p);
     la2::la2_dlam_reduce<<<static_cast<unsigned>((H + 255) / 256), 256, 0, cs>>>(p);
     launches += 2;
+    if (cudaGetLastError() != cudaSuccess) return LA2_ERR_CUDA;
+    t_last_launches = launches;
+    return LA2_OK;
+}
+
+
+size_t la2_norm_workspace_bytes(int B, int H, int T, int d, int e, int block, la2_dtype dtype,
+                                int is_bwd) {
+    bool empty = false;
+    if (common_checks(B, H, T, d, e, block, dtype, &empty) != LA2_OK || d > 128)
+        return static_cast<size_t>(-1);
+    if (empty) return 0;
+    const long long seqs = static_cast<long long>(B) * H;
+    size_t n = align256(la2_workspace_bytes(B, H, T, d, e, block, dtype, is_bwd));
+    if (is_bwd) n += 2 * align256(static_cast<size_t>(seqs) * T * sizeof(float));
+    return n + nz_chunk_bytes(seqs, T, d);
+}
+
+la2_status la2_fwd_norm(const void* q, const void* k, const void* v, const float* decay, float* y,
+                        float* den, int B, int H, int T, int d, int e, int block, la2_dtype dtype,
+                        la2_layout layout, void* workspace, size_t workspace_bytes,
+                        la2_stream_t stream) {
+    t_last_launches = 0;
+    bool empty = false;
+    la2_status st = norm_checks(q, k, v, decay, B, H, T, d, e, block, dtype, layout, &empty);
+    if (st != LA2_OK || empty) return st;
+    if (!y || (reinterpret_cast<uintptr_t>(den) & 3u)) return LA2_ERR_INVALID_ARG;
+    const size_t need = la2_norm_workspace_bytes(B, H, T, d, e, block, dtype, 0);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return LA2_ERR_WORKSPACE;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return LA2_ERR_INVALID_ARG;
+    const size_t fws = align256(la2_workspace_bytes(B, H, T, d, e, block, dtype, 0));
+    // the numerator (the normalised form's instantiation: hi + lo operands at every (d, e))
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y) ||
+        (reinterpret_cast<uintptr_t>(decay) & 3u))
+        return LA2_ERR_INVALID_ARG;
+    const RoleDesc num = {q, k, v, y, d, e, +1};
+    st = run_roles(&num, 1, decay, B, H, T, block, dtype, layout == LA2_LAYOUT_BTHD,
+                   g_schedule.load(), fws ? workspace : nullptr, fws,
+                   reinterpret_cast<cudaStream_t>(stream), Hold(), true);
+    if (st != LA2_OK) return st;
+    int launches = t_last_launches;
+    // the denominator, dividing y in place
+    char* base = static_cast<char*>(workspace);
+    la2::NzParams p = nz_params(B, H, T, d, e, layout == LA2_LAYOUT_BTHD, decay,
+                                base ? reinterpret_cast<float*>(base + fws) : nullptr);
+    p.a = k;
+    p.q = q;
+    p.y = y;
+    p.den = den;
+    p.mode = la2::kNzDen;
+    p.dir = +1;
+    if (p.nchunk > 1 && !p.chunk) return LA2_ERR_WORKSPACE;
+    const long long seqs = static_cast<long long>(B) * H;
+    const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == LA2_DTYPE_BF16) nz_launch<__nv_bfloat16>(p, seqs, cs, &launches);
+    else nz_launch<float>(p, seqs, cs, &launches);
+    if (cudaGetLastError() != cudaSuccess) return LA2_ERR_CUDA;
+    t_last_launches = launches;
+    return LA2_OK;
+}
+
+la2_status la2_bwd_norm(const void* q, const void* k, const void* v, const float* decay,
+                        const float* y, const float* den, const void* dy, void* dq, void* dk,
+                        void* dv, int B, int H, int T, int d, int e, int block, la2_dtype dtype,
+                        la2_layout layout, void* workspace, size_t workspace_bytes,
+                        la2_stream_t stream) {
+    t_last_launches = 0;
+    bool empty = false;
+    la2_status st = norm_checks(q, k, v, decay, B, H, T, d, e, block, dtype, layout, &empty);
+    if (st != LA2_OK || empty) return st;
+    if (!y || !den || !dy || !dq || !dk || !dv) return LA2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dy) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(decay) & 3u) ||
+        (reinterpret_cast<uintptr_t>(y) & 3u) || (reinterpret_cast<uintptr_t>(den) & 3u))
+        return LA2_ERR_INVALID_ARG;
+    const size_t need = la2_norm_workspace_bytes(B, H, T, d, e, block, dtype, 1);
+    if (!workspace || workspace_bytes < need) return LA2_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return LA2_ERR_INVALID_ARG;
+    int dev = 0;
+    int* status = nullptr;
+    if (!device_setup(&dev, &status)) return LA2_ERR_CUDA;
+    const long long seqs = static_cast<long long>(B) * H;
+    const size_t bws = align256(la2_workspace_bytes(B, H, T, d, e, block, dtype, 1));
+    const size_t rows = align256(static_cast<size_t>(seqs) * T * sizeof(float));
+    char* base = static_cast<char*>(workspace);
+    float* dden = reinterpret_cast<float*>(base + bws);
+    float* inv = reinterpret_cast<float*>(base + bws + rows);
+    float* chunk = reinterpret_cast<float*>(base + bws + 2 * rows);
+    const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const bool bthd = layout == LA2_LAYOUT_BTHD;
+    int launches = 0;
+    // dden_t = -(dy_t . y_t) / den_t, inv_t = 1 / den_t
+    {
+        const long long nrows = seqs * T;
+        const unsigned grid = static_cast<unsigned>(cdiv(nrows * 32, 256));
+        if (dtype == LA2_DTYPE_BF16)
+            la2::la2_nz_prep<__nv_bfloat16><<<grid, 256, 0, cs>>>(static_cast<const __nv_bfloat16*>(dy), y,
+                                                                   den, dden, inv, nrows, H, T, e, bthd);
+        else
+            la2::la2_nz_prep<float><<<grid, 256, 0, cs>>>(static_cast<const float*>(dy), y, den, dden, inv,
+                                                          nrows, H, T, e, bthd);
+        ++launches;
+        if (cudaGetLastError() != cudaSuccess) return LA2_ERR_CUDA;
+    }
+    // the numerator's backward with dnum_t = dy_t / den_t: the dq scan with
+    // dout = dy (its rows are divided by den_t afterwards), the dk and dv scans
+    // with the factor 1 / den_t on their summed position
+    RoleDesc roles[3] = {
+        {dy, v, k, dq, e, d, +1},
+        {v, dy, q, dk, e, d, -1},
+        {k, q, dy, dv, d, e, -1},
+    };
+    roles[1].colf = inv;
+    roles[2].colf = inv;
+    st = run_roles(roles, 3, decay, B, H, T, block, dtype, bthd, g_schedule.load(),
+                   bws ? workspace : nullptr, bws, cs, Hold(), true);
+    if (st != LA2_OK) return st;
+    launches += t_last_launches;
+    // dq_t = dq_t / den_t + dden_t z_t, then dk_s += sum_{t>=s} lambda^(t-s) dden_t q_t
+    la2::NzParams p = nz_params(B, H, T, d, e, bthd, decay, chunk);
+    p.w = dden;
+    p.rs = inv;
+    p.a = k;
+    p.out = static_cast<float*>(dq);
+    p.mode = la2::kNzDq;
+    p.dir = +1;
+    if (dtype == LA2_DTYPE_BF16) nz_launch<__nv_bfloat16>(p, seqs, cs, &launches);
+    else nz_launch<float>(p, seqs, cs, &launches);
+    p.a = q;
+    p.out = static_cast<float*>(dk);
+    p.mode = la2::kNzDk;
+    p.dir = -1;
+    if (dtype == LA2_DTYPE_BF16) nz_launch<__nv_bfloat16>(p, seqs, cs, &launches);
+    else nz_launch<float>(p, seqs, cs, &launches);
     if (cudaGetLastError() != cudaSuccess) return LA2_ERR_CUDA;
     t_last_launches = launches;
     return LA2_OK;

@@ -24,6 +24,7 @@ struct F32Role {
     float* fin;         // [BH, DA, DC] state the scan ends with, or null
     int da, dc, dir;
     int init_t;
+    const float* colf;  // [BH, T] factor on the summed position, or null (see scan_ws_sm100.cuh)
     // dir = +1: init is the state before position 0, fin the state after
     // position T-1.  dir = -1: init enters at position T-1 (row t weighs it by
     // lambda^(T-1-t)), and fin is lambda times the state at position 0.
@@ -134,6 +135,8 @@ la2_scan_f32(const __grid_constant__ F32Params p)
                     if (lag >= 0) {
                         for (int u = 0; u < da; ++u) s = fmaf(As[rr * da + u], Bs[cc * da + u], s);
                         s *= pw[lag];
+                        const int loc = kb * kF32Sub + cc;
+                        if (R.colf) s *= loc < len ? R.colf[static_cast<size_t>(bh) * T + t0 + loc] : 0.f;
                     }
                     Ps[z] = s;
                 }
@@ -171,7 +174,8 @@ la2_scan_f32(const __grid_constant__ F32Params p)
             __syncthreads();
             for (int z = tid; z < kF32Sub * da; z += kF32Threads) {
                 const int rr = z / da, u = z % da, loc = kb * kF32Sub + rr;
-                const float ws = loc < len ? (dir > 0 ? pw[tl - 1 - loc] : pw[loc]) : 0.f;
+                float ws = loc < len ? (dir > 0 ? pw[tl - 1 - loc] : pw[loc]) : 0.f;
+                if (R.colf && loc < len) ws *= R.colf[static_cast<size_t>(bh) * T + t0 + loc];
                 Bs[z] = loc < len ? ws * b[static_cast<size_t>(t0 + loc) * rs * da + u] : 0.f;
             }
             for (int z = tid; z < kF32Sub * dc; z += kF32Threads) {

@@ -77,6 +77,9 @@ struct Role {
     float* fin;              // [B*H, DA, DC] fp32 state the scan ends with, or null
     int dir;                 // +1 or -1
     int init_t;              // 1: init is stored transposed
+    const float* colf;       // [B*H, T] fp32 factor f_s on the summed position s, or null (1):
+                             // x_t = sum_s lambda^|t-s| (a_t . b_s) f_s c_s, applied in fp32 to
+                             // the columns of P and to the state-update weights of row s
     // dir = +1: init is the state before position 0 (row t of the output gets
     // lambda^(t+1) a_t^T init) and fin the state after position T-1.
     // dir = -1: init is a state entering at position T-1 (row t gets
@@ -136,9 +139,15 @@ __device__ __forceinline__ long long seg_slot_index(const Params& p, bool balanc
 // tf32: no hi/lo split, and w_s B is written to its own buffer, so it need
 // not wait for S.  Otherwise P and w_s B are bf16 hi + lo pairs (hi of w_s B
 // in place of B).  The state W is a bf16 hi + lo pair in both modes.
-template <int DA, int DC>
+//
+// kNorm is the instantiation the normalised form uses.  It forces the bf16
+// hi + lo mode at DA = DC = 64 as well (about 1e-5 instead of 2e-3 of rms):
+// the normalised form divides by q . z and its backward subtracts nearly equal
+// parts, which would magnify tf32's error.  It alone compiles the per-position
+// factor (Role::colf), so the other instantiations carry none of its code.
+template <int DA, int DC, bool kNorm = false>
 struct RingCfg {
-    static constexpr bool kTf32 = DA == 64 && DC == 64;
+    static constexpr bool kTf32 = DA == 64 && DC == 64 && !kNorm;
     static constexpr bool kBig = DA == 128 && DC == 128;
     static constexpr int NA = kBig ? 1 : 2;                  // A tiles
     static constexpr int NB = 2;                             // B tiles
@@ -196,9 +205,9 @@ struct RingCfg {
     }
 };
 
-template <int DA, int DC>
+template <int DA, int DC, bool kNorm = false>
 struct Smem {
-    using Q = RingCfg<DA, DC>;
+    using Q = RingCfg<DA, DC, kNorm>;
     static constexpr uint32_t kAsz = kTB * DA * 2;            // one A (or B) tile
     static constexpr uint32_t kBsz = kAsz;
     static constexpr uint32_t kCsz = kTB * DC * 2;            // one C tile
@@ -317,13 +326,13 @@ __device__ __forceinline__ uint32_t empty_par(int s, int n) {
 // kMulti: the balanced plan's CTAs, which may run several segments (a
 // separate instantiation, so that the one-segment kernel carries no loop
 // state in its registers).
-template <int DA, int DC, bool kMulti>
+template <int DA, int DC, bool kMulti, bool kNorm = false>
 __global__ void __launch_bounds__(kThreads, 1)
 la2_scan_ws(const __grid_constant__ Params p)
 {
     static_assert((DA == 64 || DA == 128) && (DC == 64 || DC == 128), "DA, DC in {64, 128}");
-    using L = Smem<DA, DC>;
-    using Q = RingCfg<DA, DC>;
+    using L = Smem<DA, DC, kNorm>;
+    using Q = RingCfg<DA, DC, kNorm>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t base = smem_u32(smem_raw);
     if (base & 1023u) {  // 128-byte swizzled tiles need a 1024-byte aligned base
@@ -743,8 +752,23 @@ la2_scan_ws(const __grid_constant__ Params p)
         // output reads that state; only the final state does.
         const int nlast = T - (nb - 1) * kTB;
         const float ws_last = r < nlast ? pw[max(nlast - 1 - r, 0)] : 0.f;
+        // the per-position factor of this thread's row of the tile of step s
+        const float* colf = (kNorm && R.colf) ? R.colf + static_cast<size_t>(bh) * T : nullptr;
+        auto f_of = [&](int s, int row) -> float {
+            const int t = tile_of(s) * kTB + row;
+            return t < T ? __ldg(colf + t) : 0.f;
+        };
         auto ws_of = [&](int s) {
-            return (dir > 0 && unit_end && s == ns - 1) ? ws_last : ws;
+            const float w = (dir > 0 && unit_end && s == ns - 1) ? ws_last : ws;
+            if constexpr (kNorm) return colf ? w * f_of(s, r) : w;
+            return w;
+        };
+        // P's columns times the factors of their positions (32 columns of block pr)
+        auto colscale = [&](int s, int pr, float (&sv)[32]) {
+            if constexpr (!kNorm) return;
+            if (colf == nullptr) return;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) sv[u] *= f_of(s, 32 * pr + u);
         };
         // P = S * lambda^|r-c| on the causal side, 0 elsewhere, 32 columns (one
         // pair of K = 16 groups) at a time.  pr == quad is the diagonal block;
@@ -860,6 +884,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                     float sv[32];
                     tmem_ld32(st + lane_off + pr * 32, sv);
                     weigh(pr, sv);
+                    colscale(s, pr, sv);
                     tmem_st32(st + lane_off + pr * 32, sv);
                 }
             } else {
@@ -901,6 +926,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                     float sv[32];
                     tmem_ld32(st + lane_off + pr * 32, sv);
                     weigh(pr, sv);
+                    colscale(s, pr, sv);
                     uint32_t pk[32];
 #pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2)
@@ -1384,7 +1410,11 @@ la2_state_ws(const __grid_constant__ Params p)
             if (s >= 2 && !wait_bar(bar(SB_D0 + slot), ph ^ 1, abort_flag, p.status, 74)) break;
             // row weight lambda^(T_B (n-1-s)) w_s(r)
             const int e = dir > 0 ? kTB * (ns - s) - 1 - r : kTB * (ns - 1 - s) + r;
-            const float wt = static_cast<float>(exp2(static_cast<double>(e) * l2));
+            float wt = static_cast<float>(exp2(static_cast<double>(e) * l2));
+            if (R.colf) {
+                const int t = tile_of(s) * kTB + r;
+                wt = t < p.T ? wt * __ldg(R.colf + static_cast<size_t>(bh) * p.T + t) : 0.f;
+            }
             const uint32_t bt = sB + slot * L::kBsz, bl = sBlo + slot * L::kBsz;
 #pragma unroll
             for (int k = 0; k < DA / 16; ++k) {

@@ -29,7 +29,8 @@ LA2_DTYPE_BF16 = 1
 EXPORTS = ("la2_workspace_bytes", "la2_fwd", "la2_fwd_state", "la2_fwd_ex", "la2_bwd", "la2_bwd_ex",
            "la2_decode", "la2_status_str", "la2_device_status", "la2_last_launch_count",
            "la2_fwd_noalloc", "la2_set_schedule", "la2_plan_info", "la2_selftest_timeout",
-           "la2_bwd_state", "la2_dlambda", "la2_dlambda_workspace_bytes")
+           "la2_bwd_state", "la2_dlambda", "la2_dlambda_workspace_bytes",
+           "la2_norm_workspace_bytes", "la2_fwd_norm", "la2_bwd_norm")
 
 LA2_LAYOUT_BHTD = 0
 LA2_LAYOUT_BTHD = 1
@@ -95,6 +96,13 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la2_dlambda_workspace_bytes.restype = sz
     lib.la2_dlambda.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
     lib.la2_dlambda.restype = i
+    lib.la2_norm_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+    lib.la2_norm_workspace_bytes.restype = sz
+    lib.la2_fwd_norm.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, sz, vp]
+    lib.la2_fwd_norm.restype = i
+    lib.la2_bwd_norm.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i,
+                                 vp, sz, vp]
+    lib.la2_bwd_norm.restype = i
     _lib = lib
     return lib
 
@@ -417,6 +425,56 @@ def la2_dlambda(q, k, v, decay, dout, init_state=None, d_final_state=None, layou
     if st != LA2_OK:
         raise LA2Error(st, "la2_dlambda")
     return d_decay
+
+
+def la2_norm_workspace_bytes(B, H, T, d, e, block, dtype, is_bwd) -> int:
+    return int(load().la2_norm_workspace_bytes(B, H, T, d, e, block, dtype, int(is_bwd)))
+
+
+def la2_fwd_norm(q, k, v, decay, layout: str = "bhtd", y=None, den=None, block: int = 128,
+                 stream=None, workspace=None):
+    """(y, den): the normalised form y_t = num_t / (q_t . z_t), z_t = decay z_{t-1} + k_t."""
+    B, H, T, d, e = _dims(q, v, layout)
+    dt = _dtype_code(q)
+    for t, n, D in ((q, "q", d), (k, "k", d), (v, "v", e)):
+        _check(t, n, _shape(layout, B, H, T, D), q.dtype)
+    _check(decay, "decay", (H,), torch.float32)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    y = torch.empty(_shape(layout, B, H, T, e), **f32) if y is None else y
+    den = torch.empty((B, H, T), **f32) if den is None else den
+    _check(y, "y", _shape(layout, B, H, T, e), torch.float32)
+    _check(den, "den", (B, H, T), torch.float32)
+    wp, wn = _workspace(la2_norm_workspace_bytes(B, H, T, d, e, block, dt, 0), q.device, workspace)
+    st = int(load().la2_fwd_norm(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(),
+                                 y.data_ptr(), den.data_ptr(), B, H, T, d, e, block, dt,
+                                 _LAYOUTS[layout], wp, wn, _stream_ptr(stream)))
+    if st != LA2_OK:
+        raise LA2Error(st, "la2_fwd_norm")
+    return y, den
+
+
+def la2_bwd_norm(q, k, v, decay, y, den, dy, layout: str = "bhtd", dq=None, dk=None, dv=None,
+                 block: int = 128, stream=None, workspace=None):
+    """(dq, dk, dv) of sum(dy * y) for (y, den) = la2_fwd_norm(q, k, v, decay)."""
+    B, H, T, d, e = _dims(q, v, layout)
+    dt = _dtype_code(q)
+    for t, n, D in ((q, "q", d), (k, "k", d), (v, "v", e), (dy, "dy", e)):
+        _check(t, n, _shape(layout, B, H, T, D), q.dtype)
+    _check(decay, "decay", (H,), torch.float32)
+    _check(y, "y", _shape(layout, B, H, T, e), torch.float32)
+    _check(den, "den", (B, H, T), torch.float32)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty(_shape(layout, B, H, T, d), **f32) if dq is None else dq
+    dk = torch.empty(_shape(layout, B, H, T, d), **f32) if dk is None else dk
+    dv = torch.empty(_shape(layout, B, H, T, e), **f32) if dv is None else dv
+    wp, wn = _workspace(la2_norm_workspace_bytes(B, H, T, d, e, block, dt, 1), q.device, workspace)
+    st = int(load().la2_bwd_norm(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(),
+                                 y.data_ptr(), den.data_ptr(), dy.data_ptr(), dq.data_ptr(),
+                                 dk.data_ptr(), dv.data_ptr(), B, H, T, d, e, block, dt,
+                                 _LAYOUTS[layout], wp, wn, _stream_ptr(stream)))
+    if st != LA2_OK:
+        raise LA2Error(st, "la2_bwd_norm")
+    return dq, dk, dv
 
 
 def la2_decode_raw(q, k, v, decay, state, out, B, H, d, e, dtype, stream=0) -> int:

@@ -308,6 +308,54 @@ la2_status la2_dlambda(const void *q, const void *k, const void *v, const float 
                        la2_layout layout, void *workspace, size_t workspace_bytes,
                        la2_stream_t stream);
 
+/*
+ * The normalised form.  The "Lightning Attention" explainer (section 1) writes
+ * causal linear attention with a denominator, and (section 2) runs its
+ * running sum z as a recurrence parallel to the state.  With the identity
+ * feature map (the explainer's default; any other feature map phi is applied to
+ * q and k by the caller before the call, since the tiling does not depend on
+ * it) and the decay on both sums:
+ *
+ *   z_t = lambda z_{t-1} + k_t,   den_t = q_t . z_t,
+ *   y_t = (sum_{s<=t} lambda^(t-s) (q_t . k_s) v_s) / den_t
+ *
+ * la2_fwd_norm writes y (fp32, the layout of v) and, unless den is NULL, den
+ * (fp32 [B, H, T]).  la2_bwd_norm takes y and den from the forward and dy (the
+ * gradient of y, the input dtype, the layout of v) and writes dq, dk, dv
+ * (fp32):
+ *
+ *   dnum_t = dy_t / den_t,   dden_t = -(dy_t . y_t) / den_t,
+ *   dq_t = sum_{s<=t} lambda^(t-s) (dnum_t . v_s) k_s + dden_t z_t,
+ *   dk_s = sum_{t>=s} lambda^(t-s) (v_s . dnum_t) q_t + sum_{t>=s} lambda^(t-s) dden_t q_t,
+ *   dv_s = sum_{t>=s} lambda^(t-s) (k_s . q_t) dnum_t.
+ *
+ * dnum enters the tensor-core scans without being rounded to the input type:
+ * the dk and dv scans weigh their summed position t by 1/den_t in fp32 (in
+ * their masks and state updates), and the dq scan's rows are divided by den_t
+ * afterwards.  This matters because dq and dk are each the difference of two
+ * nearly equal parts when y depends weakly on q and k.  The sums over
+ * positions of d-vectors (z, and the dk term in dden) are SIMT scans.
+ *
+ * The caller keeps den_t away from zero (e.g. with a positive feature map);
+ * nothing is checked.  Support as la2_fwd (d <= 128 for both dtypes' paths),
+ * both layouts.  workspace: at least la2_norm_workspace_bytes(..., is_bwd)
+ * bytes, 256-byte aligned; the backward's grows with T (two fp32 values per
+ * position: dden and 1/den).  Asynchronous on `stream`.
+ */
+size_t la2_norm_workspace_bytes(int B, int H, int T, int d, int e, int block, la2_dtype dtype,
+                                int is_bwd);
+
+la2_status la2_fwd_norm(const void *q, const void *k, const void *v, const float *decay,
+                        float *y, float *den, int B, int H, int T, int d, int e, int block,
+                        la2_dtype dtype, la2_layout layout, void *workspace,
+                        size_t workspace_bytes, la2_stream_t stream);
+
+la2_status la2_bwd_norm(const void *q, const void *k, const void *v, const float *decay,
+                        const float *y, const float *den, const void *dy, void *dq, void *dk,
+                        void *dv, int B, int H, int T, int d, int e, int block, la2_dtype dtype,
+                        la2_layout layout, void *workspace, size_t workspace_bytes,
+                        la2_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 const char *la2_status_str(la2_status status);
 

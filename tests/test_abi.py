@@ -222,3 +222,18 @@ def test_dlambda_workspace_flat_in_T_and_arguments(lib):
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0, FAKE, 1, 2, 100, 200, 64, la2.LA2_DTYPE_BF16, 0,
              FAKE, 1 << 30, 0) == la2.LA2_ERR_UNSUPPORTED
     del ok
+
+
+def test_norm_workspace_and_arguments(lib):
+    ws = [la2.la2_norm_workspace_bytes(1, 8, T, 128, 128, 128, la2.LA2_DTYPE_BF16, 0)
+          for T in (4096, 65536)]
+    assert ws[0] == ws[1]                       # the forward's is flat in T
+    assert la2.la2_norm_workspace_bytes(1, 8, 64, 129, 64, 128, la2.LA2_DTYPE_F32, 0) == 2 ** 64 - 1
+    f = la2.load().la2_fwd_norm
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 256, 128, 128, 128, la2.LA2_DTYPE_BF16, 5,
+             FAKE, 1 << 30, 0) == la2.LA2_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, FAKE, 0, FAKE, 1, 2, 256, 128, 128, 128, la2.LA2_DTYPE_BF16, 0,
+             FAKE, 1 << 30, 0) == la2.LA2_ERR_INVALID_ARG
+    g = la2.load().la2_bwd_norm
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 256, 128, 128, 128,
+             la2.LA2_DTYPE_BF16, 0, 0, 0, 0) == la2.LA2_ERR_WORKSPACE
