@@ -55,10 +55,17 @@ struct DlParams {
 __device__ __forceinline__ float dl_load(const float* p) { return *p; }
 __device__ __forceinline__ float dl_load(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
-__device__ __forceinline__ size_t dl_row(const DlParams& p, int bh, int t) {
-    const int b = bh / p.H, h = bh - b * p.H;
-    return p.bthd ? (static_cast<size_t>(b) * p.T + t) * p.H + h : static_cast<size_t>(bh) * p.T + t;
-}
+// Rows of sequence bh: row(t) = base + t * stride ([B, H, T, D]: bh T + t;
+// [B, T, H, D]: (b T + t) H + h), worked out once per CTA.
+struct DlRows {
+    size_t base, stride;
+    __device__ __forceinline__ DlRows(const DlParams& p, int bh) {
+        const int b = bh / p.H, h = bh - b * p.H;
+        base = p.bthd ? static_cast<size_t>(b) * p.T * p.H + h : static_cast<size_t>(bh) * p.T;
+        stride = p.bthd ? static_cast<size_t>(p.H) : 1;
+    }
+    __device__ __forceinline__ size_t operator()(int t) const { return base + static_cast<size_t>(t) * stride; }
+};
 
 __device__ __forceinline__ void dl_cvt(uint4 w, const float*, float (&x)[4]) {
     x[0] = __uint_as_float(w.x); x[1] = __uint_as_float(w.y);
@@ -80,7 +87,7 @@ __device__ __forceinline__ void dl_cvt(uint4 w, const __nv_bfloat16*, float (&x)
 // store; otherwise element by element, loads again batched ahead of stores.
 template <typename Tin>
 __device__ __forceinline__ void dl_stage2(float* dA, const Tin* sA, int DA, float* dB, const Tin* sB, int DB,
-                                          const DlParams& p, int bh, int t0, int n) {
+                                          const DlParams& p, const DlRows& dl_row, int t0, int n) {
     if (p.vec) {
         constexpr int kE = 16 / sizeof(Tin);                   // elements per vector
         constexpr int kCh = 128 / kE;                          // vectors per smem row
@@ -89,7 +96,7 @@ __device__ __forceinline__ void dl_stage2(float* dA, const Tin* sA, int DA, floa
 #pragma unroll
         for (int m = 0; m < kPer; ++m) {
             const int z = threadIdx.x + m * kDlThreads, r = z / kCh, c = (z % kCh) * kE;
-            const size_t row = dl_row(p, bh, t0 + r);
+            const size_t row = dl_row(t0 + r);
             va[m] = (r < n && c < DA) ? __ldg(reinterpret_cast<const uint4*>(sA + row * DA + c)) : make_uint4(0, 0, 0, 0);
             vb[m] = (r < n && c < DB) ? __ldg(reinterpret_cast<const uint4*>(sB + row * DB + c)) : make_uint4(0, 0, 0, 0);
         }
@@ -117,7 +124,7 @@ __device__ __forceinline__ void dl_stage2(float* dA, const Tin* sA, int DA, floa
 #pragma unroll
         for (int m = 0; m < kPer; ++m) {
             const int z = threadIdx.x + m * kDlThreads, r = z >> 7, u = z & 127;
-            x[m] = (r < n && u < D) ? dl_load(src + dl_row(p, bh, t0 + r) * D + u) : 0.f;
+            x[m] = (r < n && u < D) ? dl_load(src + dl_row(t0 + r) * D + u) : 0.f;
         }
 #pragma unroll
         for (int m = 0; m < kPer; ++m) {
@@ -130,12 +137,12 @@ __device__ __forceinline__ void dl_stage2(float* dA, const Tin* sA, int DA, floa
 // L2 prefetch of rows [t0, t0 + n) of sequence bh of a tensor (one 128-byte
 // line per thread and call at most), so that the next staging reads L2.
 template <typename Tin>
-__device__ __forceinline__ void dl_prefetch(const Tin* src, int D, const DlParams& p, int bh, int t0, int n) {
+__device__ __forceinline__ void dl_prefetch(const Tin* src, int D, const DlRows& dl_row, int t0, int n) {
     const int lines = (D * static_cast<int>(sizeof(Tin)) + 127) / 128;
     const int z = threadIdx.x;
     if (z < n * lines) {
         const int r = z / lines, l = z % lines;
-        const char* a = reinterpret_cast<const char*>(src + dl_row(p, bh, t0 + r) * D) + 128 * l;
+        const char* a = reinterpret_cast<const char*>(src + dl_row(t0 + r) * D) + 128 * l;
         asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
     }
 }
@@ -197,6 +204,7 @@ __global__ void __launch_bounds__(kDlThreads, 1) la2_dlam_prepass(const __grid_c
     float* pw = Vs + kDlRows * kDlStride;
     const int bh = blockIdx.x / (p.nseg - 1), j = blockIdx.x % (p.nseg - 1);
     const int tid = threadIdx.x, ti = tid >> 4, tj = tid & 15;
+    const DlRows rows(p, bh);
     const double l2 = log2(static_cast<double>(p.decay[bh % p.H]));
     dl_table(pw, l2);
     const int a = j * p.seg_rows, bnd = min(p.T, a + p.seg_rows);
@@ -206,12 +214,12 @@ __global__ void __launch_bounds__(kDlThreads, 1) la2_dlam_prepass(const __grid_c
     for (int t0 = a; t0 < bnd; t0 += kDlRows) {
         const int n = min(kDlRows, bnd - t0);
         __syncthreads();
-        dl_stage2(Ks, static_cast<const Tin*>(p.k), p.d, Vs, static_cast<const Tin*>(p.v), p.e, p, bh, t0, n);
+        dl_stage2(Ks, static_cast<const Tin*>(p.k), p.d, Vs, static_cast<const Tin*>(p.v), p.e, p, rows, t0, n);
         __syncthreads();
         if (t0 + kDlRows < bnd) {
             const int nn = min(kDlRows, bnd - t0 - kDlRows);
-            dl_prefetch(static_cast<const Tin*>(p.k), p.d, p, bh, t0 + kDlRows, nn);
-            dl_prefetch(static_cast<const Tin*>(p.v), p.e, p, bh, t0 + kDlRows, nn);
+            dl_prefetch(static_cast<const Tin*>(p.k), p.d, rows, t0 + kDlRows, nn);
+            dl_prefetch(static_cast<const Tin*>(p.v), p.e, rows, t0 + kDlRows, nn);
         }
         dl_carry(W, U, Ks, Vs, n, pw, ti, tj);
     }
@@ -240,6 +248,7 @@ __global__ void __launch_bounds__(kDlThreads, 1) la2_dlam_scan(const __grid_cons
     float* pw = reinterpret_cast<float*>(red + kDlThreads / 32);         // [kDlRows + 1]
     const int bh = blockIdx.x / p.nseg, j = blockIdx.x % p.nseg;
     const int tid = threadIdx.x, ti = tid >> 4, tj = tid & 15;
+    const DlRows rows(p, bh);
     const double l2 = log2(static_cast<double>(p.decay[bh % p.H]));
     dl_table(pw, l2);
     const size_t de = static_cast<size_t>(p.d) * p.e;
@@ -277,15 +286,15 @@ __global__ void __launch_bounds__(kDlThreads, 1) la2_dlam_scan(const __grid_cons
     for (int t0 = a; t0 < bnd; t0 += kDlRows) {
         const int n = min(kDlRows, bnd - t0);
         __syncthreads();
-        dl_stage2(Qs, static_cast<const Tin*>(p.q), p.d, Ks, static_cast<const Tin*>(p.k), p.d, p, bh, t0, n);
-        dl_stage2(Vs, static_cast<const Tin*>(p.v), p.e, Gs, static_cast<const Tin*>(p.g), p.e, p, bh, t0, n);
+        dl_stage2(Qs, static_cast<const Tin*>(p.q), p.d, Ks, static_cast<const Tin*>(p.k), p.d, p, rows, t0, n);
+        dl_stage2(Vs, static_cast<const Tin*>(p.v), p.e, Gs, static_cast<const Tin*>(p.g), p.e, p, rows, t0, n);
         __syncthreads();
         if (t0 + kDlRows < bnd) {
             const int nn = min(kDlRows, bnd - t0 - kDlRows);
-            dl_prefetch(static_cast<const Tin*>(p.q), p.d, p, bh, t0 + kDlRows, nn);
-            dl_prefetch(static_cast<const Tin*>(p.k), p.d, p, bh, t0 + kDlRows, nn);
-            dl_prefetch(static_cast<const Tin*>(p.v), p.e, p, bh, t0 + kDlRows, nn);
-            dl_prefetch(static_cast<const Tin*>(p.g), p.e, p, bh, t0 + kDlRows, nn);
+            dl_prefetch(static_cast<const Tin*>(p.q), p.d, rows, t0 + kDlRows, nn);
+            dl_prefetch(static_cast<const Tin*>(p.k), p.d, rows, t0 + kDlRows, nn);
+            dl_prefetch(static_cast<const Tin*>(p.v), p.e, rows, t0 + kDlRows, nn);
+            dl_prefetch(static_cast<const Tin*>(p.g), p.e, rows, t0 + kDlRows, nn);
         }
         // inter: (r+1) lambda^r q_r^T W do_r + lambda^(r+1) q_r^T U do_r, this
         // thread's block of W and U

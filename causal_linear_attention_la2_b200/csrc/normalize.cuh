@@ -29,7 +29,7 @@
 namespace la2 {
 
 constexpr int kNzThreads = 128;  // one per feature (d <= 128)
-constexpr int kNzRows = 32;      // rows staged per step
+constexpr int kNzRows = 16;      // rows whose loads are issued together (registers bound occupancy)
 
 enum NzMode { kNzDen = 0, kNzDq = 1, kNzDk = 2 };
 
@@ -51,10 +51,17 @@ struct NzParams {
 __device__ __forceinline__ float nz_load(const float* p) { return *p; }
 __device__ __forceinline__ float nz_load(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
-__device__ __forceinline__ size_t nz_row(const NzParams& p, int bh, int t) {
-    const int b = bh / p.H, h = bh - b * p.H;
-    return p.bthd ? (static_cast<size_t>(b) * p.T + t) * p.H + h : static_cast<size_t>(bh) * p.T + t;
-}
+// Rows of sequence bh: row(t) = base + t * stride ([B, H, T, D]: bh T + t;
+// [B, T, H, D]: (b T + t) H + h), worked out once per CTA.
+struct NzRows {
+    size_t base, stride;
+    __device__ __forceinline__ NzRows(const NzParams& p, int bh) {
+        const int b = bh / p.H, h = bh - b * p.H;
+        base = p.bthd ? static_cast<size_t>(b) * p.T * p.H + h : static_cast<size_t>(bh) * p.T;
+        stride = p.bthd ? static_cast<size_t>(p.H) : 1;
+    }
+    __device__ __forceinline__ size_t operator()(int t) const { return base + static_cast<size_t>(t) * stride; }
+};
 
 // Rows of chunk j (scan order): [lo, hi) in time.
 __device__ __forceinline__ void nz_span(const NzParams& p, int j, int& lo, int& hi) {
@@ -77,16 +84,21 @@ __global__ void __launch_bounds__(kNzThreads) la2_nz_prepass(const __grid_consta
     int lo, hi;
     nz_span(p, j, lo, hi);
     const Tin* a = static_cast<const Tin*>(p.a);
+    const NzRows nz_row(p, bh);
     float x = 0.f;
     const int n = hi - lo;
+    const int ic = min(i, p.d - 1);
     for (int s0 = 0; s0 < n; s0 += kNzRows) {
         const int m = min(kNzRows, n - s0);
+        // every load of the batch first (addresses clamped into range, so that
+        // none waits behind a branch), then the recurrence
         float av[kNzRows], wv[kNzRows];
 #pragma unroll
         for (int r = 0; r < kNzRows; ++r) {
-            const int t = p.dir > 0 ? lo + s0 + r : hi - 1 - s0 - r;
-            av[r] = (r < m && i < p.d) ? nz_load(a + nz_row(p, bh, t) * p.d + i) : 0.f;
-            wv[r] = r < m ? nz_weight(p, bh, t) : 0.f;
+            const int rr = min(r, m - 1);
+            const int t = p.dir > 0 ? lo + s0 + rr : hi - 1 - s0 - rr;
+            av[r] = nz_load(a + nz_row(t) * p.d + ic);
+            wv[r] = nz_weight(p, bh, t);
         }
 #pragma unroll
         for (int r = 0; r < kNzRows; ++r)
@@ -117,18 +129,24 @@ __global__ void __launch_bounds__(kNzThreads) la2_nz_scan(const __grid_constant_
     }
     const Tin* a = static_cast<const Tin*>(p.a);
     const Tin* q = static_cast<const Tin*>(p.q);
+    const NzRows nz_row(p, bh);
     const int n = hi - lo;
+    const int ic = min(i, p.d - 1);
+    const float fi = i < p.d ? 1.f : 0.f;  // threads past d carry zeros
     for (int s0 = 0; s0 < n; s0 += kNzRows) {
         const int m = min(kNzRows, n - s0);
+        // every load of the batch first, addresses clamped into range (rows
+        // past m repeat the last row and are not used), then the recurrence
         float av[kNzRows], wv[kNzRows], qv[kNzRows];
 #pragma unroll
         for (int r = 0; r < kNzRows; ++r) {
-            const int t = p.dir > 0 ? lo + s0 + r : hi - 1 - s0 - r;
-            const bool ok = r < m && i < p.d;
-            const size_t row = nz_row(p, bh, ok ? t : lo);
-            av[r] = ok ? nz_load(a + row * p.d + i) : 0.f;
+            const int rr = min(r, m - 1);
+            const int t = p.dir > 0 ? lo + s0 + rr : hi - 1 - s0 - rr;
+            const size_t row = nz_row(t);
+            av[r] = fi * nz_load(a + row * p.d + ic);
             wv[r] = r < m ? nz_weight(p, bh, t) : 0.f;
-            qv[r] = (p.mode == kNzDen && ok) ? nz_load(q + row * p.d + i) : 0.f;
+            if (p.mode == kNzDen) qv[r] = nz_load(q + row * p.d + ic);
+            else qv[r] = p.out[row * p.d + ic];       // dq / dk mode: the row to add to
         }
         if (p.mode == kNzDen) {
             // den_t = q_t . x_t: per row a warp sum, then the four warps' sums
@@ -150,27 +168,44 @@ __global__ void __launch_bounds__(kNzThreads) la2_nz_scan(const __grid_constant_
             }
             __syncthreads();
             if (p.y) {
-                for (int z = i; z < m * p.e; z += kNzThreads) {
-                    const int r = z / p.e, c = z - r * p.e;
-                    float* yp = p.y + nz_row(p, bh, lo + s0 + r) * p.e + c;
-                    *yp = *yp / dens[r];
+                // y rows of the batch: all loads, then the divisions and stores
+                constexpr int kPer = kNzRows * 128 / kNzThreads;  // e <= 128
+                float yv[kPer];
+#pragma unroll
+                for (int u = 0; u < kPer; ++u) {
+                    const int z = i + u * kNzThreads, r = z >> 7, c = z & 127;
+                    yv[u] = (r < m && c < p.e) ? p.y[nz_row(lo + s0 + r) * p.e + c] : 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < kPer; ++u) {
+                    const int z = i + u * kNzThreads, r = z >> 7, c = z & 127;
+                    if (r < m && c < p.e) p.y[nz_row(lo + s0 + r) * p.e + c] = yv[u] / dens[r];
                 }
             }
             __syncthreads();
         } else {
             // dq: out_t = rs_t out_t + dden_t x_t (forward scan of k); dk:
-            // out_t += x_t (reverse scan of dden_t q_t)
+            // out_t += x_t (reverse scan of dden_t q_t); the rows of out were
+            // read with the batch's loads (qv), so no load waits behind a store
+            float fv[kNzRows], sv[kNzRows];
+#pragma unroll
+            for (int r = 0; r < kNzRows; ++r) {
+                const int rr = min(r, m - 1);
+                const size_t st = static_cast<size_t>(bh) * p.T + (p.dir > 0 ? lo + s0 + rr : hi - 1 - s0 - rr);
+                fv[r] = p.mode == kNzDq ? p.w[st] : 1.f;
+                sv[r] = p.mode == kNzDq ? p.rs[st] : 1.f;
+            }
 #pragma unroll
             for (int r = 0; r < kNzRows; ++r) {
                 x = fmaf(lam, x, wv[r] * av[r]);
-                if (r < m && i < p.d) {
-                    const int t = p.dir > 0 ? lo + s0 + r : hi - 1 - s0 - r;
-                    float* op = p.out + nz_row(p, bh, t) * p.d + i;
-                    if (p.mode == kNzDq) {
-                        const size_t st = static_cast<size_t>(bh) * p.T + t;
-                        *op = fmaf(p.w[st], x, *op * p.rs[st]);
-                    } else {
-                        *op += x;
+                qv[r] = fmaf(fv[r], x, qv[r] * sv[r]);
+            }
+            if (i < p.d) {
+#pragma unroll
+                for (int r = 0; r < kNzRows; ++r) {
+                    if (r < m) {
+                        const int t = p.dir > 0 ? lo + s0 + r : hi - 1 - s0 - r;
+                        p.out[nz_row(t) * p.d + i] = qv[r];
                     }
                 }
             }
