@@ -426,11 +426,13 @@ def step_line(w, fwd_ms, bwd_ms, tc, hbm, world=1):
 
 def sweep_lines(la2, w, dev_in, dev_out, lam_sweep, dev, stream, flush, args, tc, hbm):
     """The same fwd+bwd step at every sweep length (and at the TNL-15B layer),
-    on views of the resident inputs: every sweep point has B T = 131,072, and
+    with block 128 and 256, on views of the resident inputs: every sweep point has B T = 131,072, and
     its inputs drawn by the recipe are the same flat buffers reshaped (T =
     92,160, B = 1, and the 15B layer take a prefix of them)."""
     lines = []
     cases = [I.sweep_workload(T, w.block) for T in I.SWEEP_T] + [I.WORKLOADS["tnl15b"]]
+    # the pages' other block size for the sweep (T_B = 256: the phase-serial kernel)
+    cases += [I.sweep_workload(T, 256) for T in I.SWEEP_T if w.block != 256]
     for ws in cases:
         if ws.d != w.d or ws.e != w.e:
             continue

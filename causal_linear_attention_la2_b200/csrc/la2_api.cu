@@ -16,6 +16,7 @@
 #include "dlambda.cuh"
 #include "la2.h"
 #include "normalize.cuh"
+#include "scan_blk_sm100.cuh"
 #include "scan_f32.cuh"
 #include "scan_ws_sm100.cuh"
 
@@ -58,6 +59,12 @@ bool set_ws_attrs() {
            cudaFuncSetAttribute(la2::ws::la2_state_ws<DA, DC>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 la2::ws::StateSmem<DA, DC>::kBytes) == cudaSuccess;
+}
+
+template <int DA, int TB>
+bool set_blk_attrs() {
+    return cudaFuncSetAttribute(la2::blk::la2_scan_blk<DA, TB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                la2::blk::Smem<DA, TB>::kBytes) == cudaSuccess;
 }
 
 // How the bf16 kernel spreads its (sequence, role) units over CTAs.  Each CTA
@@ -221,6 +228,8 @@ bool device_setup(int* dev_out, int** status_out) {
         ok = ok && set_ws_attrs<64, 64>() && set_ws_attrs<64, 128>() && set_ws_attrs<128, 64>() &&
              set_ws_attrs<128, 128>() && set_ws_attrs<64, 64, true>() && set_ws_attrs<64, 128, true>() &&
              set_ws_attrs<128, 64, true>() && set_ws_attrs<128, 128, true>();
+        ok = ok && set_blk_attrs<64, 64>() && set_blk_attrs<64, 256>() && set_blk_attrs<128, 64>() &&
+             set_blk_attrs<128, 256>();
         ok = ok &&
              cudaFuncSetAttribute(la2::la2_dlam_scan<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(la2::dl_scan_smem_bytes())) == cudaSuccess &&
@@ -296,7 +305,6 @@ la2_status common_checks(int B, int H, int T, int d, int e, int block, la2_dtype
     if (static_cast<long long>(B) * H > (1LL << 24)) return LA2_ERR_UNSUPPORTED;
     if (dtype == LA2_DTYPE_BF16) {
         if ((d != 64 && d != 128) || (e != 64 && e != 128)) return LA2_ERR_UNSUPPORTED;
-        if (block != la2::ws::kTB) return LA2_ERR_UNSUPPORTED;
     } else {
         if (d > 128 || e > 128) return LA2_ERR_UNSUPPORTED;
     }
@@ -370,6 +378,45 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
     return LA2_OK;
 }
 
+// T_B = 64 or 256 on bf16 inputs (scan_blk_sm100.cuh): one CTA per
+// (sequence, role, 64 value columns), no segments, no workspace, no states.
+la2_status launch_bf16_blk(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
+                           int block, bool bthd, int* status, cudaStream_t stream) {
+    la2::blk::Params p;
+    std::memset(&p, 0, sizeof(p));
+    const int da = roles[0].da, dc = roles[0].dc;
+    for (int r = 0; r < n; ++r) {
+        if (roles[r].init || roles[r].fin || roles[r].colf) return LA2_ERR_UNSUPPORTED;
+        if (!make_map(&p.role[r].ta, roles[r].a, B, H, T, da, bthd) ||
+            !make_map(&p.role[r].tb, roles[r].b, B, H, T, da, bthd) ||
+            !make_map(&p.role[r].tc, roles[r].c, B, H, T, dc, bthd))
+            return LA2_ERR_CUDA;
+        p.role[r].x = static_cast<float*>(roles[r].x);
+        p.role[r].dir = roles[r].dir;
+    }
+    p.decay = decay;
+    p.status = status;
+    p.H = H;
+    p.T = T;
+    p.nroles = n;
+    p.bthd = bthd ? 1 : 0;
+    p.dc = dc;
+    p.nslice = dc / la2::blk::kDC;
+    const long long ctas = static_cast<long long>(B) * H * n * p.nslice;
+    if (ctas > 0x7fffffffLL) return LA2_ERR_UNSUPPORTED;
+    const unsigned grid = static_cast<unsigned>(ctas);
+    auto go = [&](auto kernel, size_t smem) {
+        kernel<<<grid, la2::blk::kThreads, smem, stream>>>(p);
+    };
+    if (da == 128 && block == 256) go(la2::blk::la2_scan_blk<128, 256>, la2::blk::Smem<128, 256>::kBytes);
+    else if (da == 128) go(la2::blk::la2_scan_blk<128, 64>, la2::blk::Smem<128, 64>::kBytes);
+    else if (block == 256) go(la2::blk::la2_scan_blk<64, 256>, la2::blk::Smem<64, 256>::kBytes);
+    else go(la2::blk::la2_scan_blk<64, 64>, la2::blk::Smem<64, 64>::kBytes);
+    if (cudaGetLastError() != cudaSuccess) return LA2_ERR_CUDA;
+    ++t_last_launches;
+    return LA2_OK;
+}
+
 la2_status launch_f32(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
                       int block, bool bthd, cudaStream_t stream) {
     la2::F32Params p;
@@ -424,7 +471,9 @@ la2_status for_role_groups(const RoleDesc* roles, int n, F&& f) {
     return LA2_OK;
 }
 
-size_t bf16_workspace_bytes(const RoleDesc* roles, int n, int B, int H, int T, int sched) {
+size_t bf16_workspace_bytes(const RoleDesc* roles, int n, int B, int H, int T, int sched,
+                            int block = la2::ws::kTB) {
+    if (block != la2::ws::kTB) return 0;  // the T_B = 64 / 256 kernel needs none
     size_t total = 0;
     for_role_groups(roles, n, [&](const RoleDesc* g, int m) {
         total += seg_workspace_bytes(static_cast<long long>(B) * H * m, T, g[0].da, g[0].dc, sched);
@@ -441,11 +490,17 @@ la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, in
     int dev = 0;
     int* status = nullptr;
     if (dtype == LA2_DTYPE_BF16) {
-        const size_t need = bf16_workspace_bytes(roles, n, B, H, T, sched);
+        const size_t need = bf16_workspace_bytes(roles, n, B, H, T, sched, block);
         if (need > 0 && (workspace == nullptr || ws_bytes < need)) return LA2_ERR_WORKSPACE;
     }
     if (!device_setup(&dev, &status)) return LA2_ERR_CUDA;
     if (dtype == LA2_DTYPE_F32) return launch_f32(roles, n, decay, B, H, T, block, bthd, stream);
+    if (block != la2::ws::kTB) {
+        if (norm || hold.flag) return LA2_ERR_UNSUPPORTED;
+        return for_role_groups(roles, n, [&](const RoleDesc* g, int m) {
+            return launch_bf16_blk(g, m, decay, B, H, T, block, bthd, status, stream);
+        });
+    }
     size_t off = 0;
     return for_role_groups(roles, n, [&](const RoleDesc* g, int m) {
         float* seg = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) + off) : nullptr;
@@ -508,7 +563,8 @@ size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block, la2_dty
                              {nullptr, nullptr, nullptr, nullptr, e, d, -1},
                              {nullptr, nullptr, nullptr, nullptr, d, e, -1}};
     const int sched = g_schedule.load();
-    return is_bwd ? bf16_workspace_bytes(bwd, 3, B, H, T, sched) : bf16_workspace_bytes(fwd, 1, B, H, T, sched);
+    return is_bwd ? bf16_workspace_bytes(bwd, 3, B, H, T, sched, block)
+                  : bf16_workspace_bytes(fwd, 1, B, H, T, sched, block);
 }
 
 la2_schedule la2_set_schedule(la2_schedule schedule) {
@@ -532,7 +588,13 @@ int la2_plan_info(int B, int H, int T, int d, int e, int block, la2_dtype dtype,
     for_role_groups(is_bwd ? bwd : fwd, is_bwd ? 3 : 1, [&](const RoleDesc* g, int m) {
         if (out && n < max_out) {
             const long long units = static_cast<long long>(B) * H * m;
-            const SegPlan sp = plan_segments(units, T, sched);
+            SegPlan sp = plan_segments(units, T, sched);
+            if (block != la2::ws::kTB) {
+                // T_B = 64 / 256: one CTA per (unit, 64 value columns), one segment
+                sp = SegPlan();
+                sp.seg_tiles = (T + 127) / 128;
+                sp.nctas = units * (g[0].dc / la2::blk::kDC);
+            }
             la2_plan& o = out[n];
             o.d = g[0].da;
             o.e = g[0].dc;

@@ -26,9 +26,11 @@
  *     la2_dtype).  Every tensor pointer must be 16-byte aligned.
  *   - decay is a device array of H floats (fp32) holding lambda_h in (0, 1];
  *     values outside that range are the caller's error and are not checked.
- *   - block is the tile length T_B (64, 128 or 256).  It changes the order of
- *     floating-point operations only, never the mathematical result.  T need
- *     not be a multiple of block: the last tile is short.
+ *   - block is the tile length T_B (64, 128 or 256): the state is carried
+ *     across blocks of that many positions, the products inside a block are
+ *     the masked left product.  It changes the order of floating-point
+ *     operations only, never the mathematical result.  T need not be a
+ *     multiple of block: the last tile is short.
  *   - Calls are asynchronous on `stream` (0 = legacy default stream).  Argument
  *     errors are reported synchronously and launch nothing.  A failed launch
  *     returns LA2_ERR_CUDA.  Faults detected inside a kernel (a bounded wait
@@ -151,8 +153,14 @@ int la2_plan_info(int B, int H, int T, int d, int e, int block, la2_dtype dtype,
  * Forward: out[b,h,t,:] = sum_{s<=t} decay[h]^(t-s) (q[b,h,t,:] . k[b,h,s,:]) v[b,h,s,:].
  *
  * Supported: dtype F32 with 1 <= d, e <= 128 and any block; dtype BF16 with
- * d, e in {64, 128} and block = 128.  Anything else well-formed returns
- * LA2_ERR_UNSUPPORTED.  out must not alias an input.  workspace: device
+ * d, e in {64, 128} and any block.  Anything else well-formed returns
+ * LA2_ERR_UNSUPPORTED.  On the BF16 path block = 128 runs the warp-specialised
+ * tcgen05 kernel (the fast path: overlapped pipeline, sequences cut into
+ * segments to fill the GPU); block = 64 and 256 run a phase-serial tcgen05
+ * kernel with the state carried across 64- or 256-row blocks (one CTA per
+ * sequence and 64 value columns, no segments, no initial or final state:
+ * LA2_ERR_UNSUPPORTED for la2_fwd_state / la2_bwd_state with states and for
+ * the normalised form).  out must not alias an input.  workspace: device
  * memory, 256-byte aligned, of at least la2_workspace_bytes(..., 0) bytes
  * (LA2_ERR_WORKSPACE otherwise), not used concurrently by another call.
  */

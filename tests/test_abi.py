@@ -85,8 +85,7 @@ def test_misaligned_pointers(lib, name):
     assert _fwd(**{name: FAKE + 8}) == la2.LA2_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("kw", [dict(d=96), dict(e=32), dict(d=256), dict(block=64),
-                                dict(block=256)])
+@pytest.mark.parametrize("kw", [dict(d=96), dict(e=32), dict(d=256)])
 def test_bf16_unsupported_shapes(lib, kw):
     assert _fwd(**kw) == la2.LA2_ERR_UNSUPPORTED
     assert _bwd(**kw) == la2.LA2_ERR_UNSUPPORTED
@@ -237,3 +236,12 @@ def test_norm_workspace_and_arguments(lib):
     g = la2.load().la2_bwd_norm
     assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 256, 128, 128, 128,
              la2.LA2_DTYPE_BF16, 0, 0, 0, 0) == la2.LA2_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("block", [64, 256])
+def test_bf16_other_blocks_need_no_workspace_and_reject_states(lib, block):
+    assert la2.la2_workspace_bytes(1, 2, 65536, 128, 128, block, la2.LA2_DTYPE_BF16, 0) == 0
+    assert la2.la2_workspace_bytes(1, 2, 65536, 128, 128, block, la2.LA2_DTYPE_BF16, 1) == 0
+    plan = la2.la2_plan_info(1, 2, 1000, 128, 64, block, is_bwd=True)
+    # one CTA per (sequence, role, 64 value columns), one segment each
+    assert [(g["ctas"], g["segments"], g["prepass_ctas"]) for g in plan] == [(8, 1, 0), (2, 1, 0)]

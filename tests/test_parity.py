@@ -164,6 +164,58 @@ def test_outputs_do_not_write_past_their_end(la2mod):
         assert torch.all(b[-guard:] == 7.0)
 
 
+# ------------------------------------------- bf16 with T_B = 64 and 256
+
+@pytest.mark.parametrize("block", [64, 256])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200, 256, 257, 700])
+@pytest.mark.parametrize("d,e", [(128, 128), (64, 64), (64, 128), (128, 64)])
+def test_bf16_other_blocks_ragged(la2mod, oracle_mod, block, T, d, e):
+    x = I.make_inputs(2, 3, T, d, e, "bf16", seed=T * 5 + d + e + block)
+    errs = _check(la2mod, oracle_mod, x, block, TOL["bf16"])
+    assert max(errs.values()) < 1e-3, errs  # hi + lo operands at every (d, e)
+
+
+@pytest.mark.parametrize("block", [64, 256])
+def test_bf16_other_blocks_decays_and_bitwise_repeat(la2mod, oracle_mod, block):
+    x = I.make_inputs(1, 7, 900, 128, 128, "bf16", seed=21)
+    x["lam"] = torch.tensor([2.0 ** -20, 0.3, 0.8, 0.9, 0.99, 0.999, 1.0], dtype=torch.float32)
+    _check(la2mod, oracle_mod, x, block, TOL["bf16"])
+    a = _run_gpu(la2mod, x, block)
+    b = _run_gpu(la2mod, x, block)
+    for u, w in zip(a, b):
+        assert torch.equal(u, w)
+
+
+@pytest.mark.parametrize("block", [64, 256])
+def test_bf16_other_blocks_bthd_layout_bitwise(la2mod, block):
+    dev = torch.device("cuda")
+    x = I.make_inputs(2, 3, 333, 128, 64, "bf16", seed=23)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    lam = x["lam"].to(dev)
+    o1 = la2mod.la2_fwd_ex(q, k, v, lam, "bhtd", block=block)
+    g1 = la2mod.la2_bwd_ex(q, k, v, lam, do, "bhtd", block=block)
+    qt, kt, vt, dt = (t.transpose(1, 2).contiguous() for t in (q, k, v, do))
+    o2 = la2mod.la2_fwd_ex(qt, kt, vt, lam, "bthd", block=block)
+    g2 = la2mod.la2_bwd_ex(qt, kt, vt, lam, dt, "bthd", block=block)
+    torch.cuda.synchronize()
+    assert la2mod.la2_device_status(reset=True) == 0
+    assert torch.equal(o1, o2.transpose(1, 2))
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b.transpose(1, 2))
+
+
+@pytest.mark.parametrize("block", [64, 256])
+def test_bf16_blocks_agree(la2mod, block):
+    """Every block size computes the same function: T_B changes only the order of
+    floating-point operations (the oracle's tiling pin shows it exactly)."""
+    x = I.make_inputs(2, 4, 1000, 128, 128, "bf16", seed=22)
+    ref = _run_gpu(la2mod, x, 128)
+    got = _run_gpu(la2mod, x, block)
+    for u, w in zip(got, ref):
+        rel = float((u - w).abs().max() / w.pow(2).mean().sqrt())
+        assert rel < 1e-3, rel
+
+
 # -------------------------------------------------- full-size named workloads
 
 _FLAT = {}
@@ -187,7 +239,9 @@ def _workload_inputs(w):
 
 FULL = ["tnl400m", "tnl15b", "tnl15b_nodecay", "long", "sweep_T1024_blk128",
         "sweep_T4096_blk128", "sweep_T16384_blk128", "sweep_T32768_blk128",
-        "sweep_T65536_blk128", "sweep_T131072_blk128", "sweep_T92160_blk128"]
+        "sweep_T65536_blk128", "sweep_T131072_blk128", "sweep_T92160_blk128",
+        "sweep_T1024_blk256", "sweep_T4096_blk256", "sweep_T16384_blk256", "sweep_T32768_blk256",
+        "sweep_T65536_blk256", "sweep_T92160_blk256", "sweep_T131072_blk256"]
 
 
 def _sampled(la2mod, oracle_mod, w, x):
