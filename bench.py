@@ -75,8 +75,16 @@ def flops_per_token_head(w: I.Workload) -> float:
 
 
 def elem_bytes(w: I.Workload) -> int:
-    """Bytes per input element (outputs are always fp32)."""
+    """Bytes per input element."""
     return 2 if w.dtype == "bf16" else 4
+
+
+OUT_TORCH = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def out_bytes(out_dtype: str) -> int:
+    """Bytes per output element (--out-dtype)."""
+    return 2 if out_dtype == "bf16" else 4
 
 
 def bwd_algorithmic_bytes(w: I.Workload) -> float:
@@ -86,14 +94,14 @@ def bwd_algorithmic_bytes(w: I.Workload) -> float:
     return float(w.sequences) * w.T * elem_bytes(w) * (4 * w.d + 3 * w.e)
 
 
-def bwd_written_bytes(w: I.Workload) -> float:
-    """The same with the outputs at the fp32 width the kernel writes."""
-    return float(w.sequences) * w.T * (elem_bytes(w) * (2 * w.d + 2 * w.e) + 4 * (2 * w.d + w.e))
+def bwd_written_bytes(w: I.Workload, ob: int = 4) -> float:
+    """The same with the outputs at the width the kernel writes (ob bytes)."""
+    return float(w.sequences) * w.T * (elem_bytes(w) * (2 * w.d + 2 * w.e) + ob * (2 * w.d + w.e))
 
 
-def fwd_algorithmic_bytes(w: I.Workload) -> float:
-    """la2_fwd reads q, k, v and writes fp32 o, each once."""
-    return float(w.sequences) * w.T * (elem_bytes(w) * (2 * w.d + w.e) + 4 * w.e)
+def fwd_algorithmic_bytes(w: I.Workload, ob: int = 4) -> float:
+    """la2_fwd reads q, k, v and writes o (ob bytes per element), each once."""
+    return float(w.sequences) * w.T * (elem_bytes(w) * (2 * w.d + w.e) + ob * w.e)
 
 
 class ClockSampler:
@@ -279,6 +287,7 @@ def workload_config(w, args):
             "block": w.block, "layout": getattr(args, "layout", "bhtd"),
             "global_batch": w.B * args.gpus, "seq_len": w.T,
             "parallelism": f"replicas{args.gpus}",
+            "out_dtype": getattr(args, "out_dtype", "f32"),
             "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"}
 
 
@@ -412,7 +421,7 @@ def time_steps(la2, fwd, bwd, stream, flush, steps, warmup):
     return [s.elapsed_time(m) for s, m, _ in ev], [m.elapsed_time(e) for _, m, e in ev], launches
 
 
-def step_line(w, fwd_ms, bwd_ms, tc, hbm, world=1):
+def step_line(w, fwd_ms, bwd_ms, tc, hbm, world=1, ob=4):
     """tokens/s, credited TFLOP/s and roofline figures of one workload's step."""
     f = sum(fwd_ms) / len(fwd_ms)
     b = sum(bwd_ms) / len(bwd_ms)
@@ -421,7 +430,7 @@ def step_line(w, fwd_ms, bwd_ms, tc, hbm, world=1):
     return {"tokens_per_s": w.tokens * world / (step_ms * 1e-3), "ms_per_step": step_ms,
             "fwd_ms": f, "bwd_ms": b, "tflops": tflops, "tc_frac": tflops / (tc * world),
             "bwd_hbm_frac": bwd_algorithmic_bytes(w) / (b * 1e-3) / 1e9 / hbm,
-            "bwd_hbm_frac_fp32_out": bwd_written_bytes(w) / (b * 1e-3) / 1e9 / hbm}
+            "bwd_hbm_frac_as_written": bwd_written_bytes(w, ob) / (b * 1e-3) / 1e9 / hbm}
 
 
 def sweep_lines(la2, w, dev_in, dev_out, lam_sweep, dev, stream, flush, args, tc, hbm):
@@ -445,15 +454,17 @@ def sweep_lines(la2, w, dev_in, dev_out, lam_sweep, dev, stream, flush, args, tc
         dv = dev_out[3].reshape(-1)[:nv].view(shp_v)
         lam = lam_sweep if ws.H == w.H else torch.from_numpy(ws.decays().copy()).to(dev)
 
+        od = OUT_TORCH[args.out_dtype]
+
         def fwd():
-            la2.la2_fwd(q, k, v, lam, out=out, block=ws.block)
+            la2.la2_fwd_ex(q, k, v, lam, out=out, block=ws.block, out_dtype=od)
 
         def bwd():
-            la2.la2_bwd(q, k, v, lam, do, dq=dq, dk=dk, dv=dv, block=ws.block)
+            la2.la2_bwd_ex(q, k, v, lam, do, dq=dq, dk=dk, dv=dv, block=ws.block, out_dtype=od)
 
         fm, bm, _ = time_steps(la2, fwd, bwd, stream, flush, args.sweep_steps, 3)
         ent = {"workload": ws.name, "B": ws.B, "T": ws.T, "H": ws.H, "block": ws.block}
-        ent.update(step_line(ws, fm, bm, tc, hbm))
+        ent.update(step_line(ws, fm, bm, tc, hbm, ob=out_bytes(args.out_dtype)))
         lines.append(ent)
     return lines
 
@@ -468,17 +479,19 @@ def run_ours(args, w, world, rank, local):
         x = dict(x, **{n: x[n].transpose(1, 2).contiguous() for n in ("q", "k", "v", "do")})
     q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
     lam = x["lam"].to(dev)
-    f32 = dict(dtype=torch.float32, device=dev)
-    out = torch.empty(v.shape, **f32)
-    dq, dk, dv = torch.empty(q.shape, **f32), torch.empty(k.shape, **f32), torch.empty(v.shape, **f32)
+    od = OUT_TORCH[args.out_dtype]
+    ob = out_bytes(args.out_dtype)
+    o = dict(dtype=od, device=dev)
+    out = torch.empty(v.shape, **o)
+    dq, dk, dv = torch.empty(q.shape, **o), torch.empty(k.shape, **o), torch.empty(v.shape, **o)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def fwd(qq=q, kk=k, vv=v):
-        la2.la2_fwd_ex(qq, kk, vv, lam, lay, out=out, block=w.block)
+        la2.la2_fwd_ex(qq, kk, vv, lam, lay, out=out, block=w.block, out_dtype=od)
 
     def bwd(qq=q, kk=k, vv=v, dd=do):
-        la2.la2_bwd_ex(qq, kk, vv, lam, dd, lay, dq=dq, dk=dk, dv=dv, block=w.block)
+        la2.la2_bwd_ex(qq, kk, vv, lam, dd, lay, dq=dq, dk=dk, dv=dv, block=w.block, out_dtype=od)
 
     for _ in range(args.warmup):
         flush.fill_(0.0)
@@ -502,8 +515,7 @@ def run_ours(args, w, world, rank, local):
     # The four outputs are read back into one pinned buffer, one after the
     # other (every byte still crosses PCIe; the host copy is not kept).
     hosts = {n: x[n].pin_memory() for n in ("q", "k", "v", "do")}
-    hout = torch.empty(max(t.numel() for t in (out, dq, dk, dv)), dtype=torch.float32,
-                       pin_memory=True)
+    hout = torch.empty(max(t.numel() for t in (out, dq, dk, dv)), dtype=od, pin_memory=True)
     h2d = sum(t.numel() * t.element_size() for t in hosts.values())
     d2h = sum(t.numel() * t.element_size() for t in (out, dq, dk, dv))
     e2e_steps = max(2, min(args.steps, 5))
@@ -538,7 +550,7 @@ def run_ours(args, w, world, rank, local):
     value = tokens_per_step / (step_ms * 1e-3)
     bwd_avg_ms = sum(bwd_ms) / len(bwd_ms)
     achieved = bwd_algorithmic_bytes(w) / (bwd_avg_ms * 1e-3) / 1e9
-    written = bwd_written_bytes(w) / (bwd_avg_ms * 1e-3) / 1e9
+    written = bwd_written_bytes(w, ob) / (bwd_avg_ms * 1e-3) / 1e9
     traffic = None
     try:
         with open(PROFILE_TRAFFIC) as f:
@@ -561,7 +573,8 @@ def run_ours(args, w, world, rank, local):
                      "frac": achieved / hbm, "traffic": traffic,
                      "peak_kind": f"{pk_kind} hbm_gbs",
                      "bytes": "q, k, v, dO in and dq, dk, dv out, each once at the input width",
-                     "achieved_fp32_out": written, "frac_fp32_out": written / hbm},
+                     "out_dtype": args.out_dtype,
+                     "achieved_as_written": written, "frac_as_written": written / hbm},
         "e2e": {"value": tokens_per_step / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
@@ -598,10 +611,14 @@ def main(argv=None):
     ap.add_argument("--mode", default="train", choices=["train", "decode"],
                     help="train: la2_fwd + la2_bwd (the default line); decode: la2_decode steps")
     ap.add_argument("--decode-workload", default="decode_tnl15b", choices=sorted(I.DECODE_WORKLOADS))
+    ap.add_argument("--out-dtype", default="f32", choices=sorted(OUT_TORCH),
+                    help="element type of o, dq, dk, dv (bf16 needs bf16 inputs)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be at least 3")
     w = I.WORKLOADS[args.workload]
+    if w.dtype != "bf16":
+        args.out_dtype = "f32"
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":

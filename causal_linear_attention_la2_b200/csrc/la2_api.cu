@@ -329,7 +329,7 @@ void launch_ws(const la2::ws::Params& p, const SegPlan& sp, cudaStream_t stream)
 // segment starts inside its unit.
 la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
                           bool bthd, int sched, int* status, float* seg_state, const Hold& hold,
-                          cudaStream_t stream, bool norm = false) {
+                          cudaStream_t stream, bool norm = false, bool xbf16 = false) {
     la2::ws::Params p;
     std::memset(&p, 0, sizeof(p));
     const int BH = B * H;
@@ -339,7 +339,7 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
             !make_map(&p.role[r].tb, roles[r].b, B, H, T, da, bthd) ||
             !make_map(&p.role[r].tc, roles[r].c, B, H, T, dc, bthd))
             return LA2_ERR_CUDA;
-        p.role[r].x = static_cast<float*>(roles[r].x);
+        p.role[r].x = roles[r].x;
         p.role[r].init = roles[r].init;
         p.role[r].fin = roles[r].fin;
         p.role[r].dir = roles[r].dir;
@@ -354,6 +354,7 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
     p.bthd = bthd ? 1 : 0;
     p.hold = hold.flag;
     p.hold_ns = hold.ns;
+    p.xbf16 = xbf16 ? 1 : 0;
     const SegPlan sp = plan_segments(static_cast<long long>(BH) * n, T, sched);
     p.nunits = BH * n;
     p.nseg = sp.nseg;
@@ -381,7 +382,7 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
 // T_B = 64 or 256 on bf16 inputs (scan_blk_sm100.cuh): one CTA per
 // (sequence, role, 64 value columns), no segments, no workspace, no states.
 la2_status launch_bf16_blk(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
-                           int block, bool bthd, int* status, cudaStream_t stream) {
+                           int block, bool bthd, int* status, cudaStream_t stream, bool xbf16) {
     la2::blk::Params p;
     std::memset(&p, 0, sizeof(p));
     const int da = roles[0].da, dc = roles[0].dc;
@@ -391,7 +392,7 @@ la2_status launch_bf16_blk(const RoleDesc* roles, int n, const float* decay, int
             !make_map(&p.role[r].tb, roles[r].b, B, H, T, da, bthd) ||
             !make_map(&p.role[r].tc, roles[r].c, B, H, T, dc, bthd))
             return LA2_ERR_CUDA;
-        p.role[r].x = static_cast<float*>(roles[r].x);
+        p.role[r].x = roles[r].x;
         p.role[r].dir = roles[r].dir;
     }
     p.decay = decay;
@@ -402,6 +403,7 @@ la2_status launch_bf16_blk(const RoleDesc* roles, int n, const float* decay, int
     p.bthd = bthd ? 1 : 0;
     p.dc = dc;
     p.nslice = dc / la2::blk::kDC;
+    p.xbf16 = xbf16 ? 1 : 0;
     const long long ctas = static_cast<long long>(B) * H * n * p.nslice;
     if (ctas > 0x7fffffffLL) return LA2_ERR_UNSUPPORTED;
     const unsigned grid = static_cast<unsigned>(ctas);
@@ -486,7 +488,7 @@ size_t bf16_workspace_bytes(const RoleDesc* roles, int n, int B, int H, int T, i
 la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
                      int block, la2_dtype dtype, bool bthd, int sched, void* workspace,
                      size_t ws_bytes, cudaStream_t stream, const Hold& hold = Hold(),
-                     bool norm = false) {
+                     bool norm = false, bool xbf16 = false) {
     int dev = 0;
     int* status = nullptr;
     if (dtype == LA2_DTYPE_BF16) {
@@ -494,11 +496,14 @@ la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, in
         if (need > 0 && (workspace == nullptr || ws_bytes < need)) return LA2_ERR_WORKSPACE;
     }
     if (!device_setup(&dev, &status)) return LA2_ERR_CUDA;
-    if (dtype == LA2_DTYPE_F32) return launch_f32(roles, n, decay, B, H, T, block, bthd, stream);
+    if (dtype == LA2_DTYPE_F32) {
+        if (xbf16) return LA2_ERR_UNSUPPORTED;
+        return launch_f32(roles, n, decay, B, H, T, block, bthd, stream);
+    }
     if (block != la2::ws::kTB) {
         if (norm || hold.flag) return LA2_ERR_UNSUPPORTED;
         return for_role_groups(roles, n, [&](const RoleDesc* g, int m) {
-            return launch_bf16_blk(g, m, decay, B, H, T, block, bthd, status, stream);
+            return launch_bf16_blk(g, m, decay, B, H, T, block, bthd, status, stream, xbf16);
         });
     }
     size_t off = 0;
@@ -506,7 +511,8 @@ la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, in
         float* seg = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) + off) : nullptr;
         off += seg_workspace_bytes(static_cast<long long>(B) * H * m, T, g[0].da, g[0].dc, sched);
         off = (off + 255) & ~static_cast<size_t>(255);
-        return launch_bf16_ws(g, m, decay, B, H, T, bthd, sched, status, seg, hold, stream, norm);
+        return launch_bf16_ws(g, m, decay, B, H, T, bthd, sched, status, seg, hold, stream, norm,
+                              xbf16);
     });
 }
 
@@ -613,13 +619,15 @@ int la2_plan_info(int B, int H, int T, int d, int e, int block, la2_dtype dtype,
 
 la2_status la2_fwd_ex(const void* q, const void* k, const void* v, const float* decay, void* out,
                       const float* init_state, float* final_state, int B, int H, int T, int d,
-                      int e, int block, la2_dtype dtype, la2_layout layout, void* workspace,
-                      size_t workspace_bytes, la2_stream_t stream) {
+                      int e, int block, la2_dtype dtype, la2_dtype out_dtype, la2_layout layout,
+                      void* workspace, size_t workspace_bytes, la2_stream_t stream) {
     t_last_launches = 0;
     if (layout != LA2_LAYOUT_BHTD && layout != LA2_LAYOUT_BTHD) return LA2_ERR_INVALID_ARG;
+    if (out_dtype != LA2_DTYPE_F32 && out_dtype != LA2_DTYPE_BF16) return LA2_ERR_INVALID_ARG;
     bool empty = false;
     la2_status st = common_checks(B, H, T, d, e, block, dtype, &empty);
     if (st != LA2_OK) return st;
+    if (out_dtype == LA2_DTYPE_BF16 && dtype != LA2_DTYPE_BF16) return LA2_ERR_UNSUPPORTED;
     if (empty) {
         // no position to process: the final state is the initial one (or 0)
         if (final_state && B > 0 && H > 0) {
@@ -643,7 +651,8 @@ la2_status la2_fwd_ex(const void* q, const void* k, const void* v, const float* 
     r.fin = final_state;
     return run_roles(&r, 1, decay, B, H, T, block, dtype, layout == LA2_LAYOUT_BTHD,
                      g_schedule.load(), workspace, workspace_bytes,
-                     reinterpret_cast<cudaStream_t>(stream));
+                     reinterpret_cast<cudaStream_t>(stream), Hold(), false,
+                     out_dtype == LA2_DTYPE_BF16);
 }
 
 la2_status la2_fwd_state(const void* q, const void* k, const void* v, const float* decay,
@@ -651,7 +660,7 @@ la2_status la2_fwd_state(const void* q, const void* k, const void* v, const floa
                          int T, int d, int e, int block, la2_dtype dtype, void* workspace,
                          size_t workspace_bytes, la2_stream_t stream) {
     return la2_fwd_ex(q, k, v, decay, out, init_state, final_state, B, H, T, d, e, block, dtype,
-                      LA2_LAYOUT_BHTD, workspace, workspace_bytes, stream);
+                      LA2_DTYPE_F32, LA2_LAYOUT_BHTD, workspace, workspace_bytes, stream);
 }
 
 la2_status la2_fwd(const void* q, const void* k, const void* v, const float* decay, void* out,
@@ -666,27 +675,30 @@ la2_status la2_bwd(const void* q, const void* k, const void* v, const float* dec
                    int e, int block, la2_dtype dtype, void* workspace, size_t workspace_bytes,
                    la2_stream_t stream) {
     return la2_bwd_ex(q, k, v, decay, dout, dq, dk, dv, B, H, T, d, e, block, dtype,
-                      LA2_LAYOUT_BHTD, workspace, workspace_bytes, stream);
+                      LA2_DTYPE_F32, LA2_LAYOUT_BHTD, workspace, workspace_bytes, stream);
 }
 
 la2_status la2_bwd_ex(const void* q, const void* k, const void* v, const float* decay,
                       const void* dout, void* dq, void* dk, void* dv, int B, int H, int T, int d,
-                      int e, int block, la2_dtype dtype, la2_layout layout, void* workspace,
-                      size_t workspace_bytes, la2_stream_t stream) {
+                      int e, int block, la2_dtype dtype, la2_dtype out_dtype, la2_layout layout,
+                      void* workspace, size_t workspace_bytes, la2_stream_t stream) {
     return la2_bwd_state(q, k, v, decay, dout, nullptr, nullptr, dq, dk, dv, nullptr, B, H, T, d,
-                         e, block, dtype, layout, workspace, workspace_bytes, stream);
+                         e, block, dtype, out_dtype, layout, workspace, workspace_bytes, stream);
 }
 
 la2_status la2_bwd_state(const void* q, const void* k, const void* v, const float* decay,
                          const void* dout, const float* init_state, const float* d_final_state,
                          void* dq, void* dk, void* dv, float* d_init_state, int B, int H, int T,
-                         int d, int e, int block, la2_dtype dtype, la2_layout layout,
-                         void* workspace, size_t workspace_bytes, la2_stream_t stream) {
+                         int d, int e, int block, la2_dtype dtype, la2_dtype out_dtype,
+                         la2_layout layout, void* workspace, size_t workspace_bytes,
+                         la2_stream_t stream) {
     t_last_launches = 0;
     if (layout != LA2_LAYOUT_BHTD && layout != LA2_LAYOUT_BTHD) return LA2_ERR_INVALID_ARG;
+    if (out_dtype != LA2_DTYPE_F32 && out_dtype != LA2_DTYPE_BF16) return LA2_ERR_INVALID_ARG;
     bool empty = false;
     la2_status st = common_checks(B, H, T, d, e, block, dtype, &empty);
     if (st != LA2_OK) return st;
+    if (out_dtype == LA2_DTYPE_BF16 && dtype != LA2_DTYPE_BF16) return LA2_ERR_UNSUPPORTED;
     const uintptr_t smis = reinterpret_cast<uintptr_t>(init_state) |
                            reinterpret_cast<uintptr_t>(d_final_state) |
                            reinterpret_cast<uintptr_t>(d_init_state);
@@ -728,7 +740,8 @@ la2_status la2_bwd_state(const void* q, const void* k, const void* v, const floa
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return LA2_ERR_INVALID_ARG;
     return run_roles(roles, 3, decay, B, H, T, block, dtype, layout == LA2_LAYOUT_BTHD,
                      g_schedule.load(), workspace, workspace_bytes,
-                     reinterpret_cast<cudaStream_t>(stream));
+                     reinterpret_cast<cudaStream_t>(stream), Hold(), false,
+                     out_dtype == LA2_DTYPE_BF16);
 }
 
 la2_status la2_decode(const void* q, const void* k, const void* v, const float* decay,

@@ -333,6 +333,16 @@ __device__ __forceinline__ void st_global_v2(void* p, float a, float b) {
     asm volatile("st.global.v2.f32 [%0], {%1, %2};" :: "l"(p), "f"(a), "f"(b) : "memory");
 }
 
+// Stores of packed bf16 pairs (pack_bf16x2): one pair, or four pairs (16 bytes).
+__device__ __forceinline__ void st_global_b32(void* p, uint32_t a) {
+    asm volatile("st.global.b32 [%0], %1;" :: "l"(p), "r"(a) : "memory");
+}
+__device__ __forceinline__ void st_global_v4_b32(void* p, uint32_t a, uint32_t b, uint32_t c,
+                                                 uint32_t d) {
+    asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};"
+                 :: "l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 // Packed pair arithmetic (sm_100 f32x2): (a0, a1) * (b0, b1), elementwise,
 // round to nearest.
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) {

@@ -48,6 +48,7 @@ struct Params {
     int H, T, nroles, bthd;
     int dc;              // the group's full value width (row length of the outputs)
     int nslice;          // dc / 64: CTAs per (sequence, role)
+    int xbf16;           // 1: outputs bf16 (rounded to nearest even once), 0: fp32
 };
 
 template <int DA, int TB>
@@ -133,8 +134,10 @@ la2_scan_blk(const __grid_constant__ Params p)
 
     // output rows: [B, H, T, dc] (row stride dc) or [B, T, H, dc] (stride H dc)
     const size_t xrs = p.bthd ? static_cast<size_t>(p.H) * p.dc : static_cast<size_t>(p.dc);
-    float* xg = R.x + (p.bthd ? (static_cast<size_t>(bh / p.H) * T * p.H + bh % p.H) * p.dc
-                              : static_cast<size_t>(bh) * T * p.dc) + kDC * cs;
+    const size_t xoff = (p.bthd ? (static_cast<size_t>(bh / p.H) * T * p.H + bh % p.H) * p.dc
+                                : static_cast<size_t>(bh) * T * p.dc) + kDC * cs;
+    const bool xb16 = p.xbf16 != 0;
+    char* const xg = static_cast<char*>(R.x) + xoff * (xb16 ? 2 : 4);
 
     constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);
     constexpr uint32_t kIdX = idesc_bf16_f32(128, kDC, 0, 1);
@@ -272,8 +275,14 @@ la2_scan_blk(const __grid_constant__ Params p)
             for (int u = 0; u < 32; ++u) v[u] = fmaf(f, y[u], v[u]);
         }
         const int row = tile * 128 + r;
-        if (row < T) {
-            float* dst = xg + static_cast<size_t>(row) * xrs + 32 * hf;
+        if (row < T && xb16) {
+            uint16_t* dst = reinterpret_cast<uint16_t*>(xg) + static_cast<size_t>(row) * xrs + 32 * hf;
+#pragma unroll
+            for (int u = 0; u < 32; u += 8)
+                st_global_v4_b32(dst + u, pack_bf16x2(v[u], v[u + 1]), pack_bf16x2(v[u + 2], v[u + 3]),
+                                 pack_bf16x2(v[u + 4], v[u + 5]), pack_bf16x2(v[u + 6], v[u + 7]));
+        } else if (row < T) {
+            float* dst = reinterpret_cast<float*>(xg) + static_cast<size_t>(row) * xrs + 32 * hf;
 #pragma unroll
             for (int u = 0; u < 32; u += 4) st_global_v4(dst + u, v[u], v[u + 1], v[u + 2], v[u + 3]);
         }

@@ -69,9 +69,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la2_fwd_state.restype = i
     lib.la2_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
     lib.la2_bwd.restype = i
-    lib.la2_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, sz, vp]
+    lib.la2_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, vp, sz, vp]
     lib.la2_fwd_ex.restype = i
-    lib.la2_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp, sz, vp]
+    lib.la2_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, vp, sz,
+                               vp]
     lib.la2_bwd_ex.restype = i
     lib.la2_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
     lib.la2_decode.restype = i
@@ -90,7 +91,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.la2_selftest_timeout.argtypes = [vp, vp, vp, vp, vp, i, i, i, ctypes.c_uint, vp]
     lib.la2_selftest_timeout.restype = i
     lib.la2_bwd_state.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i,
-                                  i, vp, sz, vp]
+                                  i, i, vp, sz, vp]
     lib.la2_bwd_state.restype = i
     lib.la2_dlambda_workspace_bytes.argtypes = [i, i, i, i, i, i]
     lib.la2_dlambda_workspace_bytes.restype = sz
@@ -189,6 +190,15 @@ def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype == torch.float32:
         return LA2_DTYPE_F32
     raise TypeError(f"unsupported dtype {t.dtype}; expected bfloat16 or float32")
+
+
+def _out_dtype(out_dtype) -> tuple:
+    """(torch dtype, la2_dtype code) of the outputs: fp32 (None) or bf16."""
+    if out_dtype is None or out_dtype == torch.float32:
+        return torch.float32, LA2_DTYPE_F32
+    if out_dtype == torch.bfloat16:
+        return torch.bfloat16, LA2_DTYPE_BF16
+    raise TypeError(f"unsupported out_dtype {out_dtype}; expected torch.float32 or torch.bfloat16")
 
 
 def _check(t: torch.Tensor, name: str, shape, dtype) -> None:
@@ -308,19 +318,22 @@ def _shape(layout, B, H, T, D):
 
 
 def la2_fwd_ex(q, k, v, decay, layout: str = "bhtd", init_state=None, out=None, final_state=None,
-               want_final: bool = False, block: int = 128, stream=None, workspace=None):
+               want_final: bool = False, block: int = 128, stream=None, workspace=None,
+               out_dtype=None):
     """la2_fwd_state for q, k, v (and out) laid out [B, H, T, D] ('bhtd') or
-    [B, T, H, D] ('bthd').  Returns out, or (out, final_state) with want_final
-    or a final_state buffer given."""
+    [B, T, H, D] ('bthd'), out of type out_dtype (torch.float32, the default, or
+    torch.bfloat16).  Returns out, or (out, final_state) with want_final or a
+    final_state buffer given."""
     B, H, T, d, e = _dims(q, v, layout)
     dt = _dtype_code(q)
+    odt, oc = _out_dtype(out_dtype)
     _check(q, "q", _shape(layout, B, H, T, d), q.dtype)
     _check(k, "k", _shape(layout, B, H, T, d), q.dtype)
     _check(v, "v", _shape(layout, B, H, T, e), q.dtype)
     _check(decay, "decay", (H,), torch.float32)
     f32 = dict(dtype=torch.float32, device=q.device)
-    out = torch.empty(_shape(layout, B, H, T, e), **f32) if out is None else out
-    _check(out, "out", _shape(layout, B, H, T, e), torch.float32)
+    out = torch.empty(_shape(layout, B, H, T, e), dtype=odt, device=q.device) if out is None else out
+    _check(out, "out", _shape(layout, B, H, T, e), odt)
     if final_state is None and want_final:
         final_state = torch.empty((B, H, d, e), **f32)
     fp = 0
@@ -333,31 +346,33 @@ def la2_fwd_ex(q, k, v, decay, layout: str = "bhtd", init_state=None, out=None, 
         ip = init_state.data_ptr()
     wp, wn = _workspace(la2_workspace_bytes(B, H, T, d, e, block, dt, 0), q.device, workspace)
     st = int(load().la2_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(),
-                               out.data_ptr(), ip, fp, B, H, T, d, e, block, dt, _LAYOUTS[layout],
-                               wp, wn, _stream_ptr(stream)))
+                               out.data_ptr(), ip, fp, B, H, T, d, e, block, dt, oc,
+                               _LAYOUTS[layout], wp, wn, _stream_ptr(stream)))
     if st != LA2_OK:
         raise LA2Error(st, "la2_fwd_ex")
     return (out, final_state) if final_state is not None else out
 
 
 def la2_bwd_ex(q, k, v, decay, dout, layout: str = "bhtd", dq=None, dk=None, dv=None,
-               block: int = 128, stream=None, workspace=None):
-    """la2_bwd for tensors laid out [B, H, T, D] ('bhtd') or [B, T, H, D] ('bthd')."""
+               block: int = 128, stream=None, workspace=None, out_dtype=None):
+    """la2_bwd for tensors laid out [B, H, T, D] ('bhtd') or [B, T, H, D] ('bthd'),
+    dq, dk, dv of type out_dtype (torch.float32, the default, or torch.bfloat16)."""
     B, H, T, d, e = _dims(q, v, layout)
     dt = _dtype_code(q)
+    odt, oc = _out_dtype(out_dtype)
     for t, n, D in ((q, "q", d), (k, "k", d), (v, "v", e), (dout, "dout", e)):
         _check(t, n, _shape(layout, B, H, T, D), q.dtype)
     _check(decay, "decay", (H,), torch.float32)
-    f32 = dict(dtype=torch.float32, device=q.device)
-    dq = torch.empty(_shape(layout, B, H, T, d), **f32) if dq is None else dq
-    dk = torch.empty(_shape(layout, B, H, T, d), **f32) if dk is None else dk
-    dv = torch.empty(_shape(layout, B, H, T, e), **f32) if dv is None else dv
+    o = dict(dtype=odt, device=q.device)
+    dq = torch.empty(_shape(layout, B, H, T, d), **o) if dq is None else dq
+    dk = torch.empty(_shape(layout, B, H, T, d), **o) if dk is None else dk
+    dv = torch.empty(_shape(layout, B, H, T, e), **o) if dv is None else dv
     for t, n, D in ((dq, "dq", d), (dk, "dk", d), (dv, "dv", e)):
-        _check(t, n, _shape(layout, B, H, T, D), torch.float32)
+        _check(t, n, _shape(layout, B, H, T, D), odt)
     wp, wn = _workspace(la2_workspace_bytes(B, H, T, d, e, block, dt, 1), q.device, workspace)
     st = int(load().la2_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(),
                                dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, T,
-                               d, e, block, dt, _LAYOUTS[layout], wp, wn, _stream_ptr(stream)))
+                               d, e, block, dt, oc, _LAYOUTS[layout], wp, wn, _stream_ptr(stream)))
     if st != LA2_OK:
         raise LA2Error(st, "la2_bwd_ex")
     return dq, dk, dv
@@ -365,21 +380,24 @@ def la2_bwd_ex(q, k, v, decay, dout, layout: str = "bhtd", dq=None, dk=None, dv=
 
 def la2_bwd_state(q, k, v, decay, dout, init_state=None, d_final_state=None, layout: str = "bhtd",
                   dq=None, dk=None, dv=None, d_init_state=None, want_d_init: bool = True,
-                  block: int = 128, stream=None, workspace=None):
+                  block: int = 128, stream=None, workspace=None, out_dtype=None):
     """(dq, dk, dv, d_init_state) of sum(dout * out) + sum(d_final_state * final_state) for
     the forward la2_fwd_ex(q, k, v, decay, layout, init_state); states [B, H, d, e] fp32
-    (None = zero).  d_init_state is None unless want_d_init or a buffer is given."""
+    (None = zero), dq, dk, dv of type out_dtype (torch.float32 or torch.bfloat16).
+    d_init_state is None unless want_d_init or a buffer is given."""
     B, H, T, d, e = _dims(q, v, layout)
     dt = _dtype_code(q)
+    odt, oc = _out_dtype(out_dtype)
     for t, n, D in ((q, "q", d), (k, "k", d), (v, "v", e), (dout, "dout", e)):
         _check(t, n, _shape(layout, B, H, T, D), q.dtype)
     _check(decay, "decay", (H,), torch.float32)
     f32 = dict(dtype=torch.float32, device=q.device)
-    dq = torch.empty(_shape(layout, B, H, T, d), **f32) if dq is None else dq
-    dk = torch.empty(_shape(layout, B, H, T, d), **f32) if dk is None else dk
-    dv = torch.empty(_shape(layout, B, H, T, e), **f32) if dv is None else dv
+    o = dict(dtype=odt, device=q.device)
+    dq = torch.empty(_shape(layout, B, H, T, d), **o) if dq is None else dq
+    dk = torch.empty(_shape(layout, B, H, T, d), **o) if dk is None else dk
+    dv = torch.empty(_shape(layout, B, H, T, e), **o) if dv is None else dv
     for t, n, D in ((dq, "dq", d), (dk, "dk", d), (dv, "dv", e)):
-        _check(t, n, _shape(layout, B, H, T, D), torch.float32)
+        _check(t, n, _shape(layout, B, H, T, D), odt)
     if d_init_state is None and want_d_init:
         d_init_state = torch.empty((B, H, d, e), **f32)
     ptrs = []
@@ -391,7 +409,7 @@ def la2_bwd_state(q, k, v, decay, dout, init_state=None, d_final_state=None, lay
     wp, wn = _workspace(la2_workspace_bytes(B, H, T, d, e, block, dt, 1), q.device, workspace)
     st = int(load().la2_bwd_state(q.data_ptr(), k.data_ptr(), v.data_ptr(), decay.data_ptr(),
                                   dout.data_ptr(), ptrs[0], ptrs[1], dq.data_ptr(), dk.data_ptr(),
-                                  dv.data_ptr(), ptrs[2], B, H, T, d, e, block, dt,
+                                  dv.data_ptr(), ptrs[2], B, H, T, d, e, block, dt, oc,
                                   _LAYOUTS[layout], wp, wn, _stream_ptr(stream)))
     if st != LA2_OK:
         raise LA2Error(st, "la2_bwd_state")

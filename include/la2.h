@@ -22,8 +22,9 @@
  *     never allocates, frees or retains them past the call.
  *   - q, k, dq, dk are [B, H, T, d] contiguous (d fastest); v, out, dout, dv
  *     are [B, H, T, e] contiguous.  The inputs q, k, v, dout have the element
- *     type `dtype`; the outputs out, dq, dk, dv are always fp32 (see
- *     la2_dtype).  Every tensor pointer must be 16-byte aligned.
+ *     type `dtype`; the outputs out, dq, dk, dv are fp32, or, through the
+ *     `_ex` / la2_bwd_state calls' out_dtype, bf16 (see la2_dtype).  Every
+ *     tensor pointer must be 16-byte aligned.
  *   - decay is a device array of H floats (fp32) holding lambda_h in (0, 1];
  *     values outside that range are the caller's error and are not checked.
  *   - block is the tile length T_B (64, 128 or 256): the state is carried
@@ -63,11 +64,18 @@ typedef enum {
 } la2_status;
 
 /*
- * Input element type.  Outputs are fp32 in both cases: the accuracy contract
- * of this library is max|out - exact| <= 2e-2 * rms(exact) for bf16 inputs
- * (1e-5 for fp32 inputs), and the outputs of this operation have
- * max/rms ~ 10, where a bf16 result's own rounding (half an ulp, up to 2^-5
- * of rms) would already exceed that bound.
+ * Element type of the inputs (`dtype`) and of the outputs (`out_dtype`, in
+ * la2_fwd_ex, la2_bwd_ex and la2_bwd_state; fp32 in every other call).
+ *
+ * With fp32 outputs the accuracy contract is max|out - exact| <= 2e-2 *
+ * rms(exact) for bf16 inputs (1e-5 for fp32 inputs).  The outputs of this
+ * operation have max/rms ~ 10, so a bf16 result's own rounding (up to 2^-8 of
+ * the value, i.e. up to ~2^-5 of rms) does not fit inside that bound; with
+ * out_dtype = BF16 each fp32 result is rounded to nearest even once, in the
+ * kernel's output epilogue, and the contract is
+ *     |out - exact| <= 2e-2 * rms(exact) + 2^-8 * |exact|   element by element.
+ * BF16 outputs need BF16 inputs (fp32 inputs with BF16 outputs:
+ * LA2_ERR_UNSUPPORTED); they halve the bytes the kernels write.
  */
 typedef enum {
     LA2_DTYPE_F32 = 0,   /* fp32 inputs; fp32 arithmetic on SIMT cores */
@@ -196,14 +204,16 @@ la2_status la2_fwd_state(const void *q, const void *k, const void *v, const floa
                          void *workspace, size_t workspace_bytes, la2_stream_t stream);
 
 /*
- * la2_fwd_state with an explicit layout of q, k, v and out (see la2_layout);
- * everything else as la2_fwd_state.  An unknown layout is LA2_ERR_INVALID_ARG.
+ * la2_fwd_state with an explicit layout of q, k, v and out (see la2_layout)
+ * and an output element type out_dtype (F32, or BF16 with BF16 inputs; see
+ * la2_dtype); everything else as la2_fwd_state.  The states stay fp32.  An
+ * unknown layout or out_dtype is LA2_ERR_INVALID_ARG.
  */
 la2_status la2_fwd_ex(const void *q, const void *k, const void *v, const float *decay,
                       void *out, const float *init_state, float *final_state,
                       int B, int H, int T, int d, int e, int block, la2_dtype dtype,
-                      la2_layout layout, void *workspace, size_t workspace_bytes,
-                      la2_stream_t stream);
+                      la2_dtype out_dtype, la2_layout layout, void *workspace,
+                      size_t workspace_bytes, la2_stream_t stream);
 
 /*
  * Backward of L = sum dout * out with respect to q, k and v (decay is not
@@ -244,13 +254,14 @@ la2_status la2_decode(const void *q, const void *k, const void *v, const float *
 
 /*
  * la2_bwd with an explicit layout of q, k, v, dout, dq, dk and dv (see
- * la2_layout); everything else as la2_bwd.
+ * la2_layout) and the element type out_dtype of dq, dk and dv (as in
+ * la2_fwd_ex); everything else as la2_bwd.
  */
 la2_status la2_bwd_ex(const void *q, const void *k, const void *v, const float *decay,
                       const void *dout, void *dq, void *dk, void *dv,
                       int B, int H, int T, int d, int e, int block, la2_dtype dtype,
-                      la2_layout layout, void *workspace, size_t workspace_bytes,
-                      la2_stream_t stream);
+                      la2_dtype out_dtype, la2_layout layout, void *workspace,
+                      size_t workspace_bytes, la2_stream_t stream);
 
 /*
  * Backward with carried states: the gradients of
@@ -275,15 +286,16 @@ la2_status la2_bwd_ex(const void *q, const void *k, const void *v, const float *
  * init_state, d_final_state: device fp32 [B, H, d, e], or NULL (zero);
  * d_init_state: device fp32 [B, H, d, e], or NULL (not computed); all 4-byte
  * aligned, d_init_state aliasing nothing else.  With T = 0, d_init_state =
- * d_final_state.  Layout, support matrix and workspace as la2_bwd_ex (the
- * same size with or without states).
+ * d_final_state.  Layout, out_dtype (of dq, dk, dv; d_init_state stays
+ * fp32), support matrix and workspace as la2_bwd_ex (the same size with or
+ * without states).
  */
 la2_status la2_bwd_state(const void *q, const void *k, const void *v, const float *decay,
                          const void *dout, const float *init_state, const float *d_final_state,
                          void *dq, void *dk, void *dv, float *d_init_state,
                          int B, int H, int T, int d, int e, int block, la2_dtype dtype,
-                         la2_layout layout, void *workspace, size_t workspace_bytes,
-                         la2_stream_t stream);
+                         la2_dtype out_dtype, la2_layout layout, void *workspace,
+                         size_t workspace_bytes, la2_stream_t stream);
 
 /*
  * Gradient with respect to the decay: d_decay[h] = sum over the batch of

@@ -197,7 +197,7 @@ def test_bwd_state_rejects_misaligned_states(lib):
         st[pos] = FAKE + 2
         r = la2.load().la2_bwd_state(FAKE, FAKE, FAKE, FAKE, FAKE, st[0], st[1], FAKE, FAKE, FAKE,
                                      st[2], 1, 2, 256, 128, 128, 128, la2.LA2_DTYPE_BF16,
-                                     la2.LA2_LAYOUT_BHTD, 0, 0, 0)
+                                     la2.LA2_DTYPE_F32, la2.LA2_LAYOUT_BHTD, 0, 0, 0)
         assert r == la2.LA2_ERR_INVALID_ARG
 
 
@@ -245,3 +245,25 @@ def test_bf16_other_blocks_need_no_workspace_and_reject_states(lib, block):
     plan = la2.la2_plan_info(1, 2, 1000, 128, 64, block, is_bwd=True)
     # one CTA per (sequence, role, 64 value columns), one segment each
     assert [(g["ctas"], g["segments"], g["prepass_ctas"]) for g in plan] == [(8, 1, 0), (2, 1, 0)]
+
+
+@pytest.mark.parametrize("call", ["fwd_ex", "bwd_ex", "bwd_state"])
+def test_out_dtype_arguments(lib, call):
+    """An unknown output type is an argument error; bf16 outputs need bf16
+    inputs (UNSUPPORTED for fp32 inputs, reported before anything is read)."""
+    L = la2.load()
+    bf, f32, lay = la2.LA2_DTYPE_BF16, la2.LA2_DTYPE_F32, la2.LA2_LAYOUT_BHTD
+
+    def go(dtype, out_dtype):
+        if call == "fwd_ex":
+            return L.la2_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0, 1, 2, 256, 128, 128, 128, dtype,
+                                out_dtype, lay, 0, 0, 0)
+        if call == "bwd_ex":
+            return L.la2_bwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 256, 128, 128,
+                                128, dtype, out_dtype, lay, 0, 0, 0)
+        return L.la2_bwd_state(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0, FAKE, FAKE, FAKE, 0, 1, 2, 256,
+                               128, 128, 128, dtype, out_dtype, lay, 0, 0, 0)
+
+    assert go(bf, 2) == la2.LA2_ERR_INVALID_ARG
+    assert go(bf, -1) == la2.LA2_ERR_INVALID_ARG
+    assert go(f32, bf) == la2.LA2_ERR_UNSUPPORTED

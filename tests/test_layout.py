@@ -68,5 +68,5 @@ def test_unknown_layout_is_rejected(la2mod):
     from causal_linear_attention_la2_b200.la2 import LA2_ERR_INVALID_ARG
     lib = la2mod.load()
     st = lib.la2_fwd_ex(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 0, 0, 1, 1, 8, 64, 64, 128, 1,
-                        7, 0, 0, 0)
+                        0, 7, 0, 0, 0)
     assert st == LA2_ERR_INVALID_ARG
