@@ -158,18 +158,18 @@ struct RingCfg {
     static constexpr int NCF = kTf32 ? 2 : 0;                // fp32 C (tf32 mode)
     static constexpr int NWB = kTf32 ? 1 : 0;                // fp32 w_s B (tf32 mode)
     static constexpr int NW = DA == 64 ? 2 : 1;              // W as its hi/lo pair
-    // DC = 64 (kOwnD): X += P C (one TMEM buffer), X_inter = A W (one) and
-    // dW (two) are separate accumulators, and the epilogue forms
-    // w_x X_inter + X; X += P C then never waits for the state, and dW of
-    // tile s+1 never waits for the update after tile s.  DC = 128: X (two
+    // DC = 64 (kOwnD): X += P C (one TMEM buffer), X_inter = A W (two) and
+    // dW (one) are separate accumulators, and the epilogue forms
+    // w_x X_inter + X; X += P C then never waits for the state, and X_inter
+    // of tile s never waits for the output of tile s-1.  DC = 128: X (two
     // buffers) holds A W, scaled by w_x in TMEM, then P C; dW borrows the X
     // buffer of the next tile.
     static constexpr bool kOwnD = DC == 64;
-    static constexpr int ND = kOwnD ? 2 : 1;                 // dW accumulators (own-D)
+    static constexpr int ND = 1;                             // dW accumulators (own-D)
     static constexpr int NX = kOwnD ? 1 : 2;                 // X accumulators in TMEM
-    static constexpr int NXW = kOwnD ? 1 : NX;               // XW_DONE barriers
+    static constexpr int NXW = kOwnD ? 2 : NX;               // XW_DONE barriers
     static constexpr int NXS = kOwnD ? 0 : NX;               // XS barriers (scaled in TMEM)
-    static constexpr int NXI = kOwnD ? 1 : 0;                // EMPTY_XI (X_inter read out)
+    static constexpr int NXI = kOwnD ? 2 : 0;                // X_inter buffers (EMPTY_XI: read out)
     static constexpr int NBS = kTf32 ? 0 : NB;
     // "full": the producer has filled the buffer; "empty": its consumers are done
     static constexpr int FULL_A = 0, EMPTY_A = FULL_A + NA;
@@ -443,12 +443,14 @@ la2_scan_ws(const __grid_constant__ Params p)
     // issued before the state update has read dW.
     auto tS = [&](int b) { return tmem + static_cast<uint32_t>(b * 128); };
     auto tX = [&](int b) { return tmem + 256 + static_cast<uint32_t>(b * DC); };
-    const uint32_t tXI = tmem + 256 + static_cast<uint32_t>(Q::NX * DC);  // X_inter (DC = 64)
+    auto tXI = [&](int s) {  // X_inter of step s (DC = 64)
+        return tmem + 256 + static_cast<uint32_t>((Q::NX + s % (Q::NXI > 0 ? Q::NXI : 1)) * DC);
+    };
     auto tD = [&](int s) {
-        return Q::kOwnD ? tmem + 256 + static_cast<uint32_t>((Q::NX + 1) * DC + (s % Q::ND) * DC)
+        return Q::kOwnD ? tmem + 256 + static_cast<uint32_t>((Q::NX + Q::NXI) * DC + (s % Q::ND) * DC)
                         : tX((s + 1) % Q::NX);
     };
-    static_assert(256 + Q::NX * DC + (Q::kOwnD ? (1 + Q::ND) * DC : 0) <= static_cast<int>(kTmemCols),
+    static_assert(256 + Q::NX * DC + (Q::kOwnD ? (Q::NXI + Q::ND) * DC : 0) <= static_cast<int>(kTmemCols),
                   "TMEM columns");
     auto tile_of = [&](int step) { return dir > 0 ? s0 + step : nb - 1 - (s0 + step); };
     // fp32 state slot of segment gg of this (sequence, role)
@@ -647,9 +649,10 @@ la2_scan_ws(const __grid_constant__ Params p)
                 // also read the dW that sat in this X buffer)
                 if (!wait_bar<Q::kTf32>(bar(Q::W_READY + sw), full_par(s, Q::NW), abort_flag, p.status, 30)) break;
                 if (!wait_bar<Q::kTf32>(bar(Q::FULL_A + sa), full_par(s, Q::NA), abort_flag, p.status, 31)) break;
-                if (Q::kOwnD) {
-                    // X_inter has been read out after tile s-1
-                    if (s >= 1 && !wait_bar<Q::kTf32>(bar(Q::EMPTY_XI), full_par(s - 1, 1), abort_flag, p.status, 32))
+                if constexpr (Q::kOwnD) {
+                    // X_inter buffer s % 2 has been read out after tile s-2
+                    if (s >= Q::NXI && !wait_bar<Q::kTf32>(bar(Q::EMPTY_XI + s % Q::NXI), empty_par(s, Q::NXI),
+                                                           abort_flag, p.status, 32))
                         break;
                 } else if (s >= Q::NX && !wait_bar<Q::kTf32>(bar(Q::EMPTY_X + s % Q::NX), empty_par(s, Q::NX),
                                                    abort_flag, p.status, 32)) {
@@ -657,7 +660,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                 }
                 LA2_TR(7, s);
                 tc_fence_after();
-                const uint32_t xt = Q::kOwnD ? tXI : tX(s % Q::NX);
+                const uint32_t xt = Q::kOwnD ? tXI(s) : tX(s % Q::NX);
                 const uint64_t da = desc_add(dA0, sa * L::kAsz), dw = desc_add(dW0, sw * 2 * L::kWsz);
 #pragma unroll
                 for (int k = 0; k < DA / 16; ++k) {
@@ -1191,7 +1194,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                 tmem_ld16x256b_x4_pair(xt + l0 + col, xt + l1 + col, v);
                 if constexpr (Q::kOwnD) {
                     float vi[32];
-                    tmem_ld16x256b_x4_pair(tXI + l0 + col, tXI + l1 + col, vi);
+                    tmem_ld16x256b_x4_pair(tXI(s) + l0 + col, tXI(s) + l1 + col, vi);
 #pragma unroll
                     for (int lh = 0; lh < 2; ++lh)
 #pragma unroll
@@ -1205,7 +1208,7 @@ la2_scan_ws(const __grid_constant__ Params p)
                 if (b == kCols / 32 - 1) {
                     tc_fence_before();
                     mbar_arrive(bar(Q::EMPTY_X + s % Q::NX));
-                    if constexpr (Q::NXI > 0) mbar_arrive(bar(Q::EMPTY_XI));
+                    if constexpr (Q::NXI > 0) mbar_arrive(bar(Q::EMPTY_XI + s % Q::NXI));
                 }
                 if (xb16) {
                     // one bf16 pair per store: a warp writes 16 bytes of each of 8 rows
