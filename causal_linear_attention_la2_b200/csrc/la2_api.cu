@@ -134,20 +134,42 @@ bool balanced_plan(long long units, int nb, SegPlan* out) {
     return true;
 }
 
+// AUTO takes the balanced plan where the uniform one runs its units in waves
+// whose last is mostly empty (at least 148 units, over a quarter of the
+// waves' SM time idle) and the units are long (>= 128 tiles), so that one
+// balanced wave saves more than its state pre-pass costs; elsewhere the
+// uniform plan.  bench.py on B200, processes alternating the schedules
+// (tokens/s, uniform -> balanced):
+//   T =  65,536, 2 x 32 sequences (bwd: 192 units, second wave 44 CTAs): 19.2 -> 20.2 M
+//   T = 131,072, 32 sequences (fwd in 4 segments, bwd 96 units): 19.4 -> 19.2 M
+//   long, 16 sequences of 65,536 (fwd in 9 segments, bwd in 3):      38.6 -> 37.8 M
+bool auto_balanced(long long units, int nb) {
+    if (units < kTargetCTAs || nb < 128) return false;
+    const long long waves = cdiv(units, kTargetCTAs);
+    return 4 * units < 3 * kTargetCTAs * waves;
+}
+
 // `sched` is the schedule setting read once at the top of the entry point, so
 // that one call sizes its workspace and launches with the same plan even if
 // another thread changes the setting meanwhile.
 SegPlan plan_segments(long long units, int T, int sched) {
     const int nb = (T + la2::ws::kTB - 1) / la2::ws::kTB;
     SegPlan b;
-    if (sched == LA2_SCHEDULE_BALANCED && balanced_plan(units, nb, &b)) return b;
+    const bool bal = sched == LA2_SCHEDULE_BALANCED || (sched == LA2_SCHEDULE_AUTO && auto_balanced(units, nb));
+    if (bal && balanced_plan(units, nb, &b)) return b;
     return uniform_plan(units, nb);
 }
 
-// Workspace bytes of one bf16 launch over `units` (sequence, role) units.
-size_t seg_workspace_bytes(long long units, int T, int da, int dc, int sched) {
+// Workspace bytes of one bf16 launch over `units` (sequence, role) units,
+// the same for every T: the balanced plan's 147 states (never fewer than the
+// uniform plan's states at the segment boundaries of every unit), or the
+// uniform plan's.  AUTO reserves the balanced size for unit counts it takes
+// the balanced plan for at some T (the set of such T, if any, contains every
+// long T, so the test at a very long T decides).
+size_t seg_workspace_bytes(long long units, int da, int dc, int sched) {
     const size_t state = static_cast<size_t>(da) * static_cast<size_t>(dc) * sizeof(float);
-    if (plan_segments(units, T, sched).balanced) return static_cast<size_t>(kTargetCTAs - 1) * state;
+    const bool bal = sched == LA2_SCHEDULE_BALANCED || (sched == LA2_SCHEDULE_AUTO && auto_balanced(units, 1 << 20));
+    if (bal) return static_cast<size_t>(kTargetCTAs - 1) * state;
     return static_cast<size_t>(max_segments(units) - 1) * static_cast<size_t>(units) * state;
 }
 
@@ -478,7 +500,7 @@ size_t bf16_workspace_bytes(const RoleDesc* roles, int n, int B, int H, int T, i
     if (block != la2::ws::kTB) return 0;  // the T_B = 64 / 256 kernel needs none
     size_t total = 0;
     for_role_groups(roles, n, [&](const RoleDesc* g, int m) {
-        total += seg_workspace_bytes(static_cast<long long>(B) * H * m, T, g[0].da, g[0].dc, sched);
+        total += seg_workspace_bytes(static_cast<long long>(B) * H * m, g[0].da, g[0].dc, sched);
         total = (total + 255) & ~static_cast<size_t>(255);
         return LA2_OK;
     });
@@ -509,7 +531,7 @@ la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, in
     size_t off = 0;
     return for_role_groups(roles, n, [&](const RoleDesc* g, int m) {
         float* seg = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) + off) : nullptr;
-        off += seg_workspace_bytes(static_cast<long long>(B) * H * m, T, g[0].da, g[0].dc, sched);
+        off += seg_workspace_bytes(static_cast<long long>(B) * H * m, g[0].da, g[0].dc, sched);
         off = (off + 255) & ~static_cast<size_t>(255);
         return launch_bf16_ws(g, m, decay, B, H, T, bthd, sched, status, seg, hold, stream, norm,
                               xbf16);

@@ -101,8 +101,8 @@ typedef enum {
  * the workspace only holds the fp32 end state of each segment that a sequence
  * is cut into so that the work fills the GPU's 148 SMs (see la2_schedule): at
  * most 147 states of d x e floats per group of roles with the same (d, e).
- * The value does not depend on T; it depends on the schedule setting in force
- * (la2_set_schedule).  0 means the call accepts workspace = NULL.  Returns
+ * The value does not depend on T (under AUTO it covers the plan AUTO takes at
+ * any T); it depends on the schedule setting in force (la2_set_schedule).  0 means the call accepts workspace = NULL.  Returns
  * (size_t)-1 for arguments the call would reject.
  */
 size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block,
@@ -116,10 +116,15 @@ size_t la2_workspace_bytes(int B, int H, int T, int d, int e, int block,
  *   BALANCED the units' 128-position tiles are laid end to end and cut into
  *            148 equal runs, one CTA each, which processes the pieces of
  *            units its run covers one after the other (one wave, equal work);
- *   AUTO     (default) the library's choice: UNIFORM.  On a B200 BALANCED
- *            was at best 3% faster on the benchmark shapes and up to 11%
- *            slower: with every SM busy each tile takes longer, and its
- *            pre-pass re-reads inputs.
+ *   AUTO     (default) the library's choice: BALANCED for at least 148
+ *            units of at least 128 tiles whose UNIFORM waves would leave over
+ *            a quarter of their SM time idle (e.g. 192 units: a second wave
+ *            of 44 CTAs), UNIFORM elsewhere.  Measured on a B200 with the
+ *            benchmark: BALANCED +5% at T = 65,536 with 64 sequences, -1% to
+ *            -2% where UNIFORM cuts few units into segments or runs one
+ *            partial wave, and up to 23% slower per pass where UNIFORM fills
+ *            its waves (every SM busy makes each tile slower, and the
+ *            pre-pass re-reads inputs).
  * A segment that starts inside its unit receives its incoming state from a
  * pre-pass over the unit's earlier positions.  Results agree between the
  * schedules to rounding (the sum is grouped differently).  Process-wide;

@@ -153,12 +153,16 @@ def test_no_workspace_when_the_grid_is_full(lib):
 
 
 def test_plan_info(lib):
-    # long-context forward: 16 units of 512 tiles, cut into 9 segments of 57 tiles
-    assert la2.la2_plan_info(1, 16, 65536, 128, 128) == [
-        {"d": 128, "e": 128, "schedule": "uniform", "units": 16, "segments": 9, "tiles_per_cta": 57,
-         "ctas": 144, "prepass_ctas": 128}]
-    # its backward: 48 units in 3 segments of 171 tiles
-    assert la2.la2_plan_info(1, 16, 65536, 128, 128, is_bwd=True)[0]["segments"] == 3
+    prev = la2.la2_set_schedule("uniform")
+    try:
+        # long-context forward: 16 units of 512 tiles, cut into 9 segments of 57 tiles
+        assert la2.la2_plan_info(1, 16, 65536, 128, 128) == [
+            {"d": 128, "e": 128, "schedule": "uniform", "units": 16, "segments": 9, "tiles_per_cta": 57,
+             "ctas": 144, "prepass_ctas": 128}]
+        # its backward: 48 units in 3 segments of 171 tiles
+        assert la2.la2_plan_info(1, 16, 65536, 128, 128, is_bwd=True)[0]["segments"] == 3
+    finally:
+        la2.la2_set_schedule(prev)
     # 15B backward: 240 units fill the GPU, no segments, no pre-pass
     p = la2.la2_plan_info(2, 40, 6144, 128, 128, is_bwd=True)
     assert len(p) == 1 and p[0]["units"] == 240 and p[0]["ctas"] == 240 and p[0]["prepass_ctas"] == 0
@@ -267,3 +271,33 @@ def test_out_dtype_arguments(lib, call):
     assert go(bf, 2) == la2.LA2_ERR_INVALID_ARG
     assert go(bf, -1) == la2.LA2_ERR_INVALID_ARG
     assert go(f32, bf) == la2.LA2_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("B,H,T,is_bwd,want", [
+    (2, 32, 65536, 1, "balanced"),   # 192 units of 512 tiles: uniform's second wave is 44 CTAs
+    (3, 50, 16384, 0, "balanced"),   # 150 units of 128 tiles: a second wave of 2 CTAs
+    (2, 32, 65536, 0, "uniform"),    # 64 units, cut into 2 segments each
+    (1, 16, 65536, 0, "uniform"),    # long forward: 16 units in 9 segments
+    (1, 32, 131072, 0, "uniform"),   # 32 units in 4 segments
+    (1, 32, 131072, 1, "uniform"),   # 96 units of 1024 tiles, one wave
+    (4, 32, 32768, 0, "uniform"),    # 128 units of 256 tiles in one wave
+    (4, 32, 32768, 1, "uniform"),    # 384 units, three waves 86% full
+    (2, 40, 6144, 0, "uniform"),     # 15B forward: 80 units of only 48 tiles
+    (2, 40, 6144, 1, "uniform"),     # 15B backward: 240 units of 48 tiles
+    (8, 16, 2048, 1, "uniform"),     # TNL-400M backward
+    (128, 32, 1024, 0, "uniform"),   # 4096 short units
+])
+def test_auto_schedule_choice(lib, B, H, T, is_bwd, want):
+    """AUTO takes the balanced plan for >= 148 units of >= 128 tiles whose
+    uniform waves leave over a quarter of their SM time idle, the uniform plan
+    elsewhere; its workspace covers the plan it takes."""
+    prev = la2.la2_set_schedule("auto")
+    try:
+        p = la2.la2_plan_info(B, H, T, 128, 128, is_bwd=bool(is_bwd))
+        assert [g["schedule"] for g in p] == [want]
+        if want == "balanced":
+            assert p[0]["ctas"] <= 148
+            ws = la2.la2_workspace_bytes(B, H, T, 128, 128, 128, la2.LA2_DTYPE_BF16, is_bwd)
+            assert ws >= 147 * 128 * 128 * 4
+    finally:
+        la2.la2_set_schedule(prev)
