@@ -50,12 +50,18 @@ EncodeTiledFn encode_fn() {
 
 template <int DA, int DC, bool kNorm = false>
 bool set_ws_attrs() {
+    constexpr size_t smem = la2::ws::Smem<DA, DC, kNorm>::kBytes;
+    if constexpr (!kNorm) {  // the bf16-output instantiations (no normalised form)
+        if (cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC, false, false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+            cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC, true, false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return false;
+    }
     return cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC, false, kNorm>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                la2::ws::Smem<DA, DC, kNorm>::kBytes) == cudaSuccess &&
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess &&
            cudaFuncSetAttribute(la2::ws::la2_scan_ws<DA, DC, true, kNorm>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                la2::ws::Smem<DA, DC, kNorm>::kBytes) == cudaSuccess &&
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess &&
            cudaFuncSetAttribute(la2::ws::la2_state_ws<DA, DC>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 la2::ws::StateSmem<DA, DC>::kBytes) == cudaSuccess;
@@ -70,19 +76,20 @@ bool set_blk_attrs() {
 // How the bf16 kernel spreads its (sequence, role) units over CTAs.  Each CTA
 // fills one SM (148 on a B200).  Two plans:
 //
-// - uniform (the default): each unit is cut into g equal segments, one CTA
-//   each; g > 1 only when there are fewer units than SMs;
-// - balanced (on request, la2_set_schedule): the units' tiles are laid end to
-//   end and CTA c takes tiles [c L, (c+1) L), L = ceil(total / 148): one wave,
-//   every SM the same work, a CTA running the end of one unit and the start of
-//   the next one after the other.
+// - uniform: each unit is cut into g equal segments, one CTA each; g > 1
+//   only when there are fewer units than SMs;
+// - balanced: the units' tiles are laid end to end and CTA c takes tiles
+//   [c L, (c+1) L), L = ceil(total / 148): one wave, every SM the same work, a
+//   CTA running the end of one unit and the start of the next one after the
+//   other.
+// The default (AUTO, auto_balanced below) takes balanced only where the
+// uniform waves leave a mostly empty last wave over long units.
 //
 // A segment that does not start its unit gets its incoming state from the
-// state pre-pass, which reads that unit's B and C up to the segment.  On a
-// B200 the balanced plan measured no faster on any benchmark shape: a tile
-// takes 20-40% longer once every SM runs the scan (at d = 128 the scan then
-// nears what the memory system delivers), a partial last wave runs faster, and
-// the pre-pass re-reads B and C.
+// state pre-pass, which reads that unit's B and C up to the segment.  Filling
+// more SMs does not always pay: a tile takes 20-40% longer once every SM runs
+// the scan (at d = 128 the scan then nears what the memory system delivers), a
+// partial last wave runs faster, and the pre-pass re-reads B and C.
 //
 // Workspace, flat in T in both plans: uniform, (g - 1) states per unit with g
 // from the number of units alone (a short sequence may use fewer); balanced,
@@ -333,17 +340,18 @@ la2_status common_checks(int B, int H, int T, int d, int e, int block, la2_dtype
     return LA2_OK;
 }
 
-template <int DA, int DC, bool kNorm = false>
+template <int DA, int DC, bool kNorm = false, bool kXb16 = false>
 void launch_ws(const la2::ws::Params& p, const SegPlan& sp, cudaStream_t stream) {
+    constexpr size_t smem = la2::ws::Smem<DA, DC, kNorm>::kBytes;
     if (sp.npre > 0)
         la2::ws::la2_state_ws<DA, DC><<<static_cast<unsigned>(sp.npre), la2::ws::kStateThreads,
                                         la2::ws::StateSmem<DA, DC>::kBytes, stream>>>(p);
     if (sp.balanced)
-        la2::ws::la2_scan_ws<DA, DC, true, kNorm><<<static_cast<unsigned>(sp.nctas), la2::ws::kThreads,
-                                                    la2::ws::Smem<DA, DC, kNorm>::kBytes, stream>>>(p);
+        la2::ws::la2_scan_ws<DA, DC, true, kNorm, kXb16>
+            <<<static_cast<unsigned>(sp.nctas), la2::ws::kThreads, smem, stream>>>(p);
     else
-        la2::ws::la2_scan_ws<DA, DC, false, kNorm><<<static_cast<unsigned>(sp.nctas), la2::ws::kThreads,
-                                                     la2::ws::Smem<DA, DC, kNorm>::kBytes, stream>>>(p);
+        la2::ws::la2_scan_ws<DA, DC, false, kNorm, kXb16>
+            <<<static_cast<unsigned>(sp.nctas), la2::ws::kThreads, smem, stream>>>(p);
 }
 
 // Launches the warp-specialised kernel over `n` roles that share (DA, DC),
@@ -376,7 +384,6 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
     p.bthd = bthd ? 1 : 0;
     p.hold = hold.flag;
     p.hold_ns = hold.ns;
-    p.xbf16 = xbf16 ? 1 : 0;
     const SegPlan sp = plan_segments(static_cast<long long>(BH) * n, T, sched);
     p.nunits = BH * n;
     p.nseg = sp.nseg;
@@ -390,6 +397,11 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
         else if (da == 128) launch_ws<128, 64, true>(p, sp, stream);
         else if (dc == 128) launch_ws<64, 128, true>(p, sp, stream);
         else launch_ws<64, 64, true>(p, sp, stream);
+    } else if (xbf16) {
+        if (da == 128 && dc == 128) launch_ws<128, 128, false, true>(p, sp, stream);
+        else if (da == 128) launch_ws<128, 64, false, true>(p, sp, stream);
+        else if (dc == 128) launch_ws<64, 128, false, true>(p, sp, stream);
+        else launch_ws<64, 64, false, true>(p, sp, stream);
     } else {
         if (da == 128 && dc == 128) launch_ws<128, 128>(p, sp, stream);
         else if (da == 128) launch_ws<128, 64>(p, sp, stream);
