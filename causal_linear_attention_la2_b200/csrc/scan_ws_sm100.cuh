@@ -49,7 +49,7 @@
 // 0 issues through predicated instructions).
 // How many buffers each operand gets depends on (DA, DC) (RingCfg): shared
 // memory holds two of most rings, and at DA = DC = 128 one A, C and W buffer
-// and two B buffers.  With DC = 64, X += P C, X_inter and dW (two buffers)
+// and two B buffers.  With DC = 64, X += P C, X_inter (two buffers) and dW
 // are separate TMEM accumulators; otherwise A W is scaled in place by w_x
 // before P C adds to it, and dW borrows the X buffer of the next tile.
 //

@@ -245,7 +245,7 @@ def la2_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, decay: torch.Tens
             workspace: torch.Tensor | None = None) -> torch.Tensor:
     """o[b,h,t] = sum_{s<=t} decay[h]^(t-s) (q[b,h,t] . k[b,h,s]) v[b,h,s], on q's device.
 
-    q, k, v: bf16 or fp32; the output is always fp32."""
+    q, k, v: bf16 or fp32; the output is fp32 (la2_fwd_ex also writes bf16)."""
     B, H, T, d = q.shape
     e = v.shape[-1]
     dt = _dtype_code(q)
