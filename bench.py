@@ -75,6 +75,15 @@ def flops_per_token_head(w: I.Workload) -> float:
     return 3.0 * (2.0 * w.block * (w.d + w.e) + 4.0 * w.d * w.e)
 
 
+def executed_flops_per_token_head(w: I.Workload) -> float:
+    """Executed fwd+bwd FLOPs per (token, head) of the measurement plan: the
+    forward's 2 T_B (d + e) + 4 d e and the backward's 2 T_B (3d + 3e) + 10 d e
+    (which recomputes Q K^T, the states and dO V^T in each of its scans)."""
+    fwd = 2.0 * w.block * (w.d + w.e) + 4.0 * w.d * w.e
+    bwd = 2.0 * w.block * (3 * w.d + 3 * w.e) + 10.0 * w.d * w.e
+    return fwd + bwd
+
+
 def elem_bytes(w: I.Workload) -> int:
     """Bytes per input element."""
     return 2 if w.dtype == "bf16" else 4
@@ -396,10 +405,12 @@ def run_decode(args, world, rank, local):
 
 def time_steps(la2, fwd, bwd, stream, flush, steps, warmup):
     """CUDA-event times of `steps` fwd and bwd calls after `warmup` untimed
-    ones, the L2 flushed (outside the events) before each; returns the per-step
-    fwd and bwd times in ms and the kernels launched in the timed steps."""
+    ones, the L2 flushed (outside the events) before each unless flush is
+    None; returns the per-step fwd and bwd times in ms and the kernels
+    launched in the timed steps."""
     for _ in range(warmup):
-        flush.fill_(0.0)
+        if flush is not None:
+            flush.fill_(0.0)
         fwd()
         bwd()
     torch.cuda.synchronize()
@@ -408,7 +419,8 @@ def time_steps(la2, fwd, bwd, stream, flush, steps, warmup):
            torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     launches = 0
     for i in range(steps):
-        flush.fill_(float(i))
+        if flush is not None:
+            flush.fill_(float(i))
         s, m, e = ev[i]
         s.record(stream)
         fwd()
@@ -523,6 +535,10 @@ def run_ours(args, w, world, rank, local):
     barrier(world)
     clk = clocks.stop() if clocks else None
     step_ms = max_over_ranks(sum(fwd_ms) / len(fwd_ms) + sum(bwd_ms) / len(bwd_ms), world)
+    # the same steps back to back without the L2 flush (context only: every
+    # workload but tiny_f32 holds more than the 126 MB L2)
+    nf_f, nf_b, _ = time_steps(la2, fwd, bwd, stream, None, args.steps, 1)
+    step_ms_no_flush = max_over_ranks(sum(nf_f) / len(nf_f) + sum(nf_b) / len(nf_b), world)
 
     # end to end through the public API: pinned host in -> device -> host out.
     # The four outputs are read back into one pinned buffer, one after the
@@ -559,6 +575,7 @@ def run_ours(args, w, world, rank, local):
     pk, pk_kind = peaks()
     hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     tc = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    tc_sus = float(pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     tokens_per_step = w.tokens * world
     value = tokens_per_step / (step_ms * 1e-3)
     bwd_avg_ms = sum(bwd_ms) / len(bwd_ms)
@@ -580,6 +597,9 @@ def run_ours(args, w, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic", "config": workload_config(w, args),
         "tflops": tflops, "tc_frac": tflops / (tc * world), "tc_peak_tflops": tc,
+        "tc_frac_sustained": tflops / (tc_sus * world), "tc_peak_sustained_tflops": tc_sus,
+        "tflops_executed": executed_flops_per_token_head(w) * w.T * w.sequences * world / (step_ms * 1e-3) / 1e12,
+        "ms_per_step_no_l2_flush": step_ms_no_flush,
         "fwd_ms": sum(fwd_ms) / len(fwd_ms), "bwd_ms": bwd_avg_ms,
         "roofline": {"bound": "hbm", "kernel": bwd_kernel_label(la2, w),
                      "achieved": achieved, "peak": hbm, "unit": "GB/s",
