@@ -414,20 +414,24 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
 }
 
 // T_B = 64 or 256 on bf16 inputs (scan_blk_sm100.cuh): one CTA per
-// (sequence, role, 64 value columns), no segments, no workspace, no states.
+// (sequence, role, 64 value columns), no segments, no workspace; carried
+// states as in the T_B = 128 kernel, no per-position factor (colf).
 la2_status launch_bf16_blk(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
                            int block, bool bthd, int* status, cudaStream_t stream, bool xbf16) {
     la2::blk::Params p;
     std::memset(&p, 0, sizeof(p));
     const int da = roles[0].da, dc = roles[0].dc;
     for (int r = 0; r < n; ++r) {
-        if (roles[r].init || roles[r].fin || roles[r].colf) return LA2_ERR_UNSUPPORTED;
+        if (roles[r].colf) return LA2_ERR_UNSUPPORTED;  // the normalised form: T_B = 128 only
         if (!make_map(&p.role[r].ta, roles[r].a, B, H, T, da, bthd) ||
             !make_map(&p.role[r].tb, roles[r].b, B, H, T, da, bthd) ||
             !make_map(&p.role[r].tc, roles[r].c, B, H, T, dc, bthd))
             return LA2_ERR_CUDA;
         p.role[r].x = roles[r].x;
         p.role[r].dir = roles[r].dir;
+        p.role[r].init = roles[r].init;
+        p.role[r].fin = roles[r].fin;
+        p.role[r].init_t = roles[r].init_t;
     }
     p.decay = decay;
     p.status = status;

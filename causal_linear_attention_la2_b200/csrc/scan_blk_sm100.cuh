@@ -30,7 +30,13 @@
 // memory), every hand-off an mbarrier or a block barrier: simple and exact, not
 // overlapped like the T_B = 128 kernel.  Operands the kernel forms (P, w_s B,
 // the state) enter the tensor cores as bf16 hi + lo pairs; the state is kept in
-// fp32 registers.  No initial or final state and no segments.
+// fp32 registers.  Carried states as in the T_B = 128 kernel (ws::Role): an
+// initial state (forward: before position 0; reverse: entering at position
+// T-1, so the reverse scan's first block weighs it by lambda^(n-1-r) over its
+// n rows and decays it by lambda^(n-1)), read transposed with init_t; the
+// final state (forward: after position T-1, the last block's update using its
+// true row count; reverse: lambda times the state at position 0).  No
+// segments.
 #pragma once
 #include "ptx_sm100.cuh"
 #include "scan_ws_sm100.cuh"
@@ -42,7 +48,7 @@ constexpr int kThreads = 256;
 constexpr int kDC = 64;  // value columns per CTA
 
 struct Params {
-    ws::Role role[3];    // maps, output and direction of each role (init, fin, colf unused)
+    ws::Role role[3];    // maps, output, direction and carried states of each role (colf unused)
     const float* decay;  // [H]
     int* status;         // device status word
     int H, T, nroles, bthd;
@@ -236,8 +242,8 @@ la2_scan_blk(const __grid_constant__ Params p)
             st_shared_v4(sLo + off, l[0], l[1], l[2], l[3]);
         }
     };
-    // W <- f W + dW (dW in TMEM at t): the fp32 state in registers, its hi/lo
-    // pair to sw (the next A W MMA's operand)
+    // W <- f W + dW (dW in TMEM at t; d = null: W <- f W): the fp32 state in
+    // registers, its hi/lo pair to sw (the next A W MMA's operand)
     auto update_w = [&](uint32_t t, float f, uint32_t sw) {
         float d[32];
         tmem_ld32(t + lane_off + 32 * hf, d);
@@ -255,6 +261,28 @@ la2_scan_blk(const __grid_constant__ Params p)
                     wreg[u] = w.x;
                     wreg[u + 1] = w.y;
                     split_pack2v(w, h[z], l[z]);
+                }
+                st_shared_v4(sw + o0, h[0], h[1], h[2], h[3]);
+                st_shared_v4(sw + o1, h[4], h[5], h[6], h[7]);
+                st_shared_v4(sw + L::kWsz + o0, l[0], l[1], l[2], l[3]);
+                st_shared_v4(sw + L::kWsz + o1, l[4], l[5], l[6], l[7]);
+            }
+        }
+    };
+    // W <- f W without a dW (the hi/lo pair rewritten from the registers)
+    auto scale_w = [&](float f, uint32_t sw) {
+        if (owns_w_row) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int col = 32 * hf + 16 * hh;
+                const uint32_t o0 = ws::sw128(wrow, col >> 3), o1 = ws::sw128(wrow, (col >> 3) + 1);
+                uint32_t h[8], l[8];
+#pragma unroll
+                for (int z = 0; z < 8; ++z) {
+                    const int u = 16 * hh + 2 * z;
+                    wreg[u] *= f;
+                    wreg[u + 1] *= f;
+                    split_pack2v(make_float2(wreg[u], wreg[u + 1]), h[z], l[z]);
                 }
                 st_shared_v4(sw + o0, h[0], h[1], h[2], h[3]);
                 st_shared_v4(sw + o1, h[4], h[5], h[6], h[7]);
@@ -302,14 +330,34 @@ la2_scan_blk(const __grid_constant__ Params p)
         tc_fence_after();
     };
 
+    // the initial state of this CTA's 64 value columns: row wrow, columns
+    // 64 cs + 32 hf + u of [DA][dc] (or of [dc][DA] with init_t)
+    if (R.init != nullptr) {
+        if (owns_w_row) {
+            const float* w0 = R.init + static_cast<size_t>(bh) * (DA * p.dc);
+            const int c0 = kDC * cs + 32 * hf;
+#pragma unroll
+            for (int u = 0; u < 32; ++u)
+                wreg[u] = R.init_t ? w0[static_cast<size_t>(c0 + u) * DA + wrow]
+                                   : w0[static_cast<size_t>(wrow) * p.dc + c0 + u];
+        }
+        scale_w(1.f, sW);
+        sync_tmem();
+    }
+
     if constexpr (TB == 256) {
         const uint32_t tS0 = tmem, tS1 = tmem + 128, tS2 = tmem + 256, tX0 = tmem + 384, tX1 = tmem + 448;
         const uint32_t tD = tmem;  // dW reuses S_00's columns once P_00 C_0 is done
         const int nblk = (nb + 1) / 2;
         const uint32_t sB0 = sB, sB1 = sB + L::kAsz, sC0 = sC, sC1 = sC + L::kCsz;
+        // rows of the sequence's last block (1..256): the forward scan's last
+        // update and the reverse scan's first block use them
+        const int nrow = T - 256 * (nblk - 1);
         for (int step = 0; step < nblk && ok; ++step) {
             const int m = dir > 0 ? step : nblk - 1 - step;
             const int u0 = dir > 0 ? 2 * m : 2 * m + 1, u1 = dir > 0 ? 2 * m + 1 : 2 * m;
+            const bool lastf = dir > 0 && step == nblk - 1;  // state after position T-1
+            const bool firstr = dir < 0 && step == 0;        // state entering at position T-1
             // B, C of both tiles and A of u0 (tiles past T read as zero)
             if (tid == 0) {
                 mbar_arrive_expect_tx(barT, 3 * L::kAsz + 2 * L::kCsz);
@@ -348,8 +396,11 @@ la2_scan_blk(const __grid_constant__ Params p)
             make_p(tS0, diag);
             make_p(tS1, off);
             make_p(tS2, diag);
-            scale_x(tX0, dir > 0 ? pw[r + 1] : pw[128 - r]);
-            scale_x(tX1, dir > 0 ? pw[128 + r + 1] : pw[256 - r]);
+            // rows of the reverse scan's first block weigh the entering state by
+            // lambda^(n-1-j) (block row j < n), not lambda^(256-j)
+            scale_x(tX0, dir > 0 ? pw[r + 1]
+                                 : (firstr ? (128 + r < nrow ? pw[nrow - 1 - 128 - r] : 0.f) : pw[128 - r]));
+            scale_x(tX1, dir > 0 ? pw[128 + r + 1] : (firstr ? (r < nrow ? pw[nrow - 1 - r] : 0.f) : pw[256 - r]));
             sync_tmem();
             if (tid == 0) {
                 mma_pc(tX0, tS0, sC0, false);
@@ -362,8 +413,10 @@ la2_scan_blk(const __grid_constant__ Params p)
             store_x(tX0, 0u, 0.f, u0);
             store_x(tX1, 0u, 0.f, u1);
             // dW over the block: rows of u0 weigh lambda^(255-c) (fwd) or
-            // lambda^(128+c) (rev), rows of u1 lambda^(127-c) resp. lambda^c
-            split_b(sB0, dir > 0 ? pw[255 - r] : pw[128 + r]);
+            // lambda^(128+c) (rev), rows of u1 lambda^(127-c) resp. lambda^c;
+            // the forward scan's last block, n rows, lambda^(n-1-j) for block
+            // row j < n and lambda^n for the old state
+            split_b(sB0, dir > 0 ? (lastf ? (r < nrow ? pw[nrow - 1 - r] : 0.f) : pw[255 - r]) : pw[128 + r]);
             sync_tmem();
             if (tid == 0) {
                 mma_dw(tD, sB0, sC0, 0, 8, true);
@@ -371,7 +424,7 @@ la2_scan_blk(const __grid_constant__ Params p)
             }
             wait_m(86);
             if (!ok) break;
-            split_b(sB1, dir > 0 ? pw[127 - r] : pw[r]);
+            split_b(sB1, dir > 0 ? (lastf ? (128 + r < nrow ? pw[nrow - 1 - 128 - r] : 0.f) : pw[127 - r]) : pw[r]);
             sync_tmem();
             if (tid == 0) {
                 mma_dw(tD, sB1, sC1, 0, 8, false);
@@ -379,16 +432,30 @@ la2_scan_blk(const __grid_constant__ Params p)
             }
             wait_m(87);
             if (!ok) break;
-            update_w(tD, pw[256], sW);
+            update_w(tD, lastf ? pw[nrow] : (firstr ? pw[nrow - 1] : pw[256]), sW);
             sync_tmem();
         }
     } else {
         const uint32_t tS = tmem, tX = tmem + 128, tY1 = tmem + 192, tY2 = tmem + 256, tD = tmem + 320;
+        const int nlast = T - 128 * (nb - 1);  // rows of the last 128-row tile
         for (int step = 0; step < nb && ok; ++step) {
             const int tile = dir > 0 ? step : nb - 1 - step;
             // the two 64-row blocks in scan order: f first, then s (time
             // blocks 0 = rows 0..63, 1 = rows 64..127)
             const int bf = dir > 0 ? 0 : 1;
+            // rows of f and s that hold positions of the sequence: all 64,
+            // except in the forward scan's last tile (the state after position
+            // T-1) and the reverse scan's first tile (the state entering at T-1)
+            const bool lastf = dir > 0 && step == nb - 1;
+            const bool firstr = dir < 0 && step == 0;
+            int nf = 64, nsb = 64;
+            if (lastf) {
+                nf = min(nlast, 64);
+                nsb = max(nlast - 64, 0);
+            } else if (firstr) {
+                nf = max(nlast - 64, 0);
+                nsb = min(nlast, 64);
+            }
             if (tid == 0) {
                 mbar_arrive_expect_tx(barT, 2 * L::kAsz + L::kCsz);
                 load_tile(sB, &R.tb, tile, DA, 0);
@@ -410,7 +477,10 @@ la2_scan_blk(const __grid_constant__ Params p)
                 return dir > 0 ? (c <= rr ? pw[rr - c] : 0.f) : (c >= rr ? pw[c - rr] : 0.f);
             };
             make_p(tS, diag64);
-            split_b(sB, dir > 0 ? pw[63 - (r & 63)] : pw[r & 63]);
+            // forward key weights lambda^(n-1-r') over the block's n rows (n = 64
+            // but in the last tile); reverse lambda^r'
+            const int nkb = ((r >> 6) == bf) ? nf : nsb;
+            split_b(sB, dir > 0 ? ((r & 63) < nkb ? pw[nkb - 1 - (r & 63)] : 0.f) : pw[r & 63]);
             sync_tmem();
             if (tid == 0) {
                 mma_pc(tX, tS, sC, true);
@@ -419,7 +489,11 @@ la2_scan_blk(const __grid_constant__ Params p)
             }
             wait_m(93);
             if (!ok) break;
-            update_w(tD, pw[64], sW2);  // W_mid, the state after block f
+            // W_mid, the state after block f: lambda^n_f W + dW_f forward; in
+            // the reverse scan's first tile the entering state decays from
+            // position T-1 to the start of f (lambda^(n_f-1)), or passes to s
+            // unchanged when f holds no position
+            update_w(tD, dir > 0 ? pw[nf] : (firstr ? pw[max(nf - 1, 0)] : pw[64]), sW2);
             sync_tmem();
             if (tid == 0) {
                 mma_xw(tY2, sW2);
@@ -431,12 +505,27 @@ la2_scan_blk(const __grid_constant__ Params p)
             // rows of f read W, rows of s W_mid, each with its block-local
             // weight lambda^(r'+1) (fwd) or lambda^(64-r') (rev)
             const int rb = r & 63;
-            const float wx = dir > 0 ? pw[rb + 1] : pw[64 - rb];
             const bool in_f = (r >> 6) == bf;
+            float wx = dir > 0 ? pw[rb + 1] : pw[64 - rb];
+            if (firstr) {  // the entering state: lambda^(n-1-r') over the n rows that hold it
+                if (in_f) wx = rb < nf ? pw[nf - 1 - rb] : 0.f;
+                else if (nf == 0) wx = rb < nsb ? pw[nsb - 1 - rb] : 0.f;
+            }
             store_x(tX, in_f ? tY1 : tY2, wx, tile);
-            update_w(tD, pw[64], sW);   // W after block s
+            // W after block s
+            update_w(tD, dir > 0 ? pw[nsb] : ((firstr && nf == 0) ? pw[max(nsb - 1, 0)] : pw[64]), sW);
             sync_tmem();
         }
+    }
+
+    // the final state: forward, the state after position T-1; reverse, lambda
+    // times the state at position 0
+    if (ok && R.fin != nullptr && owns_w_row) {
+        float* fin = R.fin + static_cast<size_t>(bh) * (DA * p.dc) + static_cast<size_t>(wrow) * p.dc + kDC * cs +
+                     32 * hf;
+        const float fs = dir > 0 ? 1.f : lam;
+#pragma unroll
+        for (int u = 0; u < 32; ++u) fin[u] = fs * wreg[u];
     }
 
     // tear-down

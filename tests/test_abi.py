@@ -243,7 +243,7 @@ def test_norm_workspace_and_arguments(lib):
 
 
 @pytest.mark.parametrize("block", [64, 256])
-def test_bf16_other_blocks_need_no_workspace_and_reject_states(lib, block):
+def test_bf16_other_blocks_need_no_workspace(lib, block):
     assert la2.la2_workspace_bytes(1, 2, 65536, 128, 128, block, la2.LA2_DTYPE_BF16, 0) == 0
     assert la2.la2_workspace_bytes(1, 2, 65536, 128, 128, block, la2.LA2_DTYPE_BF16, 1) == 0
     plan = la2.la2_plan_info(1, 2, 1000, 128, 64, block, is_bwd=True)

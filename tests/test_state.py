@@ -134,3 +134,46 @@ def test_no_init_matches_la2_fwd(la2mod):
     b, _ = la2mod.la2_fwd_state(q, k, v, lam, None)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+# ------------------------------------- bf16 with T_B = 64 and 256 (la2_scan_blk)
+
+@pytest.mark.parametrize("block", [64, 256])
+@pytest.mark.parametrize("T", [1, 63, 65, 128, 129, 255, 257, 700])
+@pytest.mark.parametrize("d,e", [(128, 128), (64, 64), (64, 128), (128, 64)])
+def test_bf16_other_blocks_state_in_out(la2mod, oracle_mod, block, T, d, e):
+    """The phase-serial kernel from init_state, the final state from its last
+    block's true row count (every T mod block case), fp32 state in registers."""
+    x = I.make_inputs(2, 3, T, d, e, "bf16", seed=T + 3 * d + e + block)
+    init = _init_state(2, 3, d, e, seed=T + block)
+    out, fin = _run(la2mod, x, init, block=block)
+    ro, rs = _ref(oracle_mod, x, init)
+    eo, es = _err(out, ro), _err(fin, rs)
+    assert torch.isfinite(out).all() and torch.isfinite(fin).all()
+    assert eo < 1e-3 and es < 1e-3, (eo, es)  # hi + lo operands, fp32 state
+
+
+@pytest.mark.parametrize("block", [64, 256])
+@pytest.mark.parametrize("cut", [100, 256])
+def test_other_blocks_pieces_equal_whole(la2mod, oracle_mod, block, cut):
+    T = 777
+    x = I.make_inputs(2, 4, T, 128, 128, "bf16", seed=cut + block)
+    first = {n: x[n][:, :, :cut].contiguous() for n in ("q", "k", "v")}
+    second = {n: x[n][:, :, cut:].contiguous() for n in ("q", "k", "v")}
+    first["lam"] = second["lam"] = x["lam"]
+    o1, s1 = _run(la2mod, first, None, block=block)
+    o2, s2 = _run(la2mod, second, s1.cpu(), block=block)
+    ro, rs = _ref(oracle_mod, x, None)
+    assert _err(torch.cat([o1, o2], dim=2), ro) < 1e-3
+    assert _err(s2, rs) < 1e-3
+
+
+@pytest.mark.parametrize("block", [64, 256])
+def test_other_blocks_state_decays(la2mod, oracle_mod, block):
+    """lambda from 2^-20 to 1 in one launch, with a state in and out."""
+    x = I.make_inputs(1, 7, 333, 128, 128, "bf16", seed=40 + block)
+    x["lam"] = torch.tensor([2.0 ** -20, 0.3, 0.8, 0.9, 0.99, 0.999, 1.0], dtype=torch.float32)
+    init = _init_state(1, 7, 128, 128, seed=41)
+    out, fin = _run(la2mod, x, init, block=block)
+    ro, rs = _ref(oracle_mod, x, init)
+    assert _err(out, ro) <= TOL["bf16"] and _err(fin, rs) <= TOL["bf16"]

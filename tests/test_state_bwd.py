@@ -179,3 +179,46 @@ def test_no_states_match_la2_bwd_bitwise(la2mod, d, e):
     assert b[3] is None
     for u, w in zip(a, b[:3]):
         assert torch.equal(u, w)
+
+
+# ------------------------------------- bf16 with T_B = 64 and 256 (la2_scan_blk)
+
+@pytest.mark.parametrize("block", [64, 256])
+@pytest.mark.parametrize("T", [1, 63, 65, 128, 129, 255, 257, 700])
+@pytest.mark.parametrize("d,e", [(128, 128), (64, 64), (64, 128), (128, 64)])
+def test_bf16_other_blocks_bwd_state(la2mod, oracle_mod, block, T, d, e):
+    """S0 read transposed by the dq scan, G entering at position T-1 in the dk
+    and dv scans' first (ragged) block, dS0 from the dv scan's final state."""
+    x = I.make_inputs(2, 3, T, d, e, "bf16", seed=T + 5 * d + e + block)
+    errs = _check(la2mod, oracle_mod, x, _state(2, 3, d, e, T), _state(2, 3, d, e, T + 1), TOL["bf16"],
+                  block)
+    assert max(errs.values()) < 1e-3, errs
+
+
+@pytest.mark.parametrize("block", [64, 256])
+@pytest.mark.parametrize("which", ["s0", "g"])
+def test_other_blocks_bwd_one_state_only(la2mod, oracle_mod, block, which):
+    x = I.make_inputs(1, 4, 333, 128, 128, "bf16", seed=13 + block)
+    s = _state(1, 4, 128, 128, 8)
+    _check(la2mod, oracle_mod, x, s if which == "s0" else None, s if which == "g" else None,
+           TOL["bf16"], block)
+
+
+@pytest.mark.parametrize("block", [64, 256])
+def test_other_blocks_bwd_pieces_equal_whole(la2mod, oracle_mod, block):
+    """The backward of the second piece from the carried S0 and the incoming G,
+    then of the first piece with the second's dS0 as its G: the whole
+    sequence's gradients."""
+    T, cut = 600, 257
+    x = I.make_inputs(1, 3, T, 128, 128, "bf16", seed=50 + block)
+    lam64 = np.broadcast_to(x["lam"].numpy().astype(np.float64)[None, :], (1, 3))
+    part = [{n: x[n][:, :, a:b].contiguous() for n in ("q", "k", "v", "do")} for a, b in ((0, cut), (cut, T))]
+    for pc in part:
+        pc["lam"] = x["lam"]
+    _, s1 = oracle_mod.forward_state(part[0]["q"], part[0]["k"], part[0]["v"], lam64, None)
+    g2 = _gpu(la2mod, part[1], torch.from_numpy(s1).float(), None, block)
+    g1 = _gpu(la2mod, part[0], None, g2[3].cpu(), block)
+    want = _ref(oracle_mod, x, None, None)
+    for i, n in enumerate(NAMES[:3]):
+        got = torch.cat([g1[i], g2[i]], dim=2)
+        assert _err(got, want[i]) < 1e-3, n
