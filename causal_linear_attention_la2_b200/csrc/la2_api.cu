@@ -415,14 +415,13 @@ la2_status launch_bf16_ws(const RoleDesc* roles, int n, const float* decay, int 
 
 // T_B = 64 or 256 on bf16 inputs (scan_blk_sm100.cuh): one CTA per
 // (sequence, role, 64 value columns), no segments, no workspace; carried
-// states as in the T_B = 128 kernel, no per-position factor (colf).
+// states and the per-position factor (colf) as in the T_B = 128 kernel.
 la2_status launch_bf16_blk(const RoleDesc* roles, int n, const float* decay, int B, int H, int T,
                            int block, bool bthd, int* status, cudaStream_t stream, bool xbf16) {
     la2::blk::Params p;
     std::memset(&p, 0, sizeof(p));
     const int da = roles[0].da, dc = roles[0].dc;
     for (int r = 0; r < n; ++r) {
-        if (roles[r].colf) return LA2_ERR_UNSUPPORTED;  // the normalised form: T_B = 128 only
         if (!make_map(&p.role[r].ta, roles[r].a, B, H, T, da, bthd) ||
             !make_map(&p.role[r].tb, roles[r].b, B, H, T, da, bthd) ||
             !make_map(&p.role[r].tc, roles[r].c, B, H, T, dc, bthd))
@@ -432,6 +431,7 @@ la2_status launch_bf16_blk(const RoleDesc* roles, int n, const float* decay, int
         p.role[r].init = roles[r].init;
         p.role[r].fin = roles[r].fin;
         p.role[r].init_t = roles[r].init_t;
+        p.role[r].colf = roles[r].colf;
     }
     p.decay = decay;
     p.status = status;
@@ -539,7 +539,7 @@ la2_status run_roles(const RoleDesc* roles, int n, const float* decay, int B, in
         return launch_f32(roles, n, decay, B, H, T, block, bthd, stream);
     }
     if (block != la2::ws::kTB) {
-        if (norm || hold.flag) return LA2_ERR_UNSUPPORTED;
+        if (hold.flag) return LA2_ERR_UNSUPPORTED;  // the self-test runs the T_B = 128 kernel
         return for_role_groups(roles, n, [&](const RoleDesc* g, int m) {
             return launch_bf16_blk(g, m, decay, B, H, T, block, bthd, status, stream, xbf16);
         });

@@ -35,8 +35,8 @@
 // T-1, so the reverse scan's first block weighs it by lambda^(n-1-r) over its
 // n rows and decays it by lambda^(n-1)), read transposed with init_t; the
 // final state (forward: after position T-1, the last block's update using its
-// true row count; reverse: lambda times the state at position 0).  No
-// segments.
+// true row count; reverse: lambda times the state at position 0); and the
+// per-position factor colf of the normalised form.  No segments.
 #pragma once
 #include "ptx_sm100.cuh"
 #include "scan_ws_sm100.cuh"
@@ -48,7 +48,7 @@ constexpr int kThreads = 256;
 constexpr int kDC = 64;  // value columns per CTA
 
 struct Params {
-    ws::Role role[3];    // maps, output, direction and carried states of each role (colf unused)
+    ws::Role role[3];    // maps, output, direction, carried states and per-position factor
     const float* decay;  // [H]
     int* status;         // device status word
     int H, T, nroles, bthd;
@@ -205,9 +205,18 @@ la2_scan_blk(const __grid_constant__ Params p)
             mma_bf16_ss(t, desc_add(dl, k * 2048), cd, kIdW, 1u);
         }
     };
-    // P from the S block at t: weight(row, col) per element (0 off the mask),
-    // stored back as [hi (8 columns) | lo (8 columns)] per 16 columns
-    auto make_p = [&](uint32_t t, auto weight) {
+    // the per-position factor f on the summed position (the normalised form's
+    // backward; null elsewhere): x_t = sum_s lambda^|t-s| (a_t . b_s) f_s c_s,
+    // applied to P's columns and to the state-update weights of the keys
+    const float* colf = R.colf ? R.colf + static_cast<size_t>(bh) * T : nullptr;
+    auto f_at = [&](int tile, int row) -> float {
+        const int t = tile * 128 + row;
+        return t < T ? __ldg(colf + t) : 0.f;
+    };
+    // P from the S block at t, whose columns are the keys of tile ktile:
+    // weight(row, col) per element (0 off the mask), times f of the key with
+    // colf, stored back as [hi (8 columns) | lo (8 columns)] per 16 columns
+    auto make_p = [&](uint32_t t, int ktile, auto weight) {
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
             const int col0 = 64 * hf + 32 * cc;
@@ -215,6 +224,10 @@ la2_scan_blk(const __grid_constant__ Params p)
             tmem_ld32(t + lane_off + col0, sv);
 #pragma unroll
             for (int u = 0; u < 32; ++u) sv[u] *= weight(r, col0 + u);
+            if (colf) {
+#pragma unroll
+                for (int u = 0; u < 32; ++u) sv[u] *= f_at(ktile, col0 + u);
+            }
             uint32_t pk[32];
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2)
@@ -225,9 +238,11 @@ la2_scan_blk(const __grid_constant__ Params p)
             tmem_st32u(t + lane_off + col0, pk);
         }
     };
-    // hi(w_s B) in place and lo(w_s B) into sLo, row r's weight w (this
-    // thread: half hf of the row's 16-byte chunks)
-    auto split_b = [&](uint32_t sb, float w) {
+    // hi(w_s B) in place and lo(w_s B) into sLo, row r's weight w, times f
+    // of that key (tile ktile) with colf (this thread: half hf of the row's
+    // 16-byte chunks)
+    auto split_b = [&](uint32_t sb, int ktile, float w) {
+        if (colf) w *= f_at(ktile, r);
 #pragma unroll
         for (int k = 0; k < DA / 16; ++k) {
             const int chunk = hf * (DA / 16) + k;
@@ -393,9 +408,9 @@ la2_scan_blk(const __grid_constant__ Params p)
                 return dir > 0 ? (c <= rr ? pw[rr - c] : 0.f) : (c >= rr ? pw[c - rr] : 0.f);
             };
             auto off = [&](int rr, int c) -> float { return dir > 0 ? pw[128 + rr - c] : pw[128 + c - rr]; };
-            make_p(tS0, diag);
-            make_p(tS1, off);
-            make_p(tS2, diag);
+            make_p(tS0, u0, diag);
+            make_p(tS1, u0, off);
+            make_p(tS2, u1, diag);
             // rows of the reverse scan's first block weigh the entering state by
             // lambda^(n-1-j) (block row j < n), not lambda^(256-j)
             scale_x(tX0, dir > 0 ? pw[r + 1]
@@ -416,7 +431,7 @@ la2_scan_blk(const __grid_constant__ Params p)
             // lambda^(128+c) (rev), rows of u1 lambda^(127-c) resp. lambda^c;
             // the forward scan's last block, n rows, lambda^(n-1-j) for block
             // row j < n and lambda^n for the old state
-            split_b(sB0, dir > 0 ? (lastf ? (r < nrow ? pw[nrow - 1 - r] : 0.f) : pw[255 - r]) : pw[128 + r]);
+            split_b(sB0, u0, dir > 0 ? (lastf ? (r < nrow ? pw[nrow - 1 - r] : 0.f) : pw[255 - r]) : pw[128 + r]);
             sync_tmem();
             if (tid == 0) {
                 mma_dw(tD, sB0, sC0, 0, 8, true);
@@ -424,7 +439,8 @@ la2_scan_blk(const __grid_constant__ Params p)
             }
             wait_m(86);
             if (!ok) break;
-            split_b(sB1, dir > 0 ? (lastf ? (128 + r < nrow ? pw[nrow - 1 - 128 - r] : 0.f) : pw[127 - r]) : pw[r]);
+            split_b(sB1, u1,
+                    dir > 0 ? (lastf ? (128 + r < nrow ? pw[nrow - 1 - 128 - r] : 0.f) : pw[127 - r]) : pw[r]);
             sync_tmem();
             if (tid == 0) {
                 mma_dw(tD, sB1, sC1, 0, 8, false);
@@ -476,11 +492,11 @@ la2_scan_blk(const __grid_constant__ Params p)
                 if ((rr >> 6) != (c >> 6)) return 0.f;
                 return dir > 0 ? (c <= rr ? pw[rr - c] : 0.f) : (c >= rr ? pw[c - rr] : 0.f);
             };
-            make_p(tS, diag64);
+            make_p(tS, tile, diag64);
             // forward key weights lambda^(n-1-r') over the block's n rows (n = 64
             // but in the last tile); reverse lambda^r'
             const int nkb = ((r >> 6) == bf) ? nf : nsb;
-            split_b(sB, dir > 0 ? ((r & 63) < nkb ? pw[nkb - 1 - (r & 63)] : 0.f) : pw[r & 63]);
+            split_b(sB, tile, dir > 0 ? ((r & 63) < nkb ? pw[nkb - 1 - (r & 63)] : 0.f) : pw[r & 63]);
             sync_tmem();
             if (tid == 0) {
                 mma_pc(tX, tS, sC, true);

@@ -172,7 +172,7 @@ int la2_plan_info(int B, int H, int T, int d, int e, int block, la2_dtype dtype,
  * segments to fill the GPU); block = 64 and 256 run a phase-serial tcgen05
  * kernel with the state carried across 64- or 256-row blocks in fp32
  * registers (one CTA per sequence and 64 value columns, no segments; carried
- * states as with block = 128; the normalised form is LA2_ERR_UNSUPPORTED).  out must not alias an input.  workspace: device
+ * states and the normalised form as with block = 128).  out must not alias an input.  workspace: device
  * memory, 256-byte aligned, of at least la2_workspace_bytes(..., 0) bytes
  * (LA2_ERR_WORKSPACE otherwise), not used concurrently by another call.
  */

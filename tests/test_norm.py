@@ -161,3 +161,22 @@ def test_norm_full_size_15b(la2mod, oracle_mod):
     w = I.WORKLOADS["tnl15b"]
     x = _inputs(w.B, w.H, w.T, w.d, w.e, w.dtype, seed=0)
     _check(la2mod, oracle_mod, x, TOL[w.dtype], heads=([0, 1, 1], [0, 20, 39]))
+
+
+# ------------------------------------- bf16 with T_B = 64 and 256 (la2_scan_blk)
+
+@pytest.mark.parametrize("block", [64, 256])
+@pytest.mark.parametrize("T", [1, 65, 129, 257, 700])
+@pytest.mark.parametrize("d,e", [(128, 128), (64, 64), (64, 128), (128, 64)])
+def test_norm_bf16_other_blocks(la2mod, oracle_mod, block, T, d, e):
+    """The numerator scans of the phase-serial kernel, the backward's dk and dv
+    with the factor 1 / den on the summed position."""
+    _check(la2mod, oracle_mod, _inputs(2, 3, T, d, e, "bf16", seed=T + d + e + block), TOL["bf16"],
+           block=block)
+
+
+@pytest.mark.parametrize("block", [64, 256])
+def test_norm_other_blocks_decays(la2mod, oracle_mod, block):
+    x = _inputs(1, 5, 700, 128, 128, "bf16", seed=4 + block)
+    x["lam"] = torch.tensor([2.0 ** -20, 0.3, 0.9, 0.999, 1.0], dtype=torch.float32)
+    _check(la2mod, oracle_mod, x, TOL["bf16"], block=block)
