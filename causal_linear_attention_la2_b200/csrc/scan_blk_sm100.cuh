@@ -165,6 +165,12 @@ la2_scan_blk(const __grid_constant__ Params p)
         for (int gg = 0; gg < cols / 64; ++gg)
             ws::load_box(dst + gg * 16384, map, barT, x0 + gg * 64, tile * 128, bh, p.H, p.bthd);
     };
+    // an L2 prefetch of a tile that a later phase loads (the phases do not
+    // overlap, so without it every load would wait for HBM)
+    auto prefetch_tile = [&](const CUtensorMap* map, int tile, int cols, int x0) {
+        if (tile < 0 || tile * 128 >= T) return;
+        for (int gg = 0; gg < cols / 64; ++gg) ws::prefetch_box(map, x0 + gg * 64, tile * 128, bh, p.H, p.bthd);
+    };
     // S (128 x 128, fp32) = A B^T into TMEM column t
     auto mma_s = [&](uint32_t t, uint32_t sb) {
         const uint64_t db = sdesc_sw128(sb, 16, 1024);
@@ -381,6 +387,16 @@ la2_scan_blk(const __grid_constant__ Params p)
                 load_tile(sC0, &R.tc, u0, kDC, kDC * cs);
                 load_tile(sC1, &R.tc, u1, kDC, kDC * cs);
                 load_tile(sA, &R.ta, u0, DA, 0);
+                // A of u1 (loaded after the first MMAs) and the next block's tiles
+                prefetch_tile(&R.ta, u1, DA, 0);
+                if (step + 1 < nblk) {
+                    const int m2 = dir > 0 ? step + 1 : nblk - 2 - step;
+                    for (int uu = 2 * m2; uu < 2 * m2 + 2; ++uu) {
+                        prefetch_tile(&R.tb, uu, DA, 0);
+                        prefetch_tile(&R.tc, uu, kDC, kDC * cs);
+                        prefetch_tile(&R.ta, uu, DA, 0);
+                    }
+                }
             }
             wait_t(81);
             if (tid == 0) {
@@ -477,6 +493,11 @@ la2_scan_blk(const __grid_constant__ Params p)
                 load_tile(sB, &R.tb, tile, DA, 0);
                 load_tile(sC, &R.tc, tile, kDC, kDC * cs);
                 load_tile(sA, &R.ta, tile, DA, 0);
+                // the next tile's B, C and A
+                const int nt = dir > 0 ? tile + 1 : tile - 1;
+                prefetch_tile(&R.tb, nt, DA, 0);
+                prefetch_tile(&R.tc, nt, kDC, kDC * cs);
+                prefetch_tile(&R.ta, nt, DA, 0);
             }
             wait_t(91);
             if (tid == 0) {
