@@ -159,12 +159,16 @@ struct RingCfg {
     // DC = 64 (kOwnD): X += P C (one TMEM buffer), X_inter = A W (two) and
     // dW (one) are separate accumulators, and the epilogue forms
     // w_x X_inter + X; X += P C then never waits for the state, and X_inter
-    // of tile s never waits for the output of tile s-1.  DC = 128: X (two
-    // buffers) holds A W, scaled by w_x in TMEM, then P C; dW borrows the X
-    // buffer of the next tile.
+    // of tile s never waits for the output of tile s-1.  DC = 128 (kWT): X
+    // (one buffer) holds A W, scaled by w_x in TMEM, then P C; the state W
+    // itself lives in TMEM in fp32 (128 columns): the epilogue writes
+    // lambda^T_B W back after reading W for its hi/lo pair, and dW of the
+    // next tile accumulates onto it, so W <- lambda^T_B W + dW costs no
+    // shared-memory read of the state and dW never waits for the output.
     static constexpr bool kOwnD = DC == 64;
+    static constexpr bool kWT = DC == 128;
     static constexpr int ND = 1;                             // dW accumulators (own-D)
-    static constexpr int NX = kOwnD ? 1 : 2;                 // X accumulators in TMEM
+    static constexpr int NX = 1;                             // X accumulators in TMEM
     static constexpr int NXW = kOwnD ? 2 : NX;               // XW_DONE barriers
     static constexpr int NXS = kOwnD ? 0 : NX;               // XS barriers (scaled in TMEM)
     static constexpr int NXI = kOwnD ? 2 : 0;                // X_inter buffers (EMPTY_XI: read out)
@@ -440,20 +444,18 @@ la2_scan_ws(const __grid_constant__ Params p)
         named_barrier_sync(1, kThreads - 128);
     }
     // TMEM: S / P in two buffers (128 columns each), X in NX buffers (DC each),
-    // then (DC = 64) X_inter and ND dW buffers; otherwise dW of tile s goes to the X buffer of
-    // tile s+1: X of tile s-1 has been read out of it, and X of tile s+1 is not
-    // issued before the state update has read dW.
+    // then (DC = 64) NXI X_inter buffers, then ND dW buffers (DC = 128: the
+    // fp32 state, onto which dW accumulates).
     auto tS = [&](int b) { return tmem + static_cast<uint32_t>(b * 128); };
     auto tX = [&](int b) { return tmem + 256 + static_cast<uint32_t>(b * DC); };
     auto tXI = [&](int s) {  // X_inter of step s (DC = 64)
         return tmem + 256 + static_cast<uint32_t>((Q::NX + s % (Q::NXI > 0 ? Q::NXI : 1)) * DC);
     };
+    // dW (DC = 64) or the fp32 state W that dW accumulates onto (DC = 128)
     auto tD = [&](int s) {
-        return Q::kOwnD ? tmem + 256 + static_cast<uint32_t>((Q::NX + Q::NXI) * DC + (s % Q::ND) * DC)
-                        : tX((s + 1) % Q::NX);
+        return tmem + 256 + static_cast<uint32_t>((Q::NX + Q::NXI) * DC + (s % Q::ND) * DC);
     };
-    static_assert(256 + Q::NX * DC + (Q::kOwnD ? (Q::NXI + Q::ND) * DC : 0) <= static_cast<int>(kTmemCols),
-                  "TMEM columns");
+    static_assert(256 + (Q::NX + Q::NXI + Q::ND) * DC <= static_cast<int>(kTmemCols), "TMEM columns");
     auto tile_of = [&](int step) { return dir > 0 ? s0 + step : nb - 1 - (s0 + step); };
     // fp32 state slot of segment gg of this (sequence, role)
     auto seg_slot = [&](int gg) {
@@ -698,17 +700,14 @@ la2_scan_ws(const __grid_constant__ Params p)
                     if (!wait_bar<Q::kTf32>(bar(Q::BS + sb), full_par(s, Q::NB), abort_flag, p.status, 33)) break;
                     if (!wait_bar<Q::kTf32>(bar(Q::FULL_C + sc), full_par(s, Q::NC), abort_flag, p.status, 34)) break;
                 }
-                if (Q::kOwnD) {
+                if constexpr (Q::kWT) {
+                    // the state holds lambda(s) W_s: written by the epilogue's set-up
+                    // (s = 0) or by the update after tile s-1
+                    if (!wait_bar<Q::kTf32>(bar(Q::EMPTY_D), full_par(s, 1), abort_flag, p.status, 36)) break;
+                } else if (s >= Q::ND && !wait_bar<Q::kTf32>(bar(Q::EMPTY_D + s % Q::ND), empty_par(s, Q::ND),
+                                                             abort_flag, p.status, 35)) {
                     // the update after tile s - ND has read this dW buffer
-                    if (s >= Q::ND && !wait_bar<Q::kTf32>(bar(Q::EMPTY_D + s % Q::ND), empty_par(s, Q::ND),
-                                                abort_flag, p.status, 35))
-                        break;
-                } else {
-                    // X buffer (s+1) % 2 has been read out after tile s-1
-                    static_assert(Q::kOwnD || Q::NX == 2, "dW shares the X buffers only with NX = 2");
-                    if (s >= 1 && !wait_bar<Q::kTf32>(bar(Q::EMPTY_X + ((s + 1) % Q::NX)), full_par(s - 1, Q::NX),
-                                            abort_flag, p.status, 36))
-                        break;
+                    break;
                 }
                 LA2_TR(8, s);
                 tc_fence_after();
@@ -728,7 +727,7 @@ la2_scan_ws(const __grid_constant__ Params p)
 #pragma unroll
                     for (int k = 0; k < kTB / 16; ++k) {
                         const uint64_t cdesc = desc_add(dc, k * 2048);
-                        mma_bf16_ss_w(dt, desc_add(db, k * 2048), cdesc, kIdW, k > 0, leader);
+                        mma_bf16_ss_w(dt, desc_add(db, k * 2048), cdesc, kIdW, (Q::kWT || k > 0) ? 1u : 0u, leader);
                         mma_bf16_ss_w(dt, desc_add(dl, k * 2048), cdesc, kIdW, 1, leader);
                     }
                     mma_commit_w(bar(Q::D_DONE + (s % Q::ND)), leader);
@@ -977,7 +976,15 @@ la2_scan_ws(const __grid_constant__ Params p)
         // with f_i = lambda^(T_B n_i) (n_i tiles in segment i: L, except for
         // segment 0, which ends at step L - ph) and W_in(0) the given initial
         // state (or 0), as its hi/lo bf16 pair in W buffer 0
-        if ((sj > 0 || R.init != nullptr) && owns_w_row) {
+        // the state's old-value factor before the dW of step s: lambda^T_B,
+        // lambda^n for the forward scan's last (n-row) tile, lambda^(n-1) for the
+        // reverse scan's first tile (an entering state at position T-1)
+        const bool has_last = dir > 0 && unit_end;
+        auto lam_of = [&](int s) -> float {
+            return (has_last && s == ns - 1) ? pw[nlast] : ((first_rev && s == 0) ? pw[nlast - 1] : lamTB);
+        };
+        {
+            const bool mine = (sj > 0 || R.init != nullptr) && owns_w_row;
             const double l2 = log2(static_cast<double>(lam));
             const float fL = static_cast<float>(exp2(static_cast<double>(kTB) * p.seg_tiles * l2));
             // segment 0 has n0 tiles; in the reverse direction its first tile
@@ -987,36 +994,55 @@ la2_scan_ws(const __grid_constant__ Params p)
                                       : static_cast<double>(kTB) * (n0 - 1) + (nlast - 1);
             const float f0 = static_cast<float>(exp2(e0 * l2));
             const float* w0 = R.init ? R.init + static_cast<size_t>(bh) * (DA * DC) : nullptr;
+            // DC = 128: the fp32 state in TMEM starts as lambda(0) W_in, so that dW
+            // of step 0 accumulates onto it (every lane stores; rows a thread
+            // does not own are 0)
+            const float f0s = lam_of(0);
+            float wt[Q::kWT ? 32 : 1];
 #pragma unroll
             for (int k = 0; k < kCols / 16; ++k) {
                 const uint32_t col = c0 + k * 16;
                 float w[16];
-                if (w0 && R.init_t) {
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) w[u] = w0[static_cast<size_t>(col + u) * DA + wrow];
-                } else {
+                for (int u = 0; u < 16; ++u) w[u] = 0.f;
+                if (mine) {
+                    if (w0 && R.init_t) {
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) w[u] = w0 ? w0[static_cast<size_t>(wrow) * DC + col + u] : 0.f;
+                        for (int u = 0; u < 16; ++u) w[u] = w0[static_cast<size_t>(col + u) * DA + wrow];
+                    } else if (w0) {
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) w[u] = w0[static_cast<size_t>(wrow) * DC + col + u];
+                    }
+                    for (int gp = 0; gp < sj; ++gp) {
+                        const float f = gp == 0 ? f0 : fL;
+                        const float* src = seg_slot(gp) + static_cast<size_t>(wrow) * DC + col;
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) w[u] = fmaf(f, w[u], src[u]);
+                    }
+                    if constexpr (kWReg) {
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) wreg[16 * (k & 1) + u] = w[u];
+                    }
+                    const uint32_t grpo = (col >> 6) * (DA * 128);
+                    const int q = (col & 63) >> 3;
+                    uint32_t h[8], l[8];
+#pragma unroll
+                    for (int z = 0; z < 8; ++z) split_pack2(w[2 * z], w[2 * z + 1], h[z], l[z]);
+                    st_shared_v4(sW + grpo + sw128(wrow, q), h[0], h[1], h[2], h[3]);
+                    st_shared_v4(sW + grpo + sw128(wrow, q + 1), h[4], h[5], h[6], h[7]);
+                    st_shared_v4(sW + L::kWsz + grpo + sw128(wrow, q), l[0], l[1], l[2], l[3]);
+                    st_shared_v4(sW + L::kWsz + grpo + sw128(wrow, q + 1), l[4], l[5], l[6], l[7]);
                 }
-                for (int gp = 0; gp < sj; ++gp) {
-                    const float f = gp == 0 ? f0 : fL;
-                    const float* src = seg_slot(gp) + static_cast<size_t>(wrow) * DC + col;
+                if constexpr (Q::kWT) {
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) w[u] = fmaf(f, w[u], src[u]);
+                    for (int u = 0; u < 16; ++u) wt[16 * (k & 1) + u] = f0s * w[u];
+                    if (k & 1) tmem_st32(tD(0) + lane_off + col - 16, wt);
                 }
-                if constexpr (kWReg) {
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) wreg[16 * (k & 1) + u] = w[u];
-                }
-                const uint32_t grpo = (col >> 6) * (DA * 128);
-                const int q = (col & 63) >> 3;
-                uint32_t h[8], l[8];
-#pragma unroll
-                for (int z = 0; z < 8; ++z) split_pack2(w[2 * z], w[2 * z + 1], h[z], l[z]);
-                st_shared_v4(sW + grpo + sw128(wrow, q), h[0], h[1], h[2], h[3]);
-                st_shared_v4(sW + grpo + sw128(wrow, q + 1), h[4], h[5], h[6], h[7]);
-                st_shared_v4(sW + L::kWsz + grpo + sw128(wrow, q), l[0], l[1], l[2], l[3]);
-                st_shared_v4(sW + L::kWsz + grpo + sw128(wrow, q + 1), l[4], l[5], l[6], l[7]);
+            }
+            if constexpr (Q::kWT) {
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(Q::EMPTY_D));
             }
         }
         fence_proxy_async_smem();
@@ -1053,10 +1079,8 @@ la2_scan_ws(const __grid_constant__ Params p)
         // W <- lambda^T_B W + dW, from W buffer s % NW into (s+1) % NW.  The
         // state is kept as its hi + lo bf16 pair (a 16-bit significand, ~2^-17
         // relative per update), which is also the next tile's MMA operand.
-        const bool has_last = dir > 0 && unit_end;
         auto update = [&](int s) -> bool {
-            const bool last = has_last && s == ns - 1;
-            const float lam_s = last ? pw[nlast] : ((first_rev && s == 0) ? pw[nlast - 1] : lamTB);
+            const float lam_s = lam_of(s);
             if (!wait_bar<Q::kTf32>(bar(Q::D_DONE + (s % Q::ND)), full_par(s, Q::ND), abort_flag, p.status, 51))
                 return false;
             // the X MMA that last read the W buffer written here is done
@@ -1068,8 +1092,54 @@ la2_scan_ws(const __grid_constant__ Params p)
             const uint32_t wsrc = sW + (s % Q::NW) * 2 * L::kWsz;
             const uint32_t wdst = sW + ((s + 1) % Q::NW) * 2 * L::kWsz;
             const uint32_t dt = tD(s);
+            if constexpr (Q::kWT) {
+                // W_{s+1} = lambda(s) W_s + dW_s, accumulated in fp32 in TMEM: its
+                // hi/lo pair to the next A W's buffer, the final state from it,
+                // and lambda(s+1) W_{s+1} written back for the next dW
+                const bool more = s + 1 < ns;
+                const float lam_n = more ? lam_of(s + 1) : 1.f;
+                const bool fin_now = unit_end && s == ns - 1 && R.fin != nullptr && owns_w_row;
+                float* const fin = R.fin ? R.fin + static_cast<size_t>(bh) * (DA * DC) + static_cast<size_t>(wrow) * DC
+                                         : nullptr;
+                const float fs = dir > 0 ? 1.f : lam;
 #pragma unroll 1
-            for (int k = 0; k < kCols / 32; ++k) {
+                for (int k = 0; k < kCols / 32; ++k) {
+                    float w[32];
+                    tmem_ld32(dt + lane_off + c0 + k * 32, w);
+                    if (owns_w_row) {
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const uint32_t col = c0 + k * 32 + hh * 16;
+                            const uint32_t o0 = (col >> 6) * (DA * 128) + sw128(wrow, (col & 63) >> 3);
+                            const uint32_t o1 = (col >> 6) * (DA * 128) + sw128(wrow, ((col & 63) >> 3) + 1);
+                            uint32_t h[8], l[8];
+#pragma unroll
+                            for (int z = 0; z < 8; ++z)
+                                split_pack2v(make_float2(w[16 * hh + 2 * z], w[16 * hh + 2 * z + 1]), h[z], l[z]);
+                            st_shared_v4(wdst + o0, h[0], h[1], h[2], h[3]);
+                            st_shared_v4(wdst + o1, h[4], h[5], h[6], h[7]);
+                            st_shared_v4(wdst + L::kWsz + o0, l[0], l[1], l[2], l[3]);
+                            st_shared_v4(wdst + L::kWsz + o1, l[4], l[5], l[6], l[7]);
+                        }
+                    }
+                    if (fin_now) {
+                        // the final state in fp32; a reverse scan hands on lambda
+                        // times its state at position 0
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) fin[c0 + k * 32 + u] = fs * w[u];
+                    }
+                    if (more) {
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) w[u] *= lam_n;
+                        tmem_st32(dt + lane_off + c0 + k * 32, w);
+                    }
+                }
+                if (more) tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(Q::EMPTY_D));
+            }
+#pragma unroll 1
+            for (int k = 0; k < (Q::kWT ? 0 : kCols / 32); ++k) {
                 float d[32];
                 tmem_ld32(dt + lane_off + c0 + k * 32, d);
                 if (tid == 384 && k == 0) LA2_TR(23, s);
@@ -1125,10 +1195,10 @@ la2_scan_ws(const __grid_constant__ Params p)
                     }
                 }
             }
-            if (unit_end && s == ns - 1 && R.fin && owns_w_row) {
-                // the final state: fp32 from registers (32 columns per thread),
-                // else from the hi + lo pair just written; a reverse scan hands
-                // on lambda times its state at position 0
+            if (!Q::kWT && unit_end && s == ns - 1 && R.fin && owns_w_row) {
+                // the final state: fp32 from registers (32 columns per thread;
+                // DC = 128 wrote it above from TMEM); a reverse scan hands on
+                // lambda times its state at position 0
                 float* fin = R.fin + static_cast<size_t>(bh) * (DA * DC) + static_cast<size_t>(wrow) * DC;
                 const float fs = dir > 0 ? 1.f : lam;
                 if constexpr (kWReg) {
