@@ -51,7 +51,8 @@
 // memory holds two of most rings, and at DA = DC = 128 one A, C and W buffer
 // and two B buffers.  With DC = 64, X += P C, X_inter (two buffers) and dW
 // are separate TMEM accumulators; otherwise A W is scaled in place by w_x
-// before P C adds to it, and dW borrows the X buffer of the next tile.
+// before P C adds to it (one X buffer), and the fp32 state itself sits in
+// TMEM, dW accumulating onto it.
 //
 // Every hand-off is an mbarrier: each buffer has a "full" barrier its
 // producer completes and an "empty" barrier its consumers complete, so a
